@@ -1,0 +1,529 @@
+// Oracle for the gated-AdaLN DiT block over video latent tokens.
+//
+// TEST INFRASTRUCTURE ONLY. This file is the plain, slow, obviously-correct CPU
+// statement of what the block computes. Only the test suite, the smoke check and
+// the CPU-baseline leg of the benchmark may load it. The CUDA library shares no
+// code, header, table or helper with it, and nothing here reads from the CUDA
+// side.
+//
+// Sources (web pages about the h3.c / h3-metal engine for MiniMax-H3):
+//   [README]  "h3-metal: Apple Silicon을 위한 네이티브 MiniMax-H3 추론"
+//             sections "Int8 양자화", "Metal 4 및 TensorOps",
+//             "속도 및 품질 트레이드오프" (control table, Token Reduction row)
+//   [MLX]     "h3.c與MLX路線對比：MiniMax-H3在Apple Silicon上的兩種推理實現工程取捨"
+//             section "性能上限" (AdaLN gating, RoPE and quantization fused ahead
+//             of the projections)
+//   [BLOG]    "맥북에서 AI 영상 생성 모델 돌리기 - MiniMax H3 로컬 실행과 30초
+//             애니메이션 만들기", section "int8 이 뭔가요" (one F32 scale per
+//             output channel for weights, one F32 scale per row for activations,
+//             computed at run time)
+// The pages give the block only in outline. Every dimension, the LayerNorm eps,
+// the GELU form, the RoPE split and the modulation formula come from the
+// workload specification this project is built against (synthetic model
+// dimensions); each reading of a silent point is listed where it is used.
+//
+// Precision: every floating-point step is carried in fp64, except
+//   * the int8 decisions, which the pages fix in F32 (scale = absmax/127 in
+//     float, code = round-half-even(v / scale) in float), and
+//   * the roundings to bf16 that the method itself defines: the quantizer's input
+//     row is a bf16 activation, the block's input/output residual stream is bf16,
+//     and the merged tokens of token reduction are a bf16 block input.
+// int8 GEMMs accumulate exactly (int32 while no partial sum can overflow it,
+// else int64 with an overflow count).
+//
+// Parallelism: optional OpenMP over independent rows/heads; with
+// OMP_NUM_THREADS=1 it runs single-threaded with identical results (no
+// reduction crosses threads).
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <cstdlib>
+#include <vector>
+#include <algorithm>
+
+extern "C" {
+
+// ---------------------------------------------------------------------------
+// bf16 <-> fp64.  bf16 = the top 16 bits of an IEEE binary32.
+// ---------------------------------------------------------------------------
+double orc_bf16_to_f64(uint16_t b) {
+  uint32_t u = (uint32_t)b << 16;
+  float f;
+  std::memcpy(&f, &u, 4);
+  return (double)f;
+}
+
+// Round a double to the nearest bf16, ties to even, in ONE rounding step.
+// bf16 keeps 8 significant bits; normal exponents go down to 2^-126 and
+// subnormals are spaced 2^-133 apart. Values beyond the largest finite bf16
+// after rounding become infinity.
+uint16_t orc_f64_to_bf16(double v) {
+  if (std::isnan(v)) return 0x7FC0;
+  const bool neg = std::signbit(v);
+  double a = std::fabs(v);
+  double r;
+  if (a == 0.0) {
+    r = 0.0;
+  } else {
+    int e;
+    std::frexp(a, &e);              // a = m * 2^e, 0.5 <= m < 1
+    int q = e - 8;                  // quantum 2^(e-8) keeps 8 significant bits
+    if (q < -133) q = -133;         // subnormal spacing
+    r = std::nearbyint(std::ldexp(a, -q));  // default mode: ties to even
+    r = std::ldexp(r, q);
+  }
+  const double max_bf16 = std::ldexp(255.0, 120);  // (2 - 2^-7) * 2^127
+  float f = (r > max_bf16) ? INFINITY : (float)r;   // r is bf16-exact, so exact in float
+  uint32_t u;
+  std::memcpy(&u, &f, 4);
+  uint16_t b = (uint16_t)(u >> 16);
+  if (neg) b |= 0x8000;
+  return b;
+}
+
+void orc_bf16_round(const double* v, int64_t n, uint16_t* out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = orc_f64_to_bf16(v[i]);
+}
+
+void orc_bf16_decode(const uint16_t* b, int64_t n, double* out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = orc_bf16_to_f64(b[i]);
+}
+
+// ---------------------------------------------------------------------------
+// Symmetric int8 quantization with one F32 scale per row ([BLOG] "int8 이 뭔가요";
+// [README] "Int8 양자화": dynamic activation quantization, per-output-channel
+// weight scales). The same rule serves activations (row = token) and weights
+// (row = output channel).
+//   scale = absmax(row) / 127            (float division)
+//   code  = clamp(rint(v / scale), -127, 127)   (float division, ties to even)
+// An all-zero row has scale 0 and codes 0 (no division). -128 is never produced.
+// ---------------------------------------------------------------------------
+void orc_quantize_rows(const float* v, int64_t rows, int64_t cols, int8_t* q, float* s) {
+#pragma omp parallel for schedule(static)
+  for (int64_t r = 0; r < rows; ++r) {
+    const float* row = v + r * cols;
+    float absmax = 0.0f;
+    for (int64_t c = 0; c < cols; ++c) absmax = std::max(absmax, std::fabs(row[c]));
+    const float scale = absmax / 127.0f;
+    s[r] = scale;
+    for (int64_t c = 0; c < cols; ++c) {
+      if (absmax == 0.0f) { q[r * cols + c] = 0; continue; }
+      float t = std::nearbyint(row[c] / scale);
+      t = std::min(127.0f, std::max(-127.0f, t));
+      q[r * cols + c] = (int8_t)t;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Exact int8 GEMM: C[m][n] = sum_k A[m][k] * W[n][k]  (both operands row-major,
+// W stored [out][in]). Accumulates in int64; returns the number of results that
+// do not fit int32 (0 when every accumulator is representable).
+// ---------------------------------------------------------------------------
+int64_t orc_gemm_i8(const int8_t* A, const int8_t* W, int64_t M, int64_t N, int64_t K, int32_t* C) {
+  // |a*w| <= 128*128, so while K * 16384 <= INT32_MAX no partial sum can leave
+  // int32 and the int32 sum below is exact; longer rows use int64.
+  int64_t overflow = 0;
+  const bool fits32 = K * 16384 <= (int64_t)INT32_MAX;
+#pragma omp parallel for schedule(dynamic, 4) reduction(+ : overflow)
+  for (int64_t m = 0; m < M; ++m) {
+    const int8_t* a = A + m * K;
+    for (int64_t n = 0; n < N; ++n) {
+      const int8_t* w = W + n * K;
+      if (fits32) {
+        int32_t acc = 0;
+        for (int64_t k = 0; k < K; ++k) acc += (int32_t)a[k] * (int32_t)w[k];
+        C[m * N + n] = acc;
+      } else {
+        int64_t acc = 0;
+        for (int64_t k = 0; k < K; ++k) acc += (int64_t)a[k] * (int64_t)w[k];
+        if (acc > INT32_MAX || acc < INT32_MIN) ++overflow;
+        C[m * N + n] = (int32_t)acc;
+      }
+    }
+  }
+  return overflow;
+}
+
+// fp64 GEMM on doubles: C[m][n] = sum_k A[m][k] * W[n][k]  (for the bf16-QKV variant).
+void orc_gemm_f64(const double* A, const double* W, int64_t M, int64_t N, int64_t K, double* C) {
+#pragma omp parallel for schedule(dynamic, 4)
+  for (int64_t m = 0; m < M; ++m) {
+    const double* a = A + m * K;
+    for (int64_t n = 0; n < N; ++n) {
+      const double* w = W + n * K;
+      double acc = 0.0;
+      for (int64_t k = 0; k < K; ++k) acc += a[k] * w[k];
+      C[m * N + n] = acc;
+    }
+  }
+}
+
+// Dequantization of an int8 GEMM result: out = acc * s_tok[row] * s_ch[col] + bias[col].
+void orc_dequant(const int32_t* acc, int64_t rows, int64_t cols, const float* s_tok,
+                 const float* s_ch, const float* bias, double* out) {
+#pragma omp parallel for schedule(static)
+  for (int64_t r = 0; r < rows; ++r)
+    for (int64_t c = 0; c < cols; ++c)
+      out[r * cols + c] = (double)acc[r * cols + c] * (double)s_tok[r] * (double)s_ch[c] +
+                          (bias ? (double)bias[c] : 0.0);
+}
+
+// ---------------------------------------------------------------------------
+// AdaLN modulation Linear: mod[j] = sum_k W_ada[j][k] * c[k] + b[j], j in [0, 6d).
+// W_ada is bf16 [6d][d]. The six d-long chunks are, in order:
+// shift_attn, scale_attn, gate_attn, shift_mlp, scale_mlp, gate_mlp
+// (the original DiT ordering; the pages name gated AdaLN ([README] "Int8 양자화",
+// fused kernels bullet; [MLX] "性能上限") but not the chunk order; no SiLU on c,
+// the specification says only "Linear").
+// ---------------------------------------------------------------------------
+void orc_adaln_linear(const uint16_t* w_ada, const float* b_ada, const float* c, int64_t d,
+                      double* mod) {
+#pragma omp parallel for schedule(static)
+  for (int64_t j = 0; j < 6 * d; ++j) {
+    double acc = 0.0;
+    for (int64_t k = 0; k < d; ++k) acc += orc_bf16_to_f64(w_ada[j * d + k]) * (double)c[k];
+    mod[j] = acc + (b_ada ? (double)b_ada[j] : 0.0);
+  }
+}
+
+// LayerNorm without affine: y = (x - mean) / sqrt(var + eps), biased variance.
+void orc_layernorm(const double* x, int64_t rows, int64_t d, double eps, double* y) {
+#pragma omp parallel for schedule(static)
+  for (int64_t r = 0; r < rows; ++r) {
+    const double* xr = x + r * d;
+    double mean = 0.0;
+    for (int64_t i = 0; i < d; ++i) mean += xr[i];
+    mean /= (double)d;
+    double var = 0.0;
+    for (int64_t i = 0; i < d; ++i) var += (xr[i] - mean) * (xr[i] - mean);
+    var /= (double)d;
+    const double inv = 1.0 / std::sqrt(var + eps);
+    for (int64_t i = 0; i < d; ++i) y[r * d + i] = (xr[i] - mean) * inv;
+  }
+}
+
+// Modulation: h = y * (1 + scale) + shift, then rounded to bf16 because the
+// quantizer's input row is a bf16 activation (reading: the pages quantize bf16
+// activations; the rounding point is not stated).
+void orc_modulate_bf16(const double* y, int64_t rows, int64_t d, const double* shift,
+                       const double* scale, uint16_t* h) {
+#pragma omp parallel for schedule(static)
+  for (int64_t r = 0; r < rows; ++r)
+    for (int64_t i = 0; i < d; ++i)
+      h[r * d + i] = orc_f64_to_bf16(y[r * d + i] * (1.0 + scale[i]) + shift[i]);
+}
+
+// Latent grid positions of token i (flattened t-major, then h, then w).
+void orc_grid_positions(int64_t T, int64_t H, int64_t W, int32_t* tp, int32_t* hp, int32_t* wp) {
+  for (int64_t i = 0; i < T * H * W; ++i) {
+    tp[i] = (int32_t)(i / (H * W));
+    hp[i] = (int32_t)((i / W) % H);
+    wp[i] = (int32_t)(i % W);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// 3D RoPE, in place on rows of n_heads*dh channels (channel = head*dh + lane).
+// [MLX] "性能上限" says RoPE is folded into the kernel before the projections;
+// the split and pairing are readings: lanes [0,rt) rotate by the frame index t,
+// [rt, rt+rh) by the row index h, [rt+rh, dh) by the column index w. Inside a
+// segment of length r, lanes (2j, 2j+1) form a pair with frequency
+// theta^(-2j/r), and (x0, x1) -> (x0 cos a - x1 sin a, x0 sin a + x1 cos a),
+// a = position * frequency.
+// ---------------------------------------------------------------------------
+void orc_rope_3d(double* x, int64_t rows, const int32_t* tp, const int32_t* hp, const int32_t* wp,
+                 int n_heads, int dh, int rt, int rh, int rw, double theta) {
+  (void)rw;
+#pragma omp parallel for schedule(static)
+  for (int64_t r = 0; r < rows; ++r) {
+    for (int hd = 0; hd < n_heads; ++hd) {
+      double* v = x + r * (int64_t)n_heads * dh + (int64_t)hd * dh;
+      for (int lane = 0; lane < dh; lane += 2) {
+        int seg_start, seg_len;
+        int32_t pos;
+        if (lane < rt) { seg_start = 0; seg_len = rt; pos = tp[r]; }
+        else if (lane < rt + rh) { seg_start = rt; seg_len = rh; pos = hp[r]; }
+        else { seg_start = rt + rh; seg_len = dh - rt - rh; pos = wp[r]; }
+        const int j = (lane - seg_start) / 2;
+        const double freq = std::pow(theta, -2.0 * j / (double)seg_len);
+        const double a = (double)pos * freq;
+        const double c = std::cos(a), s = std::sin(a);
+        const double x0 = v[lane], x1 = v[lane + 1];
+        v[lane] = x0 * c - x1 * s;
+        v[lane + 1] = x0 * s + x1 * c;
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Full non-causal softmax attention per head (the pages' per-step time grows
+// roughly as frames^1.9, [BLOG] "★ 긴 영상은 나눠 찍는 게 훨씬 쌉니다", which is the
+// signature of full attention over all latent tokens).
+//   O[i] = sum_j softmax_j(Q[i].K[j] / sqrt(dh)) V[j]
+// Q: [nq][n_heads*dh] query rows; K, V: [L][n_heads*dh]; O: [nq][n_heads*dh].
+// The softmax subtracts the row maximum before exponentiating.
+// ---------------------------------------------------------------------------
+void orc_attention(const double* Q, const double* K, const double* V, int64_t nq, int64_t L,
+                   int n_heads, int dh, double* O) {
+  const int64_t D = (int64_t)n_heads * dh;
+  const double inv_sqrt = 1.0 / std::sqrt((double)dh);
+#pragma omp parallel for collapse(2) schedule(dynamic, 1)
+  for (int64_t i = 0; i < nq; ++i) {
+    for (int hd = 0; hd < n_heads; ++hd) {
+      std::vector<double> sc((size_t)L);
+      const double* q = Q + i * D + (int64_t)hd * dh;
+      double mx = -INFINITY;
+      for (int64_t j = 0; j < L; ++j) {
+        const double* k = K + j * D + (int64_t)hd * dh;
+        double dot = 0.0;
+        for (int e = 0; e < dh; ++e) dot += q[e] * k[e];
+        sc[(size_t)j] = dot * inv_sqrt;
+        mx = std::max(mx, sc[(size_t)j]);
+      }
+      double sum = 0.0;
+      for (int64_t j = 0; j < L; ++j) { sc[(size_t)j] = std::exp(sc[(size_t)j] - mx); sum += sc[(size_t)j]; }
+      double* o = O + i * D + (int64_t)hd * dh;
+      for (int e = 0; e < dh; ++e) o[e] = 0.0;
+      for (int64_t j = 0; j < L; ++j) {
+        const double p = sc[(size_t)j] / sum;
+        const double* v = V + j * D + (int64_t)hd * dh;
+        for (int e = 0; e < dh; ++e) o[e] += p * v[e];
+      }
+    }
+  }
+}
+
+// GELU, tanh form: 0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3))).
+void orc_gelu_tanh(const double* x, int64_t n, double* y) {
+  const double k = std::sqrt(2.0 / M_PI);
+  for (int64_t i = 0; i < n; ++i) {
+    const double v = x[i];
+    y[i] = 0.5 * v * (1.0 + std::tanh(k * (v + 0.044715 * v * v * v)));
+  }
+}
+
+// Gated residual: out = x + gate * y (gate broadcast over rows).
+void orc_gated_residual(const double* x, const double* y, const double* gate, int64_t rows,
+                        int64_t d, double* out) {
+  for (int64_t r = 0; r < rows; ++r)
+    for (int64_t i = 0; i < d; ++i) out[r * d + i] = x[r * d + i] + gate[i] * y[r * d + i];
+}
+
+// ---------------------------------------------------------------------------
+// Token reduction ([README] control table, "Token Reduction": horizontally
+// adjacent video tokens are paired in the middle blocks).
+// pair:   xm[t,h,k] = bf16((x[t,h,2k] + x[t,h,2k+1]) / 2)   (the merged tokens are
+//         a bf16 block input)
+// unpair: out[t,h,2k+j] = x[t,h,2k+j] + (ym[t,h,k] - xm[t,h,k]),  j in {0,1}
+//         (the block's delta on the merged token is added back at both of its
+//         positions of the unmerged residual)
+// Layout [B][T][H][W][d]; W must be even.
+// ---------------------------------------------------------------------------
+void orc_token_pair(const uint16_t* x, int64_t B, int64_t T, int64_t H, int64_t W, int64_t d,
+                    uint16_t* xm) {
+  const int64_t Wm = W / 2;
+  for (int64_t row = 0; row < B * T * H; ++row)
+    for (int64_t k = 0; k < Wm; ++k)
+      for (int64_t i = 0; i < d; ++i) {
+        const double a = orc_bf16_to_f64(x[(row * W + 2 * k) * d + i]);
+        const double b = orc_bf16_to_f64(x[(row * W + 2 * k + 1) * d + i]);
+        xm[(row * Wm + k) * d + i] = orc_f64_to_bf16((a + b) / 2.0);
+      }
+}
+
+void orc_token_unpair(const uint16_t* x, const uint16_t* xm, const double* ym, int64_t B, int64_t T,
+                      int64_t H, int64_t W, int64_t d, double* out) {
+  const int64_t Wm = W / 2;
+  for (int64_t row = 0; row < B * T * H; ++row)
+    for (int64_t w = 0; w < W; ++w)
+      for (int64_t i = 0; i < d; ++i) {
+        const int64_t m = (row * Wm + w / 2) * d + i;
+        out[(row * W + w) * d + i] =
+            orc_bf16_to_f64(x[(row * W + w) * d + i]) + (ym[m] - orc_bf16_to_f64(xm[m]));
+      }
+}
+
+// ---------------------------------------------------------------------------
+// One DiT block, forward.
+// ---------------------------------------------------------------------------
+typedef struct {
+  int64_t B, T, H, W;          // latent grid, L = T*H*W tokens per batch item
+  int64_t d, n_heads, head_dim, d_ff;
+  int rope_t, rope_h, rope_w;
+  double rope_theta, ln_eps;
+  int qkv_int8;                // 1: int8 QKV (default); 0: bf16 QKV
+} orc_dims;
+
+typedef struct {
+  const uint16_t* w_ada; const float* b_ada;        // bf16 [6d][d], fp32 [6d] or NULL
+  const int8_t* wqkv; const float* sqkv;            // int8 [3d][d] + fp32 [3d]
+  const uint16_t* wqkv_bf16;                        // bf16 [3d][d] (qkv_int8 == 0)
+  const float* bqkv;                                // fp32 [3d] or NULL
+  const int8_t* wo; const float* so; const float* bo;  // [d][d]
+  const int8_t* w1; const float* s1; const float* b1;  // [d_ff][d]
+  const int8_t* w2; const float* s2; const float* b2;  // [d][d_ff]
+} orc_weights;
+
+// Optional intermediate dumps (each pointer may be NULL).
+typedef struct {
+  double* mod;        // [B][6d]
+  uint16_t* h1;       // [B*L][d]  modulated LN output (attention branch), bf16
+  double* qkv;        // [B*L][3d] Q,K,V after dequant and RoPE (token-major)
+  double* attn;       // [n_rows][d] attention output before rounding
+  double* x1;         // [n_rows][d] residual after the attention branch
+  uint16_t* h2;       // [n_rows][d] modulated LN output (MLP branch), bf16
+  double* gelu;       // [n_rows][d_ff] GELU output before rounding
+} orc_trace;
+
+// Block forward. x: bf16 [B][L][d]. c: fp32 [B][d]. The result is written for
+// the rows listed in `rows` (indices into B*L; all rows in order when rows is
+// NULL and n_rows == B*L) as fp64 [n_rows][d].
+//
+// Order of steps (gated AdaLN, [README] "Int8 양자화" fused-kernel bullet; [MLX]
+// "性能上限"):
+//   mod = AdaLN Linear(c)
+//   h1  = bf16(LN(x) * (1 + scale_a) + shift_a);  A1, s1 = quant(h1)
+//   QKV = deq(A1 Wqkv^T) + b;  RoPE(Q), RoPE(K)   (or bf16 h1 @ bf16 Wqkv^T)
+//   O   = attention(Q, K, V);  A2, s2 = quant(bf16(O))
+//   x1  = x + gate_a * (deq(A2 Wo^T) + bo)
+//   h2  = bf16(LN(x1) * (1 + scale_m) + shift_m);  A3, s3 = quant(h2)
+//   G   = GELU(deq(A3 W1^T) + b1);  A4, s4 = quant(bf16(G))
+//   out = x1 + gate_m * (deq(A4 W2^T) + b2)
+// Returns 0, or -1 if an int8 accumulator overflowed int32.
+int orc_block_forward(const orc_dims* dm, const orc_weights* wt, const float* c, const uint16_t* x,
+                      const int64_t* rows, int64_t n_rows, double* out, orc_trace* tr) {
+  const int64_t B = dm->B, L = dm->T * dm->H * dm->W, d = dm->d, F = dm->d_ff;
+  const int64_t R = B * L, nh = dm->n_heads, dh = dm->head_dim;
+  int64_t overflow = 0;
+
+  // AdaLN modulation vectors per batch item.
+  std::vector<double> mod((size_t)(B * 6 * d));
+  for (int64_t b = 0; b < B; ++b) orc_adaln_linear(wt->w_ada, wt->b_ada, c + b * d, d, &mod[(size_t)(b * 6 * d)]);
+  auto chunk = [&](int64_t b, int k) { return &mod[(size_t)(b * 6 * d + k * d)]; };
+
+  // Attention branch input for ALL tokens (K and V need every row).
+  std::vector<double> xd((size_t)(R * d));
+  orc_bf16_decode(x, R * d, xd.data());
+  std::vector<double> y((size_t)(R * d));
+  orc_layernorm(xd.data(), R, d, dm->ln_eps, y.data());
+  std::vector<uint16_t> h1((size_t)(R * d));
+  for (int64_t b = 0; b < B; ++b)
+    orc_modulate_bf16(&y[(size_t)(b * L * d)], L, d, chunk(b, 0), chunk(b, 1), &h1[(size_t)(b * L * d)]);
+
+  std::vector<double> qkv((size_t)(R * 3 * d));
+  if (dm->qkv_int8) {
+    std::vector<float> h1f((size_t)(R * d));
+    for (int64_t i = 0; i < R * d; ++i) h1f[(size_t)i] = (float)orc_bf16_to_f64(h1[(size_t)i]);
+    std::vector<int8_t> A1((size_t)(R * d));
+    std::vector<float> s1((size_t)R);
+    orc_quantize_rows(h1f.data(), R, d, A1.data(), s1.data());
+    std::vector<int32_t> acc((size_t)(R * 3 * d));
+    overflow += orc_gemm_i8(A1.data(), wt->wqkv, R, 3 * d, d, acc.data());
+    orc_dequant(acc.data(), R, 3 * d, s1.data(), wt->sqkv, wt->bqkv, qkv.data());
+  } else {
+    std::vector<double> hd((size_t)(R * d)), wd((size_t)(3 * d * d));
+    orc_bf16_decode(h1.data(), R * d, hd.data());
+    orc_bf16_decode(wt->wqkv_bf16, 3 * d * d, wd.data());
+    orc_gemm_f64(hd.data(), wd.data(), R, 3 * d, d, qkv.data());
+    if (wt->bqkv)
+      for (int64_t r = 0; r < R; ++r)
+        for (int64_t o = 0; o < 3 * d; ++o) qkv[(size_t)(r * 3 * d + o)] += wt->bqkv[o];
+  }
+
+  // Split into token-major Q, K, V ([R][d] each; channel = head*dh + lane) and rotate Q, K.
+  std::vector<double> Q((size_t)(R * d)), K((size_t)(R * d)), V((size_t)(R * d));
+  for (int64_t r = 0; r < R; ++r)
+    for (int64_t i = 0; i < d; ++i) {
+      Q[(size_t)(r * d + i)] = qkv[(size_t)(r * 3 * d + i)];
+      K[(size_t)(r * d + i)] = qkv[(size_t)(r * 3 * d + d + i)];
+      V[(size_t)(r * d + i)] = qkv[(size_t)(r * 3 * d + 2 * d + i)];
+    }
+  std::vector<int32_t> tp((size_t)L), hp((size_t)L), wp((size_t)L);
+  orc_grid_positions(dm->T, dm->H, dm->W, tp.data(), hp.data(), wp.data());
+  for (int64_t b = 0; b < B; ++b) {
+    orc_rope_3d(&Q[(size_t)(b * L * d)], L, tp.data(), hp.data(), wp.data(), (int)nh, (int)dh,
+                dm->rope_t, dm->rope_h, dm->rope_w, dm->rope_theta);
+    orc_rope_3d(&K[(size_t)(b * L * d)], L, tp.data(), hp.data(), wp.data(), (int)nh, (int)dh,
+                dm->rope_t, dm->rope_h, dm->rope_w, dm->rope_theta);
+  }
+  if (tr && tr->mod) std::memcpy(tr->mod, mod.data(), mod.size() * sizeof(double));
+  if (tr && tr->h1) std::memcpy(tr->h1, h1.data(), h1.size() * sizeof(uint16_t));
+  if (tr && tr->qkv)
+    for (int64_t r = 0; r < R; ++r)
+      for (int64_t i = 0; i < d; ++i) {
+        tr->qkv[r * 3 * d + i] = Q[(size_t)(r * d + i)];
+        tr->qkv[r * 3 * d + d + i] = K[(size_t)(r * d + i)];
+        tr->qkv[r * 3 * d + 2 * d + i] = V[(size_t)(r * d + i)];
+      }
+
+  // From here on only the requested rows are carried.
+  std::vector<int64_t> sel((size_t)n_rows);
+  for (int64_t i = 0; i < n_rows; ++i) sel[(size_t)i] = rows ? rows[i] : i;
+
+  // Attention for the selected query rows, each against the keys of its own batch item.
+  std::vector<double> O((size_t)(n_rows * d));
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t i = 0; i < n_rows; ++i) {
+    const int64_t r = sel[(size_t)i], b = r / L;
+    orc_attention(&Q[(size_t)(r * d)], &K[(size_t)(b * L * d)], &V[(size_t)(b * L * d)], 1, L,
+                  (int)nh, (int)dh, &O[(size_t)(i * d)]);
+  }
+  if (tr && tr->attn) std::memcpy(tr->attn, O.data(), O.size() * sizeof(double));
+
+  // Attention output projection with gated residual.
+  std::vector<float> Of((size_t)(n_rows * d));
+  for (int64_t i = 0; i < n_rows * d; ++i) Of[(size_t)i] = (float)orc_bf16_to_f64(orc_f64_to_bf16(O[(size_t)i]));
+  std::vector<int8_t> A2((size_t)(n_rows * d));
+  std::vector<float> s2((size_t)n_rows);
+  orc_quantize_rows(Of.data(), n_rows, d, A2.data(), s2.data());
+  std::vector<int32_t> acc2((size_t)(n_rows * d));
+  overflow += orc_gemm_i8(A2.data(), wt->wo, n_rows, d, d, acc2.data());
+  std::vector<double> yo((size_t)(n_rows * d));
+  orc_dequant(acc2.data(), n_rows, d, s2.data(), wt->so, wt->bo, yo.data());
+  std::vector<double> x1((size_t)(n_rows * d));
+  for (int64_t i = 0; i < n_rows; ++i) {
+    const int64_t r = sel[(size_t)i], b = r / L;
+    orc_gated_residual(&xd[(size_t)(r * d)], &yo[(size_t)(i * d)], chunk(b, 2), 1, d, &x1[(size_t)(i * d)]);
+  }
+  if (tr && tr->x1) std::memcpy(tr->x1, x1.data(), x1.size() * sizeof(double));
+
+  // MLP branch.
+  std::vector<double> y2((size_t)(n_rows * d));
+  orc_layernorm(x1.data(), n_rows, d, dm->ln_eps, y2.data());
+  std::vector<uint16_t> h2((size_t)(n_rows * d));
+  for (int64_t i = 0; i < n_rows; ++i) {
+    const int64_t b = sel[(size_t)i] / L;
+    orc_modulate_bf16(&y2[(size_t)(i * d)], 1, d, chunk(b, 3), chunk(b, 4), &h2[(size_t)(i * d)]);
+  }
+  if (tr && tr->h2) std::memcpy(tr->h2, h2.data(), h2.size() * sizeof(uint16_t));
+  std::vector<float> h2f((size_t)(n_rows * d));
+  for (int64_t i = 0; i < n_rows * d; ++i) h2f[(size_t)i] = (float)orc_bf16_to_f64(h2[(size_t)i]);
+  std::vector<int8_t> A3((size_t)(n_rows * d));
+  std::vector<float> s3((size_t)n_rows);
+  orc_quantize_rows(h2f.data(), n_rows, d, A3.data(), s3.data());
+  std::vector<int32_t> acc3((size_t)(n_rows * F));
+  overflow += orc_gemm_i8(A3.data(), wt->w1, n_rows, F, d, acc3.data());
+  std::vector<double> pre((size_t)(n_rows * F)), g((size_t)(n_rows * F));
+  orc_dequant(acc3.data(), n_rows, F, s3.data(), wt->s1, wt->b1, pre.data());
+  orc_gelu_tanh(pre.data(), n_rows * F, g.data());
+  if (tr && tr->gelu) std::memcpy(tr->gelu, g.data(), g.size() * sizeof(double));
+  std::vector<float> gf((size_t)(n_rows * F));
+  for (int64_t i = 0; i < n_rows * F; ++i) gf[(size_t)i] = (float)orc_bf16_to_f64(orc_f64_to_bf16(g[(size_t)i]));
+  std::vector<int8_t> A4((size_t)(n_rows * F));
+  std::vector<float> s4((size_t)n_rows);
+  orc_quantize_rows(gf.data(), n_rows, F, A4.data(), s4.data());
+  std::vector<int32_t> acc4((size_t)(n_rows * d));
+  overflow += orc_gemm_i8(A4.data(), wt->w2, n_rows, d, F, acc4.data());
+  std::vector<double> y4((size_t)(n_rows * d));
+  orc_dequant(acc4.data(), n_rows, d, s4.data(), wt->s2, wt->b2, y4.data());
+  for (int64_t i = 0; i < n_rows; ++i) {
+    const int64_t b = sel[(size_t)i] / L;
+    orc_gated_residual(&x1[(size_t)(i * d)], &y4[(size_t)(i * d)], chunk(b, 5), 1, d, &out[i * d]);
+  }
+  return overflow ? -1 : 0;
+}
+
+}  // extern "C"

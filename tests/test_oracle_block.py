@@ -1,0 +1,107 @@
+"""Block-level pins of the CPU oracle (no GPU needed).
+
+The steps are pinned one by one in test_oracle_pins.py; these check how the
+block composes them: the gate chunks really gate (a zero gate gives an exact
+identity), a sampled-row evaluation equals the full evaluation on those rows,
+batch items are independent, and the quantities fed between steps have the
+sizes the method implies.
+"""
+import numpy as np
+import pytest
+
+import oracle as O
+from video_diffusion_transformer_adaln_b200 import synth
+
+WL = synth.WORKLOADS["d256_L512"].with_(T=1, H=8, W=8)  # 64 tokens, d=256: seconds on one core
+
+
+def _weights(wl, block=0, zero_gates=False):
+    raw = synth.block_weights(wl, block)
+    w = {"w_ada": raw["w_ada"], "b_ada": raw["b_ada"].copy()}
+    if zero_gates:
+        d = wl.d
+        w["b_ada"][2 * d:3 * d] = 0
+        w["b_ada"][5 * d:6 * d] = 0
+    for name, sname in (("wqkv", "sqkv"), ("wo", "so"), ("w1", "s1"), ("w2", "s2")):
+        w[name], w[sname] = O.quantize_rows(raw[name])
+    if "wqkv_bf16" in raw:
+        w["wqkv_bf16"] = raw["wqkv_bf16"]
+    return w
+
+
+def _dims(wl):
+    return O.Dims(wl.B, wl.T, wl.H, wl.W, wl.d, wl.n_heads, wl.head_dim, wl.d_ff, wl.rope,
+                  wl.rope_theta, wl.ln_eps, wl.qkv_int8)
+
+
+def test_zero_gates_give_exact_identity():
+    wl = WL
+    x = synth.x_input(wl)
+    out = O.block_forward(_dims(wl), _weights(wl, zero_gates=True), synth.cond(wl), x)
+    assert np.array_equal(out, O.bf16_decode(x).reshape(-1, wl.d))
+
+
+def test_zero_mlp_gate_leaves_attention_residual():
+    wl = WL
+    w = _weights(wl)
+    w["b_ada"][5 * wl.d:] = 0
+    x = synth.x_input(wl)
+    out, tr = O.block_forward(_dims(wl), w, synth.cond(wl), x, trace=True)
+    assert np.array_equal(out, tr["x1"])
+    assert not np.array_equal(out, O.bf16_decode(x).reshape(-1, wl.d))
+
+
+def test_sampled_rows_equal_full_rows():
+    wl = WL
+    w = _weights(wl)
+    x, c = synth.x_input(wl), synth.cond(wl)
+    full = O.block_forward(_dims(wl), w, c, x)
+    rows = synth.sample_rows(wl.L, 9)
+    part = O.block_forward(_dims(wl), w, c, x, rows=rows)
+    assert np.array_equal(part, full[rows])
+
+
+def test_batch_items_are_independent():
+    wl = WL
+    w = _weights(wl)
+    wl2 = wl.with_(B=2)
+    x2, c2 = synth.x_input(wl2), synth.cond(wl2)
+    out2 = O.block_forward(_dims(wl2), w, c2, x2)
+    for b in range(2):
+        ob = O.block_forward(_dims(wl), w, c2[b:b + 1], x2[b:b + 1])
+        assert np.array_equal(out2[b * wl.L:(b + 1) * wl.L], ob)
+
+
+def test_trace_quantities_are_consistent():
+    wl = WL
+    w = _weights(wl)
+    x, c = synth.x_input(wl), synth.cond(wl)
+    out, tr = O.block_forward(_dims(wl), w, c, x, trace=True)
+    d = wl.d
+    # mod = AdaLN Linear(c), gates = the seeded gate biases (gate rows are zero)
+    assert np.max(np.abs(tr["mod"][0] - O.adaln_linear(w["w_ada"], w["b_ada"], c[0]))) == 0
+    assert np.max(np.abs(tr["mod"][0, 2 * d:3 * d] - w["b_ada"][2 * d:3 * d])) < 1e-12
+    # h1 = bf16(LN(x) (1 + scale) + shift)
+    y = O.layernorm(O.bf16_decode(x).reshape(-1, d), wl.ln_eps)
+    assert np.array_equal(tr["h1"], O.modulate_bf16(y, tr["mod"][0, :d], tr["mod"][0, d:2 * d]))
+    # Q and K are rotated (norm per pair preserved vs unrotated projections), V is not
+    q1, s1 = O.quantize_rows(O.bf16_decode(tr["h1"]).astype(np.float32))
+    raw = O.dequant(O.gemm_i8(q1, w["wqkv"]), s1, w["sqkv"])
+    assert np.max(np.abs(tr["qkv"][:, 2 * d:] - raw[:, 2 * d:])) == 0
+    qk = tr["qkv"][:, :2 * d]
+    assert np.max(np.abs(np.hypot(qk[:, 0::2], qk[:, 1::2]) - np.hypot(raw[:, :2 * d:2], raw[:, 1:2 * d:2]))) < 1e-9
+    assert not np.allclose(qk, raw[:, :2 * d])
+    # GELU output feeds a per-row quantizer of width d_ff
+    assert tr["gelu"].shape == (wl.L, wl.d_ff)
+    assert np.isfinite(out).all()
+
+
+def test_bf16_qkv_variant_runs_and_differs_slightly():
+    wl = WL.with_(qkv_int8=False)
+    w = _weights(wl)
+    x, c = synth.x_input(wl), synth.cond(wl)
+    a = O.block_forward(_dims(wl), w, c, x)
+    b = O.block_forward(_dims(WL), _weights(WL), c, x)
+    xd = O.bf16_decode(x).reshape(-1, wl.d)
+    rel = np.linalg.norm((a - xd) - (b - xd)) / np.linalg.norm(a - xd)
+    assert 0 < rel < 0.1  # int8 vs bf16 QKV: close but not identical deltas
