@@ -1,0 +1,237 @@
+/*
+ * h3b — forward pass of one gated-AdaLN DiT block over video latent tokens, on
+ * NVIDIA B200 (sm_100a). C ABI: plain pointers and sizes, no framework types.
+ *
+ * The method (web pages about the h3.c / h3-metal MiniMax-H3 engine):
+ *   "h3-metal: Apple Silicon을 위한 네이티브 MiniMax-H3 추론"
+ *       section "Int8 양자화": int8 MLP and QKV with dynamic per-row activation
+ *       quantization and per-output-channel weight scales; the activation
+ *       quantizer is fused into the preceding gated-AdaLN kernel.
+ *       section "Metal 4 및 TensorOps": Q/K/V routed straight into a head-major
+ *       attention input.
+ *       section "속도 및 품질 트레이드오프" (Token Reduction row): horizontally
+ *       adjacent video tokens are paired in the middle blocks.
+ *   "h3.c與MLX路線對比：MiniMax-H3在Apple Silicon上的兩種推理實現工程取捨"
+ *       section "性能上限": AdaLN gating, RoPE and quantization folded into the
+ *       kernel ahead of the projections.
+ *   "맥북에서 AI 영상 생성 모델 돌리기 - MiniMax H3 로컬 실행과 30초 애니메이션 만들기"
+ *       section "int8 이 뭔가요": one F32 scale per output channel (weights),
+ *       one F32 scale per row computed at run time (activations).
+ * Dimensions, LayerNorm eps, GELU form and the RoPE split are parameters; the
+ * pages do not state them.
+ *
+ * Conventions for every entry point
+ *   - All tensor pointers are DEVICE pointers on the current CUDA device, owned
+ *     by the caller; the library never allocates device memory for the block and
+ *     keeps no state beyond per-device kernel attributes and one device-side
+ *     error word (h3b_device_error).
+ *   - Every call is asynchronous on `stream` (NULL = legacy default stream).
+ *   - bf16 tensors are passed as `void*` (IEEE bfloat16 bit patterns).
+ *   - Matrices are row-major. Weights are [out][in] (each output channel's input
+ *     weights contiguous).
+ *   - Arguments are validated on the host BEFORE any launch; on failure nothing
+ *     is launched and a negative h3b_status is returned. Launch failures are
+ *     reported as H3B_ERR_CUDA. Kernel faults surface at the caller's next
+ *     synchronization, as for any CUDA launch.
+ *   - Every device pointer must be 16-byte aligned.
+ *   - Device-side waits are bounded. A wait that runs out records a nonzero code
+ *     in the device error word and the kernel returns; read it with
+ *     h3b_device_error after synchronizing.
+ */
+#ifndef H3B_H
+#define H3B_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define H3B_API __attribute__((visibility("default")))
+#else
+#define H3B_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* h3b_stream; /* == cudaStream_t */
+
+typedef enum {
+  H3B_OK = 0,
+  H3B_ERR_ARG = -1,          /* NULL pointer or nonsensical value */
+  H3B_ERR_SHAPE = -2,        /* unsupported dimensions */
+  H3B_ERR_ALIGN = -3,        /* pointer not 16-byte aligned */
+  H3B_ERR_WORKSPACE = -4,    /* workspace smaller than h3b_workspace_size */
+  H3B_ERR_ARCH = -5,         /* current device is not compute capability 10.0 */
+  H3B_ERR_CUDA = -6,         /* a CUDA runtime/driver call failed */
+  H3B_ERR_DEVICE_CHECK = -7  /* the device error word is set */
+} h3b_status;
+
+/* Block dimensions.
+ *   Latent grid T x H x W per batch item, flattened t-major, then h, then w:
+ *   token l = (t*H + h)*W + w, L = T*H*W. B independent batch items.
+ *   d = n_heads * head_dim; head_dim in {64, 128}; d % 256 == 0, d <= 8192;
+ *   d_ff % 256 == 0, d_ff <= 32768.
+ *   RoPE: rope_t + rope_h + rope_w == head_dim, each even (3D RoPE; lanes
+ *   [0,rope_t) rotate with t, the next rope_h with h, the rest with w; pair
+ *   (2j, 2j+1) of a segment of length r has frequency rope_theta^(-2j/r)).
+ *   ln_eps: LayerNorm epsilon (no affine, biased variance).
+ *   qkv_int8: 1 = int8 QKV projection (default), 0 = bf16 QKV projection. */
+typedef struct {
+  int B, T, H, W;
+  int d, n_heads, head_dim, d_ff;
+  int rope_t, rope_h, rope_w;
+  float rope_theta, ln_eps;
+  int qkv_int8;
+} h3b_dims;
+
+/* Weights of one block (device pointers). int8 codes with one F32 scale per
+ * output channel (quantize them with h3b_quantize_weights). Biases may be NULL
+ * (zero). b_ada may be NULL.
+ *   w_ada     bf16 [6d][d]   AdaLN Linear; output chunks in order
+ *                            shift_attn, scale_attn, gate_attn, shift_mlp,
+ *                            scale_mlp, gate_mlp
+ *   b_ada     fp32 [6d]
+ *   wqkv      int8 [3d][d] + sqkv fp32 [3d]   (qkv_int8 == 1)
+ *   wqkv_bf16 bf16 [3d][d]                    (qkv_int8 == 0)
+ *   bqkv      fp32 [3d]; output channel o -> part o/d (Q, K, V),
+ *             head (o % d)/head_dim, lane o % head_dim
+ *   wo int8 [d][d]       + so fp32 [d],    bo fp32 [d]
+ *   w1 int8 [d_ff][d]    + s1 fp32 [d_ff], b1 fp32 [d_ff]
+ *   w2 int8 [d][d_ff]    + s2 fp32 [d],    b2 fp32 [d] */
+typedef struct {
+  const void* w_ada; const float* b_ada;
+  const int8_t* wqkv; const float* sqkv; const void* wqkv_bf16; const float* bqkv;
+  const int8_t* wo; const float* so; const float* bo;
+  const int8_t* w1; const float* s1; const float* b1;
+  const int8_t* w2; const float* s2; const float* b2;
+} h3b_block_weights;
+
+H3B_API const char* h3b_status_string(h3b_status s);
+
+/* Human-readable detail of the last failing call on this host thread (the
+ * failed check or CUDA call); empty when none. Owned by the library. */
+H3B_API const char* h3b_last_error_detail(void);
+
+/* Bytes of scratch workspace h3b_block_forward / h3b_blocks_forward need for
+ * these dimensions (regions aliased by lifetime). */
+H3B_API h3b_status h3b_workspace_size(const h3b_dims* dims, size_t* bytes);
+
+/* One block forward, in place on the residual stream x (bf16 [B][L][d]).
+ *   mod = AdaLN Linear(c)                                  c: fp32 [B][d]
+ *   A1,s1 = quant(bf16(LN(x)(1+scale_attn)+shift_attn))    (fused kernel)
+ *   Q,K,V = deq(A1 Wqkv^T)+bqkv, 3D RoPE on Q,K, written head-major
+ *   O = softmax(Q K^T / sqrt(head_dim)) V   (non-causal, per batch item, head)
+ *   x += gate_attn * (deq(quant(O) Wo^T) + bo)
+ *   A3,s3 = quant(bf16(LN(x)(1+scale_mlp)+shift_mlp))
+ *   G = bf16(GELU_tanh(deq(A3 W1^T)+b1))
+ *   x += gate_mlp * (deq(quant(G) W2^T) + b2)
+ * ws: device workspace of at least h3b_workspace_size bytes (256-byte aligned). */
+H3B_API h3b_status h3b_block_forward(const h3b_dims* dims, const h3b_block_weights* w, const float* c,
+                             void* x, void* ws, size_t ws_bytes, h3b_stream stream);
+
+/* n_blocks blocks in sequence on one residual stream x; block i uses w[i]
+ * (HOST array of n_blocks weight structs holding device pointers) and
+ * c + i*B*d (device, fp32 [n_blocks][B][d]). Same workspace as one block. */
+H3B_API h3b_status h3b_blocks_forward(const h3b_dims* dims, const h3b_block_weights* w, int n_blocks,
+                              const float* c, void* x, void* ws, size_t ws_bytes,
+                              h3b_stream stream);
+
+/* Token reduction ("Token Reduction" row of the control table): horizontally
+ * adjacent tokens w = 2k, 2k+1 of each (t, h) row are merged by their mean.
+ *   full: dims of the UNMERGED grid (W even).
+ *   x  bf16 [B][T][H][W][d] -> xm bf16 [B][T][H][W/2][d], xm = bf16((a+b)/2).
+ *   xm_copy: optional second destination receiving the same merged tokens
+ *   (e.g. the buffer the block then updates in place), or NULL. */
+H3B_API h3b_status h3b_token_pair(const h3b_dims* full, const void* x, void* xm, void* xm_copy,
+                          h3b_stream stream);
+
+/* out[t,h,2k+j] = bf16(x[t,h,2k+j] + (ym[t,h,k] - xm[t,h,k])), j in {0,1}:
+ * the block's delta on each merged token is added at both of its positions of
+ * the unmerged residual. out may alias x. */
+H3B_API h3b_status h3b_token_unpair(const h3b_dims* full, const void* x, const void* xm, const void* ym,
+                            void* out, h3b_stream stream);
+
+/* Per-output-channel weight quantization (offline): w fp32 [rows][cols] ->
+ * q int8 [rows][cols], s fp32 [rows]; s = absmax/127 (float),
+ * q = clamp(round-half-even(w/s), -127, 127); an all-zero row gives s = 0,
+ * q = 0. cols % 16 == 0. */
+H3B_API h3b_status h3b_quantize_weights(const float* w, int rows, int cols, int8_t* q, float* s,
+                                h3b_stream stream);
+
+/* Reads (and optionally clears) the device error word of the current device.
+ * Synchronizes the device. *code == 0 means no bounded wait ran out. */
+H3B_API h3b_status h3b_device_error(unsigned int* code, int clear);
+
+/* ---------------------------------------------------------------------------
+ * Step entry points. Each runs one step of the block on caller buffers; the
+ * block entry points above chain exactly these kernels. They exist so every
+ * step can be checked on its own.
+ * ------------------------------------------------------------------------- */
+
+/* AdaLN Linear: mod[b][j] = sum_k w_ada[j][k] c[b][k] + b_ada[j]; mod fp32 [B][6d]. */
+H3B_API h3b_status h3b_adaln_modulation(const h3b_dims* dims, const void* w_ada, const float* b_ada,
+                                const float* c, float* mod, h3b_stream stream);
+
+/* Fused LayerNorm + modulation + per-row int8 quantization over rows of x
+ * (bf16 [rows][d]); shift/scale fp32 [d] broadcast over rows_per_item rows,
+ * then advance by mod_stride floats per batch item (rows_per_item = L,
+ * mod_stride = 6d when reading a mod buffer; rows_per_item = rows for one set).
+ *   h = bf16(LN(x)(1+scale)+shift); s = absmax(h)/127; q = rint(h/s)
+ * q int8 [rows][d], s fp32 [rows]; h_out bf16 [rows][d] or NULL (writes h);
+ * absmax_zero: fp32 [rows] set to 0, or NULL. write_codes = 0 skips q/s. */
+H3B_API h3b_status h3b_ln_modulate_quantize(const void* x, int rows, int d, float eps, const float* shift,
+                                    const float* scale, int rows_per_item, int mod_stride,
+                                    int8_t* q, float* s, void* h_out, float* absmax_zero,
+                                    int write_codes, h3b_stream stream);
+
+/* Per-row int8 quantization of bf16 rows (h bf16 [rows][cols]). If absmax is
+ * non-NULL it holds each row's max |h| (as produced by the attention and GELU
+ * steps) and the row is read once; otherwise it is computed here. */
+H3B_API h3b_status h3b_quantize_rows(const void* h, int rows, int cols, const float* absmax, int8_t* q,
+                             float* s, h3b_stream stream);
+
+/* int8 GEMM on tensor cores, C[m][n] = sum_k A[m][k] W[n][k] (exact int32).
+ * A int8 [M][K], W int8 [N][K], C int32 [M][N]; M >= 1, N % 16 == 0, K % 16 == 0. */
+H3B_API h3b_status h3b_gemm_i8_s32(const int8_t* A, const int8_t* W, int32_t* C, int M, int N, int K,
+                           h3b_stream stream);
+
+/* int8 GEMM with dequantizing epilogue: out bf16 [M][N] = bf16(C*sA[m]*sW[n] + bias[n]). */
+H3B_API h3b_status h3b_gemm_i8_dequant(const int8_t* A, const float* sA, const int8_t* W, const float* sW,
+                               const float* bias, void* out, int M, int N, int K,
+                               h3b_stream stream);
+
+/* QKV projection with 3D RoPE, written head-major:
+ *   qkv bf16 [3][B][n_heads][L][head_dim] (part, batch item, head, token, lane).
+ * int8 (dims->qkv_int8 == 1): A int8 [B*L][d] + sA, w->wqkv + w->sqkv.
+ * bf16 (dims->qkv_int8 == 0): A bf16 [B*L][d] (sA ignored), w->wqkv_bf16.
+ * rope_ws: device scratch of at least h3b_rope_table_bytes(dims) bytes. */
+H3B_API h3b_status h3b_qkv_projection(const h3b_dims* dims, const void* A, const float* sA,
+                              const h3b_block_weights* w, void* qkv, void* rope_ws,
+                              h3b_stream stream);
+H3B_API size_t h3b_rope_table_bytes(const h3b_dims* dims);
+
+/* Non-causal attention per batch item and head on the head-major qkv buffer.
+ * o bf16 [B][L][d] (token-major, head h at columns [h*head_dim, (h+1)*head_dim));
+ * absmax fp32 [B*L]: each row's max |o| is max-combined into it (zero it first). */
+H3B_API h3b_status h3b_attention(const h3b_dims* dims, const void* qkv, void* o, float* absmax,
+                         h3b_stream stream);
+
+/* int8 GEMM with gated residual epilogue, in place on x bf16 [M][N]:
+ *   x[m][n] = bf16(x[m][n] + gate[m / rows_per_item][n] * (C*sA[m]*sW[n] + bias[n]))
+ * gate fp32, rows of gate_stride floats per batch item. */
+H3B_API h3b_status h3b_gemm_i8_gated_residual(const int8_t* A, const float* sA, const int8_t* W,
+                                      const float* sW, const float* bias, const float* gate,
+                                      int rows_per_item, int gate_stride, void* x, int M, int N,
+                                      int K, h3b_stream stream);
+
+/* int8 GEMM with GELU epilogue: g bf16 [M][N] = bf16(GELU_tanh(C*sA[m]*sW[n] + bias[n]));
+ * absmax fp32 [M] max-combined with each row's max |g| (zero it first). */
+H3B_API h3b_status h3b_gemm_i8_gelu(const int8_t* A, const float* sA, const int8_t* W, const float* sW,
+                            const float* bias, void* g, float* absmax, int M, int N, int K,
+                            h3b_stream stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* H3B_H */

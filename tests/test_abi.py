@@ -1,0 +1,114 @@
+"""The C ABI without a GPU: the library loads, exports every entry point the
+header declares, and rejects bad arguments on the host before any launch."""
+import ctypes as C
+import os
+import re
+
+import pytest
+import torch
+
+from video_diffusion_transformer_adaln_b200 import build, h3b, synth
+from video_diffusion_transformer_adaln_b200.runtime import dims_of
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "h3b.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return h3b.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(h3b_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = declared_functions()
+    assert len(names) >= 19
+    for n in names:
+        assert hasattr(L, n), n
+    # and the binding wraps each of them under the same name
+    for n in names:
+        assert hasattr(h3b, n) or n in ("h3b_status_string", "h3b_last_error_detail"), n
+
+
+def test_status_strings(L):
+    for code in h3b.STATUS:
+        assert h3b.status_string(code)
+
+
+def _dims(**kw):
+    wl = synth.WORKLOADS["d256_L512"]
+    d = dims_of(wl)
+    for k, v in kw.items():
+        setattr(d, k, v)
+    return d
+
+
+def test_workspace_size_host_only(L):
+    n = h3b.h3b_workspace_size(_dims())
+    wl = synth.WORKLOADS["d256_L512"]
+    R, D, F = wl.L, wl.d, wl.d_ff
+    # at least the int8 activations (R x F) and the bf16 Q/K/V + attention output (8 R D bytes)
+    assert n >= R * F + 8 * R * D
+    big = h3b.h3b_workspace_size(dims_of(synth.WORKLOADS["d5120_L18432"]))
+    assert 1.0e9 < big < 1.3e9
+
+
+@pytest.mark.parametrize("field,value", [("head_dim", 96), ("d", 300), ("d_ff", 1000), ("rope_t", 15),
+                                         ("B", 0), ("W", 0), ("n_heads", 3), ("B", 9)])
+def test_bad_dims_are_rejected(L, field, value):
+    with pytest.raises(h3b.H3BError) as e:
+        h3b.h3b_workspace_size(_dims(**{field: value}))
+    assert e.value.status in (-1, -2)
+
+
+def test_block_forward_validation_order(L):
+    d = _dims()
+    w = h3b.BlockWeights()
+    for n in h3b.WEIGHT_FIELDS:
+        setattr(w, n, 0x10000)
+    x = 0x20000
+    c = 0x30000
+    ws = 0x40000
+    need = h3b.h3b_workspace_size(d)
+    # NULL x
+    assert L.h3b_block_forward(C.byref(d), C.byref(w), c, None, ws, need, None) == -1
+    # misaligned x / workspace
+    assert L.h3b_block_forward(C.byref(d), C.byref(w), c, x + 2, ws, need, None) == -3
+    assert L.h3b_block_forward(C.byref(d), C.byref(w), c, x, ws + 16, need, None) == -3
+    # workspace too small
+    assert L.h3b_block_forward(C.byref(d), C.byref(w), c, x, ws, need - 1, None) == -4
+    # bad shape
+    bad = _dims(d_ff=100)
+    assert L.h3b_block_forward(C.byref(bad), C.byref(w), c, x, ws, need, None) == -2
+    # missing weight (placeholder pointers are never dereferenced: validation
+    # fails before any launch, on a GPU host as well)
+    w.w1 = None
+    st = L.h3b_block_forward(C.byref(d), C.byref(w), c, x, ws, need, None)
+    assert st in (-1, -5, -6)  # weights are checked after the device query on a GPU-less host
+
+
+def test_token_pair_validation(L):
+    full = _dims(W=15)
+    assert L.h3b_token_pair(C.byref(full), 0x1000, 0x2000, None, None) == -2
+    full = _dims()
+    assert L.h3b_token_pair(C.byref(full), None, 0x2000, None, None) == -1
+    assert L.h3b_token_pair(C.byref(full), 0x1008, 0x2000, None, None) == -3
+
+
+def test_gemm_validation(L):
+    assert L.h3b_gemm_i8_s32(0x1000, 0x2000, 0x3000, 128, 24, 128, None) == -2   # N % 16
+    assert L.h3b_gemm_i8_s32(0x1000, 0x2000, 0x3000, 128, 256, 100, None) == -2  # K % 16
+    assert L.h3b_gemm_i8_s32(0x1001, 0x2000, 0x3000, 128, 256, 128, None) == -3
+    assert L.h3b_gemm_i8_s32(None, 0x2000, 0x3000, 128, 256, 128, None) == -1
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="would launch on the placeholder pointers")
+def test_valid_call_without_a_b200_launches_nothing(L):
+    # On a host without a compute-capability-10.0 device the call stops at the
+    # device query with ARCH or CUDA status; it never reports success.
+    assert L.h3b_quantize_weights(0x1000, 4, 16, 0x2000, 0x3000, None) in (-5, -6)

@@ -1,0 +1,286 @@
+"""Step-by-step parity of the CUDA kernels against the CPU oracle, on the same
+seeded inputs (every input is generated on the host; no oracle input comes
+from the GPU except where a test re-quantizes the GPU's own bf16 quantizer
+input to check the bit-exact decision).
+
+Bars: integer/byte work bit-exact; bf16 outputs within the rounding the kernel
+performs (stated per test)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from gpu_helpers import (bf16_dev, bf16_host, bf16_ulp_diff, no_device_error, oracle_weights, rel_l2,
+                         require_gpu, to_dev)
+from video_diffusion_transformer_adaln_b200 import h3b, synth
+from video_diffusion_transformer_adaln_b200.runtime import DeviceBlock, dims_of, quantize_weight
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    require_gpu()
+    h3b.h3b_device_error(clear=True)
+    yield
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+# ----------------------------------------------------------------------------- quantizers
+
+@pytest.mark.parametrize("rows,cols", [(1, 16), (768, 256), (256, 1024), (37, 8192), (1000, 48)])
+def test_weight_quantizer_bit_exact(rows, cols):
+    r = _rng(rows * 7 + cols)
+    w = (r.standard_normal((rows, cols)) * r.uniform(0.001, 10, (rows, 1))).astype(np.float32)
+    w[0, :3] = [127.0, 2.5, -3.5] if cols >= 3 else w[0, :3]
+    if rows > 3:
+        w[3] = 0.0
+    q, s = quantize_weight(to_dev(w))
+    qo, so = O.quantize_rows(w)
+    assert np.array_equal(q.cpu().numpy(), qo)
+    assert np.array_equal(s.cpu().numpy(), so)
+    no_device_error()
+
+
+@pytest.mark.parametrize("rows,cols,with_absmax", [(33, 1024, False), (33, 1024, True), (512, 256, False),
+                                                   (129, 20480, True), (5, 16, False)])
+def test_row_quantizer_bit_exact(rows, cols, with_absmax):
+    r = _rng(rows + cols)
+    h = synth.f32_to_bf16_bits((r.standard_normal((rows, cols)) * r.uniform(0.01, 30, (rows, 1))).astype(np.float32))
+    h[1] = 0  # an all-zero row
+    hf = synth.bf16_bits_to_f32(h)
+    q = torch.empty((rows, cols), dtype=torch.int8, device="cuda")
+    s = torch.empty(rows, dtype=torch.float32, device="cuda")
+    am = to_dev(np.abs(hf).max(axis=1).astype(np.float32)) if with_absmax else None
+    h3b.h3b_quantize_rows(bf16_dev(h), q, s, absmax=am)
+    qo, so = O.quantize_rows(hf)
+    assert np.array_equal(q.cpu().numpy(), qo)
+    assert np.array_equal(s.cpu().numpy(), so)
+    no_device_error()
+
+
+@pytest.mark.parametrize("rows,d,items", [(512, 256, 1), (37, 2048, 1), (64, 5120, 1), (96, 256, 3), (8, 8192, 2)])
+def test_ln_modulate_quantize(rows, d, items):
+    r = _rng(rows * d)
+    wl = synth.WORKLOADS["d256_L512"].with_(d=d, n_heads=d // 64)
+    x = synth.f32_to_bf16_bits(r.standard_normal((rows, d)).astype(np.float32) *
+                               np.where(np.isin(np.arange(d), synth.outlier_channels(wl)), 16, 1).astype(np.float32))
+    mod = r.standard_normal((items, 6 * d)).astype(np.float32)
+    rpi = (rows + items - 1) // items
+    q = torch.empty((rows, d), dtype=torch.int8, device="cuda")
+    s = torch.empty(rows, dtype=torch.float32, device="cuda")
+    h = torch.empty((rows, d), dtype=torch.bfloat16, device="cuda")
+    az = torch.full((rows,), 7.0, dtype=torch.float32, device="cuda")
+    md = to_dev(mod)
+    h3b.h3b_ln_modulate_quantize(bf16_dev(x), rows, d, 1e-6, md[:, 3 * d:], md[:, 4 * d:], rpi, 6 * d, q, s,
+                                 h_out=h, absmax_zero=az)
+    hg = bf16_host(h)
+    # (1) the int8 decision is bit-exact given the kernel's own bf16 quantizer input
+    qo, so = O.quantize_rows(synth.bf16_bits_to_f32(hg))
+    assert np.array_equal(q.cpu().numpy(), qo) and np.array_equal(s.cpu().numpy(), so)
+    assert np.all(az.cpu().numpy() == 0)
+    # (2) the bf16 quantizer input matches the oracle's fp64 LN + modulation to one
+    #     bf16 rounding (fp32 LN statistics may move a value across a rounding boundary)
+    y = O.layernorm(O.bf16_decode(x), 1e-6)
+    ho = np.empty_like(hg)
+    for i in range(rows):
+        it = i // rpi
+        ho[i] = O.modulate_bf16(y[i:i + 1], mod[it, 3 * d:4 * d].astype(np.float64),
+                                mod[it, 4 * d:5 * d].astype(np.float64))[0]
+    ulp = bf16_ulp_diff(hg, ho)
+    assert ulp.max() <= 1 and (ulp > 0).mean() < 0.02
+    no_device_error()
+
+
+def test_adaln_modulation():
+    wl = synth.WORKLOADS["d2048_L4096"].with_(B=2)
+    raw = synth.block_weights(wl)
+    c = synth.cond(wl)
+    mod = torch.empty((2, 6 * wl.d), dtype=torch.float32, device="cuda")
+    h3b.h3b_adaln_modulation(dims_of(wl), bf16_dev(raw["w_ada"]), to_dev(raw["b_ada"]), to_dev(c), mod)
+    for b in range(2):
+        ref = O.adaln_linear(raw["w_ada"], raw["b_ada"], c[b])
+        assert np.max(np.abs(mod[b].cpu().numpy() - ref)) <= 1e-5 * np.max(np.abs(ref)) + 1e-6
+    no_device_error()
+
+
+# ----------------------------------------------------------------------------- int8 GEMM
+
+@pytest.mark.parametrize("M,N,K", [(128, 256, 128), (512, 768, 256), (300, 272, 144), (1, 16, 16),
+                                   (1024, 1536, 2048), (256, 512, 20480), (129, 6144, 2048)])
+def test_gemm_i8_s32_bit_exact(M, N, K):
+    r = _rng(M + N + K)
+    A = r.integers(-128, 128, (M, K), dtype=np.int8)
+    W = r.integers(-128, 128, (N, K), dtype=np.int8)
+    C_ = torch.empty((M, N), dtype=torch.int32, device="cuda")
+    h3b.h3b_gemm_i8_s32(to_dev(A), to_dev(W), C_)
+    assert np.array_equal(C_.cpu().numpy(), O.gemm_i8(A, W))
+    no_device_error()
+
+
+def _quant_operands(M, N, K, seed):
+    r = _rng(seed)
+    a = (r.standard_normal((M, K)) * r.uniform(0.1, 5, (M, 1))).astype(np.float32)
+    w = (r.standard_normal((N, K)) / np.sqrt(K)).astype(np.float32)
+    qa, sa = O.quantize_rows(a)
+    qw, sw = O.quantize_rows(w)
+    bias = r.standard_normal(N).astype(np.float32) * 0.1
+    return qa, sa, qw, sw, bias
+
+
+@pytest.mark.parametrize("M,N,K", [(512, 768, 256), (200, 1040, 512)])
+def test_gemm_i8_dequant(M, N, K):
+    qa, sa, qw, sw, bias = _quant_operands(M, N, K, 11)
+    out = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    h3b.h3b_gemm_i8_dequant(to_dev(qa), to_dev(sa), to_dev(qw), to_dev(sw), to_dev(bias), out)
+    ref = O.dequant(O.gemm_i8(qa, qw), sa, sw, bias)
+    ulp = bf16_ulp_diff(bf16_host(out), O.bf16_round(ref))
+    assert ulp.max() <= 1
+    no_device_error()
+
+
+@pytest.mark.parametrize("M,N,K", [(512, 1024, 256), (77, 8192, 2048)])
+def test_gemm_i8_gelu(M, N, K):
+    qa, sa, qw, sw, bias = _quant_operands(M, N, K, 12)
+    g = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    am = torch.zeros(M, dtype=torch.float32, device="cuda")
+    h3b.h3b_gemm_i8_gelu(to_dev(qa), to_dev(sa), to_dev(qw), to_dev(sw), to_dev(bias), g, am)
+    gg = bf16_host(g)
+    ref = O.gelu_tanh(O.dequant(O.gemm_i8(qa, qw), sa, sw, bias))
+    assert rel_l2(O.bf16_decode(gg), ref) < 4e-3
+    assert np.max(np.abs(O.bf16_decode(gg) - ref)) <= 2 ** -7 * np.max(np.abs(ref)) + 1e-3
+    # the reported absmax is exactly the max |g| of the written bf16 row
+    assert np.array_equal(am.cpu().numpy(), np.abs(O.bf16_decode(gg)).max(axis=1).astype(np.float32))
+    no_device_error()
+
+
+@pytest.mark.parametrize("M,N,K,items", [(512, 256, 256, 1), (256, 2048, 8192, 2), (100, 512, 1024, 1)])
+def test_gemm_i8_gated_residual(M, N, K, items):
+    qa, sa, qw, sw, bias = _quant_operands(M, N, K, 13)
+    r = _rng(14)
+    x = synth.f32_to_bf16_bits(r.standard_normal((M, N)).astype(np.float32))
+    gate = r.standard_normal((items, 3 * N)).astype(np.float32)
+    rpi = (M + items - 1) // items
+    xd = bf16_dev(x)
+    gd = to_dev(gate)
+    h3b.h3b_gemm_i8_gated_residual(to_dev(qa), to_dev(sa), to_dev(qw), to_dev(sw), to_dev(bias), gd[:, N:], rpi,
+                                   3 * N, xd)
+    y = O.dequant(O.gemm_i8(qa, qw), sa, sw, bias)
+    ref = np.empty((M, N))
+    for i in range(M):
+        ref[i] = O.gated_residual(O.bf16_decode(x[i:i + 1]), y[i:i + 1], gate[i // rpi, N:2 * N])[0]
+    ulp = bf16_ulp_diff(bf16_host(xd), O.bf16_round(ref))
+    assert ulp.max() <= 1
+    # a zero gate leaves x bit-identical
+    xd2 = bf16_dev(x)
+    h3b.h3b_gemm_i8_gated_residual(to_dev(qa), to_dev(sa), to_dev(qw), to_dev(sw), to_dev(bias),
+                                   torch.zeros((items, N), device="cuda"), rpi, N, xd2)
+    assert np.array_equal(bf16_host(xd2), x)
+    no_device_error()
+
+
+# ----------------------------------------------------------------------------- QKV + RoPE
+
+def _qkv_reference(wl, A_f32, sA, raw_w):
+    """Oracle Q,K,V (token-major [R][3d]) after dequant and RoPE."""
+    d = wl.d
+    if wl.qkv_int8:
+        qa, _ = O.quantize_rows(A_f32) if sA is None else (A_f32, None)
+        w, s = O.quantize_rows(raw_w["wqkv"])
+        acc = O.gemm_i8(qa, w)
+        qkv = O.dequant(acc, sA, s)
+    else:
+        qkv = O.gemm_f64(O.bf16_decode(A_f32), O.bf16_decode(raw_w["wqkv_bf16"]))
+    t, h, w_ = O.grid_positions(wl.T, wl.H, wl.W)
+    t, h, w_ = (np.tile(a, wl.B) for a in (t, h, w_))
+    Q = O.rope_3d(qkv[:, :d], t, h, w_, wl.n_heads, wl.head_dim, wl.rope)
+    K = O.rope_3d(qkv[:, d:2 * d], t, h, w_, wl.n_heads, wl.head_dim, wl.rope)
+    return np.concatenate([Q, K, qkv[:, 2 * d:]], axis=1)
+
+
+def _head_major_to_token_major(qkv_dev, wl):
+    B, H, L, dh = wl.B, wl.n_heads, wl.L, wl.head_dim
+    a = O.bf16_decode(bf16_host(qkv_dev)).reshape(3, B, H, L, dh)
+    return a.transpose(1, 3, 0, 2, 4).reshape(B * L, 3 * H * dh)
+
+
+@pytest.mark.parametrize("name,B,qkv_int8", [("d256_L512", 1, True), ("d256_L512", 2, True),
+                                              ("d2048_L4096", 1, True), ("d256_L512", 1, False)])
+def test_qkv_projection_rope_head_major(name, B, qkv_int8):
+    wl = synth.WORKLOADS[name].with_(B=B, qkv_int8=qkv_int8)
+    if name == "d2048_L4096":
+        wl = wl.with_(T=2, H=16, W=16)  # 512 tokens keep the oracle GEMM quick
+    raw = synth.block_weights(wl)
+    r = _rng(21)
+    R, d = wl.B * wl.L, wl.d
+    dims = dims_of(wl)
+    qkv = torch.empty(3 * R * d, dtype=torch.bfloat16, device="cuda")
+    rope_ws = torch.empty(h3b.h3b_rope_table_bytes(dims), dtype=torch.uint8, device="cuda")
+    blk = DeviceBlock.from_host(raw, qkv_int8=qkv_int8)
+    if qkv_int8:
+        a = (r.standard_normal((R, d)) * 2).astype(np.float32)
+        qa, sa = O.quantize_rows(a)
+        h3b.h3b_qkv_projection(dims, to_dev(qa), to_dev(sa), blk.struct, qkv, rope_ws)
+        ref = _qkv_reference(wl, qa, sa, raw)
+    else:
+        a = synth.f32_to_bf16_bits((r.standard_normal((R, d)) * 2).astype(np.float32))
+        h3b.h3b_qkv_projection(dims, bf16_dev(a), None, blk.struct, qkv, rope_ws)
+        ref = _qkv_reference(wl, a, None, raw)
+    got = _head_major_to_token_major(qkv, wl)
+    assert np.max(np.abs(got - ref)) <= 2 ** -8 * np.max(np.abs(ref)) * 2
+    assert rel_l2(got, ref) < 4e-3
+    no_device_error()
+
+
+# ----------------------------------------------------------------------------- attention
+
+@pytest.mark.parametrize("B,H,L,dh,n_q", [(1, 4, 512, 64, 512), (1, 2, 200, 128, 200), (2, 2, 777, 128, 128),
+                                          (1, 16, 4096, 128, 96), (1, 1, 128, 64, 128), (1, 1, 1, 128, 1)])
+def test_attention(B, H, L, dh, n_q):
+    r = _rng(B * H * L * dh)
+    # head-major bf16 Q, K, V with a spread of score magnitudes
+    qkv_bits = synth.f32_to_bf16_bits((r.standard_normal((3, B, H, L, dh)) *
+                                       r.uniform(0.3, 2.0, (3, B, H, 1, 1))).astype(np.float32))
+    wl = synth.Workload("attn", 1, 1, L, H * dh, H, dh, 256, (0, 0, dh), 0, B=B)
+    dims = dims_of(wl)
+    o = torch.empty((B, L, H * dh), dtype=torch.bfloat16, device="cuda")
+    am = torch.zeros(B * L, dtype=torch.float32, device="cuda")
+    h3b.h3b_attention(dims, bf16_dev(qkv_bits), o, am)
+    og = O.bf16_decode(bf16_host(o))
+    q = O.bf16_decode(qkv_bits)
+    rows = synth.sample_rows(L, n_q)
+    for b in range(B):
+        tm = lambda part: q[part, b].transpose(1, 0, 2).reshape(L, H * dh)
+        ref = O.attention(tm(0)[rows], tm(1), tm(2), H, dh)
+        got = og[b, rows]
+        assert rel_l2(got, ref) < 1e-2
+        assert np.max(np.abs(got - ref)) < 2e-2 * np.max(np.abs(ref)) + 1e-3
+    assert np.array_equal(am.cpu().numpy(), np.abs(og).max(axis=2).reshape(-1).astype(np.float32))
+    no_device_error()
+
+
+# ----------------------------------------------------------------------------- token pairing
+
+@pytest.mark.parametrize("B,T,H,W,d", [(1, 2, 16, 16, 256), (2, 1, 3, 6, 8), (1, 8, 48, 48, 5120)])
+def test_token_pair_unpair(B, T, H, W, d):
+    r = _rng(B * T * H * W)
+    x = synth.f32_to_bf16_bits(r.standard_normal((B, T, H, W, d)).astype(np.float32))
+    full = h3b.make_dims(B, T, H, W, d, 1, 64, 256, (0, 0, 64))
+    xm = torch.empty((B, T, H, W // 2, d), dtype=torch.bfloat16, device="cuda")
+    xm2 = torch.empty_like(xm)
+    xd = bf16_dev(x)
+    h3b.h3b_token_pair(full, xd, xm, xm2)
+    xo = O.token_pair(x, B, T, H, W, d)
+    assert np.array_equal(bf16_host(xm), xo) and np.array_equal(bf16_host(xm2), xo)
+    ym_bits = synth.f32_to_bf16_bits(r.standard_normal((B, T, H, W // 2, d)).astype(np.float32))
+    out = torch.empty_like(xd)
+    h3b.h3b_token_unpair(full, xd, xm, bf16_dev(ym_bits), out)
+    ref = O.token_unpair(x, xo, O.bf16_decode(ym_bits), B, T, H, W, d)
+    assert bf16_ulp_diff(bf16_host(out), O.bf16_round(ref)).max() <= 1
+    # identity block: unpair(x, xm, xm) == x exactly
+    h3b.h3b_token_unpair(full, xd, xm, xm, out)
+    assert np.array_equal(bf16_host(out), x)
+    no_device_error()

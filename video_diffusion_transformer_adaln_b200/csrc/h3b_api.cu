@@ -1,0 +1,566 @@
+// The C ABI of the h3b library (declared in include/h3b.h): argument
+// validation, workspace planning, TMA descriptor encoding and the launch
+// sequence of one gated-AdaLN DiT block forward.
+//
+// Method references (web pages on the h3.c / h3-metal engine):
+//   "h3-metal: Apple Silicon을 위한 네이티브 MiniMax-H3 추론", sections
+//     "Int8 양자화" (gated AdaLN with the activation quantizer fused ahead of
+//     the int8 QKV and MLP projections), "Metal 4 및 TensorOps" (head-major
+//     Q/K/V) and "속도 및 품질 트레이드오프" (Token Reduction, Active DiT Blocks).
+//   "h3.c與MLX路線對比：MiniMax-H3在Apple Silicon上的兩種推理實現工程取捨",
+//     section "性能上限" (AdaLN gating, RoPE and quantization folded into the
+//     preceding kernels; activation memory reused by lifetime).
+#include <algorithm>
+#include <mutex>
+#include <string>
+
+#include "h3b.h"
+#include "h3b_common.cuh"
+#include "h3b_internal.h"
+
+// Device error word: kernels OR a nonzero code into it when a bounded wait
+// runs out. Host code reaches it through its device address (per device).
+__device__ unsigned int g_h3b_error_word;
+
+namespace h3b {
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  bool init = false;
+  bool arch_ok = false;
+  int sms = 0;
+  unsigned* err = nullptr;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+thread_local std::string g_detail;
+
+h3b_status cuda_fail(cudaError_t e, const char* where) {
+  g_detail = std::string(where) + ": " + cudaGetErrorName(e) + " (" + cudaGetErrorString(e) + ")";
+  return H3B_ERR_CUDA;
+}
+h3b_status fail(h3b_status s, const std::string& why) {
+  g_detail = why;
+  return s;
+}
+
+// Per-device facts, read once: compute capability (10.0 required), SM count,
+// and the device address of the error word.
+h3b_status device_info(DeviceInfo** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(H3B_ERR_ARG, "device index out of range");
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DeviceInfo& di = g_dev[dev];
+  if (!di.init) {
+    int major = 0, minor = 0, sms = 0;
+    if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+      return cuda_fail(e, "cudaDeviceGetAttribute");
+    di.arch_ok = (major == 10 && minor == 0);
+    di.sms = sms;
+    if (di.arch_ok) {
+      void* p = nullptr;
+      if ((e = cudaGetSymbolAddress(&p, g_h3b_error_word)) != cudaSuccess)
+        return cuda_fail(e, "cudaGetSymbolAddress(error word)");
+      di.err = static_cast<unsigned*>(p);
+    }
+    di.init = true;
+  }
+  if (!di.arch_ok) return fail(H3B_ERR_ARCH, "device is not compute capability 10.0 (sm_100a)");
+  *out = &di;
+  return H3B_OK;
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+h3b_status check_dims(const h3b_dims* d) {
+  if (!d) return fail(H3B_ERR_ARG, "dims is NULL");
+  if (d->B < 1 || d->T < 1 || d->H < 1 || d->W < 1) return fail(H3B_ERR_SHAPE, "B, T, H, W must be >= 1");
+  if (d->B > 8) return fail(H3B_ERR_SHAPE, "B must be <= 8");
+  if (d->head_dim != 64 && d->head_dim != 128) return fail(H3B_ERR_SHAPE, "head_dim must be 64 or 128");
+  if (d->n_heads < 1 || d->d != d->n_heads * d->head_dim) return fail(H3B_ERR_SHAPE, "d != n_heads * head_dim");
+  if (d->d % 256 != 0 || d->d > 8192) return fail(H3B_ERR_SHAPE, "d must be a multiple of 256, <= 8192");
+  if (d->d_ff < 256 || d->d_ff % 256 != 0 || d->d_ff > 32768)
+    return fail(H3B_ERR_SHAPE, "d_ff must be a multiple of 256 in [256, 32768]");
+  if (d->rope_t < 0 || d->rope_h < 0 || d->rope_w < 0 || (d->rope_t | d->rope_h | d->rope_w) & 1 ||
+      d->rope_t + d->rope_h + d->rope_w != d->head_dim)
+    return fail(H3B_ERR_SHAPE, "rope split must be even parts summing to head_dim");
+  if (!(d->rope_theta > 0.0f) || !(d->ln_eps >= 0.0f)) return fail(H3B_ERR_ARG, "rope_theta > 0 and ln_eps >= 0");
+  const long long L = (long long)d->T * d->H * d->W;
+  if (L * d->B * (long long)d->d_ff > (1LL << 40)) return fail(H3B_ERR_SHAPE, "problem too large");
+  if (L * d->B >= (1LL << 31)) return fail(H3B_ERR_SHAPE, "too many tokens");
+  return H3B_OK;
+}
+
+struct WsLayout {
+  size_t mod, rope, sA, absmax, act, r1, total;
+};
+
+size_t rope_bytes(const h3b_dims& d) {
+  return sizeof(float2) * ((size_t)d.T * (d.rope_t / 2) + (size_t)d.H * (d.rope_h / 2) +
+                           (size_t)d.W * (d.rope_w / 2));
+}
+
+WsLayout ws_layout(const h3b_dims& d) {
+  WsLayout w{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += align256(bytes);
+    return o;
+  };
+  const size_t R = (size_t)d.B * d.T * d.H * d.W;
+  const size_t D = d.d, F = d.d_ff;
+  w.mod = take((size_t)d.B * 6 * D * 4);
+  w.rope = take(rope_bytes(d));
+  w.sA = take(R * 4);
+  w.absmax = take(R * 4);
+  // int8 activations (A1..A4 in turn, up to R x F), or the bf16 QKV input.
+  w.act = take(std::max(R * std::max(D, F), d.qkv_int8 ? (size_t)0 : R * D * 2));
+  // Q/K/V + attention output, later reused for the GELU output.
+  w.r1 = take(std::max(3 * R * D * 2 + R * D * 2, R * F * 2));
+  w.total = off;
+  return w;
+}
+
+h3b_status check_weights(const h3b_dims& d, const h3b_block_weights* w) {
+  if (!w) return fail(H3B_ERR_ARG, "weights is NULL");
+  const void* req[] = {w->w_ada, w->wo, w->so, w->w1, w->s1, w->w2, w->s2};
+  for (const void* p : req) {
+    if (!p) return fail(H3B_ERR_ARG, "a required weight pointer is NULL");
+    if (!aligned16(p)) return fail(H3B_ERR_ALIGN, "weight pointer not 16-byte aligned");
+  }
+  if (d.qkv_int8) {
+    if (!w->wqkv || !w->sqkv) return fail(H3B_ERR_ARG, "wqkv/sqkv NULL");
+    if (!aligned16(w->wqkv) || !aligned16(w->sqkv)) return fail(H3B_ERR_ALIGN, "wqkv/sqkv alignment");
+  } else {
+    if (!w->wqkv_bf16) return fail(H3B_ERR_ARG, "wqkv_bf16 NULL");
+    if (!aligned16(w->wqkv_bf16)) return fail(H3B_ERR_ALIGN, "wqkv_bf16 alignment");
+  }
+  const void* opt[] = {w->b_ada, w->bqkv, w->bo, w->b1, w->b2};
+  for (const void* p : opt)
+    if (p && !aligned16(p)) return fail(H3B_ERR_ALIGN, "bias pointer not 16-byte aligned");
+  return H3B_OK;
+}
+
+#define H3B_CK(call, where)                        \
+  do {                                             \
+    cudaError_t e_ = (call);                       \
+    if (e_ != cudaSuccess) return cuda_fail(e_, where); \
+  } while (0)
+
+GemmArgs base_args(int M, int N, int K, unsigned* err) {
+  GemmArgs a{};
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.rows_per_item = M > 0 ? M : 1;
+  a.err = err;
+  return a;
+}
+
+// The block's launch sequence on one stream (workspace regions per ws_layout).
+h3b_status run_block(const h3b_dims& d, const h3b_block_weights& w, const float* c, void* x,
+                     uint8_t* ws, const WsLayout& lay, bool rope_ready, const DeviceInfo& di,
+                     cudaStream_t st) {
+  const int D = d.d, F = d.d_ff, L = d.T * d.H * d.W, R = d.B * L;
+  float* mod = reinterpret_cast<float*>(ws + lay.mod);
+  float2* rope = reinterpret_cast<float2*>(ws + lay.rope);
+  float* sA = reinterpret_cast<float*>(ws + lay.sA);
+  float* absmax = reinterpret_cast<float*>(ws + lay.absmax);
+  int8_t* act = reinterpret_cast<int8_t*>(ws + lay.act);
+  uint8_t* r1 = ws + lay.r1;
+  void* qkv = r1;
+  void* o = r1 + (size_t)3 * R * D * 2;
+  void* g = r1;
+
+  // a1: AdaLN modulation vectors
+  H3B_CK(launch_adaln_gemv(w.w_ada, w.b_ada, c, d.B, D, mod, st), "adaln_gemv");
+  if (!rope_ready)
+    H3B_CK(launch_rope_table(rope, d.T, d.H, d.W, d.rope_t, d.rope_h, d.rope_w, d.rope_theta, st), "rope_table");
+  // a2: LN + modulation + quantization (or the bf16 activation for bf16 QKV)
+  if (d.qkv_int8)
+    H3B_CK(launch_ln_mod_quant(x, R, D, d.ln_eps, mod, mod + D, L, 6 * D, act, sA, nullptr, absmax, 1, st), "ln_mod_quant");
+  else
+    H3B_CK(launch_ln_mod_quant(x, R, D, d.ln_eps, mod, mod + D, L, 6 * D, nullptr, nullptr, act, absmax, 0, st), "ln_mod");
+  // a3: QKV projection + 3D RoPE, head-major
+  {
+    GemmArgs a = base_args(R, 3 * D, D, di.err);
+    a.sA = sA;
+    a.sW = w.sqkv;
+    a.bias = w.bqkv;
+    a.out = qkv;
+    a.B = d.B; a.L = L; a.T = d.T; a.H = d.H; a.W = d.W; a.d = D;
+    a.n_heads = d.n_heads; a.head_dim = d.head_dim;
+    a.rope_t = d.rope_t; a.rope_h = d.rope_h; a.rope_w = d.rope_w; a.rope = rope;
+    H3B_CK(launch_gemm(d.qkv_int8 != 0, EPI_QKV, act, d.qkv_int8 ? (const void*)w.wqkv : w.wqkv_bf16, a, di.sms, st), "gemm_qkv");
+  }
+  // a4: attention; a5: quantize its output
+  {
+    AttnArgs a{d.B, L, d.n_heads, d.head_dim, qkv, o, absmax, di.err};
+    H3B_CK(launch_attention(a, st), "attention");
+  }
+  H3B_CK(launch_quant_rows_bf16(o, R, D, absmax, act, sA, st), "quant_o");
+  // a6: output projection + gated residual (gate_attn = chunk 2)
+  {
+    GemmArgs a = base_args(R, D, D, di.err);
+    a.sA = sA; a.sW = w.so; a.bias = w.bo; a.out = x;
+    a.gate = mod + 2 * D; a.rows_per_item = L; a.gate_stride = 6 * D;
+    H3B_CK(launch_gemm(true, EPI_RESID, act, w.wo, a, di.sms, st), "gemm_wo");
+  }
+  // a7: LN + modulation + quantization for the MLP (chunks 3, 4)
+  H3B_CK(launch_ln_mod_quant(x, R, D, d.ln_eps, mod + 3 * D, mod + 4 * D, L, 6 * D, act, sA, nullptr, absmax, 1, st), "ln_mod_quant_mlp");
+  // a8: W1 + GELU (+ row absmax), then requantize
+  {
+    GemmArgs a = base_args(R, F, D, di.err);
+    a.sA = sA; a.sW = w.s1; a.bias = w.b1; a.out = g; a.absmax = absmax;
+    H3B_CK(launch_gemm(true, EPI_GELU, act, w.w1, a, di.sms, st), "gemm_w1");
+  }
+  H3B_CK(launch_quant_rows_bf16(g, R, F, absmax, act, sA, st), "quant_g");
+  // a9: W2 + gated residual (gate_mlp = chunk 5)
+  {
+    GemmArgs a = base_args(R, D, F, di.err);
+    a.sA = sA; a.sW = w.s2; a.bias = w.b2; a.out = x;
+    a.gate = mod + 5 * D; a.rows_per_item = L; a.gate_stride = 6 * D;
+    H3B_CK(launch_gemm(true, EPI_RESID, act, w.w2, a, di.sms, st), "gemm_w2");
+  }
+  return H3B_OK;
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------------------
+// TMA descriptors (driver entry point fetched through the runtime).
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+bool make_tmap_2d(CUtensorMap* map, const void* base, int elem_bytes, uint64_t cols, uint64_t rows,
+                  uint64_t row_stride_bytes, uint32_t box_cols, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {row_stride_bytes};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUtensorMapDataType dt = elem_bytes == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  return fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_tmap_3d(CUtensorMap* map, const void* base, int elem_bytes, uint64_t d0, uint64_t d1, uint64_t d2,
+                  uint32_t box0, uint32_t box1) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {d0, d1, d2};
+  const cuuint64_t strides[2] = {d0 * elem_bytes, d0 * d1 * elem_bytes};
+  const cuuint32_t box[3] = {box0, box1, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUtensorMapDataType dt = elem_bytes == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  return fn(map, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace h3b
+
+using namespace h3b;
+
+// ===========================================================================
+// C ABI
+// ===========================================================================
+extern "C" {
+
+const char* h3b_status_string(h3b_status s) {
+  switch (s) {
+    case H3B_OK: return "ok";
+    case H3B_ERR_ARG: return "invalid argument";
+    case H3B_ERR_SHAPE: return "unsupported shape";
+    case H3B_ERR_ALIGN: return "pointer not 16-byte aligned";
+    case H3B_ERR_WORKSPACE: return "workspace too small";
+    case H3B_ERR_ARCH: return "device is not sm_100a (compute capability 10.0)";
+    case H3B_ERR_CUDA: return "CUDA error";
+    case H3B_ERR_DEVICE_CHECK: return "device error word set";
+  }
+  return "unknown status";
+}
+
+const char* h3b_last_error_detail(void) { return g_detail.c_str(); }
+
+h3b_status h3b_workspace_size(const h3b_dims* dims, size_t* bytes) {
+  h3b_status s = check_dims(dims);
+  if (s != H3B_OK) return s;
+  if (!bytes) return fail(H3B_ERR_ARG, "bytes is NULL");
+  *bytes = ws_layout(*dims).total;
+  return H3B_OK;
+}
+
+size_t h3b_rope_table_bytes(const h3b_dims* dims) {
+  if (check_dims(dims) != H3B_OK) return 0;
+  return rope_bytes(*dims);
+}
+
+static h3b_status block_common(const h3b_dims* dims, const float* c, void* x, void* ws, size_t ws_bytes,
+                               WsLayout* lay, DeviceInfo** di) {
+  h3b_status s = check_dims(dims);
+  if (s != H3B_OK) return s;
+  if (!c || !x || !ws) return fail(H3B_ERR_ARG, "c, x and ws must be non-NULL");
+  if (!aligned16(c) || !aligned16(x)) return fail(H3B_ERR_ALIGN, "c/x not 16-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return fail(H3B_ERR_ALIGN, "workspace not 256-byte aligned");
+  *lay = ws_layout(*dims);
+  if (ws_bytes < lay->total) return fail(H3B_ERR_WORKSPACE, "workspace smaller than h3b_workspace_size");
+  return device_info(di);
+}
+
+h3b_status h3b_block_forward(const h3b_dims* dims, const h3b_block_weights* w, const float* c, void* x,
+                             void* ws, size_t ws_bytes, h3b_stream stream) {
+  WsLayout lay;
+  DeviceInfo* di = nullptr;
+  h3b_status s = block_common(dims, c, x, ws, ws_bytes, &lay, &di);
+  if (s != H3B_OK) return s;
+  if ((s = check_weights(*dims, w)) != H3B_OK) return s;
+  return run_block(*dims, *w, c, x, static_cast<uint8_t*>(ws), lay, false, *di, stream);
+}
+
+h3b_status h3b_blocks_forward(const h3b_dims* dims, const h3b_block_weights* w, int n_blocks, const float* c,
+                              void* x, void* ws, size_t ws_bytes, h3b_stream stream) {
+  WsLayout lay;
+  DeviceInfo* di = nullptr;
+  h3b_status s = block_common(dims, c, x, ws, ws_bytes, &lay, &di);
+  if (s != H3B_OK) return s;
+  if (n_blocks < 0 || (n_blocks > 0 && !w)) return fail(H3B_ERR_ARG, "n_blocks < 0 or weights NULL");
+  for (int i = 0; i < n_blocks; ++i)
+    if ((s = check_weights(*dims, &w[i])) != H3B_OK) return s;
+  const size_t c_stride = (size_t)dims->B * dims->d;
+  for (int i = 0; i < n_blocks; ++i) {
+    s = run_block(*dims, w[i], c + i * c_stride, x, static_cast<uint8_t*>(ws), lay, i > 0, *di, stream);
+    if (s != H3B_OK) return s;
+  }
+  return H3B_OK;
+}
+
+static h3b_status check_pair_dims(const h3b_dims* full) {
+  if (!full) return fail(H3B_ERR_ARG, "dims is NULL");
+  if (full->B < 1 || full->T < 1 || full->H < 1 || full->W < 2) return fail(H3B_ERR_SHAPE, "bad grid");
+  if (full->W % 2 != 0) return fail(H3B_ERR_SHAPE, "W must be even for token pairing");
+  if (full->d < 8 || full->d % 8 != 0) return fail(H3B_ERR_SHAPE, "d must be a multiple of 8");
+  return H3B_OK;
+}
+
+h3b_status h3b_token_pair(const h3b_dims* full, const void* x, void* xm, void* xm_copy, h3b_stream stream) {
+  h3b_status s = check_pair_dims(full);
+  if (s != H3B_OK) return s;
+  if (!x || !xm) return fail(H3B_ERR_ARG, "x and xm must be non-NULL");
+  if (!aligned16(x) || !aligned16(xm) || (xm_copy && !aligned16(xm_copy))) return fail(H3B_ERR_ALIGN, "alignment");
+  DeviceInfo* di = nullptr;
+  if ((s = device_info(&di)) != H3B_OK) return s;
+  const long long lines = (long long)full->B * full->T * full->H;
+  H3B_CK(launch_token_pair(x, xm, xm_copy, lines, full->W, full->d, di->sms, stream), "token_pair");
+  return H3B_OK;
+}
+
+h3b_status h3b_token_unpair(const h3b_dims* full, const void* x, const void* xm, const void* ym, void* out,
+                            h3b_stream stream) {
+  h3b_status s = check_pair_dims(full);
+  if (s != H3B_OK) return s;
+  if (!x || !xm || !ym || !out) return fail(H3B_ERR_ARG, "NULL pointer");
+  if (!aligned16(x) || !aligned16(xm) || !aligned16(ym) || !aligned16(out)) return fail(H3B_ERR_ALIGN, "alignment");
+  DeviceInfo* di = nullptr;
+  if ((s = device_info(&di)) != H3B_OK) return s;
+  const long long lines = (long long)full->B * full->T * full->H;
+  H3B_CK(launch_token_unpair(x, xm, ym, out, lines, full->W, full->d, di->sms, stream), "token_unpair");
+  return H3B_OK;
+}
+
+h3b_status h3b_quantize_weights(const float* w, int rows, int cols, int8_t* q, float* s, h3b_stream stream) {
+  if (!w || !q || !s) return fail(H3B_ERR_ARG, "NULL pointer");
+  if (rows < 0 || cols < 16 || cols % 16 != 0) return fail(H3B_ERR_SHAPE, "cols must be a positive multiple of 16");
+  if (!aligned16(w) || !aligned16(q)) return fail(H3B_ERR_ALIGN, "alignment");
+  DeviceInfo* di = nullptr;
+  h3b_status st = device_info(&di);
+  if (st != H3B_OK) return st;
+  H3B_CK(launch_quant_rows_f32(w, rows, cols, q, s, stream), "quantize_weights");
+  return H3B_OK;
+}
+
+h3b_status h3b_device_error(unsigned int* code, int clear) {
+  if (!code) return fail(H3B_ERR_ARG, "code is NULL");
+  DeviceInfo* di = nullptr;
+  h3b_status s = device_info(&di);
+  if (s != H3B_OK) return s;
+  H3B_CK(cudaDeviceSynchronize(), "cudaDeviceSynchronize");
+  H3B_CK(cudaMemcpy(code, di->err, sizeof(unsigned), cudaMemcpyDeviceToHost), "read error word");
+  if (clear) H3B_CK(cudaMemset(di->err, 0, sizeof(unsigned)), "clear error word");
+  return *code ? H3B_ERR_DEVICE_CHECK : H3B_OK;
+}
+
+// ---- step entry points ------------------------------------------------------
+
+h3b_status h3b_adaln_modulation(const h3b_dims* dims, const void* w_ada, const float* b_ada, const float* c,
+                                float* mod, h3b_stream stream) {
+  h3b_status s = check_dims(dims);
+  if (s != H3B_OK) return s;
+  if (!w_ada || !c || !mod) return fail(H3B_ERR_ARG, "NULL pointer");
+  if (!aligned16(w_ada) || !aligned16(c) || !aligned16(mod)) return fail(H3B_ERR_ALIGN, "alignment");
+  DeviceInfo* di = nullptr;
+  if ((s = device_info(&di)) != H3B_OK) return s;
+  H3B_CK(launch_adaln_gemv(w_ada, b_ada, c, dims->B, dims->d, mod, stream), "adaln_gemv");
+  return H3B_OK;
+}
+
+h3b_status h3b_ln_modulate_quantize(const void* x, int rows, int d, float eps, const float* shift,
+                                    const float* scale, int rows_per_item, int mod_stride, int8_t* q, float* s,
+                                    void* h_out, float* absmax_zero, int write_codes, h3b_stream stream) {
+  if (!x || !shift || !scale || (write_codes && (!q || !s))) return fail(H3B_ERR_ARG, "NULL pointer");
+  if (rows < 0 || d < 256 || d % 256 != 0 || d > 8192) return fail(H3B_ERR_SHAPE, "d must be a multiple of 256, <= 8192");
+  if (rows_per_item < 1 || mod_stride < 0 || mod_stride % 4 != 0) return fail(H3B_ERR_ARG, "rows_per_item/mod_stride");
+  if (!aligned16(x) || !aligned16(shift) || !aligned16(scale) || (q && !aligned16(q)) || (h_out && !aligned16(h_out)))
+    return fail(H3B_ERR_ALIGN, "alignment");
+  DeviceInfo* di = nullptr;
+  h3b_status st = device_info(&di);
+  if (st != H3B_OK) return st;
+  H3B_CK(launch_ln_mod_quant(x, rows, d, eps, shift, scale, rows_per_item, mod_stride, q, s, h_out, absmax_zero,
+                             write_codes, stream), "ln_mod_quant");
+  return H3B_OK;
+}
+
+h3b_status h3b_quantize_rows(const void* h, int rows, int cols, const float* absmax, int8_t* q, float* s,
+                             h3b_stream stream) {
+  if (!h || !q || !s) return fail(H3B_ERR_ARG, "NULL pointer");
+  if (rows < 0 || cols < 16 || cols % 16 != 0) return fail(H3B_ERR_SHAPE, "cols must be a positive multiple of 16");
+  if (!aligned16(h) || !aligned16(q)) return fail(H3B_ERR_ALIGN, "alignment");
+  DeviceInfo* di = nullptr;
+  h3b_status st = device_info(&di);
+  if (st != H3B_OK) return st;
+  H3B_CK(launch_quant_rows_bf16(h, rows, cols, absmax, q, s, stream), "quantize_rows");
+  return H3B_OK;
+}
+
+static h3b_status gemm_common(const void* A, const void* W, const void* out, int M, int N, int K,
+                              DeviceInfo** di) {
+  if (!A || !W || !out) return fail(H3B_ERR_ARG, "NULL pointer");
+  if (M < 0 || N < 16 || N % 16 != 0 || K < 16 || K % 16 != 0)
+    return fail(H3B_ERR_SHAPE, "need M >= 0, N and K positive multiples of 16");
+  if (!aligned16(A) || !aligned16(W) || !aligned16(out)) return fail(H3B_ERR_ALIGN, "alignment");
+  return device_info(di);
+}
+
+h3b_status h3b_gemm_i8_s32(const int8_t* A, const int8_t* W, int32_t* C, int M, int N, int K, h3b_stream stream) {
+  DeviceInfo* di = nullptr;
+  h3b_status s = gemm_common(A, W, C, M, N, K, &di);
+  if (s != H3B_OK) return s;
+  GemmArgs a = base_args(M, N, K, di->err);
+  a.out = C;
+  H3B_CK(launch_gemm(true, EPI_S32, A, W, a, di->sms, stream), "gemm_i8_s32");
+  return H3B_OK;
+}
+
+h3b_status h3b_gemm_i8_dequant(const int8_t* A, const float* sA, const int8_t* W, const float* sW,
+                               const float* bias, void* out, int M, int N, int K, h3b_stream stream) {
+  DeviceInfo* di = nullptr;
+  h3b_status s = gemm_common(A, W, out, M, N, K, &di);
+  if (s != H3B_OK) return s;
+  if (!sA || !sW) return fail(H3B_ERR_ARG, "scales NULL");
+  if (!aligned16(sW) || (bias && !aligned16(bias))) return fail(H3B_ERR_ALIGN, "alignment");
+  GemmArgs a = base_args(M, N, K, di->err);
+  a.sA = sA; a.sW = sW; a.bias = bias; a.out = out;
+  H3B_CK(launch_gemm(true, EPI_DEQ, A, W, a, di->sms, stream), "gemm_i8_dequant");
+  return H3B_OK;
+}
+
+h3b_status h3b_qkv_projection(const h3b_dims* dims, const void* A, const float* sA, const h3b_block_weights* w,
+                              void* qkv, void* rope_ws, h3b_stream stream) {
+  h3b_status s = check_dims(dims);
+  if (s != H3B_OK) return s;
+  if (!A || !w || !qkv || !rope_ws) return fail(H3B_ERR_ARG, "NULL pointer");
+  if (dims->qkv_int8 && (!w->wqkv || !w->sqkv || !sA)) return fail(H3B_ERR_ARG, "int8 QKV needs wqkv, sqkv, sA");
+  if (!dims->qkv_int8 && !w->wqkv_bf16) return fail(H3B_ERR_ARG, "bf16 QKV needs wqkv_bf16");
+  if (!aligned16(A) || !aligned16(qkv) || !aligned16(rope_ws) || (w->bqkv && !aligned16(w->bqkv)) ||
+      (w->sqkv && !aligned16(w->sqkv)))
+    return fail(H3B_ERR_ALIGN, "alignment");
+  DeviceInfo* di = nullptr;
+  if ((s = device_info(&di)) != H3B_OK) return s;
+  const int L = dims->T * dims->H * dims->W, D = dims->d;
+  float2* rope = static_cast<float2*>(rope_ws);
+  H3B_CK(launch_rope_table(rope, dims->T, dims->H, dims->W, dims->rope_t, dims->rope_h, dims->rope_w,
+                           dims->rope_theta, stream), "rope_table");
+  GemmArgs a = base_args(dims->B * L, 3 * D, D, di->err);
+  a.sA = sA; a.sW = w->sqkv; a.bias = w->bqkv; a.out = qkv;
+  a.B = dims->B; a.L = L; a.T = dims->T; a.H = dims->H; a.W = dims->W; a.d = D;
+  a.n_heads = dims->n_heads; a.head_dim = dims->head_dim;
+  a.rope_t = dims->rope_t; a.rope_h = dims->rope_h; a.rope_w = dims->rope_w; a.rope = rope;
+  H3B_CK(launch_gemm(dims->qkv_int8 != 0, EPI_QKV, A, dims->qkv_int8 ? (const void*)w->wqkv : w->wqkv_bf16, a,
+                     di->sms, stream), "qkv_projection");
+  return H3B_OK;
+}
+
+h3b_status h3b_attention(const h3b_dims* dims, const void* qkv, void* o, float* absmax, h3b_stream stream) {
+  // Attention alone needs only the grid, the batch and the head shape.
+  if (!dims) return fail(H3B_ERR_ARG, "dims is NULL");
+  if (dims->B < 1 || dims->T < 1 || dims->H < 1 || dims->W < 1 || dims->n_heads < 1)
+    return fail(H3B_ERR_SHAPE, "B, T, H, W, n_heads must be >= 1");
+  if (dims->head_dim != 64 && dims->head_dim != 128) return fail(H3B_ERR_SHAPE, "head_dim must be 64 or 128");
+  if ((long long)dims->B * dims->n_heads > 65535) return fail(H3B_ERR_SHAPE, "B * n_heads must be <= 65535");
+  if ((long long)dims->T * dims->H * dims->W >= (1LL << 31)) return fail(H3B_ERR_SHAPE, "too many tokens");
+  h3b_status s = H3B_OK;
+  if (!qkv || !o || !absmax) return fail(H3B_ERR_ARG, "NULL pointer");
+  if (!aligned16(qkv) || !aligned16(o)) return fail(H3B_ERR_ALIGN, "alignment");
+  DeviceInfo* di = nullptr;
+  if ((s = device_info(&di)) != H3B_OK) return s;
+  AttnArgs a{dims->B, dims->T * dims->H * dims->W, dims->n_heads, dims->head_dim, qkv, o, absmax, di->err};
+  H3B_CK(launch_attention(a, stream), "attention");
+  return H3B_OK;
+}
+
+h3b_status h3b_gemm_i8_gated_residual(const int8_t* A, const float* sA, const int8_t* W, const float* sW,
+                                      const float* bias, const float* gate, int rows_per_item, int gate_stride,
+                                      void* x, int M, int N, int K, h3b_stream stream) {
+  DeviceInfo* di = nullptr;
+  h3b_status s = gemm_common(A, W, x, M, N, K, &di);
+  if (s != H3B_OK) return s;
+  if (!sA || !sW || !gate) return fail(H3B_ERR_ARG, "scales/gate NULL");
+  if (rows_per_item < 1 || gate_stride < 0 || gate_stride % 4 != 0) return fail(H3B_ERR_ARG, "rows_per_item/gate_stride");
+  if (!aligned16(sW) || !aligned16(gate) || (bias && !aligned16(bias))) return fail(H3B_ERR_ALIGN, "alignment");
+  GemmArgs a = base_args(M, N, K, di->err);
+  a.sA = sA; a.sW = sW; a.bias = bias; a.out = x;
+  a.gate = gate; a.rows_per_item = rows_per_item; a.gate_stride = gate_stride;
+  H3B_CK(launch_gemm(true, EPI_RESID, A, W, a, di->sms, stream), "gemm_i8_gated_residual");
+  return H3B_OK;
+}
+
+h3b_status h3b_gemm_i8_gelu(const int8_t* A, const float* sA, const int8_t* W, const float* sW, const float* bias,
+                            void* g, float* absmax, int M, int N, int K, h3b_stream stream) {
+  DeviceInfo* di = nullptr;
+  h3b_status s = gemm_common(A, W, g, M, N, K, &di);
+  if (s != H3B_OK) return s;
+  if (!sA || !sW || !absmax) return fail(H3B_ERR_ARG, "scales/absmax NULL");
+  if (!aligned16(sW) || (bias && !aligned16(bias))) return fail(H3B_ERR_ALIGN, "alignment");
+  GemmArgs a = base_args(M, N, K, di->err);
+  a.sA = sA; a.sW = sW; a.bias = bias; a.out = g; a.absmax = absmax;
+  H3B_CK(launch_gemm(true, EPI_GELU, A, W, a, di->sms, stream), "gemm_i8_gelu");
+  return H3B_OK;
+}
+
+}  // extern "C"

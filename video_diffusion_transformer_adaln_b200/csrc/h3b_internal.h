@@ -1,0 +1,77 @@
+// Internal launcher interface between the C ABI (h3b_api.cu) and the kernel
+// translation units. Host-only declarations; every launcher enqueues on `st`
+// and returns the launch status.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace h3b {
+
+// ---- memory-bound row kernels (k_rowops.cu)
+cudaError_t launch_adaln_gemv(const void* W, const float* bias, const float* c, int B, int d,
+                              float* mod, cudaStream_t st);
+cudaError_t launch_ln_mod_quant(const void* x, int rows, int d, float eps, const float* shift,
+                                const float* scale, int rows_per_item, int mod_stride, int8_t* q,
+                                float* s, void* h_out, float* absmax_zero, int write_codes,
+                                cudaStream_t st);
+cudaError_t launch_quant_rows_bf16(const void* h, int rows, int cols, const float* absmax,
+                                   int8_t* q, float* s, cudaStream_t st);
+cudaError_t launch_quant_rows_f32(const float* w, int rows, int cols, int8_t* q, float* s,
+                                  cudaStream_t st);
+cudaError_t launch_token_pair(const void* x, void* xm, void* xm2, long long lines, int W, int d,
+                              int sms, cudaStream_t st);
+cudaError_t launch_token_unpair(const void* x, const void* xm, const void* ym, void* out,
+                                long long lines, int W, int d, int sms, cudaStream_t st);
+cudaError_t launch_rope_table(float2* tab, int T, int H, int W, int rt, int rh, int rw,
+                              double theta, cudaStream_t st);
+
+// ---- tensor-core GEMM (k_gemm.cu)
+enum GemmEpilogue : int {
+  EPI_S32 = 0,    // int32 accumulators out
+  EPI_DEQ = 1,    // bf16(acc * sA * sW + bias)
+  EPI_QKV = 2,    // dequant + 3D RoPE on Q, K; head-major Q/K/V
+  EPI_RESID = 3,  // x = bf16(x + gate * (acc * sA * sW + bias))
+  EPI_GELU = 4,   // g = bf16(gelu_tanh(acc * sA * sW + bias)), row absmax
+};
+
+struct GemmArgs {
+  int M, N, K;
+  const float* sA;  // [M] per-row activation scales (int8 operands only)
+  const float* sW;  // [N] per-output-channel weight scales (int8 operands only)
+  const float* bias;
+  void* out;
+  float* absmax;      // EPI_GELU
+  const float* gate;  // EPI_RESID: gate[item * gate_stride + n]
+  int rows_per_item, gate_stride;
+  // EPI_QKV
+  int B, L, T, H, W, d, n_heads, head_dim, rope_t, rope_h, rope_w;
+  const float2* rope;  // table from launch_rope_table
+  unsigned* err;       // device error word
+};
+
+// A [M][K] and W [N][K] row-major, int8 (kInt8) or bf16.
+cudaError_t launch_gemm(bool int8_operands, GemmEpilogue epi, const void* A, const void* W,
+                        const GemmArgs& args, int sms, cudaStream_t st);
+
+// ---- attention (k_attention.cu)
+struct AttnArgs {
+  int B, L, n_heads, head_dim;
+  const void* qkv;  // bf16 [3][B][n_heads][L][head_dim]
+  void* o;          // bf16 [B][L][n_heads*head_dim]
+  float* absmax;    // [B*L]
+  unsigned* err;
+};
+cudaError_t launch_attention(const AttnArgs& a, cudaStream_t st);
+
+// ---- TMA descriptor construction (h3b_api.cu)
+// Row-major 2D tensor of `rows` x `cols` elements of `elem_bytes` each,
+// `row_stride_bytes` apart; box of box_cols x box_rows with 128-byte swizzle.
+bool make_tmap_2d(CUtensorMap* map, const void* base, int elem_bytes, uint64_t cols,
+                  uint64_t rows, uint64_t row_stride_bytes, uint32_t box_cols, uint32_t box_rows);
+// 3D tensor [d2][d1][d0] (d0 innermost), box of box0 x box1 x 1, 128-byte swizzle.
+bool make_tmap_3d(CUtensorMap* map, const void* base, int elem_bytes, uint64_t d0, uint64_t d1,
+                  uint64_t d2, uint32_t box0, uint32_t box1);
+
+}  // namespace h3b

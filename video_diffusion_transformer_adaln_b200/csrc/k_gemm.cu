@@ -1,0 +1,358 @@
+// Tensor-core GEMM for the block's projections on sm_100a:
+//   C[m][n] = sum_k A[m][k] * W[n][k]
+// with int8 operands (tcgen05.mma kind::i8, exact int32 accumulation) or bf16
+// operands (kind::f16, fp32 accumulation), and the block's epilogues fused:
+// per-token x per-channel dequantization, QKV with 3D RoPE written head-major,
+// GELU with the per-row absmax the next quantizer needs, and the gated
+// residual update of the bf16 residual stream.
+//
+// Method references (web pages on the h3.c / h3-metal engine):
+//   "h3-metal: Apple Silicon을 위한 네이티브 MiniMax-H3 추론", section "Int8 양자화"
+//     (int8 MLP and QKV; per-output-channel weight scales, per-row dynamic
+//     activation scales) and section "Metal 4 및 TensorOps" (Q/K/V routed
+//     directly into a head-major attention input).
+//   "h3.c與MLX路線對比：MiniMax-H3在Apple Silicon上的兩種推理實現工程取捨",
+//     section "性能上限" (RoPE folded into the kernel of the projections).
+//
+// Design (B200): persistent kernel, one 128x256 output tile at a time per CTA,
+// tiles rastered in groups of 16 M-blocks for L2 reuse. Warp 0 streams A/B
+// tiles with TMA (128-byte swizzle) into a 4-stage shared-memory ring; warp 1
+// issues tcgen05.mma from one thread into a double-buffered TMEM accumulator
+// (2 x 256 columns); warps 2-5 drain the other accumulator (tcgen05.ld) and
+// run the epilogue while the next tile's MMAs proceed. Every wait is bounded.
+#include "h3b_common.cuh"
+#include "h3b_internal.h"
+
+namespace h3b {
+namespace gemm {
+constexpr int BM = 128, BN = 256, BKB = 128, STAGES = 4;
+constexpr int A_BYTES = BM * BKB;
+constexpr int B_BYTES = BN * BKB;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int GROUP_M = 16;
+constexpr int kThreads = 192;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr int kBars = 2 * STAGES + 4 + 1;
+constexpr size_t SMEM_BYTES = (size_t)STAGES * STAGE_BYTES + 1024 + kBars * 8 + 16;
+}  // namespace gemm
+
+__device__ __forceinline__ void tile_coords(int t, int n_m, int n_n, int& mb, int& nb) {
+  const int per_group = gemm::GROUP_M * n_n;
+  const int g = t / per_group;
+  const int first = g * gemm::GROUP_M;
+  const int gm = min(gemm::GROUP_M, n_m - first);
+  const int r = t - g * per_group;
+  mb = first + r % gm;
+  nb = r / gm;
+}
+
+__device__ __forceinline__ float gelu_tanh_f(float x) {
+  // 0.5 x (1 + tanh(u)) == x / (1 + exp(-2u)),  u = sqrt(2/pi) (x + 0.044715 x^3)
+  const float u = 0.7978845608028654f * fmaf(0.044715f * x, x * x, x);
+  return x / (1.0f + __expf(-2.0f * u));
+}
+
+__device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const float (&v)[32], int valid) {
+  uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int g = 0; g < 4; ++g) {
+    if (g * 8 >= valid) break;
+    d4[g] = make_uint4(pack_bf16x2(v[8 * g + 0], v[8 * g + 1]), pack_bf16x2(v[8 * g + 2], v[8 * g + 3]),
+                       pack_bf16x2(v[8 * g + 4], v[8 * g + 5]), pack_bf16x2(v[8 * g + 6], v[8 * g + 7]));
+  }
+}
+
+// Epilogue of one 128x256 tile for the thread owning TMEM lane = tile row.
+template <bool kInt8, int kEpi>
+__device__ __forceinline__ void epilogue_tile(const GemmArgs& p, uint32_t tbase, int row, bool row_ok,
+                                              int n0) {
+  float sa = 1.0f;
+  if (kInt8 && kEpi != EPI_S32 && row_ok) sa = __ldg(p.sA + row);
+  int item = 0, l = 0, pt = 0, ph = 0, pw = 0;
+  if (kEpi == EPI_QKV) {
+    item = row / p.L;
+    l = row - item * p.L;
+    pt = l / (p.H * p.W);
+    ph = (l / p.W) % p.H;
+    pw = l % p.W;
+  } else if (kEpi == EPI_RESID) {
+    item = row / p.rows_per_item;
+  }
+  float amax = 0.0f;
+#pragma unroll 1
+  for (int c = 0; c < gemm::BN / 32; ++c) {
+    const int col0 = n0 + c * 32;
+    if (col0 >= p.N) break;  // uniform across the warp
+    uint32_t r[32];
+    tmem_ld32(tbase + c * 32, r);
+    tmem_ld_wait();
+    if (!row_ok) continue;
+    const int valid = min(32, p.N - col0);
+    if (kEpi == EPI_S32) {
+      uint4* d4 = reinterpret_cast<uint4*>(static_cast<int32_t*>(p.out) + (size_t)row * p.N + col0);
+#pragma unroll
+      for (int g = 0; g < 8; ++g)
+        if (g * 4 < valid) d4[g] = make_uint4(r[4 * g], r[4 * g + 1], r[4 * g + 2], r[4 * g + 3]);
+      continue;
+    }
+    float v[32];
+    if (kInt8) {
+      const float4* sw4 = reinterpret_cast<const float4*>(p.sW + col0);
+#pragma unroll
+      for (int g = 0; g < 8; ++g) {
+        const float4 s = (4 * g < valid) ? __ldg(sw4 + g) : make_float4(0.f, 0.f, 0.f, 0.f);
+        v[4 * g + 0] = (float)(int)r[4 * g + 0] * sa * s.x;
+        v[4 * g + 1] = (float)(int)r[4 * g + 1] * sa * s.y;
+        v[4 * g + 2] = (float)(int)r[4 * g + 2] * sa * s.z;
+        v[4 * g + 3] = (float)(int)r[4 * g + 3] * sa * s.w;
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+    }
+    if (p.bias) {
+      const float4* b4 = reinterpret_cast<const float4*>(p.bias + col0);
+#pragma unroll
+      for (int g = 0; g < 8; ++g) {
+        if (4 * g >= valid) break;
+        const float4 b = __ldg(b4 + g);
+        v[4 * g] += b.x; v[4 * g + 1] += b.y; v[4 * g + 2] += b.z; v[4 * g + 3] += b.w;
+      }
+    }
+    if (kEpi == EPI_DEQ) {
+      store_bf16x32(static_cast<__nv_bfloat16*>(p.out) + (size_t)row * p.N + col0, v, valid);
+    } else if (kEpi == EPI_GELU) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        v[i] = round_bf16(gelu_tanh_f(v[i]));
+        amax = fmaxf(amax, fabsf(v[i]));
+      }
+      store_bf16x32(static_cast<__nv_bfloat16*>(p.out) + (size_t)row * p.N + col0, v, valid);
+    } else if (kEpi == EPI_RESID) {
+      __nv_bfloat16* xp = static_cast<__nv_bfloat16*>(p.out) + (size_t)row * p.N + col0;
+      const float4* g4 = reinterpret_cast<const float4*>(p.gate + (size_t)item * p.gate_stride + col0);
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        if (g * 8 >= valid) break;
+        const uint4 xv = reinterpret_cast<const uint4*>(xp)[g];
+        const float4 ga = __ldg(g4 + 2 * g), gb = __ldg(g4 + 2 * g + 1);
+        const float gg[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+        const uint32_t xu[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          v[8 * g + 2 * e] = fmaf(gg[2 * e], v[8 * g + 2 * e], bf16_lo(xu[e]));
+          v[8 * g + 2 * e + 1] = fmaf(gg[2 * e + 1], v[8 * g + 2 * e + 1], bf16_hi(xu[e]));
+        }
+      }
+      store_bf16x32(xp, v, valid);
+    } else if (kEpi == EPI_QKV) {
+      const int part = col0 / p.d;
+      const int rem = col0 - part * p.d;
+      const int head = rem / p.head_dim;
+      const int lane0 = rem - head * p.head_dim;
+      if (part < 2) {
+        const int off_h = p.T * (p.rope_t / 2), off_w = off_h + p.H * (p.rope_h / 2);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int pl = lane0 + 2 * i;
+          int idx;
+          if (pl < p.rope_t) idx = pt * (p.rope_t / 2) + pl / 2;
+          else if (pl < p.rope_t + p.rope_h) idx = off_h + ph * (p.rope_h / 2) + (pl - p.rope_t) / 2;
+          else idx = off_w + pw * (p.rope_w / 2) + (pl - p.rope_t - p.rope_h) / 2;
+          const float2 cs = __ldg(p.rope + idx);
+          const float x0 = v[2 * i], x1 = v[2 * i + 1];
+          v[2 * i] = x0 * cs.x - x1 * cs.y;
+          v[2 * i + 1] = x0 * cs.y + x1 * cs.x;
+        }
+      }
+      __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.out) +
+                           ((((size_t)part * p.B + item) * p.n_heads + head) * p.L + l) * p.head_dim + lane0;
+      store_bf16x32(dst, v, 32);
+    }
+  }
+  if (kEpi == EPI_GELU && row_ok)
+    atomicMax(reinterpret_cast<unsigned*>(p.absmax) + row, __float_as_uint(amax));
+}
+
+template <bool kInt8, int kEpi>
+__global__ void __launch_bounds__(gemm::kThreads, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                const GemmArgs p) {
+  using namespace gemm;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kBars);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = smem_u32(bars);
+  auto full = [&](int s) { return bar0 + 8u * s; };
+  auto empty = [&](int s) { return bar0 + 8u * (STAGES + s); };
+  auto tfull = [&](int a) { return bar0 + 8u * (2 * STAGES + a); };
+  auto tempty = [&](int a) { return bar0 + 8u * (2 * STAGES + 2 + a); };
+  const uint32_t drain = bar0 + 8u * (2 * STAGES + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_m = (p.M + BM - 1) / BM, n_n = (p.N + BN - 1) / BN;
+  const int n_tiles = n_m * n_n;
+  constexpr int BKE = kInt8 ? BKB : BKB / 2;  // K elements per stage
+  const int nk = (p.K + BKE - 1) / BKE;
+  constexpr uint32_t IDESC = kInt8 ? instr_desc(2, 1, 0, 0, BM, BN) : instr_desc(1, 1, 0, 0, BM, BN);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) { mbar_init(full(s), 1); mbar_init(empty(s), 1); }
+    for (int a = 0; a < 2; ++a) { mbar_init(tfull(a), 1); mbar_init(tempty(a), 4); }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) { tma_prefetch_desc(&tmA); tma_prefetch_desc(&tmB); }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer
+      int s = 0;
+      uint32_t ph = 0;
+      uint32_t issued = 0, issued_ph = 0;  // per-stage bitmask of the last issued phase
+      bool ok = true;
+      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
+        int mb, nb;
+        tile_coords(t, n_m, n_n, mb, nb);
+        for (int kb = 0; kb < nk; ++kb) {
+          if (*abort_flag || !mbar_wait(empty(s), ph ^ 1u, p.err, ERR_WAIT_MMA)) { ok = false; break; }
+          mbar_arrive_expect_tx(full(s), STAGE_BYTES);
+          const uint32_t a_dst = sbase + s * STAGE_BYTES;
+          tma_load_2d(a_dst, &tmA, full(s), kb * BKE, mb * BM);
+          tma_load_2d(a_dst + A_BYTES, &tmB, full(s), kb * BKE, nb * BN);
+          issued |= 1u << s;
+          issued_ph = (issued_ph & ~(1u << s)) | (ph << s);
+          if (++s == STAGES) { s = 0; ph ^= 1u; }
+        }
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        for (int i = 0; i < STAGES; ++i)  // let in-flight tiles land before the CTA exits
+          if (issued & (1u << i)) mbar_wait(full(i), (issued_ph >> i) & 1u, p.err, ERR_WAIT_DRAIN, kDrainLimitNs);
+      } else {
+        // tail: every filled stage has been consumed (its commit has arrived)
+        for (int i = 0; i < STAGES; ++i)
+          if (issued & (1u << i)) mbar_wait(empty(i), (issued_ph >> i) & 1u, p.err, ERR_WAIT_MMA);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- MMA issuer
+      int s = 0;
+      uint32_t ph = 0;
+      int tl = 0;
+      bool ok = true;
+      bool any = false;
+      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++tl) {
+        const int acc = tl & 1;
+        const uint32_t aph = (tl >> 1) & 1;
+        if (*abort_flag || !mbar_wait(tempty(acc), aph ^ 1u, p.err, ERR_WAIT_EPI)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (*abort_flag || !mbar_wait(full(s), ph, p.err, ERR_WAIT_TMA)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a_addr = sbase + s * STAGE_BYTES;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint64_t ad = smem_desc_sw128(a_addr + k * 32, 16, 1024);
+            const uint64_t bd = smem_desc_sw128(a_addr + A_BYTES + k * 32, 16, 1024);
+            if (kInt8) mma_i8(d_tmem, ad, bd, IDESC, (kb | k) != 0);
+            else mma_f16(d_tmem, ad, bd, IDESC, (kb | k) != 0);
+          }
+          any = true;
+          tc_commit(empty(s));
+          if (++s == STAGES) { s = 0; ph ^= 1u; }
+        }
+        if (!ok) break;
+        tc_commit(tfull(acc));
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        if (any) {  // wait for the MMAs already issued before TMEM is released
+          tc_commit(drain);
+          mbar_wait(drain, 0, p.err, ERR_WAIT_DRAIN, kDrainLimitNs);
+        }
+      }
+    }
+  } else {
+    // ---------------- epilogue warps 2..5 (TMEM lane quadrant = warp % 4)
+    const int quad = warp & 3;
+    int tl = 0;
+    for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++tl) {
+      int mb, nb;
+      tile_coords(t, n_m, n_n, mb, nb);
+      const int acc = tl & 1;
+      const uint32_t aph = (tl >> 1) & 1;
+      if (*abort_flag || !mbar_wait(tfull(acc), aph, p.err, ERR_WAIT_MMA)) { *abort_flag = 1; break; }
+      tc_fence_after();
+      const int row = mb * BM + quad * 32 + lane;
+      const uint32_t tbase = tmem_base + ((uint32_t)(quad * 32) << 16) + acc * BN;
+      epilogue_tile<kInt8, kEpi>(p, tbase, row, row < p.M, nb * BN);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty(acc));
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+template <bool kInt8, int kEpi>
+static cudaError_t launch_one(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& a,
+                              int grid, cudaStream_t st) {
+  auto k = gemm_kernel<kInt8, kEpi>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gemm::SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  k<<<grid, gemm::kThreads, gemm::SMEM_BYTES, st>>>(ta, tb, a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gemm(bool int8_operands, GemmEpilogue epi, const void* A, const void* W,
+                        const GemmArgs& a, int sms, cudaStream_t st) {
+  using namespace gemm;
+  if (a.M == 0) return cudaSuccess;
+  const int eb = int8_operands ? 1 : 2;
+  const uint32_t bke = int8_operands ? BKB : BKB / 2;
+  CUtensorMap ta, tb;
+  if (!make_tmap_2d(&ta, A, eb, (uint64_t)a.K, (uint64_t)a.M, (uint64_t)a.K * eb, bke, BM))
+    return cudaErrorInvalidValue;
+  if (!make_tmap_2d(&tb, W, eb, (uint64_t)a.K, (uint64_t)a.N, (uint64_t)a.K * eb, bke, BN))
+    return cudaErrorInvalidValue;
+  const int n_tiles = ((a.M + BM - 1) / BM) * ((a.N + BN - 1) / BN);
+  const int grid = n_tiles < sms ? n_tiles : sms;
+  if (int8_operands) {
+    switch (epi) {
+      case EPI_S32: return launch_one<true, EPI_S32>(ta, tb, a, grid, st);
+      case EPI_DEQ: return launch_one<true, EPI_DEQ>(ta, tb, a, grid, st);
+      case EPI_QKV: return launch_one<true, EPI_QKV>(ta, tb, a, grid, st);
+      case EPI_RESID: return launch_one<true, EPI_RESID>(ta, tb, a, grid, st);
+      case EPI_GELU: return launch_one<true, EPI_GELU>(ta, tb, a, grid, st);
+    }
+  } else {
+    switch (epi) {
+      case EPI_DEQ: return launch_one<false, EPI_DEQ>(ta, tb, a, grid, st);
+      case EPI_QKV: return launch_one<false, EPI_QKV>(ta, tb, a, grid, st);
+      default: break;
+    }
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace h3b
