@@ -1,0 +1,514 @@
+#!/usr/bin/env python
+"""Benchmark of the gated-AdaLN DiT block forward on B200.
+
+One step = one forward of the whole block (AdaLN GEMV, fused LN+modulation+
+int8 quantizer, int8 QKV GEMM with 3D RoPE, bf16 attention, quantizer, int8
+output projection with gated residual, fused LN+quantizer, int8 W1 + GELU,
+quantizer, int8 W2 with gated residual) over one synthetic latent of the
+chosen workload, through the library's C ABI. Token-reduction workloads add
+the pair/unpair kernels around the block; depth-50 workloads run 50 distinct
+blocks per step.
+
+Prints one JSON line (rank 0). Under torchrun each rank runs its own
+independent latent (replicas; no data-path collective): the value is the
+total tokens/s of all ranks over the slowest rank's device time.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl h3b|reference]
+"""
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from video_diffusion_transformer_adaln_b200 import build as cuda_build  # noqa: E402
+from video_diffusion_transformer_adaln_b200 import h3b, synth  # noqa: E402
+from video_diffusion_transformer_adaln_b200.runtime import (DeviceBlock, bf16_from_bits, dims_of,  # noqa: E402
+                                                            workspace)
+
+METRIC = "DiT block tokens/s (int8 MLP+QKV, bf16 attn); % of B200 INT8/BF16/HBM roofline"
+UNIT = "tokens/s"
+DEFAULT_WORKLOAD = "d2048_L4096"
+L2_FLUSH_BYTES = 512 << 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# the recipe's nominal dense ratio of 8-bit to bf16 tensor throughput (4.5 / 2.25 PFLOP/s)
+INT8_OVER_BF16 = 2.0
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {k: float(p[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_work(name, wl):
+    """Algorithmic work of one launch: (amount, unit, bound). Tensor-core
+    kernels count useful multiply-adds x 2; memory-bound kernels count the
+    bytes they must move (read once + write once)."""
+    B, L, d, F = wl.B, wl.L, wl.d, wl.d_ff
+    if wl.token_pair:
+        L = wl.L // 2  # the block runs on the merged grid
+    R = B * L
+    if name == "gemm_qkv":
+        return 2.0 * R * 3 * d * d, "op", "tensor_i8" if wl.qkv_int8 else "tensor_bf16"
+    if name == "gemm_wo":
+        return 2.0 * R * d * d, "op", "tensor_i8"
+    if name in ("gemm_w1", "gemm_w2"):
+        return 2.0 * R * d * F, "op", "tensor_i8"
+    if name == "attention":
+        return 4.0 * B * L * L * d, "flop", "tensor_bf16"
+    if name in ("ln_mod_quant", "ln_mod_quant_mlp"):
+        return R * (2.0 * d + d + 4 + 4), "byte", "hbm"
+    if name == "ln_mod":
+        return R * (2.0 * d + 2 * d + 4), "byte", "hbm"
+    if name == "quant_o":
+        return R * (2.0 * d + d + 8), "byte", "hbm"
+    if name == "quant_g":
+        return R * (2.0 * F + F + 8), "byte", "hbm"
+    if name == "adaln_gemv":
+        return 12.0 * d * d + B * (4.0 * d + 24 * d), "byte", "hbm"
+    if name == "token_pair":
+        full = wl.B * wl.L * wl.d
+        return 2.0 * full + 2 * 2.0 * full / 2, "byte", "hbm"
+    if name == "token_unpair":
+        full = wl.B * wl.L * wl.d
+        return 2.0 * full + 2 * 2.0 * full / 2 + 2.0 * full, "byte", "hbm"
+    return 0.0, "byte", "hbm"
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons, with host timestamps."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.proc = None
+        self.t0 = self.t1 = None
+
+    def start(self):
+        try:
+            uuid = str(torch.cuda.get_device_properties(self.dev).uuid)
+            sel = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "50", "-i", sel], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+            self.started = time.time()
+        except Exception:
+            self.proc = None
+
+    def mark(self, which):
+        setattr(self, which, time.time())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.12)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            return None
+        rows = [r.split(",") for r in out.strip().splitlines() if r.strip()]
+        rows = [[c.strip() for c in r] for r in rows if len(r) >= 8]
+        if not rows:
+            return None
+        mhz = [float(r[0]) for r in rows if r[0].replace(".", "").isdigit()]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            for n, v in zip(names, r[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        busy = [m for m in mhz if m > 0.5 * max(mhz)] or mhz
+        return {"sm_mhz": statistics.median(busy) if busy else None,
+                "sm_max_mhz": float(rows[0][1]) if rows[0][1].replace(".", "").isdigit() else None,
+                "reasons": sorted(reasons), "samples": len(rows),
+                "window": "nvidia-smi every 50 ms from warm-up start to the end of the timed steps"}
+
+
+# ----------------------------------------------------------------------------- workload
+
+class Workload:
+    """Device buffers and the step callable for one named workload on this rank."""
+
+    def __init__(self, name, rank):
+        self.wl = synth.WORKLOADS[name]
+        wl = self.wl
+        seed = synth.BASE_SEED + rank  # one independent latent per rank
+        self.name = name
+        x_bits = synth.x_input(wl, seed)
+        self.x_ref = bf16_from_bits(x_bits, "cuda")
+        self.x = self.x_ref.clone()
+        if wl.n_blocks > 1:
+            g = torch.Generator(device="cuda").manual_seed(synth.BASE_SEED)
+            self.blocks = [DeviceBlock.random_on_device(wl, g) for _ in range(wl.n_blocks)]
+            self.c = torch.randn((wl.n_blocks, wl.B, wl.d), generator=g, device="cuda")
+        else:
+            self.blocks = [DeviceBlock.from_host(synth.block_weights(wl), qkv_int8=wl.qkv_int8)]
+            self.c = torch.from_numpy(synth.cond(wl, 0, seed)).cuda()
+        self.full = dims_of(wl)
+        self.dims = dims_of(wl.merged()) if wl.token_pair else self.full
+        self.ws = workspace(self.dims)
+        if wl.token_pair:
+            shp = (wl.B, wl.T, wl.H, wl.W // 2, wl.d)
+            self.xm = torch.empty(shp, dtype=torch.bfloat16, device="cuda")
+            self.ym = torch.empty_like(self.xm)
+        self.tokens = wl.B * wl.L
+
+    def step(self, x=None, c=None):
+        x = self.x if x is None else x
+        c = self.c if c is None else c
+        wl = self.wl
+        if wl.token_pair:
+            h3b.h3b_token_pair(self.full, x, self.xm, self.ym)
+            h3b.h3b_block_forward(self.dims, self.blocks[0].struct, c, self.ym, self.ws)
+            h3b.h3b_token_unpair(self.full, x, self.xm, self.ym, x)
+        elif wl.n_blocks > 1:
+            h3b.h3b_blocks_forward(self.dims, [b.struct for b in self.blocks], c, x, self.ws)
+        else:
+            h3b.h3b_block_forward(self.dims, self.blocks[0].struct, c, x, self.ws)
+
+
+# ----------------------------------------------------------------------------- CPU oracle leg
+
+class OracleRunner:
+    """The CPU oracle on a bounded sample of the workload: steps a1-a3 (AdaLN,
+    LN+quantizer, QKV projection with RoPE) for every token, then steps a4-a9
+    for n sampled tokens. The full-block time is extrapolated as
+    t(a1-a3, all tokens) + t(a4-a9 per token) x tokens."""
+
+    def __init__(self, wl):
+        import oracle as O  # the CPU oracle: benchmark baseline leg only
+
+        self.O = O
+        if wl.n_blocks > 1 or wl.token_pair:
+            wl = wl.with_(n_blocks=1, token_pair=False)
+        self.wl = wl
+        raw, self.c, self.x = synth.block_weights(wl), synth.cond(wl), synth.x_input(wl)
+        w = {"w_ada": raw["w_ada"], "b_ada": raw["b_ada"]}
+        for name, sname in (("wqkv", "sqkv"), ("wo", "so"), ("w1", "s1"), ("w2", "s2")):
+            w[name], w[sname] = O.quantize_rows(raw[name])
+        if not wl.qkv_int8:
+            w["wqkv_bf16"] = raw["wqkv_bf16"]
+        self.w = w
+        self.dm = O.Dims(wl.B, wl.T, wl.H, wl.W, wl.d, wl.n_heads, wl.head_dim, wl.d_ff, wl.rope,
+                         wl.rope_theta, wl.ln_eps, wl.qkv_int8)
+        self.R = wl.B * wl.L
+        self.t_kv = None
+
+    def run(self, n_rows):
+        rows = synth.sample_rows(self.R, n_rows) if n_rows else np.zeros(0, np.int64)
+        t0 = time.perf_counter()
+        self.O.block_forward(self.dm, self.w, self.c, self.x, rows=rows)
+        return time.perf_counter() - t0
+
+    def measure_kv(self):
+        self.t_kv = self.run(0)
+        return self.t_kv
+
+    def estimate(self, n_rows):
+        """Extrapolated full-block seconds from one sampled run."""
+        if self.t_kv is None:
+            self.measure_kv()
+        t = self.run(n_rows)
+        return self.t_kv + max(t - self.t_kv, 0.0) / n_rows * self.R
+
+    def sample_text(self, n_rows):
+        return (f"a1-a3 over all {self.R} tokens + a4-a9 on {n_rows} sampled tokens, "
+                f"extrapolated to {self.R} tokens")
+
+    def threads(self):
+        return self.O.threads()
+
+
+# ----------------------------------------------------------------------------- arms
+
+def dist_init():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v, world):
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([float(v)], device="cuda", dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(v, world):
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([float(v)], device="cuda", dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def run_h3b(args, rank, world, local):
+    cuda_build.build()
+    h3b.lib()
+    peaks, peak_src = load_peaks()
+    W = Workload(args.workload, rank)
+    wl = W.wl
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    h3b.h3b_device_error(clear=True)
+
+    def prep():
+        W.x.copy_(W.x_ref)
+        flush.zero_()
+
+    sampler = ClockSampler(local) if rank == 0 else None
+    if sampler:
+        sampler.start()
+    for _ in range(args.warmup):
+        prep()
+        W.step()
+    torch.cuda.synchronize()
+    barrier(world)
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    h3b.h3b_profile_read()  # drop anything recorded during warm-up
+    h3b.h3b_profile_enable(True)
+    torch.cuda.synchronize()
+    barrier(world)
+    for i in range(args.steps):
+        prep()  # restore the input and flush L2 outside the timed events
+        ev[i][0].record()
+        W.step()
+        ev[i][1].record()
+    torch.cuda.synchronize()
+    barrier(world)
+    h3b.h3b_profile_enable(False)
+    clocks = sampler.stop() if sampler else None
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    total_ms = max_over_ranks(sum(step_ms), world)
+    prof = h3b.h3b_profile_read()
+    err = h3b.h3b_device_error(clear=True)
+    if err:
+        raise RuntimeError(f"device error word set during the benchmark: {err:#x}")
+
+    tokens_all = sum_over_ranks(W.tokens * args.steps, world)
+    value = tokens_all / (total_ms / 1e3)
+
+    # ---- end to end: pinned host input -> device -> block -> host output, same API
+    x_host = torch.empty(W.x.shape, dtype=torch.bfloat16, pin_memory=True)
+    x_host.copy_(W.x_ref.cpu())
+    c_host = torch.empty(W.c.shape, dtype=W.c.dtype, pin_memory=True)
+    c_host.copy_(W.c.cpu())
+    out_host = torch.empty_like(x_host, pin_memory=True)
+    c_dev = torch.empty_like(W.c)
+    e2e_steps = max(3, min(args.steps, 20))
+    for _ in range(2):
+        W.x.copy_(x_host, non_blocking=True)
+        c_dev.copy_(c_host, non_blocking=True)
+        W.step(c=c_dev)
+        out_host.copy_(W.x, non_blocking=True)
+    torch.cuda.synchronize()
+    barrier(world)
+    eev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(e2e_steps)]
+    for i in range(e2e_steps):
+        flush.zero_()
+        eev[i][0].record()
+        W.x.copy_(x_host, non_blocking=True)
+        c_dev.copy_(c_host, non_blocking=True)
+        W.step(c=c_dev)
+        out_host.copy_(W.x, non_blocking=True)
+        eev[i][1].record()
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in eev), world)
+    e2e_value = sum_over_ranks(W.tokens * e2e_steps, world) / (e2e_ms / 1e3)
+    h2d = x_host.numel() * x_host.element_size() + c_host.numel() * c_host.element_size()
+    d2h = out_host.numel() * out_host.element_size()
+
+    # ---- roofline of the dominant kernel (live per-kernel device times)
+    ktot = sum(ms for _, ms in prof.values()) or 1.0
+    shares = {k: round(ms / ktot, 4) for k, (n, ms) in sorted(prof.items(), key=lambda kv: -kv[1][1])}
+    dom = max(prof.items(), key=lambda kv: kv[1][1])[0] if prof else None
+    roof = None
+    if dom:
+        n_launch, ms = prof[dom]
+        per_launch_s = ms / n_launch / 1e3
+        work, unit, bound = kernel_work(dom, wl)
+        if bound == "hbm":
+            achieved, peak, runit, rb = work / per_launch_s / 1e9, peaks["hbm_gbs"], "GB/s", "hbm"
+        else:
+            achieved = work / per_launch_s / 1e12
+            peak = peaks["bf16_tflops"] * (INT8_OVER_BF16 if bound == "tensor_i8" else 1.0)
+            runit, rb = ("TOP/s" if bound == "tensor_i8" else "TFLOP/s"), "tensor"
+        roof = {"bound": rb, "kernel": dom, "achieved": round(achieved, 2), "peak": round(peak, 1), "unit": runit,
+                "frac": round(achieved / peak, 4), "traffic": traffic_for(dom, wl, n_launch),
+                "peak_source": f"{peak_src} ({'bf16 burst x 2 nominal int8/bf16 ratio' if bound == 'tensor_i8' else 'bf16 burst' if bound == 'tensor_bf16' else 'copy bandwidth'})",
+                "work_per_launch": work, "work_unit": unit, "launch_ms": round(per_launch_s * 1e3, 4)}
+    all_roof = {}
+    for k, (n, ms) in prof.items():
+        work, unit, bound = kernel_work(k, wl)
+        if work <= 0:
+            continue
+        s = ms / n / 1e3
+        if bound == "hbm":
+            all_roof[k] = {"GB/s": round(work / s / 1e9, 1), "frac": round(work / s / 1e9 / peaks["hbm_gbs"], 3)}
+        else:
+            pk = peaks["bf16_tflops"] * (INT8_OVER_BF16 if bound == "tensor_i8" else 1.0)
+            all_roof[k] = {("TOP/s" if bound == "tensor_i8" else "TFLOP/s"): round(work / s / 1e12, 1),
+                           "frac": round(work / s / 1e12 / pk, 3)}
+
+    gpu_launches = int(sum(n for n, _ in prof.values()))
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        orc = OracleRunner(wl)
+        est_s = orc.estimate(args.cpu_rows)
+        cpu = {"value": round(W.tokens / est_s, 2), "unit": UNIT, "cores": orc.threads(),
+               "kind": "oracle", "sample": orc.sample_text(args.cpu_rows)}
+
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "int8+bf16", "data": "synthetic",
+        "config": {"workload": args.workload, "batch": wl.B, "grid_THW": [wl.T, wl.H, wl.W], "tokens": wl.L,
+                   "d": wl.d, "heads": wl.n_heads, "head_dim": wl.head_dim, "d_ff": wl.d_ff,
+                   "blocks_per_step": wl.n_blocks, "token_pair": wl.token_pair,
+                   "qkv": "int8" if wl.qkv_int8 else "bf16", "attention": "bf16",
+                   "l2": "flushed between steps (512 MiB write outside the timed events)",
+                   "parallelism": "replicas: one independent latent per GPU, no collective"},
+        "roofline": roof, "kernel_share": shares, "kernel_roofline": all_roof,
+        "cpu_baseline": cpu,
+        "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "steps": e2e_steps},
+        "gpu_launches": gpu_launches, "clocks": clocks,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_reference(args, rank, world, local):
+    """The CPU oracle as the reference arm (rank 0 only)."""
+    if rank != 0:
+        return
+    wl = synth.WORKLOADS[args.workload]
+    orc = OracleRunner(wl)
+    orc.measure_kv()
+    est = []
+    for i in range(args.warmup + args.steps):
+        e = orc.estimate(args.ref_rows)
+        if i >= args.warmup:
+            est.append(e)
+    sample, threads = orc.sample_text(args.ref_rows), orc.threads()
+    tokens = wl.B * wl.L
+    ms = 1e3 * sum(est) / len(est)
+    value = tokens / (ms / 1e3)
+    line = {"metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms, 2), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64 (int8 decisions in f32)", "data": "synthetic", "impl": "reference",
+            "config": {"workload": args.workload, "tokens": wl.L, "d": wl.d, "heads": wl.n_heads,
+                       "head_dim": wl.head_dim, "d_ff": wl.d_ff},
+            "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+_TRAFFIC = None
+
+
+def traffic_for(kernel, wl, n_launch):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, scaled to
+    this workload when it was captured on a smaller case of the same kernel; None
+    when no capture exists or the kernel source changed since it was taken."""
+    global _TRAFFIC
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if _TRAFFIC is None:
+        try:
+            with open(path) as f:
+                _TRAFFIC = json.load(f)
+        except Exception:
+            _TRAFFIC = {}
+    ent = _TRAFFIC.get(kernel)
+    if not ent:
+        return None
+    src = os.path.join(ROOT, "video_diffusion_transformer_adaln_b200", "csrc", ent.get("source", ""))
+    try:
+        import hashlib
+        with open(src, "rb") as f:
+            if hashlib.sha256(f.read()).hexdigest()[:16] != ent.get("source_sha256_16"):
+                return None
+    except Exception:
+        return None
+    if ent.get("workload") == wl.name:
+        return ent.get("bytes_per_launch")
+    scale = ent.get("scale_to", {}).get(wl.name)
+    return None if scale is None else ent["bytes_per_launch"] * scale
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--impl", default="h3b", choices=["h3b", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-rows", type=int, default=256, help="sampled tokens for the oracle baseline")
+    ap.add_argument("--ref-rows", type=int, default=16, help="sampled tokens per reference-arm step")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        run_reference(args, rank, world, 0)
+        return
+    rank, world, local = dist_init()
+    if world != args.gpus and rank == 0:
+        log(f"note: --gpus {args.gpus} but WORLD_SIZE={world}; using WORLD_SIZE")
+    try:
+        run_h3b(args, rank, world, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

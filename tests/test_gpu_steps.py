@@ -83,15 +83,18 @@ def test_ln_modulate_quantize(rows, d, items):
     assert np.array_equal(q.cpu().numpy(), qo) and np.array_equal(s.cpu().numpy(), so)
     assert np.all(az.cpu().numpy() == 0)
     # (2) the bf16 quantizer input matches the oracle's fp64 LN + modulation to one
-    #     bf16 rounding (fp32 LN statistics may move a value across a rounding boundary)
+    #     bf16 ulp of the value (at most 2^-7 |h|), plus the fp32 error of y*(1+scale)+shift when
+    #     the two terms nearly cancel (bounded relative to the row's magnitude)
     y = O.layernorm(O.bf16_decode(x), 1e-6)
     ho = np.empty_like(hg)
     for i in range(rows):
         it = i // rpi
         ho[i] = O.modulate_bf16(y[i:i + 1], mod[it, 3 * d:4 * d].astype(np.float64),
                                 mod[it, 4 * d:5 * d].astype(np.float64))[0]
-    ulp = bf16_ulp_diff(hg, ho)
-    assert ulp.max() <= 1 and (ulp > 0).mean() < 0.02
+    hgd, hod = O.bf16_decode(hg), O.bf16_decode(ho)
+    bound = 2.0 ** -7 * np.abs(hod) + 2.0 ** -16 * np.abs(hod).max(axis=1, keepdims=True)
+    assert np.all(np.abs(hgd - hod) <= bound)
+    assert (hg != ho).mean() < 0.02
     no_device_error()
 
 
@@ -172,8 +175,11 @@ def test_gemm_i8_gated_residual(M, N, K, items):
     ref = np.empty((M, N))
     for i in range(M):
         ref[i] = O.gated_residual(O.bf16_decode(x[i:i + 1]), y[i:i + 1], gate[i // rpi, N:2 * N])[0]
-    ulp = bf16_ulp_diff(bf16_host(xd), O.bf16_round(ref))
-    assert ulp.max() <= 1
+    # one bf16 rounding of the result, plus the fp32 error of x + gate*y when the
+    # two terms nearly cancel (relative to the terms' magnitude)
+    got = O.bf16_decode(bf16_host(xd))
+    terms = np.abs(O.bf16_decode(x)) + np.abs(np.stack([gate[i // rpi, N:2 * N] for i in range(M)]) * y)
+    assert np.all(np.abs(got - ref) <= 2.0 ** -8 * np.abs(ref) + 2.0 ** -20 * terms + 1e-30)
     # a zero gate leaves x bit-identical
     xd2 = bf16_dev(x)
     h3b.h3b_gemm_i8_gated_residual(to_dev(qa), to_dev(sa), to_dev(qw), to_dev(sw), to_dev(bias),

@@ -13,6 +13,7 @@
 #include <algorithm>
 #include <mutex>
 #include <string>
+#include <vector>
 
 #include "h3b.h"
 #include "h3b_common.cuh"
@@ -149,10 +150,56 @@ h3b_status check_weights(const h3b_dims& d, const h3b_block_weights* w) {
   return H3B_OK;
 }
 
-#define H3B_CK(call, where)                        \
-  do {                                             \
-    cudaError_t e_ = (call);                       \
-    if (e_ != cudaSuccess) return cuda_fail(e_, where); \
+// ---------------------------------------------------------------------------
+// Kernel-level timing (h3b_profile_*): event pairs around each launch.
+// ---------------------------------------------------------------------------
+struct ProfRec {
+  const char* name;
+  cudaEvent_t a, b;
+};
+std::mutex g_prof_mu;
+bool g_prof_on = false;
+std::vector<ProfRec> g_prof_recs;
+std::vector<cudaEvent_t> g_prof_free;
+
+cudaEvent_t prof_event() {
+  if (!g_prof_free.empty()) {
+    cudaEvent_t e = g_prof_free.back();
+    g_prof_free.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+  return e;
+}
+
+// Scoped bracket: records a start event now and an end event when the launch
+// has been enqueued (only while profiling is on).
+struct ProfScope {
+  const char* name;
+  cudaStream_t st;
+  cudaEvent_t a = nullptr;
+  ProfScope(const char* n, cudaStream_t s) : name(n), st(s) {
+    if (!g_prof_on) return;
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    a = prof_event();
+    if (a) cudaEventRecord(a, st);
+  }
+  ~ProfScope() {
+    if (!a) return;
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    cudaEvent_t b = prof_event();
+    if (!b) return;
+    cudaEventRecord(b, st);
+    g_prof_recs.push_back({name, a, b});
+  }
+};
+
+#define H3B_CK(call, where)                                 \
+  do {                                                      \
+    ProfScope prof_scope_(where, st);                       \
+    cudaError_t e_ = (call);                                \
+    if (e_ != cudaSuccess) return cuda_fail(e_, where);     \
   } while (0)
 
 GemmArgs base_args(int M, int N, int K, unsigned* err) {
@@ -377,6 +424,7 @@ h3b_status h3b_token_pair(const h3b_dims* full, const void* x, void* xm, void* x
   DeviceInfo* di = nullptr;
   if ((s = device_info(&di)) != H3B_OK) return s;
   const long long lines = (long long)full->B * full->T * full->H;
+  cudaStream_t st = stream;
   H3B_CK(launch_token_pair(x, xm, xm_copy, lines, full->W, full->d, di->sms, stream), "token_pair");
   return H3B_OK;
 }
@@ -390,22 +438,25 @@ h3b_status h3b_token_unpair(const h3b_dims* full, const void* x, const void* xm,
   DeviceInfo* di = nullptr;
   if ((s = device_info(&di)) != H3B_OK) return s;
   const long long lines = (long long)full->B * full->T * full->H;
+  cudaStream_t st = stream;
   H3B_CK(launch_token_unpair(x, xm, ym, out, lines, full->W, full->d, di->sms, stream), "token_unpair");
   return H3B_OK;
 }
 
 h3b_status h3b_quantize_weights(const float* w, int rows, int cols, int8_t* q, float* s, h3b_stream stream) {
+  cudaStream_t st = stream;
   if (!w || !q || !s) return fail(H3B_ERR_ARG, "NULL pointer");
   if (rows < 0 || cols < 16 || cols % 16 != 0) return fail(H3B_ERR_SHAPE, "cols must be a positive multiple of 16");
   if (!aligned16(w) || !aligned16(q)) return fail(H3B_ERR_ALIGN, "alignment");
   DeviceInfo* di = nullptr;
-  h3b_status st = device_info(&di);
-  if (st != H3B_OK) return st;
+  h3b_status hs = device_info(&di);
+  if (hs != H3B_OK) return hs;
   H3B_CK(launch_quant_rows_f32(w, rows, cols, q, s, stream), "quantize_weights");
   return H3B_OK;
 }
 
 h3b_status h3b_device_error(unsigned int* code, int clear) {
+  cudaStream_t st = nullptr;
   if (!code) return fail(H3B_ERR_ARG, "code is NULL");
   DeviceInfo* di = nullptr;
   h3b_status s = device_info(&di);
@@ -420,6 +471,7 @@ h3b_status h3b_device_error(unsigned int* code, int clear) {
 
 h3b_status h3b_adaln_modulation(const h3b_dims* dims, const void* w_ada, const float* b_ada, const float* c,
                                 float* mod, h3b_stream stream) {
+  cudaStream_t st = stream;
   h3b_status s = check_dims(dims);
   if (s != H3B_OK) return s;
   if (!w_ada || !c || !mod) return fail(H3B_ERR_ARG, "NULL pointer");
@@ -433,14 +485,15 @@ h3b_status h3b_adaln_modulation(const h3b_dims* dims, const void* w_ada, const f
 h3b_status h3b_ln_modulate_quantize(const void* x, int rows, int d, float eps, const float* shift,
                                     const float* scale, int rows_per_item, int mod_stride, int8_t* q, float* s,
                                     void* h_out, float* absmax_zero, int write_codes, h3b_stream stream) {
+  cudaStream_t st = stream;
   if (!x || !shift || !scale || (write_codes && (!q || !s))) return fail(H3B_ERR_ARG, "NULL pointer");
   if (rows < 0 || d < 256 || d % 256 != 0 || d > 8192) return fail(H3B_ERR_SHAPE, "d must be a multiple of 256, <= 8192");
   if (rows_per_item < 1 || mod_stride < 0 || mod_stride % 4 != 0) return fail(H3B_ERR_ARG, "rows_per_item/mod_stride");
   if (!aligned16(x) || !aligned16(shift) || !aligned16(scale) || (q && !aligned16(q)) || (h_out && !aligned16(h_out)))
     return fail(H3B_ERR_ALIGN, "alignment");
   DeviceInfo* di = nullptr;
-  h3b_status st = device_info(&di);
-  if (st != H3B_OK) return st;
+  h3b_status hs = device_info(&di);
+  if (hs != H3B_OK) return hs;
   H3B_CK(launch_ln_mod_quant(x, rows, d, eps, shift, scale, rows_per_item, mod_stride, q, s, h_out, absmax_zero,
                              write_codes, stream), "ln_mod_quant");
   return H3B_OK;
@@ -448,12 +501,13 @@ h3b_status h3b_ln_modulate_quantize(const void* x, int rows, int d, float eps, c
 
 h3b_status h3b_quantize_rows(const void* h, int rows, int cols, const float* absmax, int8_t* q, float* s,
                              h3b_stream stream) {
+  cudaStream_t st = stream;
   if (!h || !q || !s) return fail(H3B_ERR_ARG, "NULL pointer");
   if (rows < 0 || cols < 16 || cols % 16 != 0) return fail(H3B_ERR_SHAPE, "cols must be a positive multiple of 16");
   if (!aligned16(h) || !aligned16(q)) return fail(H3B_ERR_ALIGN, "alignment");
   DeviceInfo* di = nullptr;
-  h3b_status st = device_info(&di);
-  if (st != H3B_OK) return st;
+  h3b_status hs = device_info(&di);
+  if (hs != H3B_OK) return hs;
   H3B_CK(launch_quant_rows_bf16(h, rows, cols, absmax, q, s, stream), "quantize_rows");
   return H3B_OK;
 }
@@ -468,6 +522,7 @@ static h3b_status gemm_common(const void* A, const void* W, const void* out, int
 }
 
 h3b_status h3b_gemm_i8_s32(const int8_t* A, const int8_t* W, int32_t* C, int M, int N, int K, h3b_stream stream) {
+  cudaStream_t st = stream;
   DeviceInfo* di = nullptr;
   h3b_status s = gemm_common(A, W, C, M, N, K, &di);
   if (s != H3B_OK) return s;
@@ -479,6 +534,7 @@ h3b_status h3b_gemm_i8_s32(const int8_t* A, const int8_t* W, int32_t* C, int M, 
 
 h3b_status h3b_gemm_i8_dequant(const int8_t* A, const float* sA, const int8_t* W, const float* sW,
                                const float* bias, void* out, int M, int N, int K, h3b_stream stream) {
+  cudaStream_t st = stream;
   DeviceInfo* di = nullptr;
   h3b_status s = gemm_common(A, W, out, M, N, K, &di);
   if (s != H3B_OK) return s;
@@ -492,6 +548,7 @@ h3b_status h3b_gemm_i8_dequant(const int8_t* A, const float* sA, const int8_t* W
 
 h3b_status h3b_qkv_projection(const h3b_dims* dims, const void* A, const float* sA, const h3b_block_weights* w,
                               void* qkv, void* rope_ws, h3b_stream stream) {
+  cudaStream_t st = stream;
   h3b_status s = check_dims(dims);
   if (s != H3B_OK) return s;
   if (!A || !w || !qkv || !rope_ws) return fail(H3B_ERR_ARG, "NULL pointer");
@@ -517,6 +574,7 @@ h3b_status h3b_qkv_projection(const h3b_dims* dims, const void* A, const float* 
 }
 
 h3b_status h3b_attention(const h3b_dims* dims, const void* qkv, void* o, float* absmax, h3b_stream stream) {
+  cudaStream_t st = stream;
   // Attention alone needs only the grid, the batch and the head shape.
   if (!dims) return fail(H3B_ERR_ARG, "dims is NULL");
   if (dims->B < 1 || dims->T < 1 || dims->H < 1 || dims->W < 1 || dims->n_heads < 1)
@@ -537,6 +595,7 @@ h3b_status h3b_attention(const h3b_dims* dims, const void* qkv, void* o, float* 
 h3b_status h3b_gemm_i8_gated_residual(const int8_t* A, const float* sA, const int8_t* W, const float* sW,
                                       const float* bias, const float* gate, int rows_per_item, int gate_stride,
                                       void* x, int M, int N, int K, h3b_stream stream) {
+  cudaStream_t st = stream;
   DeviceInfo* di = nullptr;
   h3b_status s = gemm_common(A, W, x, M, N, K, &di);
   if (s != H3B_OK) return s;
@@ -552,6 +611,7 @@ h3b_status h3b_gemm_i8_gated_residual(const int8_t* A, const float* sA, const in
 
 h3b_status h3b_gemm_i8_gelu(const int8_t* A, const float* sA, const int8_t* W, const float* sW, const float* bias,
                             void* g, float* absmax, int M, int N, int K, h3b_stream stream) {
+  cudaStream_t st = stream;
   DeviceInfo* di = nullptr;
   h3b_status s = gemm_common(A, W, g, M, N, K, &di);
   if (s != H3B_OK) return s;
@@ -561,6 +621,41 @@ h3b_status h3b_gemm_i8_gelu(const int8_t* A, const float* sA, const int8_t* W, c
   a.sA = sA; a.sW = sW; a.bias = bias; a.out = g; a.absmax = absmax;
   H3B_CK(launch_gemm(true, EPI_GELU, A, W, a, di->sms, stream), "gemm_i8_gelu");
   return H3B_OK;
+}
+
+h3b_status h3b_profile_enable(int enable) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  g_prof_on = enable != 0;
+  return H3B_OK;
+}
+
+int h3b_profile_read(h3b_kernel_time* out, int max_entries) {
+  if (!out || max_entries < 0) return H3B_ERR_ARG;
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  int n = 0;
+  for (const ProfRec& r : g_prof_recs) {
+    float ms = 0.0f;
+    cudaError_t e = cudaEventSynchronize(r.b);
+    if (e == cudaSuccess) e = cudaEventElapsedTime(&ms, r.a, r.b);
+    if (e != cudaSuccess) return cuda_fail(e, "profile event");
+    int k = 0;
+    while (k < n && std::string(out[k].name) != r.name) ++k;
+    if (k == n) {
+      if (n == max_entries) continue;
+      out[n].name = r.name;
+      out[n].launches = 0;
+      out[n].total_ms = 0.0;
+      ++n;
+    }
+    out[k].launches += 1;
+    out[k].total_ms += ms;
+  }
+  for (const ProfRec& r : g_prof_recs) {
+    g_prof_free.push_back(r.a);
+    g_prof_free.push_back(r.b);
+  }
+  g_prof_recs.clear();
+  return n;
 }
 
 }  // extern "C"

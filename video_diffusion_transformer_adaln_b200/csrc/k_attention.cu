@@ -209,7 +209,10 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
     bool ok = true;
     for (int j = 0; j < nkv; ++j) {
       const int sb = j & 1;
-      if (*abort_flag || !mbar_wait(s_full(sb), (j >> 1) & 1, a.err, ERR_WAIT_MMA)) { ok = false; break; }
+      // tcgen05.ld/st are warp-collective (.sync.aligned): every decision that
+      // guards them is made uniform across the warp.
+      const bool s_ok = !*abort_flag && mbar_wait(s_full(sb), (j >> 1) & 1, a.err, ERR_WAIT_MMA);
+      if (!__all_sync(0xFFFFFFFFu, s_ok)) { ok = false; break; }
       tc_fence_after();
       uint32_t sr[BKV];
 #pragma unroll
@@ -255,8 +258,11 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
       }
       l_run = fmaf(l_run, alpha, rowsum);
 
-      if (j > 0 && !mbar_wait(pv_done, (j - 1) & 1, a.err, ERR_WAIT_MMA)) { ok = false; break; }
-      if (rescale) {
+      const bool pv_ok = (j == 0) || mbar_wait(pv_done, (j - 1) & 1, a.err, ERR_WAIT_MMA);
+      if (!__all_sync(0xFFFFFFFFu, pv_ok)) { ok = false; break; }
+      // The whole warp rescales its rows of O if any row's max moved; rows that
+      // kept their max use alpha = 1.
+      if (__any_sync(0xFFFFFFFFu, rescale)) {
         tc_fence_after();
 #pragma unroll
         for (int c = 0; c < DH / 32; ++c) {
@@ -282,7 +288,8 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(p_full);
     }
-    if (ok && mbar_wait(pv_done, (nkv - 1) & 1, a.err, ERR_WAIT_MMA)) {
+    const bool fin = ok && mbar_wait(pv_done, (nkv - 1) & 1, a.err, ERR_WAIT_MMA);
+    if (__all_sync(0xFFFFFFFFu, fin)) {
       tc_fence_after();
       const int q = qt * BQ + row;
       const int b = bh / a.n_heads, h = bh - b * a.n_heads;

@@ -296,7 +296,9 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
       tile_coords(t, n_m, n_n, mb, nb);
       const int acc = tl & 1;
       const uint32_t aph = (tl >> 1) & 1;
-      if (*abort_flag || !mbar_wait(tfull(acc), aph, p.err, ERR_WAIT_MMA)) { *abort_flag = 1; break; }
+      // tcgen05.ld is warp-collective: the wait outcome is made warp-uniform.
+      const bool t_ok = !*abort_flag && mbar_wait(tfull(acc), aph, p.err, ERR_WAIT_MMA);
+      if (!__all_sync(0xFFFFFFFFu, t_ok)) { *abort_flag = 1; break; }
       tc_fence_after();
       const int row = mb * BM + quad * 32 + lane;
       const uint32_t tbase = tmem_base + ((uint32_t)(quad * 32) << 16) + acc * BN;

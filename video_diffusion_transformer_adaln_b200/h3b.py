@@ -46,6 +46,10 @@ class BlockWeights(C.Structure):
     _fields_ = [(n, C.c_void_p) for n in WEIGHT_FIELDS]
 
 
+class KernelTime(C.Structure):
+    _fields_ = [("name", C.c_char_p), ("launches", C.c_int), ("total_ms", C.c_double)]
+
+
 _LIB = None
 
 
@@ -91,6 +95,10 @@ def _declare(L):
         f.argtypes = args
     L.h3b_rope_table_bytes.restype = sz
     L.h3b_rope_table_bytes.argtypes = [vp]
+    L.h3b_profile_enable.restype = i32
+    L.h3b_profile_enable.argtypes = [i32]
+    L.h3b_profile_read.restype = i32
+    L.h3b_profile_read.argtypes = [C.POINTER(KernelTime), i32]
 
 
 def _p(t: Optional[torch.Tensor]):
@@ -231,3 +239,18 @@ def h3b_gemm_i8_gelu(A, sA, W, sW, bias, g, absmax, stream=None):
     N = W.shape[0]
     _check(lib().h3b_gemm_i8_gelu(_p(A), _p(sA), _p(W), _p(sW), _p(bias), _p(g), _p(absmax), M, N, K, _s(stream)),
            "h3b_gemm_i8_gelu")
+
+
+# --------------------------------------------------------------------------- profiling
+
+def h3b_profile_enable(on: bool = True):
+    _check(lib().h3b_profile_enable(1 if on else 0), "h3b_profile_enable")
+
+
+def h3b_profile_read(max_entries: int = 64) -> Dict[str, tuple]:
+    """{kernel name: (launches, total device ms)} since the last read."""
+    arr = (KernelTime * max_entries)()
+    n = lib().h3b_profile_read(arr, max_entries)
+    if n < 0:
+        _check(n, "h3b_profile_read")
+    return {arr[i].name.decode(): (arr[i].launches, arr[i].total_ms) for i in range(n)}
