@@ -49,6 +49,9 @@ struct GemmArgs {
   int B, L, T, H, W, d, n_heads, head_dim, rope_t, rope_h, rope_w;
   const float2* rope;  // table from launch_rope_table
   unsigned* err;       // device error word
+  // tile raster (set by launch_gemm): groups of `group` M-tiles (raster_n == 0)
+  // or of `group` N-tiles (raster_n == 1)
+  int raster_n, group;
 };
 
 // A [M][K] and W [N][K] row-major, int8 (kInt8) or bf16.

@@ -13,21 +13,28 @@
 //     section "★ 긴 영상은 나눠 찍는 게 훨씬 쌉니다": cost grows about as
 //     frames^1.9, i.e. full attention over every latent token.
 //
-// Design (B200): one CTA per (128-query tile, batch item x head). Warp 0 loads
-// Q once and streams K/V tiles of 128 keys with TMA (2-stage rings, 128-byte
-// swizzle); warp 1 issues tcgen05.mma from one thread: S = Q K^T into one of
-// two TMEM score buffers, then O += P V into a TMEM accumulator, with the next
-// tile's S issued ahead of the current P V. Warps 2-5 (one query row per
-// thread) read S from TMEM, run the online softmax in fp32 with exp2, write P
-// as bf16 into shared memory in the MMA operand layout, and rescale O in TMEM
-// only when a row's running max grows by more than 2^8 (otherwise the stale
-// max is kept; the final division by the row sum is exact either way).
+// Design (B200). One CTA per (256 queries, batch item x head): two query tiles
+// g = 0, 1 of 128 rows share every K/V tile.
+//   warp 0     TMA: Q0 and Q1 once, then K_j and V_j (128 keys) into 2-stage rings
+//   warp 1     tcgen05.mma from one thread, in the order
+//                S0(0) S1(0) | PV0(0) S0(1) PV1(0) S1(1) | PV0(1) S0(2) ...
+//              so the tensor core always has the other tile's work queued
+//   warps 2-5  softmax of tile 0, warps 6-9 softmax of tile 1 (thread = row)
+// Tensor memory (512 columns): S0 | S1 | O0 | O1. Each softmax thread reads its
+// row of S_g, writes P_g = exp2(S*c - m) as bf16 pairs over the first 64
+// columns of S_g, and the P V product takes its A operand from tensor memory.
+// A commit tracks every earlier MMA of the issuing thread, so when S_g(j) is
+// complete, PV_g(j-1) is complete too: O_g can be rescaled then without another
+// barrier. The running max is kept until a row's max grows by more than 2^8
+// (then O_g and the row sum are rescaled); the final division by the row sum
+// is exact either way. Every wait is bounded and every decision guarding a
+// warp-collective TMEM access is warp-uniform.
 #include "h3b_common.cuh"
 #include "h3b_internal.h"
 
 namespace h3b {
 namespace attn {
-constexpr int BQ = 128, BKV = 128, kThreads = 192;
+constexpr int BQ = 128, BKV = 128, kThreads = 320;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int BOX = 16384;  // one TMA box: 128 rows x 128 bytes
 }  // namespace attn
@@ -37,21 +44,35 @@ __device__ __forceinline__ float fast_exp2(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+// tcgen05.mma with the A operand in tensor memory (kind::f16, bf16 inputs).
+__device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                           uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 
 template <int DH>
 struct AttnLayout {
-  static constexpr int NBOX = DH / 64;                // TMA boxes per Q/K/V tile
-  static constexpr int TILE = attn::BKV * DH * 2;     // bytes of one Q/K/V tile
-  static constexpr int Q_OFF = 0;
-  static constexpr int K_OFF = Q_OFF + TILE;
-  static constexpr int V_OFF = K_OFF + 2 * TILE;
-  static constexpr int P_OFF = V_OFF + 2 * TILE;
-  static constexpr int BAR_OFF = P_OFF + attn::BQ * attn::BKV * 2;
-  static constexpr int NBARS = 1 + 8 + 2 + 2 + 1 + 1 + 1;
-  // At least 120 KB so that two CTAs never share an SM: each holds all 512
-  // TMEM columns for its lifetime.
+  static constexpr int NBOX = DH / 64;             // TMA boxes per Q/K/V tile
+  static constexpr int TILE = attn::BKV * DH * 2;  // bytes of one Q/K/V tile
+  static constexpr int Q_OFF = 0;                  // Q0, Q1
+  static constexpr int K_OFF = Q_OFF + 2 * TILE;   // K stages 0, 1
+  static constexpr int V_OFF = K_OFF + 2 * TILE;   // V stages 0, 1
+  static constexpr int BAR_OFF = V_OFF + 2 * TILE;
+  static constexpr int NBARS = 16;
   static constexpr size_t SMEM_NEED = (size_t)BAR_OFF + NBARS * 8 + 16 + 1024;
+  // At least 120 KB so two CTAs never share an SM: each holds all 512 TMEM columns.
   static constexpr size_t SMEM = SMEM_NEED > 120 * 1024 ? SMEM_NEED : 120 * 1024;
+  // tensor memory columns: S0, S1, O0, O1
+  static constexpr uint32_t S_COL0 = 0, S_COL1 = 128, O_COL0 = 256, O_COL1 = 256 + DH;
 };
 
 template <int DH>
@@ -64,16 +85,14 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
   const uint32_t sb0 = smem_u32(smem);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::BAR_OFF);
   const uint32_t bar0 = smem_u32(bars);
-  // barrier slots
   const uint32_t q_full = bar0;
   auto k_full = [&](int s) { return bar0 + 8u * (1 + s); };
   auto k_empty = [&](int s) { return bar0 + 8u * (3 + s); };
   auto v_full = [&](int s) { return bar0 + 8u * (5 + s); };
   auto v_empty = [&](int s) { return bar0 + 8u * (7 + s); };
-  auto s_full = [&](int b) { return bar0 + 8u * (9 + b); };
-  auto s_empty = [&](int b) { return bar0 + 8u * (11 + b); };
-  const uint32_t p_full = bar0 + 8u * 13;
-  const uint32_t pv_done = bar0 + 8u * 14;
+  auto s_full = [&](int g) { return bar0 + 8u * (9 + g); };
+  auto p_full = [&](int g) { return bar0 + 8u * (11 + g); };
+  auto fin = [&](int g) { return bar0 + 8u * (13 + g); };
   const uint32_t drain = bar0 + 8u * 15;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + Lay::NBARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -91,10 +110,8 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
     for (int s = 0; s < 2; ++s) {
       mbar_init(k_full(s), 1); mbar_init(k_empty(s), 1);
       mbar_init(v_full(s), 1); mbar_init(v_empty(s), 1);
-      mbar_init(s_full(s), 1); mbar_init(s_empty(s), 4);
+      mbar_init(s_full(s), 1); mbar_init(p_full(s), 4); mbar_init(fin(s), 1);
     }
-    mbar_init(p_full, 4);
-    mbar_init(pv_done, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -108,17 +125,16 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t O_COL = 256;
 
   if (warp == 0) {
     if (lane == 0) {
       // ---------------- TMA producer
       bool ok = true;
-      uint32_t filled = 0;  // bit s: K stage s, bit 2+s: V stage s, bit 4: Q; bit 5+: last parity
-      uint32_t fill_ph = 0;
-      mbar_arrive_expect_tx(q_full, Lay::TILE);
-      for (int b = 0; b < Lay::NBOX; ++b)
-        tma_load_3d(sb0 + Lay::Q_OFF + b * BOX, &tm, q_full, b * 64, qt * BQ, bh);
+      uint32_t filled = 0, fill_ph = 0;  // bits s (K stage s) and 2+s (V stage s)
+      mbar_arrive_expect_tx(q_full, 2 * Lay::TILE);
+      for (int g = 0; g < 2; ++g)
+        for (int b = 0; b < Lay::NBOX; ++b)
+          tma_load_3d(sb0 + Lay::Q_OFF + g * Lay::TILE + b * BOX, &tm, q_full, b * 64, qt * 2 * BQ + g * BQ, bh);
       for (int j = 0; j < nkv && ok; ++j) {
         const int s = j & 1;
         const uint32_t ph = (j >> 1) & 1;
@@ -143,7 +159,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
           if (filled & (4u << s)) mbar_wait(v_full(s), (fill_ph >> (2 + s)) & 1u, a.err, ERR_WAIT_DRAIN, kDrainLimitNs);
         }
       } else {
-        for (int s = 0; s < 2; ++s) {  // tail: all issued tiles consumed
+        for (int s = 0; s < 2; ++s) {  // tail: every issued tile has been consumed
           if (filled & (1u << s)) mbar_wait(k_empty(s), (fill_ph >> s) & 1u, a.err, ERR_WAIT_MMA);
           if (filled & (4u << s)) mbar_wait(v_empty(s), (fill_ph >> (2 + s)) & 1u, a.err, ERR_WAIT_MMA);
         }
@@ -152,45 +168,54 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       // ---------------- MMA issuer
-      bool ok = mbar_wait(q_full, 0, a.err, ERR_WAIT_TMA);
       bool any = false;
-      auto issue_pv = [&](int i) -> bool {
-        const int s = i & 1;
-        if (*abort_flag || !mbar_wait(p_full, i & 1, a.err, ERR_WAIT_EPI)) return false;
-        if (!mbar_wait(v_full(s), (i >> 1) & 1, a.err, ERR_WAIT_TMA)) return false;
-        tc_fence_after();
-        const uint32_t p_addr = sb0 + Lay::P_OFF;
-        const uint32_t v_addr = sb0 + Lay::V_OFF + s * Lay::TILE;
-#pragma unroll
-        for (int k = 0; k < BKV / 16; ++k) {
-          const uint64_t ad = smem_desc_sw128(p_addr + (k >> 2) * BOX + (k & 3) * 32, 16, 1024);
-          const uint64_t bd = smem_desc_sw128(v_addr + k * 2048, BOX, 1024);
-          mma_f16(tmem + O_COL, ad, bd, IDESC_PV, (i > 0 || k > 0) ? 1u : 0u);
-        }
-        tc_commit(v_empty(s));
-        tc_commit(pv_done);
-        return true;
-      };
-      for (int j = 0; j < nkv && ok; ++j) {
+      auto issue_s = [&](int g, int j) -> bool {  // S_g(j) = Q_g K_j^T
         const int s = j & 1;
-        const int sb = j & 1;
-        if (*abort_flag || !mbar_wait(k_full(s), (j >> 1) & 1, a.err, ERR_WAIT_TMA)) { ok = false; break; }
-        if (!mbar_wait(s_empty(sb), ((j >> 1) & 1) ^ 1u, a.err, ERR_WAIT_EPI)) { ok = false; break; }
+        if (g == 0 && (*abort_flag || !mbar_wait(k_full(s), (j >> 1) & 1, a.err, ERR_WAIT_TMA))) return false;
         tc_fence_after();
-        const uint32_t q_addr = sb0 + Lay::Q_OFF;
+        const uint32_t q_addr = sb0 + Lay::Q_OFF + g * Lay::TILE;
         const uint32_t k_addr = sb0 + Lay::K_OFF + s * Lay::TILE;
+        const uint32_t s_col = g == 0 ? Lay::S_COL0 : Lay::S_COL1;
 #pragma unroll
         for (int k = 0; k < DH / 16; ++k) {
           const uint64_t ad = smem_desc_sw128(q_addr + (k >> 2) * BOX + (k & 3) * 32, 16, 1024);
           const uint64_t bd = smem_desc_sw128(k_addr + (k >> 2) * BOX + (k & 3) * 32, 16, 1024);
-          mma_f16(tmem + sb * BKV, ad, bd, IDESC_S, k > 0 ? 1u : 0u);
+          mma_f16(tmem + s_col, ad, bd, IDESC_S, k > 0 ? 1u : 0u);
         }
         any = true;
-        tc_commit(k_empty(s));
-        tc_commit(s_full(sb));
-        if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
+        tc_commit(s_full(g));
+        if (g == 1) tc_commit(k_empty(s));
+        return true;
+      };
+      auto issue_pv = [&](int g, int j) -> bool {  // O_g += P_g(j) V_j
+        const int s = j & 1;
+        if (*abort_flag || !mbar_wait(p_full(g), j & 1, a.err, ERR_WAIT_EPI)) return false;
+        if (g == 0 && !mbar_wait(v_full(s), (j >> 1) & 1, a.err, ERR_WAIT_TMA)) return false;
+        tc_fence_after();
+        const uint32_t v_addr = sb0 + Lay::V_OFF + s * Lay::TILE;
+        const uint32_t o_col = g == 0 ? Lay::O_COL0 : Lay::O_COL1;
+        const uint32_t s_col = g == 0 ? Lay::S_COL0 : Lay::S_COL1;
+#pragma unroll
+        for (int k = 0; k < BKV / 16; ++k) {
+          const uint64_t bd = smem_desc_sw128(v_addr + k * 2048, BOX, 1024);
+          mma_f16_ts(tmem + o_col, tmem + s_col + k * 8, bd, IDESC_PV, (j > 0 || k > 0) ? 1u : 0u);
+        }
+        if (g == 1) tc_commit(v_empty(s));
+        return true;
+      };
+      bool ok = mbar_wait(q_full, 0, a.err, ERR_WAIT_TMA);
+      ok = ok && issue_s(0, 0) && issue_s(1, 0);
+      for (int j = 0; j < nkv && ok; ++j) {
+        ok = issue_pv(0, j);
+        if (!ok) break;
+        if (j + 1 < nkv) ok = issue_s(0, j + 1);
+        else tc_commit(fin(0));
+        if (!ok) break;
+        ok = issue_pv(1, j);
+        if (!ok) break;
+        if (j + 1 < nkv) ok = issue_s(1, j + 1);
+        else tc_commit(fin(1));
       }
-      if (ok) ok = issue_pv(nkv - 1);
       if (!ok) {
         *abort_flag = 1;
         if (any) {
@@ -200,39 +225,41 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
       }
     }
   } else {
-    // ---------------- softmax warps 2..5: thread = query row
+    // ---------------- softmax warps: 2-5 -> tile 0, 6-9 -> tile 1 (thread = query row)
+    const int g = (warp - 2) >> 2;
     const int quad = warp & 3;
     const int row = quad * 32 + lane;
     const uint32_t t_lane = (uint32_t)(quad * 32) << 16;
-    uint8_t* P = smem + Lay::P_OFF;
+    const uint32_t s_col = g == 0 ? Lay::S_COL0 : Lay::S_COL1;
+    const uint32_t o_col = g == 0 ? Lay::O_COL0 : Lay::O_COL1;
+    const float2 c2 = make_float2(scale_log2, scale_log2);
     float m_run = -INFINITY, l_run = 0.0f;
     bool ok = true;
     for (int j = 0; j < nkv; ++j) {
-      const int sb = j & 1;
-      // tcgen05.ld/st are warp-collective (.sync.aligned): every decision that
-      // guards them is made uniform across the warp.
-      const bool s_ok = !*abort_flag && mbar_wait(s_full(sb), (j >> 1) & 1, a.err, ERR_WAIT_MMA);
+      const bool s_ok = !*abort_flag && mbar_wait(s_full(g), j & 1, a.err, ERR_WAIT_MMA);
       if (!__all_sync(0xFFFFFFFFu, s_ok)) { ok = false; break; }
       tc_fence_after();
       uint32_t sr[BKV];
 #pragma unroll
       for (int c = 0; c < BKV / 32; ++c)
-        tmem_ld32(tmem + t_lane + sb * BKV + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
+        tmem_ld32(tmem + t_lane + s_col + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
       tmem_ld_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(s_empty(sb));
 
       const int nvalid = min(BKV, L - j * BKV);
-      float mx = -INFINITY;
-      if (nvalid == BKV) {
-#pragma unroll
-        for (int i = 0; i < BKV; ++i) mx = fmaxf(mx, __uint_as_float(sr[i]));
-      } else {
+      if (nvalid < BKV) {  // uniform: only the last, partial key tile
 #pragma unroll
         for (int i = 0; i < BKV; ++i)
-          if (i < nvalid) mx = fmaxf(mx, __uint_as_float(sr[i]));
+          if (i >= nvalid) sr[i] = __float_as_uint(-INFINITY);
       }
+      // row max with 8 independent partial maxima
+      float pm[8];
+#pragma unroll
+      for (int t = 0; t < 8; ++t) pm[t] = __uint_as_float(sr[t]);
+#pragma unroll
+      for (int i = 8; i < BKV; i += 16)
+#pragma unroll
+        for (int t = 0; t < 8; ++t) pm[t] = max3f(pm[t], __uint_as_float(sr[i + t]), __uint_as_float(sr[i + 8 + t]));
+      const float mx = fmaxf(max3f(pm[0], pm[1], pm[2]), max3f(max3f(pm[3], pm[4], pm[5]), pm[6], pm[7]));
       const float mxs = mx * scale_log2;
       float alpha = 1.0f;
       bool rescale = false;
@@ -243,75 +270,71 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         m_run = mxs;
         rescale = true;
       }
-      float rowsum = 0.0f;
+      // p = exp2(s * c - m), packed to bf16 pairs in place; sum with 4 packed accumulators
+      const float2 nm2 = make_float2(-m_run, -m_run);
+      float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
       for (int i = 0; i < BKV; i += 2) {
-        float p0 = fast_exp2(fmaf(__uint_as_float(sr[i]), scale_log2, -m_run));
-        float p1 = fast_exp2(fmaf(__uint_as_float(sr[i + 1]), scale_log2, -m_run));
-        if (nvalid < BKV) {
-          if (i >= nvalid) p0 = 0.0f;
-          if (i + 1 >= nvalid) p1 = 0.0f;
-        }
-        const uint32_t pk = pack_bf16x2(p0, p1);
-        rowsum += bf16_lo(pk) + bf16_hi(pk);
-        sr[i >> 1] = pk;  // packed P overwrites the consumed scores
+        const float2 t = __ffma2_rn(make_float2(__uint_as_float(sr[i]), __uint_as_float(sr[i + 1])), c2, nm2);
+        const float2 p = make_float2(fast_exp2(t.x), fast_exp2(t.y));
+        acc[(i >> 1) & 3] = __fadd2_rn(acc[(i >> 1) & 3], p);
+        sr[i >> 1] = pack_bf16x2(p.x, p.y);
       }
-      l_run = fmaf(l_run, alpha, rowsum);
+      const float2 a01 = __fadd2_rn(acc[0], acc[1]), a23 = __fadd2_rn(acc[2], acc[3]);
+      const float2 a03 = __fadd2_rn(a01, a23);
+      l_run = fmaf(l_run, alpha, a03.x + a03.y);
 
-      const bool pv_ok = (j == 0) || mbar_wait(pv_done, (j - 1) & 1, a.err, ERR_WAIT_MMA);
-      if (!__all_sync(0xFFFFFFFFu, pv_ok)) { ok = false; break; }
-      // The whole warp rescales its rows of O if any row's max moved; rows that
-      // kept their max use alpha = 1.
+      // S_g(j) complete => PV_g(j-1) complete: O_g is stable until P_g(j) is published.
       if (__any_sync(0xFFFFFFFFu, rescale)) {
-        tc_fence_after();
 #pragma unroll
         for (int c = 0; c < DH / 32; ++c) {
           uint32_t o[32];
-          tmem_ld32(tmem + t_lane + O_COL + c * 32, o);
+          tmem_ld32(tmem + t_lane + o_col + c * 32, o);
           tmem_ld_wait();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-          tmem_st32(tmem + t_lane + O_COL + c * 32, o);
+          for (int e = 0; e < 32; e += 2) {
+            const float2 v = __fmul2_rn(make_float2(__uint_as_float(o[e]), __uint_as_float(o[e + 1])),
+                                        make_float2(alpha, alpha));
+            o[e] = __float_as_uint(v.x);
+            o[e + 1] = __float_as_uint(v.y);
+          }
+          tmem_st32(tmem + t_lane + o_col + c * 32, o);
         }
-        tmem_st_wait();
       }
-      // P row -> shared memory, K-major 128-byte-swizzled operand layout:
-      // keys [64b, 64b+64) of row r live in box b at r*128, 16-byte chunk c at (c ^ (r & 7)).
-#pragma unroll
-      for (int ch = 0; ch < BKV / 8; ++ch) {
-        const int b = ch >> 3, c = ch & 7;
-        uint4* dst = reinterpret_cast<uint4*>(P + b * BOX + row * 128 + ((c ^ (row & 7)) << 4));
-        *dst = make_uint4(sr[4 * ch], sr[4 * ch + 1], sr[4 * ch + 2], sr[4 * ch + 3]);
-      }
-      fence_proxy_async_smem();
+      // P_g(j) over the first 64 columns of S_g: column c holds keys 2c (low half) and 2c+1.
+      tmem_st32(tmem + t_lane + s_col, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+      tmem_st32(tmem + t_lane + s_col + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+      tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
+      if (lane == 0) mbar_arrive(p_full(g));
     }
-    const bool fin = ok && mbar_wait(pv_done, (nkv - 1) & 1, a.err, ERR_WAIT_MMA);
-    if (__all_sync(0xFFFFFFFFu, fin)) {
+    const bool f_ok = ok && mbar_wait(fin(g), 0, a.err, ERR_WAIT_MMA);
+    if (__all_sync(0xFFFFFFFFu, f_ok)) {
       tc_fence_after();
-      const int q = qt * BQ + row;
+      const int q = qt * 2 * BQ + g * BQ + row;
       const int b = bh / a.n_heads, h = bh - b * a.n_heads;
       const float inv_l = 1.0f / l_run;
+      const float2 il2 = make_float2(inv_l, inv_l);
       float amax = 0.0f;
       const int dm = a.n_heads * DH;
       __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.o) + ((size_t)b * L + q) * dm + h * DH;
 #pragma unroll
       for (int c = 0; c < DH / 32; ++c) {
         uint32_t o[32];
-        tmem_ld32(tmem + t_lane + O_COL + c * 32, o);
+        tmem_ld32(tmem + t_lane + o_col + c * 32, o);
         tmem_ld_wait();
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          pk[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
-          amax = fmaxf(amax, fmaxf(fabsf(bf16_lo(pk[e])), fabsf(bf16_hi(pk[e]))));
+          const float2 v = __fmul2_rn(make_float2(__uint_as_float(o[2 * e]), __uint_as_float(o[2 * e + 1])), il2);
+          pk[e] = pack_bf16x2(v.x, v.y);
+          amax = max3f(amax, fabsf(bf16_lo(pk[e])), fabsf(bf16_hi(pk[e])));
         }
         if (q < L) {
           uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
 #pragma unroll
-          for (int g = 0; g < 4; ++g) d4[g] = make_uint4(pk[4 * g], pk[4 * g + 1], pk[4 * g + 2], pk[4 * g + 3]);
+          for (int gg = 0; gg < 4; ++gg) d4[gg] = make_uint4(pk[4 * gg], pk[4 * gg + 1], pk[4 * gg + 2], pk[4 * gg + 3]);
         }
       }
       if (q < L) atomicMax(reinterpret_cast<unsigned*>(a.absmax) + (size_t)b * L + q, __float_as_uint(amax));
@@ -337,7 +360,7 @@ static cudaError_t launch_attn(const AttnArgs& a, cudaStream_t st) {
   auto k = attention_kernel<DH>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Lay::SMEM);
   if (e != cudaSuccess) return e;
-  const dim3 grid((a.L + attn::BQ - 1) / attn::BQ, a.B * a.n_heads);
+  const dim3 grid((a.L + 2 * attn::BQ - 1) / (2 * attn::BQ), a.B * a.n_heads);
   const float scale_log2 = 1.4426950408889634f / sqrtf((float)DH);
   k<<<grid, attn::kThreads, Lay::SMEM, st>>>(tm, a, scale_log2);
   return cudaGetLastError();

@@ -15,11 +15,13 @@
 //     section "性能上限" (RoPE folded into the kernel of the projections).
 //
 // Design (B200): persistent kernel, one 128x256 output tile at a time per CTA,
-// tiles rastered in groups of 16 M-blocks for L2 reuse. Warp 0 streams A/B
-// tiles with TMA (128-byte swizzle) into a 4-stage shared-memory ring; warp 1
-// issues tcgen05.mma from one thread into a double-buffered TMEM accumulator
-// (2 x 256 columns); warps 2-5 drain the other accumulator (tcgen05.ld) and
-// run the epilogue while the next tile's MMAs proceed. Every wait is bounded.
+// tiles rastered in L2-sized groups (a band of A stripes or of W slices stays
+// resident). Warp 0 streams A/B tiles with TMA (128-byte swizzle) into a
+// 4-stage shared-memory ring; warp 1 issues tcgen05.mma from one thread into a
+// double-buffered TMEM accumulator (2 x 256 columns); warps 2-9 (two per
+// sub-partition, each half of the columns) drain the other accumulator
+// (tcgen05.ld) and run the epilogue while the next tile's MMAs proceed. Every
+// wait is bounded.
 #include "h3b_common.cuh"
 #include "h3b_internal.h"
 
@@ -29,27 +31,52 @@ constexpr int BM = 128, BN = 256, BKB = 128, STAGES = 4;
 constexpr int A_BYTES = BM * BKB;
 constexpr int B_BYTES = BN * BKB;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int GROUP_M = 16;
-constexpr int kThreads = 192;
+constexpr int kEpiWarps = 8;  // two per sub-partition, each half of the tile's columns
+constexpr int kThreads = 64 + 32 * kEpiWarps;
+constexpr size_t kL2Budget = 48ull << 20;  // operand bytes the raster keeps resident in L2
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int kBars = 2 * STAGES + 4 + 1;
 constexpr size_t SMEM_BYTES = (size_t)STAGES * STAGE_BYTES + 1024 + kBars * 8 + 16;
 }  // namespace gemm
 
-__device__ __forceinline__ void tile_coords(int t, int n_m, int n_n, int& mb, int& nb) {
-  const int per_group = gemm::GROUP_M * n_n;
-  const int g = t / per_group;
-  const int first = g * gemm::GROUP_M;
-  const int gm = min(gemm::GROUP_M, n_m - first);
-  const int r = t - g * per_group;
-  mb = first + r % gm;
-  nb = r / gm;
+// Tile t -> (M-tile, N-tile). Tiles are rastered in groups: `group` M-tiles
+// with the M index fastest (their A stripes stay in L2 while W streams), or
+// `group` N-tiles with the N index fastest (their W slices stay resident
+// while A streams).
+__device__ __forceinline__ void tile_coords(int t, int n_m, int n_n, int raster_n, int group, int& mb,
+                                            int& nb) {
+  if (!raster_n) {
+    const int per_group = group * n_n;
+    const int g = t / per_group;
+    const int first = g * group;
+    const int gm = min(group, n_m - first);
+    const int r = t - g * per_group;
+    mb = first + r % gm;
+    nb = r / gm;
+  } else {
+    const int per_group = group * n_m;
+    const int g = t / per_group;
+    const int first = g * group;
+    const int gn = min(group, n_n - first);
+    const int r = t - g * per_group;
+    nb = first + r % gn;
+    mb = r / gn;
+  }
 }
 
-__device__ __forceinline__ float gelu_tanh_f(float x) {
-  // 0.5 x (1 + tanh(u)) == x / (1 + exp(-2u)),  u = sqrt(2/pi) (x + 0.044715 x^3)
-  const float u = 0.7978845608028654f * fmaf(0.044715f * x, x * x, x);
-  return x / (1.0f + __expf(-2.0f * u));
+// GELU, tanh form: 0.5 x (1 + tanh(u)) = x / (1 + exp(-2u)) with
+// u = sqrt(2/pi) (x + 0.044715 x^3), i.e. x / (1 + 2^(x (k1 + k2 x^2))) with
+// k1 = -2 sqrt(2/pi) log2(e), k2 = 0.044715 k1. For very negative x the power
+// overflows and the fast reciprocal returns the limit 0.
+constexpr float kGeluK1 = -2.0f * 0.7978845608028654f * 1.4426950408889634f;
+constexpr float kGeluK2 = 0.044715f * kGeluK1;
+__device__ __forceinline__ float2 gelu_tanh2(float2 x) {
+  const float2 x2 = __fmul2_rn(x, x);
+  const float2 t = __fmul2_rn(x, __ffma2_rn(x2, make_float2(kGeluK2, kGeluK2), make_float2(kGeluK1, kGeluK1)));
+  float e0, e1;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e0) : "f"(t.x));
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e1) : "f"(t.y));
+  return make_float2(__fdividef(x.x, 1.0f + e0), __fdividef(x.y, 1.0f + e1));
 }
 
 __device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const float (&v)[32], int valid) {
@@ -65,7 +92,7 @@ __device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const float (&
 // Epilogue of one 128x256 tile for the thread owning TMEM lane = tile row.
 template <bool kInt8, int kEpi>
 __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, uint32_t tbase, int row, bool row_ok,
-                                              int n0) {
+                                              int n0, int c_begin, int c_end) {
   float sa = 1.0f;
   if (kInt8 && kEpi != EPI_S32 && row_ok) sa = __ldg(p.sA + row);
   int item = 0, l = 0, pt = 0, ph = 0, pw = 0;
@@ -80,7 +107,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, uint32_t tbase,
   }
   float amax = 0.0f;
 #pragma unroll 1
-  for (int c = 0; c < gemm::BN / 32; ++c) {
+  for (int c = c_begin; c < c_end; ++c) {
     const int col0 = n0 + c * 32;
     if (col0 >= p.N) break;  // uniform across the warp
     uint32_t r[32];
@@ -98,13 +125,15 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, uint32_t tbase,
     float v[32];
     if (kInt8) {
       const float4* sw4 = reinterpret_cast<const float4*>(p.sW + col0);
+      const float2 sa2 = make_float2(sa, sa);
 #pragma unroll
       for (int g = 0; g < 8; ++g) {
         const float4 s = (4 * g < valid) ? __ldg(sw4 + g) : make_float4(0.f, 0.f, 0.f, 0.f);
-        v[4 * g + 0] = (float)(int)r[4 * g + 0] * sa * s.x;
-        v[4 * g + 1] = (float)(int)r[4 * g + 1] * sa * s.y;
-        v[4 * g + 2] = (float)(int)r[4 * g + 2] * sa * s.z;
-        v[4 * g + 3] = (float)(int)r[4 * g + 3] * sa * s.w;
+        const float2 lo = __fmul2_rn(__fmul2_rn(make_float2((float)(int)r[4 * g], (float)(int)r[4 * g + 1]), sa2),
+                                     make_float2(s.x, s.y));
+        const float2 hi = __fmul2_rn(__fmul2_rn(make_float2((float)(int)r[4 * g + 2], (float)(int)r[4 * g + 3]), sa2),
+                                     make_float2(s.z, s.w));
+        v[4 * g + 0] = lo.x; v[4 * g + 1] = lo.y; v[4 * g + 2] = hi.x; v[4 * g + 3] = hi.y;
       }
     } else {
 #pragma unroll
@@ -123,9 +152,11 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, uint32_t tbase,
       store_bf16x32(static_cast<__nv_bfloat16*>(p.out) + (size_t)row * p.N + col0, v, valid);
     } else if (kEpi == EPI_GELU) {
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        v[i] = round_bf16(gelu_tanh_f(v[i]));
-        amax = fmaxf(amax, fabsf(v[i]));
+      for (int i = 0; i < 32; i += 2) {
+        const float2 gv = gelu_tanh2(make_float2(v[i], v[i + 1]));
+        v[i] = round_bf16(gv.x);
+        v[i + 1] = round_bf16(gv.y);
+        amax = fmaxf(amax, fmaxf(fabsf(v[i]), fabsf(v[i + 1])));
       }
       store_bf16x32(static_cast<__nv_bfloat16*>(p.out) + (size_t)row * p.N + col0, v, valid);
     } else if (kEpi == EPI_RESID) {
@@ -201,7 +232,7 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) { mbar_init(full(s), 1); mbar_init(empty(s), 1); }
-    for (int a = 0; a < 2; ++a) { mbar_init(tfull(a), 1); mbar_init(tempty(a), 4); }
+    for (int a = 0; a < 2; ++a) { mbar_init(tfull(a), 1); mbar_init(tempty(a), kEpiWarps); }
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -225,7 +256,7 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
       bool ok = true;
       for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
         int mb, nb;
-        tile_coords(t, n_m, n_n, mb, nb);
+        tile_coords(t, n_m, n_n, p.raster_n, p.group, mb, nb);
         for (int kb = 0; kb < nk; ++kb) {
           if (*abort_flag || !mbar_wait(empty(s), ph ^ 1u, p.err, ERR_WAIT_MMA)) { ok = false; break; }
           mbar_arrive_expect_tx(full(s), STAGE_BYTES);
@@ -288,12 +319,14 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
       }
     }
   } else {
-    // ---------------- epilogue warps 2..5 (TMEM lane quadrant = warp % 4)
+    // ---------------- epilogue warps 2..9: TMEM lane quadrant = warp % 4; warps
+    // 2-5 take columns [0, 128) of the tile, warps 6-9 columns [128, 256)
     const int quad = warp & 3;
+    const int half = (warp - 2) >> 2;
     int tl = 0;
     for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++tl) {
       int mb, nb;
-      tile_coords(t, n_m, n_n, mb, nb);
+      tile_coords(t, n_m, n_n, p.raster_n, p.group, mb, nb);
       const int acc = tl & 1;
       const uint32_t aph = (tl >> 1) & 1;
       // tcgen05.ld is warp-collective: the wait outcome is made warp-uniform.
@@ -302,7 +335,7 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
       tc_fence_after();
       const int row = mb * BM + quad * 32 + lane;
       const uint32_t tbase = tmem_base + ((uint32_t)(quad * 32) << 16) + acc * BN;
-      epilogue_tile<kInt8, kEpi>(p, tbase, row, row < p.M, nb * BN);
+      epilogue_tile<kInt8, kEpi>(p, tbase, row, row < p.M, nb * BN, half * (BN / 64), (half + 1) * (BN / 64));
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(tempty(acc));
@@ -337,20 +370,35 @@ cudaError_t launch_gemm(bool int8_operands, GemmEpilogue epi, const void* A, con
     return cudaErrorInvalidValue;
   if (!make_tmap_2d(&tb, W, eb, (uint64_t)a.K, (uint64_t)a.N, (uint64_t)a.K * eb, bke, BN))
     return cudaErrorInvalidValue;
-  const int n_tiles = ((a.M + BM - 1) / BM) * ((a.N + BN - 1) / BN);
+  const int n_m = (a.M + BM - 1) / BM, n_n = (a.N + BN - 1) / BN;
+  const int n_tiles = n_m * n_n;
   const int grid = n_tiles < sms ? n_tiles : sms;
+  // Raster: keep either a band of A stripes or a band of W slices resident in L2,
+  // whichever makes the other operand's repeated streaming cheaper.
+  GemmArgs args = a;
+  {
+    const double stripe_a = (double)BM * a.K * eb, slice_w = (double)BN * a.K * eb;
+    const double bytes_a = (double)a.M * a.K * eb, bytes_w = (double)a.N * a.K * eb;
+    int gm = (int)(kL2Budget / stripe_a), gn = (int)(kL2Budget / slice_w);
+    gm = gm < 1 ? 1 : (gm > n_m ? n_m : gm);
+    gn = gn < 1 ? 1 : (gn > n_n ? n_n : gn);
+    const double traffic_m = bytes_a + ((n_m + gm - 1) / gm) * bytes_w;
+    const double traffic_n = bytes_w + ((n_n + gn - 1) / gn) * bytes_a;
+    args.raster_n = traffic_n < traffic_m ? 1 : 0;
+    args.group = args.raster_n ? gn : gm;
+  }
   if (int8_operands) {
     switch (epi) {
-      case EPI_S32: return launch_one<true, EPI_S32>(ta, tb, a, grid, st);
-      case EPI_DEQ: return launch_one<true, EPI_DEQ>(ta, tb, a, grid, st);
-      case EPI_QKV: return launch_one<true, EPI_QKV>(ta, tb, a, grid, st);
-      case EPI_RESID: return launch_one<true, EPI_RESID>(ta, tb, a, grid, st);
-      case EPI_GELU: return launch_one<true, EPI_GELU>(ta, tb, a, grid, st);
+      case EPI_S32: return launch_one<true, EPI_S32>(ta, tb, args, grid, st);
+      case EPI_DEQ: return launch_one<true, EPI_DEQ>(ta, tb, args, grid, st);
+      case EPI_QKV: return launch_one<true, EPI_QKV>(ta, tb, args, grid, st);
+      case EPI_RESID: return launch_one<true, EPI_RESID>(ta, tb, args, grid, st);
+      case EPI_GELU: return launch_one<true, EPI_GELU>(ta, tb, args, grid, st);
     }
   } else {
     switch (epi) {
-      case EPI_DEQ: return launch_one<false, EPI_DEQ>(ta, tb, a, grid, st);
-      case EPI_QKV: return launch_one<false, EPI_QKV>(ta, tb, a, grid, st);
+      case EPI_DEQ: return launch_one<false, EPI_DEQ>(ta, tb, args, grid, st);
+      case EPI_QKV: return launch_one<false, EPI_QKV>(ta, tb, args, grid, st);
       default: break;
     }
   }

@@ -40,6 +40,18 @@ __device__ __forceinline__ int quant_code(float v, float scale, float absmax) {
   int c = __float2int_rn(__fdiv_rn(v, scale));
   return max(-127, min(127, c));
 }
+// The same decision without a division per element: t = v * RN(1/scale)
+// differs from RN(v / scale) by less than 2^-15.4 for |t| <= 127.5, so when t
+// is farther than 2^-14 from a half-integer both round to the same integer;
+// only then-near ties take the correctly rounded division. Bit-identical to
+// quant_code for every input (absmax > 0).
+constexpr float kTieGuard = 0.5f - 1.0f / 16384.0f;
+__device__ __forceinline__ int quant_code_fast(float v, float scale, float rcp) {
+  float t = v * rcp;
+  float c = rintf(t);
+  if (fabsf(t - c) > kTieGuard) c = rintf(__fdiv_rn(v, scale));
+  return max(-127, min(127, (int)c));
+}
 __device__ __forceinline__ uint32_t pack4_i8(int a, int b, int c, int d) {
   return (uint32_t)(a & 0xFF) | ((uint32_t)(b & 0xFF) << 8) | ((uint32_t)(c & 0xFF) << 16) |
          ((uint32_t)(d & 0xFF) << 24);
@@ -52,45 +64,43 @@ __device__ __forceinline__ uint32_t pack4_i8(int a, int b, int c, int d) {
 // ---------------------------------------------------------------------------
 constexpr int kGemvMaxB = 8;
 
+// One warp per output row j; the row's d/8 16-byte vectors (NV per lane) are
+// all requested before any is used, so each warp keeps its whole row in flight.
+template <int NV>
 __global__ void __launch_bounds__(256) adaln_gemv_kernel(const __nv_bfloat16* __restrict__ W,
                                                          const float* __restrict__ bias,
-                                                         const float* __restrict__ c, int B, int d,
+                                                         const float* __restrict__ c, int B,
                                                          float* __restrict__ mod) {
+  constexpr int d = NV * 256;
   extern __shared__ float cs[];  // [B][d]
   for (int i = threadIdx.x; i < B * d; i += blockDim.x) cs[i] = c[i];
-  __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int j = blockIdx.x * 8 + warp;
-  if (j >= 6 * d) return;
-  const uint4* wr = reinterpret_cast<const uint4*>(W + (size_t)j * d);
-  const int nvec = d / 8;
+  const bool valid = j < 6 * d;
+  const uint4* wr = reinterpret_cast<const uint4*>(W + (size_t)(valid ? j : 0) * d);
+  uint4 w4[NV];
+#pragma unroll
+  for (int i = 0; i < NV; ++i) w4[i] = __ldcs(wr + lane + 32 * i);
+  __syncthreads();
+  if (!valid) return;
   float acc[kGemvMaxB];
 #pragma unroll
   for (int b = 0; b < kGemvMaxB; ++b) acc[b] = 0.0f;
-  for (int v0 = lane; v0 < nvec; v0 += 32 * 4) {
-    uint4 w4[4];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int v = v0 + 32 * u;
-      if (v < nvec) w4[u] = __ldcs(wr + v);
-    }
+  for (int i = 0; i < NV; ++i) {
+    const uint32_t ww[4] = {w4[i].x, w4[i].y, w4[i].z, w4[i].w};
+    const int v = lane + 32 * i;
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int v = v0 + 32 * u;
-      if (v >= nvec) break;
-      const uint32_t ww[4] = {w4[u].x, w4[u].y, w4[u].z, w4[u].w};
-#pragma unroll
-      for (int b = 0; b < kGemvMaxB; ++b) {
-        if (b >= B) break;
-        const float* cb = cs + b * d + v * 8;
-        float a = acc[b];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          a = fmaf(bf16_lo(ww[e]), cb[2 * e], a);
-          a = fmaf(bf16_hi(ww[e]), cb[2 * e + 1], a);
-        }
-        acc[b] = a;
-      }
+    for (int b = 0; b < kGemvMaxB; ++b) {
+      if (b >= B) break;
+      const float4 c0 = *reinterpret_cast<const float4*>(cs + b * d + v * 8);
+      const float4 c1 = *reinterpret_cast<const float4*>(cs + b * d + v * 8 + 4);
+      float a = acc[b];
+      a = fmaf(bf16_lo(ww[0]), c0.x, a); a = fmaf(bf16_hi(ww[0]), c0.y, a);
+      a = fmaf(bf16_lo(ww[1]), c0.z, a); a = fmaf(bf16_hi(ww[1]), c0.w, a);
+      a = fmaf(bf16_lo(ww[2]), c1.x, a); a = fmaf(bf16_hi(ww[2]), c1.y, a);
+      a = fmaf(bf16_lo(ww[3]), c1.z, a); a = fmaf(bf16_hi(ww[3]), c1.w, a);
+      acc[b] = a;
     }
   }
 #pragma unroll
@@ -102,91 +112,136 @@ __global__ void __launch_bounds__(256) adaln_gemv_kernel(const __nv_bfloat16* __
 }
 
 // ---------------------------------------------------------------------------
-// Fused LayerNorm + modulation + per-row int8 quantization. One warp per row;
-// the row stays in registers (NV 16-byte vectors per lane, d = 256*NV).
+// Fused LayerNorm + modulation + per-row int8 quantization. A row of
+// d = 8 * VPT * G channels is held in registers by a group of G threads
+// (VPT 16-byte vectors each); a 256-thread block serves 256 / G rows.
 //   y = (x - mean) * rsqrt(var + eps)          (fp32, two-pass variance)
 //   h = bf16(y * (1 + scale) + shift)
 //   s = absmax(h) / 127, q = rint(h / s)       (binary32 decision)
 // ---------------------------------------------------------------------------
-template <int NV>
-__global__ void __launch_bounds__(256, (NV <= 4 ? 4 : (NV <= 12 ? 2 : 1))) ln_mod_quant_kernel(
+template <int G>
+__device__ __forceinline__ float group_sum(float v, float* red) {
+  v = warp_sum(v);
+  if (G == 32) return v;
+  constexpr int NW = G / 32;
+  const int warp = threadIdx.x >> 5;
+  if ((threadIdx.x & 31) == 0) red[warp] = v;
+  __syncthreads();
+  const int first = (warp / NW) * NW;
+  float t = 0.0f;
+#pragma unroll
+  for (int i = 0; i < NW; ++i) t += red[first + i];
+  __syncthreads();
+  return t;
+}
+template <int G>
+__device__ __forceinline__ float group_max(float v, float* red) {
+  v = warp_max(v);
+  if (G == 32) return v;
+  constexpr int NW = G / 32;
+  const int warp = threadIdx.x >> 5;
+  if ((threadIdx.x & 31) == 0) red[warp] = v;
+  __syncthreads();
+  const int first = (warp / NW) * NW;
+  float t = 0.0f;
+#pragma unroll
+  for (int i = 0; i < NW; ++i) t = fmaxf(t, red[first + i]);
+  __syncthreads();
+  return t;
+}
+
+__device__ __forceinline__ float2 bf16x2_to_f2(uint32_t u) { return make_float2(bf16_lo(u), bf16_hi(u)); }
+
+template <int VPT, int G>
+__global__ void __launch_bounds__(256) ln_mod_quant_kernel(
     const __nv_bfloat16* __restrict__ x, int rows, float eps, const float* __restrict__ shift,
     const float* __restrict__ scale, int rows_per_item, int mod_stride, int8_t* __restrict__ q,
     float* __restrict__ s, __nv_bfloat16* __restrict__ h_out, float* __restrict__ absmax_zero,
     int write_codes) {
-  constexpr int d = NV * 256;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int row = blockIdx.x * 8 + warp;
-  if (row >= rows) return;
-  const uint4* xr = reinterpret_cast<const uint4*>(x + (size_t)row * d);
-  uint4 v[NV];
+  constexpr int RPB = 256 / G;
+  constexpr int d = VPT * G * 8;
+  __shared__ float red[8];
+  const int gt = threadIdx.x % G;
+  const int row = blockIdx.x * RPB + threadIdx.x / G;
+  const bool valid = row < rows;
+  const uint4* xr = reinterpret_cast<const uint4*>(x + (size_t)(valid ? row : 0) * d);
+  uint4 v[VPT];
 #pragma unroll
-  for (int i = 0; i < NV; ++i) v[i] = __ldcs(xr + lane + 32 * i);
+  for (int i = 0; i < VPT; ++i) v[i] = valid ? __ldcs(xr + gt + G * i) : make_uint4(0, 0, 0, 0);
 
-  float sum = 0.0f;
+  float2 acc = make_float2(0.0f, 0.0f);
 #pragma unroll
-  for (int i = 0; i < NV; ++i) {
-    const uint32_t u[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
-#pragma unroll
-    for (int e = 0; e < 4; ++e) sum += bf16_lo(u[e]) + bf16_hi(u[e]);
+  for (int i = 0; i < VPT; ++i) {
+    acc = __fadd2_rn(acc, bf16x2_to_f2(v[i].x));
+    acc = __fadd2_rn(acc, bf16x2_to_f2(v[i].y));
+    acc = __fadd2_rn(acc, bf16x2_to_f2(v[i].z));
+    acc = __fadd2_rn(acc, bf16x2_to_f2(v[i].w));
   }
-  const float mean = warp_sum(sum) * (1.0f / d);
-  float sq = 0.0f;
+  const float mean = group_sum<G>(acc.x + acc.y, red) * (1.0f / d);
+  const float2 nmean = make_float2(-mean, -mean);
+  acc = make_float2(0.0f, 0.0f);
 #pragma unroll
-  for (int i = 0; i < NV; ++i) {
+  for (int i = 0; i < VPT; ++i) {
     const uint32_t u[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      const float a = bf16_lo(u[e]) - mean, b = bf16_hi(u[e]) - mean;
-      sq = fmaf(a, a, sq);
-      sq = fmaf(b, b, sq);
+      const float2 c = __fadd2_rn(bf16x2_to_f2(u[e]), nmean);
+      acc = __ffma2_rn(c, c, acc);
     }
   }
-  const float rstd = 1.0f / sqrtf(warp_sum(sq) * (1.0f / d) + eps);
+  const float rstd = 1.0f / sqrtf(group_sum<G>(acc.x + acc.y, red) * (1.0f / d) + eps);
+  const float2 rstd2 = make_float2(rstd, rstd);
 
-  const int item = row / rows_per_item;
-  const float4* sh4 = reinterpret_cast<const float4*>(shift + (size_t)item * mod_stride);
-  const float4* sc4 = reinterpret_cast<const float4*>(scale + (size_t)item * mod_stride);
+  const int item = (valid ? row : 0) / rows_per_item;
+  const float2* sh2 = reinterpret_cast<const float2*>(shift + (size_t)item * mod_stride);
+  const float2* sc2 = reinterpret_cast<const float2*>(scale + (size_t)item * mod_stride);
   float amax = 0.0f;
 #pragma unroll
-  for (int i = 0; i < NV; ++i) {
-    const int vec = lane + 32 * i;
-    const float4 sa = __ldg(sh4 + 2 * vec), sb = __ldg(sh4 + 2 * vec + 1);
-    const float4 ca = __ldg(sc4 + 2 * vec), cb = __ldg(sc4 + 2 * vec + 1);
-    const float shv[8] = {sa.x, sa.y, sa.z, sa.w, sb.x, sb.y, sb.z, sb.w};
-    const float scv[8] = {ca.x, ca.y, ca.z, ca.w, cb.x, cb.y, cb.z, cb.w};
+  for (int i = 0; i < VPT; ++i) {
+    const int c0 = (gt + G * i) * 4;  // float2 index of the vector's first channel pair
     uint32_t u[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      const float h0 = round_bf16(fmaf((bf16_lo(u[e]) - mean) * rstd, 1.0f + scv[2 * e], shv[2 * e]));
-      const float h1 =
-          round_bf16(fmaf((bf16_hi(u[e]) - mean) * rstd, 1.0f + scv[2 * e + 1], shv[2 * e + 1]));
-      amax = fmaxf(amax, fmaxf(fabsf(h0), fabsf(h1)));
-      u[e] = pack_bf16x2(h0, h1);
+      const float2 sh = __ldg(sh2 + c0 + e);
+      const float2 sc = __ldg(sc2 + c0 + e);
+      const float2 y = __fmul2_rn(__fadd2_rn(bf16x2_to_f2(u[e]), nmean), rstd2);
+      const float2 h = __ffma2_rn(y, make_float2(1.0f + sc.x, 1.0f + sc.y), sh);
+      u[e] = pack_bf16x2(h.x, h.y);
+      amax = fmaxf(amax, fmaxf(fabsf(bf16_lo(u[e])), fabsf(bf16_hi(u[e]))));
     }
     v[i] = make_uint4(u[0], u[1], u[2], u[3]);
   }
-  amax = warp_max(amax);
+  amax = group_max<G>(amax, red);
+  if (!valid) return;
   if (h_out) {
     uint4* hr = reinterpret_cast<uint4*>(h_out + (size_t)row * d);
 #pragma unroll
-    for (int i = 0; i < NV; ++i) hr[lane + 32 * i] = v[i];
+    for (int i = 0; i < VPT; ++i) hr[gt + G * i] = v[i];
   }
-  if (absmax_zero && lane == 0) absmax_zero[row] = 0.0f;
+  if (absmax_zero && gt == 0) absmax_zero[row] = 0.0f;
   if (!write_codes) return;
   const float sc = __fdiv_rn(amax, 127.0f);
-  if (lane == 0) s[row] = sc;
+  const float rcp = __frcp_rn(sc);
+  if (gt == 0) s[row] = sc;
   uint2* qr = reinterpret_cast<uint2*>(q + (size_t)row * d);
 #pragma unroll
-  for (int i = 0; i < NV; ++i) {
+  for (int i = 0; i < VPT; ++i) {
     const uint32_t u[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
     int c[8];
+    if (!(rcp < INFINITY)) {  // absmax == 0 (codes 0) or a subnormal scale: exact division
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      c[2 * e] = quant_code(bf16_lo(u[e]), sc, amax);
-      c[2 * e + 1] = quant_code(bf16_hi(u[e]), sc, amax);
+      for (int e = 0; e < 4; ++e) {
+        c[2 * e] = quant_code(bf16_lo(u[e]), sc, amax);
+        c[2 * e + 1] = quant_code(bf16_hi(u[e]), sc, amax);
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        c[2 * e] = quant_code_fast(bf16_lo(u[e]), sc, rcp);
+        c[2 * e + 1] = quant_code_fast(bf16_hi(u[e]), sc, rcp);
+      }
     }
-    qr[lane + 32 * i] = make_uint2(pack4_i8(c[0], c[1], c[2], c[3]), pack4_i8(c[4], c[5], c[6], c[7]));
+    qr[gt + G * i] = make_uint2(pack4_i8(c[0], c[1], c[2], c[3]), pack4_i8(c[4], c[5], c[6], c[7]));
   }
 }
 
@@ -242,15 +297,27 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(const T* __restrict__ i
     amax = m;
   }
   const float sc = __fdiv_rn(amax, 127.0f);
+  const float rcp = __frcp_rn(sc);
   if (threadIdx.x == 0) s[row] = sc;
   uint2* qr = reinterpret_cast<uint2*>(q + (size_t)row * cols);
-  for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
-    float f[8];
-    load8<T>(r + v * 8, f);
-    int c[8];
+  constexpr int U = 4;  // vectors in flight per thread
+  for (int v0 = threadIdx.x; v0 < nvec; v0 += U * blockDim.x) {
+    float f[U][8];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) c[e] = quant_code(f[e], sc, amax);
-    qr[v] = make_uint2(pack4_i8(c[0], c[1], c[2], c[3]), pack4_i8(c[4], c[5], c[6], c[7]));
+    for (int u = 0; u < U; ++u) {
+      const int v = v0 + u * blockDim.x;
+      if (v < nvec) load8<T>(r + v * 8, f[u]);
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int v = v0 + u * blockDim.x;
+      if (v >= nvec) break;
+      int c[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e)
+        c[e] = (rcp < INFINITY) ? quant_code_fast(f[u][e], sc, rcp) : quant_code(f[u][e], sc, amax);
+      qr[v] = make_uint2(pack4_i8(c[0], c[1], c[2], c[3]), pack4_i8(c[4], c[5], c[6], c[7]));
+    }
   }
 }
 
@@ -331,49 +398,81 @@ __global__ void rope_table_kernel(float2* __restrict__ tab, int T, int H, int W,
 // ---------------------------------------------------------------------------
 // Launchers
 // ---------------------------------------------------------------------------
-cudaError_t launch_adaln_gemv(const void* W, const float* bias, const float* c, int B, int d,
-                              float* mod, cudaStream_t st) {
-  if (B > kGemvMaxB) return cudaErrorInvalidValue;
+template <int NV>
+static cudaError_t gemv_dispatch(const void* W, const float* bias, const float* c, int B, float* mod,
+                                 cudaStream_t st) {
+  constexpr int d = NV * 256;
   const size_t smem = (size_t)B * d * sizeof(float);
   if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(adaln_gemv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(adaln_gemv_kernel<NV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
   }
-  adaln_gemv_kernel<<<(6 * d + 7) / 8, 256, smem, st>>>(static_cast<const __nv_bfloat16*>(W), bias, c,
-                                                        B, d, mod);
+  adaln_gemv_kernel<NV><<<(6 * d + 7) / 8, 256, smem, st>>>(static_cast<const __nv_bfloat16*>(W), bias, c, B,
+                                                            mod);
   return cudaGetLastError();
 }
 
-template <int NV>
+cudaError_t launch_adaln_gemv(const void* W, const float* bias, const float* c, int B, int d,
+                              float* mod, cudaStream_t st) {
+  if (B > kGemvMaxB || d % 256 != 0) return cudaErrorInvalidValue;
+#define H3B_GV(nv) \
+  case nv:         \
+    return gemv_dispatch<nv>(W, bias, c, B, mod, st);
+  switch (d / 256) {
+    H3B_GV(1) H3B_GV(2) H3B_GV(3) H3B_GV(4) H3B_GV(5) H3B_GV(6) H3B_GV(7) H3B_GV(8)
+    H3B_GV(9) H3B_GV(10) H3B_GV(11) H3B_GV(12) H3B_GV(13) H3B_GV(14) H3B_GV(15) H3B_GV(16)
+    H3B_GV(17) H3B_GV(18) H3B_GV(19) H3B_GV(20) H3B_GV(21) H3B_GV(22) H3B_GV(23) H3B_GV(24)
+    H3B_GV(25) H3B_GV(26) H3B_GV(27) H3B_GV(28) H3B_GV(29) H3B_GV(30) H3B_GV(31) H3B_GV(32)
+    default:
+      return cudaErrorInvalidValue;
+  }
+#undef H3B_GV
+}
+
+template <int VPT, int G>
 static cudaError_t ln_dispatch(const void* x, int rows, float eps, const float* shift,
                                const float* scale, int rpi, int ms, int8_t* q, float* s, void* h,
                                float* az, int wc, cudaStream_t st) {
-  ln_mod_quant_kernel<NV><<<(rows + 7) / 8, 256, 0, st>>>(
+  constexpr int RPB = 256 / G;
+  ln_mod_quant_kernel<VPT, G><<<(rows + RPB - 1) / RPB, 256, 0, st>>>(
       static_cast<const __nv_bfloat16*>(x), rows, eps, shift, scale, rpi, ms, q, s,
       static_cast<__nv_bfloat16*>(h), az, wc);
   return cudaGetLastError();
 }
 
+// d = 256 k: a row is split over G = 128 (k % 4 == 0), 64 (k % 2 == 0) or 32
+// threads holding VPT = 32 k / G vectors of 8 channels each.
 cudaError_t launch_ln_mod_quant(const void* x, int rows, int d, float eps, const float* shift,
                                 const float* scale, int rows_per_item, int mod_stride, int8_t* q,
                                 float* s, void* h_out, float* absmax_zero, int write_codes,
                                 cudaStream_t st) {
   if (rows == 0) return cudaSuccess;
-#define H3B_LN_CASE(nv) \
-  case nv:              \
-    return ln_dispatch<nv>(x, rows, eps, shift, scale, rows_per_item, mod_stride, q, s, h_out, absmax_zero, write_codes, st);
-  switch (d / 256) {
-    H3B_LN_CASE(1) H3B_LN_CASE(2) H3B_LN_CASE(3) H3B_LN_CASE(4) H3B_LN_CASE(5) H3B_LN_CASE(6)
-    H3B_LN_CASE(7) H3B_LN_CASE(8) H3B_LN_CASE(9) H3B_LN_CASE(10) H3B_LN_CASE(11) H3B_LN_CASE(12)
-    H3B_LN_CASE(13) H3B_LN_CASE(14) H3B_LN_CASE(15) H3B_LN_CASE(16) H3B_LN_CASE(17) H3B_LN_CASE(18)
-    H3B_LN_CASE(19) H3B_LN_CASE(20) H3B_LN_CASE(21) H3B_LN_CASE(22) H3B_LN_CASE(23) H3B_LN_CASE(24)
-    H3B_LN_CASE(25) H3B_LN_CASE(26) H3B_LN_CASE(27) H3B_LN_CASE(28) H3B_LN_CASE(29) H3B_LN_CASE(30)
-    H3B_LN_CASE(31) H3B_LN_CASE(32)
-    default:
-      return cudaErrorInvalidValue;
+  const int k = d / 256;
+#define H3B_LN(vpt, g) \
+  return ln_dispatch<vpt, g>(x, rows, eps, shift, scale, rows_per_item, mod_stride, q, s, h_out, absmax_zero, write_codes, st)
+  if (k % 4 == 0) {
+    switch (k / 4) {
+      case 1: H3B_LN(1, 128); case 2: H3B_LN(2, 128); case 3: H3B_LN(3, 128); case 4: H3B_LN(4, 128);
+      case 5: H3B_LN(5, 128); case 6: H3B_LN(6, 128); case 7: H3B_LN(7, 128); case 8: H3B_LN(8, 128);
+      default: return cudaErrorInvalidValue;
+    }
+  } else if (k % 2 == 0) {
+    switch (k / 2) {
+      case 1: H3B_LN(1, 64); case 3: H3B_LN(3, 64); case 5: H3B_LN(5, 64); case 7: H3B_LN(7, 64);
+      case 9: H3B_LN(9, 64); case 11: H3B_LN(11, 64); case 13: H3B_LN(13, 64); case 15: H3B_LN(15, 64);
+      default: return cudaErrorInvalidValue;
+    }
+  } else {
+    switch (k) {
+      case 1: H3B_LN(1, 32); case 3: H3B_LN(3, 32); case 5: H3B_LN(5, 32); case 7: H3B_LN(7, 32);
+      case 9: H3B_LN(9, 32); case 11: H3B_LN(11, 32); case 13: H3B_LN(13, 32); case 15: H3B_LN(15, 32);
+      case 17: H3B_LN(17, 32); case 19: H3B_LN(19, 32); case 21: H3B_LN(21, 32); case 23: H3B_LN(23, 32);
+      case 25: H3B_LN(25, 32); case 27: H3B_LN(27, 32); case 29: H3B_LN(29, 32); case 31: H3B_LN(31, 32);
+      default: return cudaErrorInvalidValue;
+    }
   }
-#undef H3B_LN_CASE
+#undef H3B_LN
 }
 
 cudaError_t launch_quant_rows_bf16(const void* h, int rows, int cols, const float* absmax,
