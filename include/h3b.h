@@ -130,6 +130,29 @@ H3B_API h3b_status h3b_workspace_size(const h3b_dims* dims, size_t* bytes);
 H3B_API h3b_status h3b_block_forward(const h3b_dims* dims, const h3b_block_weights* w, const float* c,
                              void* x, void* ws, size_t ws_bytes, h3b_stream stream);
 
+/* Allocation-free block forward (the pages have no counterpart; this exists
+ * for callers of this library). Same computation and results as
+ * h3b_block_forward, but the scratch lives in a fixed 32 MiB device array
+ * inside this library, so the call needs no workspace and allocates nothing
+ * (no cudaMalloc/cudaFree or allocating library routine). It is meant for
+ * callers that cannot allocate device memory when they run the block: code
+ * whose device allocator belongs to a host framework that forbids side
+ * allocations, plugin or callback code that only receives input and output
+ * pointers, or latency-critical loops where an allocation could block.
+ *   - Dimensions whose h3b_workspace_size exceeds 32 MiB are rejected with
+ *     H3B_ERR_WORKSPACE before any launch (use h3b_block_forward instead).
+ *   - Every GPU that loads this library holds the 32 MiB array until the
+ *     process exits.
+ *   - The first call on a device looks up the array's device address on that
+ *     device (cudaGetSymbolAddress); make that first call before any stream
+ *     capture.
+ *   - All calls on a device share the array: calls that overlap on the GPU
+ *     (different streams or host threads) race on it; serialize them.
+ *   - Nothing in the array needs to start at zero; the block's kernels zero
+ *     the region that accumulates on every call. */
+H3B_API h3b_status h3b_block_forward_noalloc(const h3b_dims* dims, const h3b_block_weights* w,
+                                             const float* c, void* x, h3b_stream stream);
+
 /* n_blocks blocks in sequence on one residual stream x; block i uses w[i]
  * (HOST array of n_blocks weight structs holding device pointers) and
  * c + i*B*d (device, fp32 [n_blocks][B][d]). Same workspace as one block. */

@@ -285,6 +285,8 @@ h3b_status run_block(const h3b_dims& d, const h3b_block_weights& w, const float*
 // ---------------------------------------------------------------------------
 // TMA descriptors (driver entry point fetched through the runtime).
 // ---------------------------------------------------------------------------
+void set_error_detail(const std::string& why) { g_detail = why; }
+
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
                                   CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,

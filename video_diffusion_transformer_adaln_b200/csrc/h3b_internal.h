@@ -7,6 +7,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <string>
+
 namespace h3b {
 
 // ---- memory-bound row kernels (k_rowops.cu)
@@ -67,6 +69,9 @@ struct AttnArgs {
   unsigned* err;
 };
 cudaError_t launch_attention(const AttnArgs& a, cudaStream_t st);
+
+// ---- error detail reported by h3b_last_error_detail (h3b_api.cu)
+void set_error_detail(const std::string& why);
 
 // ---- TMA descriptor construction (h3b_api.cu)
 // Row-major 2D tensor of `rows` x `cols` elements of `elem_bytes` each,

@@ -74,6 +74,7 @@ def _declare(L):
     sigs = {
         "h3b_workspace_size": [vp, C.POINTER(sz)],
         "h3b_block_forward": [vp, vp, vp, vp, vp, sz, vp],
+        "h3b_block_forward_noalloc": [vp, vp, vp, vp, vp],
         "h3b_blocks_forward": [vp, vp, i32, vp, vp, vp, sz, vp],
         "h3b_token_pair": [vp, vp, vp, vp, vp],
         "h3b_token_unpair": [vp, vp, vp, vp, vp, vp],
@@ -153,6 +154,13 @@ def h3b_workspace_size(dims: Dims) -> int:
 def h3b_block_forward(dims: Dims, w: BlockWeights, c, x, ws, stream=None):
     _check(lib().h3b_block_forward(C.byref(dims), C.byref(w), _p(c), _p(x), _p(ws), ws.numel() * ws.element_size(),
                                    _s(stream)), "h3b_block_forward")
+
+
+def h3b_block_forward_noalloc(dims: Dims, w: BlockWeights, c, x, stream=None):
+    """Block forward with the library's fixed 32 MiB device scratch (no workspace,
+    no allocation); see include/h3b.h for its limits and sharing rules."""
+    _check(lib().h3b_block_forward_noalloc(C.byref(dims), C.byref(w), _p(c), _p(x), _s(stream)),
+           "h3b_block_forward_noalloc")
 
 
 def h3b_blocks_forward(dims: Dims, ws_list: Sequence[BlockWeights], c, x, ws, stream=None):
