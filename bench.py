@@ -64,10 +64,26 @@ def load_peaks():
 def kernel_work(name, wl):
     """Algorithmic work of one launch: (amount, unit, bound). Tensor-core
     kernels count useful multiply-adds x 2; memory-bound kernels count the
-    bytes they must move (read once + write once)."""
-    B, L, d, F = wl.B, wl.L, wl.d, wl.d_ff
+    bytes they must move (read once + write once). For passes that run some
+    blocks on the paired grid, block kernels average over their launches."""
+    full = wl.B * wl.L * wl.d
+    if name == "token_pair":
+        return 2.0 * full + 2 * 2.0 * full / 2, "byte", "hbm"
+    if name == "token_unpair":
+        return 2.0 * full + 2 * 2.0 * full / 2 + 2.0 * full, "byte", "hbm"
     if wl.token_pair:
-        L = wl.L // 2  # the block runs on the merged grid
+        Ls = [wl.L // 2]
+    elif wl.pair_blocks[0] < wl.pair_blocks[1]:
+        n_m = wl.pair_blocks[1] - wl.pair_blocks[0]
+        Ls = [wl.L // 2] * n_m + [wl.L] * (wl.n_blocks - n_m)
+    else:
+        Ls = [wl.L]
+    works = [_block_kernel_work(name, wl, L) for L in Ls]
+    return sum(w[0] for w in works) / len(works), works[0][1], works[0][2]
+
+
+def _block_kernel_work(name, wl, L):
+    B, d, F = wl.B, wl.d, wl.d_ff
     R = B * L
     if name == "gemm_qkv":
         return 2.0 * R * 3 * d * d, "op", "tensor_i8" if wl.qkv_int8 else "tensor_bf16"
@@ -85,14 +101,8 @@ def kernel_work(name, wl):
         return R * (2.0 * d + d + 8), "byte", "hbm"
     if name == "quant_g":
         return R * (2.0 * F + F + 8), "byte", "hbm"
-    if name == "adaln_gemv":
+    if name == "adaln_gemv":  # (its trailing blocks also fill the small RoPE table)
         return 12.0 * d * d + B * (4.0 * d + 24 * d), "byte", "hbm"
-    if name == "token_pair":
-        full = wl.B * wl.L * wl.d
-        return 2.0 * full + 2 * 2.0 * full / 2, "byte", "hbm"
-    if name == "token_unpair":
-        full = wl.B * wl.L * wl.d
-        return 2.0 * full + 2 * 2.0 * full / 2 + 2.0 * full, "byte", "hbm"
     return 0.0, "byte", "hbm"
 
 
@@ -173,7 +183,7 @@ class Workload:
         self.full = dims_of(wl)
         self.dims = dims_of(wl.merged()) if wl.token_pair else self.full
         self.ws = workspace(self.dims)
-        if wl.token_pair:
+        if wl.token_pair or wl.pair_blocks[0] < wl.pair_blocks[1]:
             shp = (wl.B, wl.T, wl.H, wl.W // 2, wl.d)
             self.xm = torch.empty(shp, dtype=torch.bfloat16, device="cuda")
             self.ym = torch.empty_like(self.xm)
@@ -187,6 +197,9 @@ class Workload:
             h3b.h3b_token_pair(self.full, x, self.xm, self.ym)
             h3b.h3b_block_forward(self.dims, self.blocks[0].struct, c, self.ym, self.ws)
             h3b.h3b_token_unpair(self.full, x, self.xm, self.ym, x)
+        elif wl.n_blocks > 1 and wl.pair_blocks[0] < wl.pair_blocks[1]:
+            h3b.h3b_blocks_forward_reduced(self.full, [b.struct for b in self.blocks], wl.pair_blocks[0],
+                                           wl.pair_blocks[1], c, x, self.xm, self.ym, self.ws)
         elif wl.n_blocks > 1:
             h3b.h3b_blocks_forward(self.dims, [b.struct for b in self.blocks], c, x, self.ws)
         else:
@@ -395,6 +408,8 @@ def run_h3b(args, rank, world, local):
                            "frac": round(work / s / 1e12 / pk, 3)}
 
     gpu_launches = int(sum(n for n, _ in prof.values()))
+    kernel_ms = {k: round(ms / args.steps, 4) for k, (n, ms) in prof.items()}
+    gap_ms = total_ms / args.steps - sum(ms for _, ms in prof.values()) / args.steps
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         orc = OracleRunner(wl)
@@ -409,10 +424,12 @@ def run_h3b(args, rank, world, local):
         "config": {"workload": args.workload, "batch": wl.B, "grid_THW": [wl.T, wl.H, wl.W], "tokens": wl.L,
                    "d": wl.d, "heads": wl.n_heads, "head_dim": wl.head_dim, "d_ff": wl.d_ff,
                    "blocks_per_step": wl.n_blocks, "token_pair": wl.token_pair,
+                   "paired_blocks": list(wl.pair_blocks),
                    "qkv": "int8" if wl.qkv_int8 else "bf16", "attention": "bf16",
                    "l2": "flushed between steps (512 MiB write outside the timed events)",
                    "parallelism": "replicas: one independent latent per GPU, no collective"},
         "roofline": roof, "kernel_share": shares, "kernel_roofline": all_roof,
+        "kernel_ms_per_step": kernel_ms, "launch_gap_ms_per_step": round(gap_ms, 4),
         "cpu_baseline": cpu,
         "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": e2e_steps},

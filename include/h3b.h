@@ -160,6 +160,21 @@ H3B_API h3b_status h3b_blocks_forward(const h3b_dims* dims, const h3b_block_weig
                               const float* c, void* x, void* ws, size_t ws_bytes,
                               h3b_stream stream);
 
+/* Multi-block pass with token reduction over a middle range of blocks
+ * ("Token Reduction" row of the control table: horizontally adjacent video
+ * tokens are paired in the middle blocks). Blocks [0, first) run on the full
+ * grid `full`; then the tokens are paired once (h3b_token_pair into xm and ym),
+ * blocks [first, last) run on the merged grid (W/2, in place on ym), the
+ * block deltas are added back at both positions once (h3b_token_unpair into
+ * x), and blocks [last, n_blocks) run on the full grid again.
+ *   0 <= first <= last <= n_blocks; full->W even when first < last.
+ *   xm, ym: bf16 [B][T][H][W/2][d] device buffers (unused when first == last).
+ *   ws: at least h3b_workspace_size(full) bytes (that covers the merged grid).
+ *   w, c: as for h3b_blocks_forward. */
+H3B_API h3b_status h3b_blocks_forward_reduced(const h3b_dims* full, const h3b_block_weights* w, int n_blocks,
+                                              int first, int last, const float* c, void* x, void* xm, void* ym,
+                                              void* ws, size_t ws_bytes, h3b_stream stream);
+
 /* Token reduction ("Token Reduction" row of the control table): horizontally
  * adjacent tokens w = 2k, 2k+1 of each (t, h) row are merged by their mean.
  *   full: dims of the UNMERGED grid (W even).

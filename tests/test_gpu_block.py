@@ -193,6 +193,45 @@ def test_blocks_forward_three_blocks_d256():
     no_device_error()
 
 
+def test_blocks_forward_reduced_middle_range_d256():
+    """Five blocks; blocks 1..3 run on the merged grid (paired once, unpaired once)."""
+    wl = synth.WORKLOADS["d256_L512"].with_(n_blocks=5)
+    first, last = 1, 4
+    x = synth.x_input(wl)
+    raws = [synth.block_weights(wl, b) for b in range(5)]
+    cs = np.stack([synth.cond(wl, b) for b in range(5)])
+    full, merged = dims_of(wl), dims_of(wl.merged())
+    blocks = [DeviceBlock.from_host(r) for r in raws]
+    xd = bf16_dev(x)
+    shape = (wl.B, wl.T, wl.H, wl.W // 2, wl.d)
+    xm = torch.empty(shape, dtype=torch.bfloat16, device="cuda")
+    ym = torch.empty_like(xm)
+    h3b.h3b_blocks_forward_reduced(full, [b.struct for b in blocks], first, last, to_dev(cs), xd, xm, ym,
+                                   workspace(full))
+    got = bf16_host(xd)
+    # the oracle composes the same pass; between blocks the stream is bf16
+    m = wl.merged()
+    xr = x
+    for b in range(first):
+        xr = O.bf16_round(O.block_forward(oracle_dims(wl), oracle_weights(raws[b]), cs[b], xr)).reshape(x.shape)
+    xmo = O.token_pair(xr, wl.B, wl.T, wl.H, wl.W, wl.d)
+    yr = xmo
+    for b in range(first, last):
+        yr = O.bf16_round(O.block_forward(oracle_dims(m), oracle_weights(raws[b]), cs[b], yr)).reshape(xmo.shape)
+    xr = O.bf16_round(O.token_unpair(xr, xmo, O.bf16_decode(yr), wl.B, wl.T, wl.H, wl.W, wl.d))
+    for b in range(last, 5):
+        out = O.block_forward(oracle_dims(wl), oracle_weights(raws[b]), cs[b], xr)
+        xr = O.bf16_round(out).reshape(x.shape)
+    _compare(got, out, x, n_blocks=5)
+    # with an empty merged range it is the plain multi-block pass, bit for bit
+    xa, xb = bf16_dev(x), bf16_dev(x)
+    h3b.h3b_blocks_forward_reduced(full, [b.struct for b in blocks], 2, 2, to_dev(cs), xa, None, None,
+                                   workspace(full))
+    blocks_forward(full, blocks, to_dev(cs), xb, workspace(full))
+    assert np.array_equal(bf16_host(xa), bf16_host(xb))
+    no_device_error()
+
+
 def test_depth50_pass_properties_d5120_T2():
     """The 50-block pass at d=5120, L=4608: finite, deterministic, equal to 50
     single-block calls; block 0's output matches the oracle on sampled rows."""

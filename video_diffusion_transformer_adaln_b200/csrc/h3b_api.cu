@@ -227,15 +227,14 @@ h3b_status run_block(const h3b_dims& d, const h3b_block_weights& w, const float*
   void* o = r1 + (size_t)3 * R * D * 2;
   void* g = r1;
 
-  // a1: AdaLN modulation vectors
-  H3B_CK(launch_adaln_gemv(w.w_ada, w.b_ada, c, d.B, D, mod, st), "adaln_gemv");
-  if (!rope_ready)
-    H3B_CK(launch_rope_table(rope, d.T, d.H, d.W, d.rope_t, d.rope_h, d.rope_w, d.rope_theta, st), "rope_table");
+  // a1: AdaLN modulation vectors (the same launch fills the RoPE table when needed)
+  H3B_CK(launch_adaln_gemv(w.w_ada, w.b_ada, c, d.B, D, mod, rope_ready ? nullptr : rope, d.T, d.H, d.W,
+                           d.rope_t, d.rope_h, d.rope_w, d.rope_theta, st), "adaln_gemv");
   // a2: LN + modulation + quantization (or the bf16 activation for bf16 QKV)
   if (d.qkv_int8)
-    H3B_CK(launch_ln_mod_quant(x, R, D, d.ln_eps, mod, mod + D, L, 6 * D, act, sA, nullptr, absmax, 1, st), "ln_mod_quant");
+    H3B_CK(launch_ln_mod_quant(x, R, D, d.ln_eps, mod, mod + D, L, 6 * D, act, sA, nullptr, absmax, 1, di.err, di.sms, st), "ln_mod_quant");
   else
-    H3B_CK(launch_ln_mod_quant(x, R, D, d.ln_eps, mod, mod + D, L, 6 * D, nullptr, nullptr, act, absmax, 0, st), "ln_mod");
+    H3B_CK(launch_ln_mod_quant(x, R, D, d.ln_eps, mod, mod + D, L, 6 * D, nullptr, nullptr, act, absmax, 0, di.err, di.sms, st), "ln_mod");
   // a3: QKV projection + 3D RoPE, head-major
   {
     GemmArgs a = base_args(R, 3 * D, D, di.err);
@@ -262,7 +261,7 @@ h3b_status run_block(const h3b_dims& d, const h3b_block_weights& w, const float*
     H3B_CK(launch_gemm(true, EPI_RESID, act, w.wo, a, di.sms, st), "gemm_wo");
   }
   // a7: LN + modulation + quantization for the MLP (chunks 3, 4)
-  H3B_CK(launch_ln_mod_quant(x, R, D, d.ln_eps, mod + 3 * D, mod + 4 * D, L, 6 * D, act, sA, nullptr, absmax, 1, st), "ln_mod_quant_mlp");
+  H3B_CK(launch_ln_mod_quant(x, R, D, d.ln_eps, mod + 3 * D, mod + 4 * D, L, 6 * D, act, sA, nullptr, absmax, 1, di.err, di.sms, st), "ln_mod_quant_mlp");
   // a8: W1 + GELU (+ row absmax), then requantize
   {
     GemmArgs a = base_args(R, F, D, di.err);
@@ -410,6 +409,48 @@ h3b_status h3b_blocks_forward(const h3b_dims* dims, const h3b_block_weights* w, 
   return H3B_OK;
 }
 
+h3b_status h3b_blocks_forward_reduced(const h3b_dims* full, const h3b_block_weights* w, int n_blocks,
+                                      int first, int last, const float* c, void* x, void* xm, void* ym,
+                                      void* ws, size_t ws_bytes, h3b_stream stream) {
+  WsLayout lay_full;
+  DeviceInfo* di = nullptr;
+  h3b_status s = block_common(full, c, x, ws, ws_bytes, &lay_full, &di);
+  if (s != H3B_OK) return s;
+  if (n_blocks < 0 || (n_blocks > 0 && !w)) return fail(H3B_ERR_ARG, "n_blocks < 0 or weights NULL");
+  if (first < 0 || first > last || last > n_blocks) return fail(H3B_ERR_ARG, "need 0 <= first <= last <= n_blocks");
+  const bool reduced = first < last;
+  h3b_dims merged = *full;
+  WsLayout lay_merged = lay_full;
+  if (reduced) {
+    if (full->W % 2 != 0) return fail(H3B_ERR_SHAPE, "W must be even for token pairing");
+    if (!xm || !ym) return fail(H3B_ERR_ARG, "xm and ym must be non-NULL");
+    if (!aligned16(xm) || !aligned16(ym)) return fail(H3B_ERR_ALIGN, "xm/ym not 16-byte aligned");
+    merged.W = full->W / 2;
+    if ((s = check_dims(&merged)) != H3B_OK) return s;
+    lay_merged = ws_layout(merged);
+  }
+  for (int i = 0; i < n_blocks; ++i)
+    if ((s = check_weights(*full, &w[i])) != H3B_OK) return s;
+  cudaStream_t st = stream;
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  const size_t c_stride = (size_t)full->B * full->d;
+  const long long lines = (long long)full->B * full->T * full->H;
+  for (int i = 0; i < first; ++i)
+    if ((s = run_block(*full, w[i], c + i * c_stride, x, wsb, lay_full, i > 0, *di, st)) != H3B_OK) return s;
+  if (reduced) {
+    H3B_CK(launch_token_pair(x, xm, ym, lines, full->W, full->d, di->sms, st), "token_pair");
+    for (int i = first; i < last; ++i)
+      if ((s = run_block(merged, w[i], c + i * c_stride, ym, wsb, lay_merged, i > first, *di, st)) != H3B_OK)
+        return s;
+    H3B_CK(launch_token_unpair(x, xm, ym, x, lines, full->W, full->d, di->sms, st), "token_unpair");
+  }
+  for (int i = last; i < n_blocks; ++i)
+    if ((s = run_block(*full, w[i], c + i * c_stride, x, wsb, lay_full, i > last || (!reduced && i > 0), *di, st)) !=
+        H3B_OK)
+      return s;
+  return H3B_OK;
+}
+
 static h3b_status check_pair_dims(const h3b_dims* full) {
   if (!full) return fail(H3B_ERR_ARG, "dims is NULL");
   if (full->B < 1 || full->T < 1 || full->H < 1 || full->W < 2) return fail(H3B_ERR_SHAPE, "bad grid");
@@ -480,7 +521,8 @@ h3b_status h3b_adaln_modulation(const h3b_dims* dims, const void* w_ada, const f
   if (!aligned16(w_ada) || !aligned16(c) || !aligned16(mod)) return fail(H3B_ERR_ALIGN, "alignment");
   DeviceInfo* di = nullptr;
   if ((s = device_info(&di)) != H3B_OK) return s;
-  H3B_CK(launch_adaln_gemv(w_ada, b_ada, c, dims->B, dims->d, mod, stream), "adaln_gemv");
+  H3B_CK(launch_adaln_gemv(w_ada, b_ada, c, dims->B, dims->d, mod, nullptr, 0, 0, 0, 0, 0, 0, 0.0, stream),
+         "adaln_gemv");
   return H3B_OK;
 }
 
@@ -497,7 +539,7 @@ h3b_status h3b_ln_modulate_quantize(const void* x, int rows, int d, float eps, c
   h3b_status hs = device_info(&di);
   if (hs != H3B_OK) return hs;
   H3B_CK(launch_ln_mod_quant(x, rows, d, eps, shift, scale, rows_per_item, mod_stride, q, s, h_out, absmax_zero,
-                             write_codes, stream), "ln_mod_quant");
+                             write_codes, di->err, di->sms, stream), "ln_mod_quant");
   return H3B_OK;
 }
 

@@ -90,9 +90,20 @@ __device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const float (&
 }
 
 // Epilogue of one 128x256 tile for the thread owning TMEM lane = tile row.
+// Residual rows this thread updates: its 128 columns of x, loaded before the
+// accumulator is ready so the global-memory latency overlaps the K loop.
+constexpr int kResidVecs = 16;  // 128 bf16 columns = 16 x 16 bytes
+__device__ __forceinline__ void prefetch_resid(const GemmArgs& p, int row, int col0, uint4 (&xp)[kResidVecs]) {
+  const bool row_ok = row < p.M;
+  const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.out) + (size_t)row * p.N + col0);
+#pragma unroll
+  for (int g = 0; g < kResidVecs; ++g)
+    xp[g] = (row_ok && col0 + 8 * g < p.N) ? src[g] : make_uint4(0, 0, 0, 0);
+}
+
 template <bool kInt8, int kEpi>
 __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, uint32_t tbase, int row, bool row_ok,
-                                              int n0, int c_begin, int c_end) {
+                                              int n0, int c_begin, int c_end, const uint4 (&xp)[kResidVecs]) {
   float sa = 1.0f;
   if (kInt8 && kEpi != EPI_S32 && row_ok) sa = __ldg(p.sA + row);
   int item = 0, l = 0, pt = 0, ph = 0, pw = 0;
@@ -106,7 +117,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, uint32_t tbase,
     item = row / p.rows_per_item;
   }
   float amax = 0.0f;
-#pragma unroll 1
+#pragma unroll
   for (int c = c_begin; c < c_end; ++c) {
     const int col0 = n0 + c * 32;
     if (col0 >= p.N) break;  // uniform across the warp
@@ -160,12 +171,12 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, uint32_t tbase,
       }
       store_bf16x32(static_cast<__nv_bfloat16*>(p.out) + (size_t)row * p.N + col0, v, valid);
     } else if (kEpi == EPI_RESID) {
-      __nv_bfloat16* xp = static_cast<__nv_bfloat16*>(p.out) + (size_t)row * p.N + col0;
+      __nv_bfloat16* xdst = static_cast<__nv_bfloat16*>(p.out) + (size_t)row * p.N + col0;
       const float4* g4 = reinterpret_cast<const float4*>(p.gate + (size_t)item * p.gate_stride + col0);
 #pragma unroll
       for (int g = 0; g < 4; ++g) {
         if (g * 8 >= valid) break;
-        const uint4 xv = reinterpret_cast<const uint4*>(xp)[g];
+        const uint4 xv = xp[(c - c_begin) * 4 + g];
         const float4 ga = __ldg(g4 + 2 * g), gb = __ldg(g4 + 2 * g + 1);
         const float gg[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
         const uint32_t xu[4] = {xv.x, xv.y, xv.z, xv.w};
@@ -175,7 +186,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, uint32_t tbase,
           v[8 * g + 2 * e + 1] = fmaf(gg[2 * e + 1], v[8 * g + 2 * e + 1], bf16_hi(xu[e]));
         }
       }
-      store_bf16x32(xp, v, valid);
+      store_bf16x32(xdst, v, valid);
     } else if (kEpi == EPI_QKV) {
       const int part = col0 / p.d;
       const int rem = col0 - part * p.d;
@@ -329,13 +340,15 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
       tile_coords(t, n_m, n_n, p.raster_n, p.group, mb, nb);
       const int acc = tl & 1;
       const uint32_t aph = (tl >> 1) & 1;
+      const int row = mb * BM + quad * 32 + lane;
+      uint4 xp[kResidVecs];
+      if (kEpi == EPI_RESID) prefetch_resid(p, row, nb * BN + half * (BN / 2), xp);
       // tcgen05.ld is warp-collective: the wait outcome is made warp-uniform.
       const bool t_ok = !*abort_flag && mbar_wait(tfull(acc), aph, p.err, ERR_WAIT_MMA);
       if (!__all_sync(0xFFFFFFFFu, t_ok)) { *abort_flag = 1; break; }
       tc_fence_after();
-      const int row = mb * BM + quad * 32 + lane;
       const uint32_t tbase = tmem_base + ((uint32_t)(quad * 32) << 16) + acc * BN;
-      epilogue_tile<kInt8, kEpi>(p, tbase, row, row < p.M, nb * BN, half * (BN / 64), (half + 1) * (BN / 64));
+      epilogue_tile<kInt8, kEpi>(p, tbase, row, row < p.M, nb * BN, half * (BN / 64), (half + 1) * (BN / 64), xp);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(tempty(acc));

@@ -52,6 +52,41 @@ __device__ __forceinline__ int quant_code_fast(float v, float scale, float rcp) 
   if (fabsf(t - c) > kTieGuard) c = rintf(__fdiv_rn(v, scale));
   return max(-127, min(127, (int)c));
 }
+// Eight codes of one 16-byte bf16 vector without a branch per element:
+// t = v * RN(1/scale); adding 1.5 * 2^23 rounds t to the nearest integer
+// (ties to even) in the low mantissa bits, whose low byte is the int8 code
+// (|t| <= 127.5 never yields -128). |t - rint(t)| is tracked; if any element
+// lies within 2^-14 of a half-integer the caller recomputes the vector with the
+// exact division (quant_code), so the result equals the binary32 decision.
+__device__ __forceinline__ uint2 quant8_fast(uint4 v, float rcp, float& worst) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  const float2 r2 = make_float2(rcp, rcp), M2 = make_float2(12582912.0f, 12582912.0f);
+  const float2 nM2 = make_float2(-12582912.0f, -12582912.0f);
+  uint32_t b[8];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float2 t = __fmul2_rn(make_float2(__uint_as_float(w[e] << 16), __uint_as_float(w[e] & 0xFFFF0000u)), r2);
+    const float2 a = __fadd2_rn(t, M2);
+    const float2 dd = __ffma2_rn(__fadd2_rn(a, nM2), make_float2(-1.0f, -1.0f), t);  // t - rint(t), exact
+    worst = fmaxf(worst, fmaxf(fabsf(dd.x), fabsf(dd.y)));
+    b[2 * e] = __float_as_uint(a.x);
+    b[2 * e + 1] = __float_as_uint(a.y);
+  }
+  const uint32_t lo = __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410);
+  const uint32_t hi = __byte_perm(__byte_perm(b[4], b[5], 0x0040), __byte_perm(b[6], b[7], 0x0040), 0x5410);
+  return make_uint2(lo, hi);
+}
+__device__ __forceinline__ uint32_t pack4_i8(int a, int b, int c, int d);
+__device__ __noinline__ uint2 quant8_exact(uint4 v, float scale, float absmax) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  int c[8];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    c[2 * e] = quant_code(__uint_as_float(w[e] << 16), scale, absmax);
+    c[2 * e + 1] = quant_code(__uint_as_float(w[e] & 0xFFFF0000u), scale, absmax);
+  }
+  return make_uint2(pack4_i8(c[0], c[1], c[2], c[3]), pack4_i8(c[4], c[5], c[6], c[7]));
+}
 __device__ __forceinline__ uint32_t pack4_i8(int a, int b, int c, int d) {
   return (uint32_t)(a & 0xFF) | ((uint32_t)(b & 0xFF) << 8) | ((uint32_t)(c & 0xFF) << 16) |
          ((uint32_t)(d & 0xFF) << 24);
@@ -66,12 +101,26 @@ constexpr int kGemvMaxB = 8;
 
 // One warp per output row j; the row's d/8 16-byte vectors (NV per lane) are
 // all requested before any is used, so each warp keeps its whole row in flight.
+struct RopeTableArgs {
+  float2* tab;  // nullptr: no table this launch
+  int T, H, W, rt, rh, rw;
+  double theta;
+};
+
+__device__ void rope_table_entries(const RopeTableArgs& r, int first, int stride);
+
 template <int NV>
 __global__ void __launch_bounds__(256) adaln_gemv_kernel(const __nv_bfloat16* __restrict__ W,
                                                          const float* __restrict__ bias,
                                                          const float* __restrict__ c, int B,
-                                                         float* __restrict__ mod) {
+                                                         float* __restrict__ mod, const RopeTableArgs rope,
+                                                         int gemv_blocks) {
   constexpr int d = NV * 256;
+  if ((int)blockIdx.x >= gemv_blocks) {  // trailing blocks fill the RoPE table
+    rope_table_entries(rope, ((int)blockIdx.x - gemv_blocks) * blockDim.x + threadIdx.x,
+                       ((int)gridDim.x - gemv_blocks) * blockDim.x);
+    return;
+  }
   extern __shared__ float cs[];  // [B][d]
   for (int i = threadIdx.x; i < B * d; i += blockDim.x) cs[i] = c[i];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -112,136 +161,210 @@ __global__ void __launch_bounds__(256) adaln_gemv_kernel(const __nv_bfloat16* __
 }
 
 // ---------------------------------------------------------------------------
-// Fused LayerNorm + modulation + per-row int8 quantization. A row of
-// d = 8 * VPT * G channels is held in registers by a group of G threads
-// (VPT 16-byte vectors each); a 256-thread block serves 256 / G rows.
+// Fused LayerNorm + modulation + per-row int8 quantization.
 //   y = (x - mean) * rsqrt(var + eps)          (fp32, two-pass variance)
 //   h = bf16(y * (1 + scale) + shift)
 //   s = absmax(h) / 127, q = rint(h / s)       (binary32 decision)
+// A row of d = 256 NV channels (32 NV 16-byte vectors) is held in registers by
+// tpr = 32 NV / VPT threads, VPT vectors each; a block holds rpp = blockDim /
+// tpr rows at a time and walks its share of the rows in passes of rpp rows,
+// all of one batch item. The item's (1 + scale, shift) pairs sit in shared
+// memory, loaded when the item changes, laid out [4][vectors] so that a warp's
+// 16-byte reads of one channel pair per vector fall in distinct banks.
+// Reductions: warp shuffles, then one shared slot per warp and a barrier
+// (slots alternate between passes, so no barrier guards their reuse).
 // ---------------------------------------------------------------------------
-template <int G>
-__device__ __forceinline__ float group_sum(float v, float* red) {
-  v = warp_sum(v);
-  if (G == 32) return v;
-  constexpr int NW = G / 32;
-  const int warp = threadIdx.x >> 5;
-  if ((threadIdx.x & 31) == 0) red[warp] = v;
-  __syncthreads();
-  const int first = (warp / NW) * NW;
-  float t = 0.0f;
-#pragma unroll
-  for (int i = 0; i < NW; ++i) t += red[first + i];
-  __syncthreads();
-  return t;
-}
-template <int G>
-__device__ __forceinline__ float group_max(float v, float* red) {
-  v = warp_max(v);
-  if (G == 32) return v;
-  constexpr int NW = G / 32;
-  const int warp = threadIdx.x >> 5;
-  if ((threadIdx.x & 31) == 0) red[warp] = v;
-  __syncthreads();
-  const int first = (warp / NW) * NW;
-  float t = 0.0f;
-#pragma unroll
-  for (int i = 0; i < NW; ++i) t = fmaxf(t, red[first + i]);
-  __syncthreads();
-  return t;
-}
-
 __device__ __forceinline__ float2 bf16x2_to_f2(uint32_t u) { return make_float2(bf16_lo(u), bf16_hi(u)); }
+__device__ __forceinline__ float max3f_row(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
 
-template <int VPT, int G>
-__global__ void __launch_bounds__(256) ln_mod_quant_kernel(
-    const __nv_bfloat16* __restrict__ x, int rows, float eps, const float* __restrict__ shift,
+constexpr int kLnMaxWarps = 32;
+
+// Lane-wise max of two bf16 pairs (both non-negative here).
+__device__ __forceinline__ uint32_t bf16x2_max(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+template <int VPT>
+__global__ void __launch_bounds__(1024, 1) ln_mod_quant_kernel(
+    const __nv_bfloat16* __restrict__ x, int rows, int vpr, float eps, const float* __restrict__ shift,
     const float* __restrict__ scale, int rows_per_item, int mod_stride, int8_t* __restrict__ q,
     float* __restrict__ s, __nv_bfloat16* __restrict__ h_out, float* __restrict__ absmax_zero,
     int write_codes) {
-  constexpr int RPB = 256 / G;
-  constexpr int d = VPT * G * 8;
-  __shared__ float red[8];
-  const int gt = threadIdx.x % G;
-  const int row = blockIdx.x * RPB + threadIdx.x / G;
-  const bool valid = row < rows;
-  const uint4* xr = reinterpret_cast<const uint4*>(x + (size_t)(valid ? row : 0) * d);
-  uint4 v[VPT];
-#pragma unroll
-  for (int i = 0; i < VPT; ++i) v[i] = valid ? __ldcs(xr + gt + G * i) : make_uint4(0, 0, 0, 0);
-
-  float2 acc = make_float2(0.0f, 0.0f);
-#pragma unroll
-  for (int i = 0; i < VPT; ++i) {
-    acc = __fadd2_rn(acc, bf16x2_to_f2(v[i].x));
-    acc = __fadd2_rn(acc, bf16x2_to_f2(v[i].y));
-    acc = __fadd2_rn(acc, bf16x2_to_f2(v[i].z));
-    acc = __fadd2_rn(acc, bf16x2_to_f2(v[i].w));
-  }
-  const float mean = group_sum<G>(acc.x + acc.y, red) * (1.0f / d);
-  const float2 nmean = make_float2(-mean, -mean);
-  acc = make_float2(0.0f, 0.0f);
-#pragma unroll
-  for (int i = 0; i < VPT; ++i) {
-    const uint32_t u[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float2 c = __fadd2_rn(bf16x2_to_f2(u[e]), nmean);
-      acc = __ffma2_rn(c, c, acc);
+  extern __shared__ float4 modp[];  // [4][vpr]: (1+sc[2c], 1+sc[2c+1], sh[2c], sh[2c+1]), c = 4 vec + e
+  __shared__ float red[2][3][kLnMaxWarps];
+  const int tpr = vpr / VPT;
+  const int rpp = blockDim.x / tpr;
+  const int sub = threadIdx.x / tpr;
+  const int t = threadIdx.x - sub * tpr;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int wpr = tpr >> 5, w0 = sub * wpr;
+  const float inv_d = 1.0f / (float)(vpr * 8);
+  const int items = (rows + rows_per_item - 1) / rows_per_item;
+  const unsigned gpi = (unsigned)((rows_per_item + rpp - 1) / rpp);
+  const unsigned total = (unsigned)items * gpi;  // passes; at most rows, so 32 bits suffice
+  int cur = -1, par = 0;
+  unsigned item = blockIdx.x / gpi, g_in = blockIdx.x % gpi;  // pass = (item, pass within item)
+  for (unsigned g = blockIdx.x; g < total; g += gridDim.x) {
+    if ((int)item != cur) {  // block-uniform
+      __syncthreads();
+      const float2* sc2 = reinterpret_cast<const float2*>(scale + (size_t)item * mod_stride);
+      const float2* sh2 = reinterpret_cast<const float2*>(shift + (size_t)item * mod_stride);
+      for (int c = threadIdx.x; c < 4 * vpr; c += blockDim.x) {
+        const float2 a = __ldg(sc2 + c), b = __ldg(sh2 + c);
+        modp[(c & 3) * vpr + (c >> 2)] = make_float4(1.0f + a.x, 1.0f + a.y, b.x, b.y);
+      }
+      cur = item;
+      __syncthreads();
     }
-  }
-  const float rstd = 1.0f / sqrtf(group_sum<G>(acc.x + acc.y, red) * (1.0f / d) + eps);
-  const float2 rstd2 = make_float2(rstd, rstd);
+    const int r_in = (int)g_in * rpp + sub;
+    const int row = (int)item * rows_per_item + r_in;
+    const bool valid = r_in < rows_per_item && row < rows;
+    const uint4* xr = reinterpret_cast<const uint4*>(x) + (size_t)(valid ? row : 0) * vpr;
+    uint4 v[VPT];
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) v[i] = valid ? __ldcs(xr + t + tpr * i) : make_uint4(0, 0, 0, 0);
 
-  const int item = (valid ? row : 0) / rows_per_item;
-  const float2* sh2 = reinterpret_cast<const float2*>(shift + (size_t)item * mod_stride);
-  const float2* sc2 = reinterpret_cast<const float2*>(scale + (size_t)item * mod_stride);
-  float amax = 0.0f;
+    float* rd = red[par][0];
+    par ^= 1;
+    // the row in fp32 pairs, converted once
+    float2 f[VPT * 4];
 #pragma unroll
-  for (int i = 0; i < VPT; ++i) {
-    const int c0 = (gt + G * i) * 4;  // float2 index of the vector's first channel pair
-    uint32_t u[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float2 sh = __ldg(sh2 + c0 + e);
-      const float2 sc = __ldg(sc2 + c0 + e);
-      const float2 y = __fmul2_rn(__fadd2_rn(bf16x2_to_f2(u[e]), nmean), rstd2);
-      const float2 h = __ffma2_rn(y, make_float2(1.0f + sc.x, 1.0f + sc.y), sh);
-      u[e] = pack_bf16x2(h.x, h.y);
-      amax = fmaxf(amax, fmaxf(fabsf(bf16_lo(u[e])), fabsf(bf16_hi(u[e]))));
+    for (int i = 0; i < VPT; ++i) {
+      f[4 * i + 0] = bf16x2_to_f2(v[i].x);
+      f[4 * i + 1] = bf16x2_to_f2(v[i].y);
+      f[4 * i + 2] = bf16x2_to_f2(v[i].z);
+      f[4 * i + 3] = bf16x2_to_f2(v[i].w);
     }
-    v[i] = make_uint4(u[0], u[1], u[2], u[3]);
-  }
-  amax = group_max<G>(amax, red);
-  if (!valid) return;
-  if (h_out) {
-    uint4* hr = reinterpret_cast<uint4*>(h_out + (size_t)row * d);
+    float2 acc = f[0];
 #pragma unroll
-    for (int i = 0; i < VPT; ++i) hr[gt + G * i] = v[i];
-  }
-  if (absmax_zero && gt == 0) absmax_zero[row] = 0.0f;
-  if (!write_codes) return;
-  const float sc = __fdiv_rn(amax, 127.0f);
-  const float rcp = __frcp_rn(sc);
-  if (gt == 0) s[row] = sc;
-  uint2* qr = reinterpret_cast<uint2*>(q + (size_t)row * d);
+    for (int e = 1; e < VPT * 4; ++e) acc = __fadd2_rn(acc, f[e]);
+    float r = warp_sum(acc.x + acc.y);
+    if (lane == 0) rd[warp] = r;
+    __syncthreads();
+    r = 0.0f;
+    for (int k = 0; k < wpr; ++k) r += rd[w0 + k];
+    const float mean = r * inv_d;
+    const float2 nmean = make_float2(-mean, -mean);
+
 #pragma unroll
-  for (int i = 0; i < VPT; ++i) {
-    const uint32_t u[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
-    int c[8];
-    if (!(rcp < INFINITY)) {  // absmax == 0 (codes 0) or a subnormal scale: exact division
+    for (int e = 0; e < VPT * 4; ++e) f[e] = __fadd2_rn(f[e], nmean);  // x - mean
+    acc = __fmul2_rn(f[0], f[0]);
+#pragma unroll
+    for (int e = 1; e < VPT * 4; ++e) acc = __ffma2_rn(f[e], f[e], acc);
+    r = warp_sum(acc.x + acc.y);
+    if (lane == 0) rd[kLnMaxWarps + warp] = r;
+    __syncthreads();
+    r = 0.0f;
+    for (int k = 0; k < wpr; ++k) r += rd[kLnMaxWarps + w0 + k];
+    const float rstd = 1.0f / sqrtf(r * inv_d + eps);
+    const float2 rstd2 = make_float2(rstd, rstd);
+
+    // h = bf16((x - mean) * rstd * (1 + scale) + shift); |h| max kept as a bf16 pair
+    uint32_t am2 = 0u;
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+      const int vec = t + tpr * i;
+      uint32_t u[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        c[2 * e] = quant_code(bf16_lo(u[e]), sc, amax);
-        c[2 * e + 1] = quant_code(bf16_hi(u[e]), sc, amax);
+        const float4 m = modp[e * vpr + vec];
+        const float2 y = __fmul2_rn(f[4 * i + e], rstd2);
+        const float2 h = __ffma2_rn(y, make_float2(m.x, m.y), make_float2(m.z, m.w));
+        u[e] = pack_bf16x2(h.x, h.y);
+        am2 = bf16x2_max(am2, u[e] & 0x7FFF7FFFu);
       }
-    } else {
+      v[i] = make_uint4(u[0], u[1], u[2], u[3]);
+    }
+    float amax = fmaxf(bf16_lo(am2), bf16_hi(am2));
+    amax = warp_max(amax);
+    if (lane == 0) rd[2 * kLnMaxWarps + warp] = amax;
+    __syncthreads();
+    amax = 0.0f;
+    for (int k = 0; k < wpr; ++k) amax = fmaxf(amax, rd[2 * kLnMaxWarps + w0 + k]);
+    if (valid) {
+      if (h_out) {
+        uint4* hr = reinterpret_cast<uint4*>(h_out) + (size_t)row * vpr;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        c[2 * e] = quant_code_fast(bf16_lo(u[e]), sc, rcp);
-        c[2 * e + 1] = quant_code_fast(bf16_hi(u[e]), sc, rcp);
+        for (int i = 0; i < VPT; ++i) hr[t + tpr * i] = v[i];
+      }
+      if (absmax_zero && t == 0) absmax_zero[row] = 0.0f;
+      if (write_codes) {
+        const float sc = __fdiv_rn(amax, 127.0f);
+        const float rcp = __frcp_rn(sc);
+        if (t == 0) s[row] = sc;
+        uint2* qr = reinterpret_cast<uint2*>(q) + (size_t)row * vpr;
+#pragma unroll
+        for (int i = 0; i < VPT; ++i) {
+          uint2 code;
+          float worst = 1.0f;
+          if (rcp < INFINITY) {
+            worst = 0.0f;
+            code = quant8_fast(v[i], rcp, worst);
+          }
+          if (worst > kTieGuard) code = quant8_exact(v[i], sc, amax);  // near-tie, zero or subnormal scale
+          qr[t + tpr * i] = code;
+        }
       }
     }
-    qr[gt + G * i] = make_uint2(pack4_i8(c[0], c[1], c[2], c[3]), pack4_i8(c[4], c[5], c[6], c[7]));
+    g_in += gridDim.x;
+    item += g_in / gpi;
+    g_in %= gpi;
+  }
+}
+
+// Per-row quantization with each row's absmax already known: a block covers
+// whole rows (rpb rows of vpr 16-byte vectors, rpb * vpr <= 1024, rpb <= 32),
+// each thread keeps up to four vectors in flight; each row's scale and its
+// reciprocal are derived once, into shared memory.
+constexpr int kQuantMaxRowsPerBlock = 32;
+__global__ void __launch_bounds__(256) quant_rows_known_absmax_kernel(const __nv_bfloat16* __restrict__ in,
+                                                                      int rows, int vpr, int rpb,
+                                                                      const float* __restrict__ absmax_in,
+                                                                      int8_t* __restrict__ q,
+                                                                      float* __restrict__ s) {
+  constexpr int U = 4;
+  __shared__ float2 srow[kQuantMaxRowsPerBlock];  // (scale, RN(1/scale)) of the block's rows
+  __shared__ float samax[kQuantMaxRowsPerBlock];
+  const unsigned row0 = blockIdx.x * (unsigned)rpb;
+  const unsigned nr = min((unsigned)rpb, (unsigned)rows - row0);
+  if (threadIdx.x < nr) {
+    const float amax = __ldg(absmax_in + row0 + threadIdx.x);
+    const float sc = __fdiv_rn(amax, 127.0f);
+    srow[threadIdx.x] = make_float2(sc, __frcp_rn(sc));
+    samax[threadIdx.x] = amax;
+    s[row0 + threadIdx.x] = sc;
+  }
+  const unsigned span = nr * (unsigned)vpr;  // vectors covered by this block
+  const size_t base = (size_t)row0 * vpr;
+  __syncthreads();
+  for (unsigned k0 = threadIdx.x; k0 < span; k0 += U * blockDim.x) {
+    uint4 raw[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const unsigned k = k0 + u * blockDim.x;
+      if (k < span) raw[u] = __ldcs(reinterpret_cast<const uint4*>(in) + base + k);
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const unsigned k = k0 + u * blockDim.x;
+      if (k >= span) break;
+      const unsigned r = rpb == 1 ? 0u : k / vpr;
+      const float2 sr = srow[r];
+      uint2 code;
+      float worst = 1.0f;
+      if (sr.y < INFINITY) {
+        worst = 0.0f;
+        code = quant8_fast(raw[u], sr.y, worst);
+      }
+      if (worst > kTieGuard) code = quant8_exact(raw[u], sr.x, samax[r]);  // near-tie, zero or subnormal scale
+      reinterpret_cast<uint2*>(q)[base + k] = code;
+    }
   }
 }
 
@@ -382,17 +505,21 @@ __global__ void token_unpair_kernel(const __nv_bfloat16* __restrict__ x,
 // entry [pos * (r/2) + j] = (cos, sin)(pos * theta^(-2j/r)), evaluated in fp64
 // and stored as fp32. Axis blocks are stored one after the other (t, h, w).
 // ---------------------------------------------------------------------------
-__global__ void rope_table_kernel(float2* __restrict__ tab, int T, int H, int W, int rt, int rh,
-                                  int rw, double theta) {
-  const int nt = T * (rt / 2), nh = H * (rh / 2), nw = W * (rw / 2);
-  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < nt + nh + nw; i += gridDim.x * blockDim.x) {
-    int idx = i, r = rt;
-    if (idx >= nt + nh) { idx -= nt + nh; r = rw; }
-    else if (idx >= nt) { idx -= nt; r = rh; }
-    const int half = r / 2, pos = idx / half, j = idx % half;
-    const double ang = (double)pos * pow(theta, -2.0 * (double)j / (double)r);
-    tab[i] = make_float2((float)cos(ang), (float)sin(ang));
+__device__ void rope_table_entries(const RopeTableArgs& r, int first, int stride) {
+  if (!r.tab) return;
+  const int nt = r.T * (r.rt / 2), nh = r.H * (r.rh / 2), nw = r.W * (r.rw / 2);
+  for (int i = first; i < nt + nh + nw; i += stride) {
+    int idx = i, len = r.rt;
+    if (idx >= nt + nh) { idx -= nt + nh; len = r.rw; }
+    else if (idx >= nt) { idx -= nt; len = r.rh; }
+    const int half = len / 2, pos = idx / half, j = idx % half;
+    const double ang = (double)pos * pow(r.theta, -2.0 * (double)j / (double)len);
+    r.tab[i] = make_float2((float)cos(ang), (float)sin(ang));
   }
+}
+
+__global__ void rope_table_kernel(const RopeTableArgs r) {
+  rope_table_entries(r, blockIdx.x * blockDim.x + threadIdx.x, gridDim.x * blockDim.x);
 }
 
 // ---------------------------------------------------------------------------
@@ -400,7 +527,7 @@ __global__ void rope_table_kernel(float2* __restrict__ tab, int T, int H, int W,
 // ---------------------------------------------------------------------------
 template <int NV>
 static cudaError_t gemv_dispatch(const void* W, const float* bias, const float* c, int B, float* mod,
-                                 cudaStream_t st) {
+                                 const RopeTableArgs& rope, cudaStream_t st) {
   constexpr int d = NV * 256;
   const size_t smem = (size_t)B * d * sizeof(float);
   if (smem > 48 * 1024) {
@@ -408,17 +535,25 @@ static cudaError_t gemv_dispatch(const void* W, const float* bias, const float* 
                                          (int)smem);
     if (e != cudaSuccess) return e;
   }
-  adaln_gemv_kernel<NV><<<(6 * d + 7) / 8, 256, smem, st>>>(static_cast<const __nv_bfloat16*>(W), bias, c, B,
-                                                            mod);
+  const int gemv_blocks = (6 * d + 7) / 8;
+  int rope_blocks = 0;
+  if (rope.tab) {
+    const int n = rope.T * (rope.rt / 2) + rope.H * (rope.rh / 2) + rope.W * (rope.rw / 2);
+    rope_blocks = (n + 255) / 256;
+  }
+  adaln_gemv_kernel<NV><<<gemv_blocks + rope_blocks, 256, smem, st>>>(static_cast<const __nv_bfloat16*>(W), bias,
+                                                                      c, B, mod, rope, gemv_blocks);
   return cudaGetLastError();
 }
 
 cudaError_t launch_adaln_gemv(const void* W, const float* bias, const float* c, int B, int d,
-                              float* mod, cudaStream_t st) {
+                              float* mod, float2* rope_tab, int T, int H, int Wd, int rt, int rh, int rw,
+                              double theta, cudaStream_t st) {
   if (B > kGemvMaxB || d % 256 != 0) return cudaErrorInvalidValue;
+  const RopeTableArgs rope{rope_tab, T, H, Wd, rt, rh, rw, theta};
 #define H3B_GV(nv) \
   case nv:         \
-    return gemv_dispatch<nv>(W, bias, c, B, mod, st);
+    return gemv_dispatch<nv>(W, bias, c, B, mod, rope, st);
   switch (d / 256) {
     H3B_GV(1) H3B_GV(2) H3B_GV(3) H3B_GV(4) H3B_GV(5) H3B_GV(6) H3B_GV(7) H3B_GV(8)
     H3B_GV(9) H3B_GV(10) H3B_GV(11) H3B_GV(12) H3B_GV(13) H3B_GV(14) H3B_GV(15) H3B_GV(16)
@@ -430,54 +565,68 @@ cudaError_t launch_adaln_gemv(const void* W, const float* bias, const float* c, 
 #undef H3B_GV
 }
 
-template <int VPT, int G>
-static cudaError_t ln_dispatch(const void* x, int rows, float eps, const float* shift,
+// Threads per row: the fewest warps w dividing NV with NV / w <= 6 vectors per
+// thread; the block holds as many rows as fit in 256 threads (at least one).
+template <int VPT>
+static cudaError_t ln_dispatch(const void* x, int rows, int nv, float eps, const float* shift,
                                const float* scale, int rpi, int ms, int8_t* q, float* s, void* h,
-                               float* az, int wc, cudaStream_t st) {
-  constexpr int RPB = 256 / G;
-  ln_mod_quant_kernel<VPT, G><<<(rows + RPB - 1) / RPB, 256, 0, st>>>(
-      static_cast<const __nv_bfloat16*>(x), rows, eps, shift, scale, rpi, ms, q, s,
-      static_cast<__nv_bfloat16*>(h), az, wc);
+                               float* az, int wc, int sms, cudaStream_t st) {
+  const int vpr = 32 * nv;
+  const int tpr = vpr / VPT;
+  const int block = tpr * (tpr >= 256 ? 1 : 256 / tpr);
+  const size_t smem = (size_t)vpr * 4 * sizeof(float4);
+  auto kern = ln_mod_quant_kernel<VPT>;
+  static int attr_done = 0;
+  if (!attr_done) {
+    // the largest row (d = 8192, 1024 vectors) needs 64 KB of (1 + scale, shift) pairs
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)(32 * 32 * 4 * sizeof(float4)));
+    if (e != cudaSuccess) return e;
+    attr_done = 1;
+  }
+  int per_sm = 0;
+  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, block, smem);
+  if (e != cudaSuccess) return e;
+  if (per_sm < 1) per_sm = 1;
+  const int rpp = block / tpr;
+  const long long passes = (long long)((rows + rpi - 1) / rpi) * ((rpi + rpp - 1) / rpp);
+  const long long grid = std::min<long long>(passes, (long long)sms * per_sm);
+  kern<<<(int)grid, block, smem, st>>>(static_cast<const __nv_bfloat16*>(x), rows, vpr, eps, shift, scale, rpi, ms,
+                                        q, s, static_cast<__nv_bfloat16*>(h), az, wc);
   return cudaGetLastError();
 }
 
-// d = 256 k: a row is split over G = 128 (k % 4 == 0), 64 (k % 2 == 0) or 32
-// threads holding VPT = 32 k / G vectors of 8 channels each.
 cudaError_t launch_ln_mod_quant(const void* x, int rows, int d, float eps, const float* shift,
                                 const float* scale, int rows_per_item, int mod_stride, int8_t* q,
-                                float* s, void* h_out, float* absmax_zero, int write_codes,
-                                cudaStream_t st) {
+                                float* s, void* h_out, float* absmax_zero, int write_codes, unsigned* err,
+                                int sms, cudaStream_t st) {
   if (rows == 0) return cudaSuccess;
-  const int k = d / 256;
-#define H3B_LN(vpt, g) \
-  return ln_dispatch<vpt, g>(x, rows, eps, shift, scale, rows_per_item, mod_stride, q, s, h_out, absmax_zero, write_codes, st)
-  if (k % 4 == 0) {
-    switch (k / 4) {
-      case 1: H3B_LN(1, 128); case 2: H3B_LN(2, 128); case 3: H3B_LN(3, 128); case 4: H3B_LN(4, 128);
-      case 5: H3B_LN(5, 128); case 6: H3B_LN(6, 128); case 7: H3B_LN(7, 128); case 8: H3B_LN(8, 128);
-      default: return cudaErrorInvalidValue;
-    }
-  } else if (k % 2 == 0) {
-    switch (k / 2) {
-      case 1: H3B_LN(1, 64); case 3: H3B_LN(3, 64); case 5: H3B_LN(5, 64); case 7: H3B_LN(7, 64);
-      case 9: H3B_LN(9, 64); case 11: H3B_LN(11, 64); case 13: H3B_LN(13, 64); case 15: H3B_LN(15, 64);
-      default: return cudaErrorInvalidValue;
-    }
-  } else {
-    switch (k) {
-      case 1: H3B_LN(1, 32); case 3: H3B_LN(3, 32); case 5: H3B_LN(5, 32); case 7: H3B_LN(7, 32);
-      case 9: H3B_LN(9, 32); case 11: H3B_LN(11, 32); case 13: H3B_LN(13, 32); case 15: H3B_LN(15, 32);
-      case 17: H3B_LN(17, 32); case 19: H3B_LN(19, 32); case 21: H3B_LN(21, 32); case 23: H3B_LN(23, 32);
-      case 25: H3B_LN(25, 32); case 27: H3B_LN(27, 32); case 29: H3B_LN(29, 32); case 31: H3B_LN(31, 32);
-      default: return cudaErrorInvalidValue;
-    }
+  const int nv = d / 256;
+  if (nv < 1 || nv > 32 || d % 256) return cudaErrorInvalidValue;
+  int w = 1;
+  while (nv % w || nv / w > 6) ++w;
+  switch (nv / w) {
+    case 1: return ln_dispatch<1>(x, rows, nv, eps, shift, scale, rows_per_item, mod_stride, q, s, h_out, absmax_zero, write_codes, sms, st);
+    case 2: return ln_dispatch<2>(x, rows, nv, eps, shift, scale, rows_per_item, mod_stride, q, s, h_out, absmax_zero, write_codes, sms, st);
+    case 3: return ln_dispatch<3>(x, rows, nv, eps, shift, scale, rows_per_item, mod_stride, q, s, h_out, absmax_zero, write_codes, sms, st);
+    case 4: return ln_dispatch<4>(x, rows, nv, eps, shift, scale, rows_per_item, mod_stride, q, s, h_out, absmax_zero, write_codes, sms, st);
+    case 5: return ln_dispatch<5>(x, rows, nv, eps, shift, scale, rows_per_item, mod_stride, q, s, h_out, absmax_zero, write_codes, sms, st);
+    case 6: return ln_dispatch<6>(x, rows, nv, eps, shift, scale, rows_per_item, mod_stride, q, s, h_out, absmax_zero, write_codes, sms, st);
+    default: return cudaErrorInvalidValue;
   }
-#undef H3B_LN
 }
 
 cudaError_t launch_quant_rows_bf16(const void* h, int rows, int cols, const float* absmax,
                                    int8_t* q, float* s, cudaStream_t st) {
   if (rows == 0) return cudaSuccess;
+  if (absmax) {
+    const int vpr = cols / 8;
+    int rpb = 1024 / vpr;
+    rpb = rpb < 1 ? 1 : (rpb > kQuantMaxRowsPerBlock ? kQuantMaxRowsPerBlock : rpb);
+    quant_rows_known_absmax_kernel<<<(rows + rpb - 1) / rpb, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(h),
+                                                                          rows, vpr, rpb, absmax, q, s);
+    return cudaGetLastError();
+  }
   quant_rows_kernel<__nv_bfloat16><<<rows, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(h), cols,
                                                         absmax, q, s);
   return cudaGetLastError();
@@ -519,7 +668,7 @@ cudaError_t launch_token_unpair(const void* x, const void* xm, const void* ym, v
 cudaError_t launch_rope_table(float2* tab, int T, int H, int W, int rt, int rh, int rw,
                               double theta, cudaStream_t st) {
   const int n = T * (rt / 2) + H * (rh / 2) + W * (rw / 2);
-  rope_table_kernel<<<(n + 255) / 256, 256, 0, st>>>(tab, T, H, W, rt, rh, rw, theta);
+  rope_table_kernel<<<(n + 255) / 256, 256, 0, st>>>(RopeTableArgs{tab, T, H, W, rt, rh, rw, theta});
   return cudaGetLastError();
 }
 

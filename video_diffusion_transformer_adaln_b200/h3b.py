@@ -76,6 +76,7 @@ def _declare(L):
         "h3b_block_forward": [vp, vp, vp, vp, vp, sz, vp],
         "h3b_block_forward_noalloc": [vp, vp, vp, vp, vp],
         "h3b_blocks_forward": [vp, vp, i32, vp, vp, vp, sz, vp],
+        "h3b_blocks_forward_reduced": [vp, vp, i32, i32, i32, vp, vp, vp, vp, vp, sz, vp],
         "h3b_token_pair": [vp, vp, vp, vp, vp],
         "h3b_token_unpair": [vp, vp, vp, vp, vp, vp],
         "h3b_quantize_weights": [vp, i32, i32, vp, vp, vp],
@@ -167,6 +168,14 @@ def h3b_blocks_forward(dims: Dims, ws_list: Sequence[BlockWeights], c, x, ws, st
     arr = (BlockWeights * len(ws_list))(*ws_list)
     _check(lib().h3b_blocks_forward(C.byref(dims), arr, len(ws_list), _p(c), _p(x), _p(ws),
                                     ws.numel() * ws.element_size(), _s(stream)), "h3b_blocks_forward")
+
+
+def h3b_blocks_forward_reduced(full: Dims, ws_list: Sequence[BlockWeights], first: int, last: int, c, x, xm, ym,
+                               ws, stream=None):
+    arr = (BlockWeights * len(ws_list))(*ws_list)
+    _check(lib().h3b_blocks_forward_reduced(C.byref(full), arr, len(ws_list), first, last, _p(c), _p(x), _p(xm),
+                                            _p(ym), _p(ws), ws.numel() * ws.element_size(), _s(stream)),
+           "h3b_blocks_forward_reduced")
 
 
 def h3b_token_pair(full: Dims, x, xm, xm_copy=None, stream=None):

@@ -44,6 +44,8 @@ class Workload:
     qkv_int8: bool = True
     rope_theta: float = 10000.0
     ln_eps: float = 1e-6
+    # multi-block pass: blocks [first, last) run on the paired grid (empty: none)
+    pair_blocks: Tuple[int, int] = (0, 0)
 
     @property
     def L(self) -> int:
@@ -54,7 +56,7 @@ class Workload:
         assert self.W % 2 == 0
         return Workload(self.name + "/merged", self.T, self.H, self.W // 2, self.d, self.n_heads,
                         self.head_dim, self.d_ff, self.rope, self.n_outliers, self.B, self.n_blocks,
-                        False, self.qkv_int8, self.rope_theta, self.ln_eps)
+                        False, self.qkv_int8, self.rope_theta, self.ln_eps, (0, 0))
 
     def with_(self, **kw) -> "Workload":
         args = dict(self.__dict__)
@@ -82,6 +84,9 @@ WORKLOADS: Dict[str, Workload] = {
 # 50 distinct blocks at d=5120 over one latent, frame sweep T in {2,4,8,12,16}
 for _T in (2, 4, 8, 12, 16):
     WORKLOADS[f"d5120_depth50_T{_T}"] = _large(_T, name=f"d5120_depth50_T{_T}", n_blocks=50)
+# the same pass with token reduction over the middle half of the blocks (13..37)
+WORKLOADS["d5120_depth50_T8_pairmid"] = _large(8, name="d5120_depth50_T8_pairmid", n_blocks=50,
+                                               pair_blocks=(13, 38))
 
 _TENSOR_IDS = {"x": 1, "outliers": 2, "c": 3, "w_ada": 4, "b_gate": 5, "wqkv": 6, "wo": 7,
                "w1": 8, "w2": 9}
