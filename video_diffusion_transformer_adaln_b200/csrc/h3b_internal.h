@@ -52,6 +52,7 @@ struct GemmArgs {
   // EPI_QKV
   int B, L, T, H, W, d, n_heads, head_dim, rope_t, rope_h, rope_w;
   const float2* rope;  // table from launch_rope_table
+  int rope_smem_entries;  // set by launch_gemm: table entries staged in shared memory (0: none)
   unsigned* err;       // device error word
   // tile raster (set by launch_gemm): groups of `group` M-tiles (raster_n == 0)
   // or of `group` N-tiles (raster_n == 1)

@@ -264,6 +264,8 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
       for (int c = 0; c < BKV / 32; ++c)
         tmem_ld32(tmem + t_lane + s_col + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
       tmem_ld_wait();
+#pragma unroll
+      for (int c = 0; c < BKV / 32; ++c) tmem_reg_fence(*reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
 
       const int nvalid = min(BKV, L - j * BKV);
       if (nvalid < BKV) {  // uniform: only the last, partial key tile
@@ -315,6 +317,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
           uint32_t o[32];
           tmem_ld32(tmem + t_lane + o_col + c * 32, o);
           tmem_ld_wait();
+          tmem_reg_fence(o);
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
             const float2 v = __fmul2_rn(make_float2(__uint_as_float(o[e]), __uint_as_float(o[e + 1])),
@@ -348,6 +351,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         uint32_t o[32];
         tmem_ld32(tmem + t_lane + o_col + c * 32, o);
         tmem_ld_wait();
+        tmem_reg_fence(o);
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {

@@ -36,7 +36,11 @@ constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr size_t kL2Budget = 48ull << 20;  // operand bytes the raster keeps resident in L2
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int kBars = 2 * STAGES + 4 + 1;
-constexpr size_t SMEM_BYTES = (size_t)STAGES * STAGE_BYTES + 1024 + kBars * 8 + 16;
+constexpr size_t CONST_OFF = (size_t)STAGES * STAGE_BYTES + 256;     // per-warp epilogue constants
+constexpr size_t ROPE_OFF = CONST_OFF + kEpiWarps * 3 * 128 * 4;     // RoPE table, when it fits
+constexpr size_t SMEM_BASE = ROPE_OFF + 1024;                         // + 1024 for the alignment slack
+constexpr size_t kSmemMax = 227 * 1024;
+constexpr int kRopeSmemMaxEntries = (int)((kSmemMax - SMEM_BASE) / 8);
 }  // namespace gemm
 
 // Tile t -> (M-tile, N-tile). Tiles are rastered in groups: `group` M-tiles
@@ -101,9 +105,42 @@ __device__ __forceinline__ void prefetch_resid(const GemmArgs& p, int row, int c
     xp[g] = (row_ok && col0 + 8 * g < p.N) ? src[g] : make_uint4(0, 0, 0, 0);
 }
 
+// Per-warp column constants of the current tile (the warp's 128 columns):
+// weight scale, bias and (gated residual) gate, staged in shared memory before
+// the accumulator wait so the epilogue reads them at shared-memory latency.
+struct EpiConst {
+  float sw[128];
+  float bias[128];
+  float gate[128];
+};
+
 template <bool kInt8, int kEpi>
-__device__ __forceinline__ void epilogue_tile(const GemmArgs& p, uint32_t tbase, int row, bool row_ok,
-                                              int n0, int c_begin, int c_end, const uint4 (&xp)[kResidVecs]) {
+__device__ __forceinline__ void stage_constants(const GemmArgs& p, EpiConst& ec, int col0, int first_row, int lane) {
+  // four consecutive columns per lane; N is a multiple of 8, so a float4 is in or out as a whole
+  const int c = col0 + 4 * lane;
+  const bool ok = c < p.N;
+  if (kInt8 && kEpi != EPI_S32)
+    *reinterpret_cast<float4*>(&ec.sw[4 * lane]) = ok ? __ldg(reinterpret_cast<const float4*>(p.sW + c))
+                                                      : make_float4(0.f, 0.f, 0.f, 0.f);
+  if (kEpi != EPI_S32 && p.bias)
+    *reinterpret_cast<float4*>(&ec.bias[4 * lane]) = ok ? __ldg(reinterpret_cast<const float4*>(p.bias + c))
+                                                        : make_float4(0.f, 0.f, 0.f, 0.f);
+  if (kEpi == EPI_RESID) {
+    const int item = min(first_row, p.M - 1) / p.rows_per_item;
+    *reinterpret_cast<float4*>(&ec.gate[4 * lane]) =
+        ok ? __ldg(reinterpret_cast<const float4*>(p.gate + (size_t)item * p.gate_stride + c))
+           : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+}
+
+// Epilogue of the warp's 32 rows x 128 columns of one 128x256 tile; the thread
+// owns TMEM lane = tile row. TMEM loads are double-buffered: chunk i+1 (32
+// columns) is requested before chunk i is processed. `rope_s` is the RoPE
+// table in shared memory (or the global table when it did not fit).
+template <bool kInt8, int kEpi>
+__device__ __forceinline__ void epilogue_tile(const GemmArgs& p, uint32_t tbase, int row, bool row_ok, int n0,
+                                              const EpiConst& ec, bool gate_uniform, const float2* rope_s,
+                                              const uint4 (&xp)[kResidVecs]) {
   float sa = 1.0f;
   if (kInt8 && kEpi != EPI_S32 && row_ok) sa = __ldg(p.sA + row);
   int item = 0, l = 0, pt = 0, ph = 0, pw = 0;
@@ -117,99 +154,114 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, uint32_t tbase,
     item = row / p.rows_per_item;
   }
   float amax = 0.0f;
+  // the gated residual keeps its 128 prefetched x columns in registers instead
+  constexpr bool kDoubleBuffer = kEpi != EPI_RESID;
+  uint32_t r[kDoubleBuffer ? 2 : 1][32];
+  tmem_ld32(tbase, r[0]);
+  tmem_ld_wait();
+  tmem_reg_fence(r[0]);
 #pragma unroll
-  for (int c = c_begin; c < c_end; ++c) {
-    const int col0 = n0 + c * 32;
+  for (int i = 0; i < 4; ++i) {
+    const int col0 = n0 + i * 32;
     if (col0 >= p.N) break;  // uniform across the warp
-    uint32_t r[32];
-    tmem_ld32(tbase + c * 32, r);
-    tmem_ld_wait();
-    if (!row_ok) continue;
-    const int valid = min(32, p.N - col0);
-    if (kEpi == EPI_S32) {
-      uint4* d4 = reinterpret_cast<uint4*>(static_cast<int32_t*>(p.out) + (size_t)row * p.N + col0);
+    const bool next = i + 1 < 4 && col0 + 32 < p.N;
+    if (kDoubleBuffer && next) tmem_ld32(tbase + (i + 1) * 32, r[(i + 1) & 1]);
+    const uint32_t (&rc)[32] = r[kDoubleBuffer ? (i & 1) : 0];
+    if (row_ok) {
+      const int valid = min(32, p.N - col0);
+      if (kEpi == EPI_S32) {
+        uint4* d4 = reinterpret_cast<uint4*>(static_cast<int32_t*>(p.out) + (size_t)row * p.N + col0);
 #pragma unroll
-      for (int g = 0; g < 8; ++g)
-        if (g * 4 < valid) d4[g] = make_uint4(r[4 * g], r[4 * g + 1], r[4 * g + 2], r[4 * g + 3]);
-      continue;
-    }
-    float v[32];
-    if (kInt8) {
-      const float4* sw4 = reinterpret_cast<const float4*>(p.sW + col0);
-      const float2 sa2 = make_float2(sa, sa);
+        for (int g = 0; g < 8; ++g)
+          if (g * 4 < valid) d4[g] = make_uint4(rc[4 * g], rc[4 * g + 1], rc[4 * g + 2], rc[4 * g + 3]);
+      } else {
+        float v[32];
+        if (kInt8) {
+          const float2 sa2 = make_float2(sa, sa);
 #pragma unroll
-      for (int g = 0; g < 8; ++g) {
-        const float4 s = (4 * g < valid) ? __ldg(sw4 + g) : make_float4(0.f, 0.f, 0.f, 0.f);
-        const float2 lo = __fmul2_rn(__fmul2_rn(make_float2((float)(int)r[4 * g], (float)(int)r[4 * g + 1]), sa2),
-                                     make_float2(s.x, s.y));
-        const float2 hi = __fmul2_rn(__fmul2_rn(make_float2((float)(int)r[4 * g + 2], (float)(int)r[4 * g + 3]), sa2),
-                                     make_float2(s.z, s.w));
-        v[4 * g + 0] = lo.x; v[4 * g + 1] = lo.y; v[4 * g + 2] = hi.x; v[4 * g + 3] = hi.y;
-      }
-    } else {
+          for (int g = 0; g < 8; ++g) {
+            const float4 sw = *reinterpret_cast<const float4*>(&ec.sw[i * 32 + 4 * g]);
+            const float2 lo = __fmul2_rn(__fmul2_rn(make_float2((float)(int)rc[4 * g], (float)(int)rc[4 * g + 1]), sa2),
+                                         make_float2(sw.x, sw.y));
+            const float2 hi = __fmul2_rn(__fmul2_rn(make_float2((float)(int)rc[4 * g + 2], (float)(int)rc[4 * g + 3]), sa2),
+                                         make_float2(sw.z, sw.w));
+            v[4 * g + 0] = lo.x; v[4 * g + 1] = lo.y; v[4 * g + 2] = hi.x; v[4 * g + 3] = hi.y;
+          }
+        } else {
 #pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-    }
-    if (p.bias) {
-      const float4* b4 = reinterpret_cast<const float4*>(p.bias + col0);
+          for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(rc[e]);
+        }
+        if (p.bias) {
 #pragma unroll
-      for (int g = 0; g < 8; ++g) {
-        if (4 * g >= valid) break;
-        const float4 b = __ldg(b4 + g);
-        v[4 * g] += b.x; v[4 * g + 1] += b.y; v[4 * g + 2] += b.z; v[4 * g + 3] += b.w;
-      }
-    }
-    if (kEpi == EPI_DEQ) {
-      store_bf16x32(static_cast<__nv_bfloat16*>(p.out) + (size_t)row * p.N + col0, v, valid);
-    } else if (kEpi == EPI_GELU) {
+          for (int g = 0; g < 8; ++g) {
+            const float4 b = *reinterpret_cast<const float4*>(&ec.bias[i * 32 + 4 * g]);
+            v[4 * g] += b.x; v[4 * g + 1] += b.y; v[4 * g + 2] += b.z; v[4 * g + 3] += b.w;
+          }
+        }
+        if (kEpi == EPI_DEQ) {
+          store_bf16x32(static_cast<__nv_bfloat16*>(p.out) + (size_t)row * p.N + col0, v, valid);
+        } else if (kEpi == EPI_GELU) {
 #pragma unroll
-      for (int i = 0; i < 32; i += 2) {
-        const float2 gv = gelu_tanh2(make_float2(v[i], v[i + 1]));
-        v[i] = round_bf16(gv.x);
-        v[i + 1] = round_bf16(gv.y);
-        amax = fmaxf(amax, fmaxf(fabsf(v[i]), fabsf(v[i + 1])));
-      }
-      store_bf16x32(static_cast<__nv_bfloat16*>(p.out) + (size_t)row * p.N + col0, v, valid);
-    } else if (kEpi == EPI_RESID) {
-      __nv_bfloat16* xdst = static_cast<__nv_bfloat16*>(p.out) + (size_t)row * p.N + col0;
-      const float4* g4 = reinterpret_cast<const float4*>(p.gate + (size_t)item * p.gate_stride + col0);
+          for (int e = 0; e < 32; e += 2) {
+            const float2 gv = gelu_tanh2(make_float2(v[e], v[e + 1]));
+            v[e] = round_bf16(gv.x);
+            v[e + 1] = round_bf16(gv.y);
+            amax = fmaxf(amax, fmaxf(fabsf(v[e]), fabsf(v[e + 1])));
+          }
+          store_bf16x32(static_cast<__nv_bfloat16*>(p.out) + (size_t)row * p.N + col0, v, valid);
+        } else if (kEpi == EPI_RESID) {
+          __nv_bfloat16* xdst = static_cast<__nv_bfloat16*>(p.out) + (size_t)row * p.N + col0;
+          const float* gsrc = gate_uniform ? &ec.gate[i * 32] : p.gate + (size_t)item * p.gate_stride + col0;
 #pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        if (g * 8 >= valid) break;
-        const uint4 xv = xp[(c - c_begin) * 4 + g];
-        const float4 ga = __ldg(g4 + 2 * g), gb = __ldg(g4 + 2 * g + 1);
-        const float gg[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
-        const uint32_t xu[4] = {xv.x, xv.y, xv.z, xv.w};
+          for (int g = 0; g < 4; ++g) {
+            if (g * 8 >= valid) break;
+            const uint4 xv = xp[i * 4 + g];
+            float4 ga, gb;
+            if (gate_uniform) {
+              ga = *reinterpret_cast<const float4*>(gsrc + 8 * g);
+              gb = *reinterpret_cast<const float4*>(gsrc + 8 * g + 4);
+            } else {
+              ga = __ldg(reinterpret_cast<const float4*>(gsrc + 8 * g));
+              gb = __ldg(reinterpret_cast<const float4*>(gsrc + 8 * g + 4));
+            }
+            const float gg[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+            const uint32_t xu[4] = {xv.x, xv.y, xv.z, xv.w};
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          v[8 * g + 2 * e] = fmaf(gg[2 * e], v[8 * g + 2 * e], bf16_lo(xu[e]));
-          v[8 * g + 2 * e + 1] = fmaf(gg[2 * e + 1], v[8 * g + 2 * e + 1], bf16_hi(xu[e]));
+            for (int e = 0; e < 4; ++e) {
+              v[8 * g + 2 * e] = fmaf(gg[2 * e], v[8 * g + 2 * e], bf16_lo(xu[e]));
+              v[8 * g + 2 * e + 1] = fmaf(gg[2 * e + 1], v[8 * g + 2 * e + 1], bf16_hi(xu[e]));
+            }
+          }
+          store_bf16x32(xdst, v, valid);
+        } else if (kEpi == EPI_QKV) {
+          const int part = col0 / p.d;
+          const int rem = col0 - part * p.d;
+          const int head = rem / p.head_dim;
+          const int lane0 = rem - head * p.head_dim;
+          if (part < 2) {
+            const int off_h = p.T * (p.rope_t / 2), off_w = off_h + p.H * (p.rope_h / 2);
+            const int base_t = pt * (p.rope_t / 2), base_h = off_h + ph * (p.rope_h / 2) - p.rope_t / 2,
+                      base_w = off_w + pw * (p.rope_w / 2) - (p.rope_t + p.rope_h) / 2;
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const int pl = lane0 + 2 * e;
+              const int idx = (pl < p.rope_t ? base_t : (pl < p.rope_t + p.rope_h ? base_h : base_w)) + (pl >> 1);
+              const float2 cs = rope_s[idx];
+              const float x0 = v[2 * e], x1 = v[2 * e + 1];
+              v[2 * e] = x0 * cs.x - x1 * cs.y;
+              v[2 * e + 1] = x0 * cs.y + x1 * cs.x;
+            }
+          }
+          __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.out) +
+                               ((((size_t)part * p.B + item) * p.n_heads + head) * p.L + l) * p.head_dim + lane0;
+          store_bf16x32(dst, v, 32);
         }
       }
-      store_bf16x32(xdst, v, valid);
-    } else if (kEpi == EPI_QKV) {
-      const int part = col0 / p.d;
-      const int rem = col0 - part * p.d;
-      const int head = rem / p.head_dim;
-      const int lane0 = rem - head * p.head_dim;
-      if (part < 2) {
-        const int off_h = p.T * (p.rope_t / 2), off_w = off_h + p.H * (p.rope_h / 2);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int pl = lane0 + 2 * i;
-          int idx;
-          if (pl < p.rope_t) idx = pt * (p.rope_t / 2) + pl / 2;
-          else if (pl < p.rope_t + p.rope_h) idx = off_h + ph * (p.rope_h / 2) + (pl - p.rope_t) / 2;
-          else idx = off_w + pw * (p.rope_w / 2) + (pl - p.rope_t - p.rope_h) / 2;
-          const float2 cs = __ldg(p.rope + idx);
-          const float x0 = v[2 * i], x1 = v[2 * i + 1];
-          v[2 * i] = x0 * cs.x - x1 * cs.y;
-          v[2 * i + 1] = x0 * cs.y + x1 * cs.x;
-        }
-      }
-      __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.out) +
-                           ((((size_t)part * p.B + item) * p.n_heads + head) * p.L + l) * p.head_dim + lane0;
-      store_bf16x32(dst, v, 32);
+    }
+    if (next) {
+      if (!kDoubleBuffer) tmem_ld32(tbase + (i + 1) * 32, r[0]);
+      tmem_ld_wait();
+      tmem_reg_fence(r[kDoubleBuffer ? ((i + 1) & 1) : 0]);
     }
   }
   if (kEpi == EPI_GELU && row_ok)
@@ -225,6 +277,8 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kBars);
+  EpiConst* epi_const = reinterpret_cast<EpiConst*>(smem + CONST_OFF);
+  float2* rope_smem = reinterpret_cast<float2*>(smem + ROPE_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const uint32_t sbase = smem_u32(smem);
   const uint32_t bar0 = smem_u32(bars);
@@ -249,6 +303,8 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) { tma_prefetch_desc(&tmA); tma_prefetch_desc(&tmB); }
+  if (kEpi == EPI_QKV)  // the whole RoPE table, once per CTA, when the launcher reserved room for it
+    for (int i = threadIdx.x; i < p.rope_smem_entries; i += blockDim.x) rope_smem[i] = __ldg(p.rope + i);
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
     tmem_relinquish();
@@ -341,14 +397,23 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
       const int acc = tl & 1;
       const uint32_t aph = (tl >> 1) & 1;
       const int row = mb * BM + quad * 32 + lane;
+      const int n0 = nb * BN + half * (BN / 2);
+      EpiConst& ec = epi_const[warp - 2];
+      // this warp finished its previous tile, so its constants buffer is free
+      stage_constants<kInt8, kEpi>(p, ec, n0, mb * BM + quad * 32, lane);
+      const int first_row = min(mb * BM + quad * 32, p.M - 1), last_row = min(mb * BM + quad * 32 + 31, p.M - 1);
+      const bool gate_uniform = kEpi == EPI_RESID && first_row / p.rows_per_item == last_row / p.rows_per_item;
       uint4 xp[kResidVecs];
-      if (kEpi == EPI_RESID) prefetch_resid(p, row, nb * BN + half * (BN / 2), xp);
+      if (kEpi == EPI_RESID) prefetch_resid(p, row, n0, xp);
+      __syncwarp();
       // tcgen05.ld is warp-collective: the wait outcome is made warp-uniform.
       const bool t_ok = !*abort_flag && mbar_wait(tfull(acc), aph, p.err, ERR_WAIT_MMA);
       if (!__all_sync(0xFFFFFFFFu, t_ok)) { *abort_flag = 1; break; }
       tc_fence_after();
-      const uint32_t tbase = tmem_base + ((uint32_t)(quad * 32) << 16) + acc * BN;
-      epilogue_tile<kInt8, kEpi>(p, tbase, row, row < p.M, nb * BN, half * (BN / 64), (half + 1) * (BN / 64), xp);
+      // this warp's 32 lanes and 128 columns of the accumulator
+      const uint32_t tbase = tmem_base + ((uint32_t)(quad * 32) << 16) + acc * BN + half * (BN / 2);
+      epilogue_tile<kInt8, kEpi>(p, tbase, row, row < p.M, n0, ec, gate_uniform,
+                                 p.rope_smem_entries > 0 ? rope_smem : p.rope, xp);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(tempty(acc));
@@ -366,9 +431,10 @@ template <bool kInt8, int kEpi>
 static cudaError_t launch_one(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& a,
                               int grid, cudaStream_t st) {
   auto k = gemm_kernel<kInt8, kEpi>;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gemm::SMEM_BYTES);
+  const size_t smem = gemm::SMEM_BASE + (size_t)a.rope_smem_entries * sizeof(float2);
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gemm::kSmemMax);
   if (e != cudaSuccess) return e;
-  k<<<grid, gemm::kThreads, gemm::SMEM_BYTES, st>>>(ta, tb, a);
+  k<<<grid, gemm::kThreads, smem, st>>>(ta, tb, a);
   return cudaGetLastError();
 }
 
@@ -389,6 +455,11 @@ cudaError_t launch_gemm(bool int8_operands, GemmEpilogue epi, const void* A, con
   // Raster: keep either a band of A stripes or a band of W slices resident in L2,
   // whichever makes the other operand's repeated streaming cheaper.
   GemmArgs args = a;
+  args.rope_smem_entries = 0;
+  if (epi == EPI_QKV && a.rope) {
+    const int entries = a.T * (a.rope_t / 2) + a.H * (a.rope_h / 2) + a.W * (a.rope_w / 2);
+    if (entries <= kRopeSmemMaxEntries) args.rope_smem_entries = entries;
+  }
   {
     const double stripe_a = (double)BM * a.K * eb, slice_w = (double)BN * a.K * eb;
     const double bytes_a = (double)a.M * a.K * eb, bytes_w = (double)a.N * a.K * eb;
