@@ -158,13 +158,13 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
       for (int j = 0; j < nkv && ok; ++j) {
         const int s = j & 1;
         const uint32_t ph = (j >> 1) & 1;
-        if (*abort_flag || !mbar_wait(k_empty(s), ph ^ 1u, a.err, ERR_WAIT_MMA)) { ok = false; break; }
+        if (!mbar_wait_or_abort(k_empty(s), ph ^ 1u, abort_flag, a.err, ERR_WAIT_MMA)) { ok = false; break; }
         mbar_arrive_expect_tx(k_full(s), Lay::TILE);
         for (int b = 0; b < Lay::NBOX; ++b)
           tma_load_3d(sb0 + Lay::K_OFF + s * Lay::TILE + b * BOX, &tm, k_full(s), b * 64, j * BKV, BH + bh);
         filled |= 1u << s;
         fill_ph = (fill_ph & ~(1u << s)) | (ph << s);
-        if (*abort_flag || !mbar_wait(v_empty(s), ph ^ 1u, a.err, ERR_WAIT_MMA)) { ok = false; break; }
+        if (!mbar_wait_or_abort(v_empty(s), ph ^ 1u, abort_flag, a.err, ERR_WAIT_MMA)) { ok = false; break; }
         mbar_arrive_expect_tx(v_full(s), Lay::TILE);
         for (int b = 0; b < Lay::NBOX; ++b)
           tma_load_3d(sb0 + Lay::V_OFF + s * Lay::TILE + b * BOX, &tm, v_full(s), b * 64, j * BKV, 2 * BH + bh);
@@ -191,7 +191,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
       bool any = false;
       auto issue_s = [&](int g, int j) -> bool {  // S_g(j) = Q_g K_j^T
         const int s = j & 1;
-        if (g == 0 && (*abort_flag || !mbar_wait(k_full(s), (j >> 1) & 1, a.err, ERR_WAIT_TMA))) return false;
+        if (g == 0 && !mbar_wait_or_abort(k_full(s), (j >> 1) & 1, abort_flag, a.err, ERR_WAIT_TMA)) return false;
         tc_fence_after();
         const uint32_t q_addr = sb0 + Lay::Q_OFF + g * Lay::TILE;
         const uint32_t k_addr = sb0 + Lay::K_OFF + s * Lay::TILE;
@@ -209,8 +209,8 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
       };
       auto issue_pv = [&](int g, int j) -> bool {  // O_g += P_g(j) V_j
         const int s = j & 1;
-        if (*abort_flag || !mbar_wait(p_full(g), j & 1, a.err, ERR_WAIT_EPI)) return false;
-        if (g == 0 && !mbar_wait(v_full(s), (j >> 1) & 1, a.err, ERR_WAIT_TMA)) return false;
+        if (!mbar_wait_or_abort(p_full(g), j & 1, abort_flag, a.err, ERR_WAIT_EPI)) return false;
+        if (g == 0 && !mbar_wait_or_abort(v_full(s), (j >> 1) & 1, abort_flag, a.err, ERR_WAIT_TMA)) return false;
         tc_fence_after();
         const uint32_t v_addr = sb0 + Lay::V_OFF + s * Lay::TILE;
         const uint32_t o_col = g == 0 ? Lay::O_COL0 : Lay::O_COL1;
@@ -256,7 +256,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
     float m_run = -INFINITY, l_run = 0.0f;
     bool ok = true;
     for (int j = 0; j < nkv; ++j) {
-      const bool s_ok = !*abort_flag && mbar_wait(s_full(g), j & 1, a.err, ERR_WAIT_MMA);
+      const bool s_ok = mbar_wait_or_abort(s_full(g), j & 1, abort_flag, a.err, ERR_WAIT_MMA);
       if (!__all_sync(0xFFFFFFFFu, s_ok)) { ok = false; break; }
       tc_fence_after();
       uint32_t sr[BKV];
@@ -336,7 +336,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(p_full(g));
     }
-    const bool f_ok = ok && mbar_wait(fin(g), 0, a.err, ERR_WAIT_MMA);
+    const bool f_ok = ok && mbar_wait_or_abort(fin(g), 0, abort_flag, a.err, ERR_WAIT_MMA);
     if (__all_sync(0xFFFFFFFFu, f_ok)) {
       tc_fence_after();
       const int q = qt * 2 * BQ + g * BQ + row;

@@ -325,7 +325,7 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
         int mb, nb;
         tile_coords(t, n_m, n_n, p.raster_n, p.group, mb, nb);
         for (int kb = 0; kb < nk; ++kb) {
-          if (*abort_flag || !mbar_wait(empty(s), ph ^ 1u, p.err, ERR_WAIT_MMA)) { ok = false; break; }
+          if (!mbar_wait_or_abort(empty(s), ph ^ 1u, abort_flag, p.err, ERR_WAIT_MMA)) { ok = false; break; }
           mbar_arrive_expect_tx(full(s), STAGE_BYTES);
           const uint32_t a_dst = sbase + s * STAGE_BYTES;
           tma_load_2d(a_dst, &tmA, full(s), kb * BKE, mb * BM);
@@ -356,11 +356,11 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
       for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++tl) {
         const int acc = tl & 1;
         const uint32_t aph = (tl >> 1) & 1;
-        if (*abort_flag || !mbar_wait(tempty(acc), aph ^ 1u, p.err, ERR_WAIT_EPI)) { ok = false; break; }
+        if (!mbar_wait_or_abort(tempty(acc), aph ^ 1u, abort_flag, p.err, ERR_WAIT_EPI)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
         for (int kb = 0; kb < nk; ++kb) {
-          if (*abort_flag || !mbar_wait(full(s), ph, p.err, ERR_WAIT_TMA)) { ok = false; break; }
+          if (!mbar_wait_or_abort(full(s), ph, abort_flag, p.err, ERR_WAIT_TMA)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a_addr = sbase + s * STAGE_BYTES;
 #pragma unroll
@@ -407,7 +407,7 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
       if (kEpi == EPI_RESID) prefetch_resid(p, row, n0, xp);
       __syncwarp();
       // tcgen05.ld is warp-collective: the wait outcome is made warp-uniform.
-      const bool t_ok = !*abort_flag && mbar_wait(tfull(acc), aph, p.err, ERR_WAIT_MMA);
+      const bool t_ok = mbar_wait_or_abort(tfull(acc), aph, abort_flag, p.err, ERR_WAIT_MMA);
       if (!__all_sync(0xFFFFFFFFu, t_ok)) { *abort_flag = 1; break; }
       tc_fence_after();
       // this warp's 32 lanes and 128 columns of the accumulator
