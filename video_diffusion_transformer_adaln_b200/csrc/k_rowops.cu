@@ -183,6 +183,14 @@ __device__ __forceinline__ float max3f_row(float a, float b, float c) {
 
 constexpr int kLnMaxWarps = 32;
 
+// 16-byte asynchronous copy global -> shared (L2 only), and the wait for all of
+// this thread's outstanding copies.
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
 // Lane-wise max of two bf16 pairs (both non-negative here).
 __device__ __forceinline__ uint32_t bf16x2_max(uint32_t a, uint32_t b) {
   uint32_t r;
@@ -197,6 +205,8 @@ __global__ void __launch_bounds__(1024, 1) ln_mod_quant_kernel(
     float* __restrict__ s, __nv_bfloat16* __restrict__ h_out, float* __restrict__ absmax_zero,
     int write_codes) {
   extern __shared__ float4 modp[];  // [4][vpr]: (1+sc[2c], 1+sc[2c+1], sh[2c], sh[2c+1]), c = 4 vec + e
+  // then the staging rows of the next pass: [rpp][vpr] 16-byte vectors, each written and read
+  // back by the same thread (cp.async), so no barrier guards them
   __shared__ float red[2][3][kLnMaxWarps];
   const int tpr = vpr / VPT;
   const int rpp = blockDim.x / tpr;
@@ -210,6 +220,17 @@ __global__ void __launch_bounds__(1024, 1) ln_mod_quant_kernel(
   const unsigned total = (unsigned)items * gpi;  // passes; at most rows, so 32 bits suffice
   int cur = -1, par = 0;
   unsigned item = blockIdx.x / gpi, g_in = blockIdx.x % gpi;  // pass = (item, pass within item)
+  uint4* stage = reinterpret_cast<uint4*>(modp + 4 * vpr) + (size_t)sub * vpr;
+  // this thread's vectors of its row in pass (it, gi) -> staging, when that row exists
+  auto prefetch = [&](unsigned gg, unsigned it, unsigned gi) {
+    const int r = (int)gi * rpp + sub, rw = (int)it * rows_per_item + r;
+    if (gg >= total || r >= rows_per_item || rw >= rows) return;
+    const uint4* src = reinterpret_cast<const uint4*>(x) + (size_t)rw * vpr;
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) cp_async16(stage + t + tpr * i, src + t + tpr * i);
+  };
+  prefetch(blockIdx.x, item, g_in);
+  cp_async_commit();
   for (unsigned g = blockIdx.x; g < total; g += gridDim.x) {
     if ((int)item != cur) {  // block-uniform
       __syncthreads();
@@ -225,10 +246,10 @@ __global__ void __launch_bounds__(1024, 1) ln_mod_quant_kernel(
     const int r_in = (int)g_in * rpp + sub;
     const int row = (int)item * rows_per_item + r_in;
     const bool valid = r_in < rows_per_item && row < rows;
-    const uint4* xr = reinterpret_cast<const uint4*>(x) + (size_t)(valid ? row : 0) * vpr;
+    cp_async_wait_all();
     uint4 v[VPT];
 #pragma unroll
-    for (int i = 0; i < VPT; ++i) v[i] = valid ? __ldcs(xr + t + tpr * i) : make_uint4(0, 0, 0, 0);
+    for (int i = 0; i < VPT; ++i) v[i] = valid ? stage[t + tpr * i] : make_uint4(0, 0, 0, 0);
 
     float* rd = red[par][0];
     par ^= 1;
@@ -241,6 +262,12 @@ __global__ void __launch_bounds__(1024, 1) ln_mod_quant_kernel(
       f[4 * i + 2] = bf16x2_to_f2(v[i].z);
       f[4 * i + 3] = bf16x2_to_f2(v[i].w);
     }
+    // the staged vectors are in registers now: start the next pass's loads
+    unsigned n_in = g_in + gridDim.x;
+    const unsigned n_item = item + n_in / gpi;
+    n_in %= gpi;
+    prefetch(g + gridDim.x, n_item, n_in);
+    cp_async_commit();
     float2 acc = f[0];
 #pragma unroll
     for (int e = 1; e < VPT * 4; ++e) acc = __fadd2_rn(acc, f[e]);
@@ -312,14 +339,15 @@ __global__ void __launch_bounds__(1024, 1) ln_mod_quant_kernel(
         }
       }
     }
-    g_in += gridDim.x;
-    item += g_in / gpi;
-    g_in %= gpi;
+    item = n_item;
+    g_in = n_in;
   }
+  cp_async_wait_all();
 }
 
 // Per-row quantization with each row's absmax already known: a block covers
-// whole rows (rpb rows of vpr 16-byte vectors, rpb * vpr <= 1024, rpb <= 32),
+// whole rows (rpb rows of vpr 16-byte vectors, rpb * vpr <= 4096 unless one row is longer,
+// rpb <= 32),
 // each thread keeps up to four vectors in flight; each row's scale and its
 // reciprocal are derived once, into shared memory.
 constexpr int kQuantMaxRowsPerBlock = 32;
@@ -343,6 +371,8 @@ __global__ void __launch_bounds__(256) quant_rows_known_absmax_kernel(const __nv
   const unsigned span = nr * (unsigned)vpr;  // vectors covered by this block
   const size_t base = (size_t)row0 * vpr;
   __syncthreads();
+  // row of vector k, advanced incrementally (k only grows): r = k / vpr without a division
+  unsigned r = 0, row_end = (unsigned)vpr;
   for (unsigned k0 = threadIdx.x; k0 < span; k0 += U * blockDim.x) {
     uint4 raw[U];
 #pragma unroll
@@ -354,7 +384,10 @@ __global__ void __launch_bounds__(256) quant_rows_known_absmax_kernel(const __nv
     for (int u = 0; u < U; ++u) {
       const unsigned k = k0 + u * blockDim.x;
       if (k >= span) break;
-      const unsigned r = rpb == 1 ? 0u : k / vpr;
+      while (k >= row_end) {
+        ++r;
+        row_end += (unsigned)vpr;
+      }
       const float2 sr = srow[r];
       uint2 code;
       float worst = 1.0f;
@@ -574,13 +607,14 @@ static cudaError_t ln_dispatch(const void* x, int rows, int nv, float eps, const
   const int vpr = 32 * nv;
   const int tpr = vpr / VPT;
   const int block = tpr * (tpr >= 256 ? 1 : 256 / tpr);
-  const size_t smem = (size_t)vpr * 4 * sizeof(float4);
+  const int rpp_d = block / tpr;
+  const size_t smem = (size_t)vpr * 4 * sizeof(float4) + (size_t)rpp_d * vpr * sizeof(uint4);
   auto kern = ln_mod_quant_kernel<VPT>;
   static int attr_done = 0;
   if (!attr_done) {
-    // the largest row (d = 8192, 1024 vectors) needs 64 KB of (1 + scale, shift) pairs
+    // the largest row (d = 8192, 1024 vectors): 64 KB of (1 + scale, shift) pairs + 16 KB staging
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)(32 * 32 * 4 * sizeof(float4)));
+                                         (int)(32 * 32 * 4 * sizeof(float4) + 32 * 32 * sizeof(uint4)));
     if (e != cudaSuccess) return e;
     attr_done = 1;
   }
@@ -621,7 +655,9 @@ cudaError_t launch_quant_rows_bf16(const void* h, int rows, int cols, const floa
   if (rows == 0) return cudaSuccess;
   if (absmax) {
     const int vpr = cols / 8;
-    int rpb = 1024 / vpr;
+    // about 4096 vectors (64 KB of input) per block: each thread keeps four 16-byte loads in
+    // flight over four rounds, and the per-block setup is amortized over several rows
+    int rpb = 4096 / vpr;
     rpb = rpb < 1 ? 1 : (rpb > kQuantMaxRowsPerBlock ? kQuantMaxRowsPerBlock : rpb);
     quant_rows_known_absmax_kernel<<<(rows + rpb - 1) / rpb, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(h),
                                                                           rows, vpr, rpb, absmax, q, s);
