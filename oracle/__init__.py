@@ -227,6 +227,7 @@ class Dims:
     rope_theta: float = 10000.0
     ln_eps: float = 1e-6
     qkv_int8: bool = True
+    wo_bf16: bool = False
 
     @property
     def L(self):
@@ -237,13 +238,14 @@ class _CDims(C.Structure):
     _fields_ = [("B", C.c_int64), ("T", C.c_int64), ("H", C.c_int64), ("W", C.c_int64),
                 ("d", C.c_int64), ("n_heads", C.c_int64), ("head_dim", C.c_int64), ("d_ff", C.c_int64),
                 ("rope_t", C.c_int), ("rope_h", C.c_int), ("rope_w", C.c_int),
-                ("rope_theta", C.c_double), ("ln_eps", C.c_double), ("qkv_int8", C.c_int)]
+                ("rope_theta", C.c_double), ("ln_eps", C.c_double), ("qkv_int8", C.c_int),
+                ("wo_bf16", C.c_int)]
 
 
 class _CWeights(C.Structure):
     _fields_ = [(n, C.c_void_p) for n in
                 ("w_ada", "b_ada", "wqkv", "sqkv", "wqkv_bf16", "bqkv", "wo", "so", "bo",
-                 "w1", "s1", "b1", "w2", "s2", "b2")]
+                 "w1", "s1", "b1", "w2", "s2", "b2", "wo_bf16")]
 
 
 class _CTrace(C.Structure):
@@ -253,7 +255,7 @@ class _CTrace(C.Structure):
 _WEIGHT_DTYPES = {"w_ada": np.uint16, "b_ada": np.float32, "wqkv": np.int8, "sqkv": np.float32,
                   "wqkv_bf16": np.uint16, "bqkv": np.float32, "wo": np.int8, "so": np.float32,
                   "bo": np.float32, "w1": np.int8, "s1": np.float32, "b1": np.float32,
-                  "w2": np.int8, "s2": np.float32, "b2": np.float32}
+                  "w2": np.int8, "s2": np.float32, "b2": np.float32, "wo_bf16": np.uint16}
 
 
 def block_forward(dims: Dims, weights: dict, c, x_bf16, rows: Optional[np.ndarray] = None,
@@ -273,7 +275,7 @@ def block_forward(dims: Dims, weights: dict, c, x_bf16, rows: Optional[np.ndarra
             setattr(cw, name, a.ctypes.data)
     cd = _CDims(dims.B, dims.T, dims.H, dims.W, d, dims.n_heads, dims.head_dim, F,
                 dims.rope[0], dims.rope[1], dims.rope[2], dims.rope_theta, dims.ln_eps,
-                1 if dims.qkv_int8 else 0)
+                1 if dims.qkv_int8 else 0, 1 if dims.wo_bf16 else 0)
     x = _c(x_bf16, np.uint16).reshape(R, d)
     c = _c(c, np.float32).reshape(dims.B, d)
     if rows is None:

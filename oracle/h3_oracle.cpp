@@ -373,6 +373,7 @@ typedef struct {
   int rope_t, rope_h, rope_w;
   double rope_theta, ln_eps;
   int qkv_int8;                // 1: int8 QKV (default); 0: bf16 QKV
+  int wo_bf16;                 // 0: int8 Wo (default); 1: bf16 Wo on the bf16 attention output
 } orc_dims;
 
 typedef struct {
@@ -383,6 +384,7 @@ typedef struct {
   const int8_t* wo; const float* so; const float* bo;  // [d][d]
   const int8_t* w1; const float* s1; const float* b1;  // [d_ff][d]
   const int8_t* w2; const float* s2; const float* b2;  // [d][d_ff]
+  const uint16_t* wo_bf16;                             // bf16 [d][d] (wo_bf16 == 1)
 } orc_weights;
 
 // Optional intermediate dumps (each pointer may be NULL).
@@ -406,7 +408,8 @@ typedef struct {
 //   h1  = bf16(LN(x) * (1 + scale_a) + shift_a);  A1, s1 = quant(h1)
 //   QKV = deq(A1 Wqkv^T) + b;  RoPE(Q), RoPE(K)   (or bf16 h1 @ bf16 Wqkv^T)
 //   O   = attention(Q, K, V);  A2, s2 = quant(bf16(O))
-//   x1  = x + gate_a * (deq(A2 Wo^T) + bo)
+//   x1  = x + gate_a * (deq(A2 Wo^T) + bo)     (or bf16(O) @ bf16 Wo^T + bo: the
+//         BF16 attention-output projection of [README] "Metal 4 및 TensorOps")
 //   h2  = bf16(LN(x1) * (1 + scale_m) + shift_m);  A3, s3 = quant(h2)
 //   G   = GELU(deq(A3 W1^T) + b1);  A4, s4 = quant(bf16(G))
 //   out = x1 + gate_m * (deq(A4 W2^T) + b2)
@@ -491,16 +494,26 @@ int orc_block_forward(const orc_dims* dm, const orc_weights* wt, const float* c,
   }
   if (tr && tr->attn) std::memcpy(tr->attn, O.data(), O.size() * sizeof(double));
 
-  // Attention output projection with gated residual.
+  // Attention output projection with gated residual. O is rounded to bf16 either way.
   std::vector<float> Of((size_t)(n_rows * d));
   for (int64_t i = 0; i < n_rows * d; ++i) Of[(size_t)i] = (float)orc_bf16_to_f64(orc_f64_to_bf16(O[(size_t)i]));
-  std::vector<int8_t> A2((size_t)(n_rows * d));
-  std::vector<float> s2((size_t)n_rows);
-  orc_quantize_rows(Of.data(), n_rows, d, A2.data(), s2.data());
-  std::vector<int32_t> acc2((size_t)(n_rows * d));
-  overflow += orc_gemm_i8(A2.data(), wt->wo, n_rows, d, d, acc2.data());
   std::vector<double> yo((size_t)(n_rows * d));
-  orc_dequant(acc2.data(), n_rows, d, s2.data(), wt->so, wt->bo, yo.data());
+  if (!dm->wo_bf16) {
+    std::vector<int8_t> A2((size_t)(n_rows * d));
+    std::vector<float> s2((size_t)n_rows);
+    orc_quantize_rows(Of.data(), n_rows, d, A2.data(), s2.data());
+    std::vector<int32_t> acc2((size_t)(n_rows * d));
+    overflow += orc_gemm_i8(A2.data(), wt->wo, n_rows, d, d, acc2.data());
+    orc_dequant(acc2.data(), n_rows, d, s2.data(), wt->so, wt->bo, yo.data());
+  } else {
+    std::vector<double> od((size_t)(n_rows * d)), wd((size_t)(d * d));
+    for (int64_t i = 0; i < n_rows * d; ++i) od[(size_t)i] = (double)Of[(size_t)i];
+    orc_bf16_decode(wt->wo_bf16, d * d, wd.data());
+    orc_gemm_f64(od.data(), wd.data(), n_rows, d, d, yo.data());
+    if (wt->bo)
+      for (int64_t r = 0; r < n_rows; ++r)
+        for (int64_t o = 0; o < d; ++o) yo[(size_t)(r * d + o)] += wt->bo[o];
+  }
   std::vector<double> x1((size_t)(n_rows * d));
   for (int64_t i = 0; i < n_rows; ++i) {
     const int64_t r = sel[(size_t)i], b = r / L;

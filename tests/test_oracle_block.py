@@ -26,12 +26,14 @@ def _weights(wl, block=0, zero_gates=False):
         w[name], w[sname] = O.quantize_rows(raw[name])
     if "wqkv_bf16" in raw:
         w["wqkv_bf16"] = raw["wqkv_bf16"]
+    if "wo_bf16" in raw:
+        w["wo_bf16"] = raw["wo_bf16"]
     return w
 
 
 def _dims(wl):
     return O.Dims(wl.B, wl.T, wl.H, wl.W, wl.d, wl.n_heads, wl.head_dim, wl.d_ff, wl.rope,
-                  wl.rope_theta, wl.ln_eps, wl.qkv_int8)
+                  wl.rope_theta, wl.ln_eps, wl.qkv_int8, wl.wo_bf16)
 
 
 def test_zero_gates_give_exact_identity():
@@ -105,3 +107,23 @@ def test_bf16_qkv_variant_runs_and_differs_slightly():
     xd = O.bf16_decode(x).reshape(-1, wl.d)
     rel = np.linalg.norm((a - xd) - (b - xd)) / np.linalg.norm(a - xd)
     assert 0 < rel < 0.1  # int8 vs bf16 QKV: close but not identical deltas
+
+
+def test_bf16_wo_projection_is_the_plain_product():
+    """bf16 output projection ([README] "Metal 4 및 TensorOps": BF16 for the attention-output
+    projection): x1 = x + gate_a * (bf16(O) @ bf16(Wo)^T), checked against a numpy product."""
+    wl = WL.with_(wo_bf16=True)
+    raw = synth.block_weights(wl)
+    w = _weights(wl)
+    x, c = synth.x_input(wl), synth.cond(wl)
+    out, tr = O.block_forward(_dims(wl), w, c, x, trace=True)
+    d = wl.d
+    ob = O.bf16_decode(O.bf16_round(tr["attn"]))
+    wo = O.bf16_decode(raw["wo_bf16"]).reshape(d, d)
+    expect = O.bf16_decode(x).reshape(-1, d) + tr["mod"][0, 2 * d:3 * d] * np.dot(ob, wo.T)
+    assert np.max(np.abs(tr["x1"] - expect)) <= 1e-12 * np.max(np.abs(expect))
+    # the int8 projection of the same draws is close but not the same
+    out8 = O.block_forward(_dims(WL), _weights(WL), c, x)
+    xd = O.bf16_decode(x).reshape(-1, d)
+    rel = np.linalg.norm((out - xd) - (out8 - xd)) / np.linalg.norm(out8 - xd)
+    assert 0 < rel < 0.1
