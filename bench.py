@@ -88,7 +88,7 @@ def _block_kernel_work(name, wl, L):
     if name == "gemm_qkv":
         return 2.0 * R * 3 * d * d, "op", "tensor_i8" if wl.qkv_int8 else "tensor_bf16"
     if name == "gemm_wo":
-        return 2.0 * R * d * d, "op", "tensor_i8"
+        return 2.0 * R * d * d, "op", "tensor_bf16" if wl.wo_bf16 else "tensor_i8"
     if name in ("gemm_w1", "gemm_w2"):
         return 2.0 * R * d * F, "op", "tensor_i8"
     if name == "attention":
@@ -227,9 +227,11 @@ class OracleRunner:
             w[name], w[sname] = O.quantize_rows(raw[name])
         if not wl.qkv_int8:
             w["wqkv_bf16"] = raw["wqkv_bf16"]
+        if wl.wo_bf16:
+            w["wo_bf16"] = raw["wo_bf16"]
         self.w = w
         self.dm = O.Dims(wl.B, wl.T, wl.H, wl.W, wl.d, wl.n_heads, wl.head_dim, wl.d_ff, wl.rope,
-                         wl.rope_theta, wl.ln_eps, wl.qkv_int8)
+                         wl.rope_theta, wl.ln_eps, wl.qkv_int8, wl.wo_bf16)
         self.R = wl.B * wl.L
         self.t_kv = None
 
@@ -425,7 +427,8 @@ def run_h3b(args, rank, world, local):
                    "d": wl.d, "heads": wl.n_heads, "head_dim": wl.head_dim, "d_ff": wl.d_ff,
                    "blocks_per_step": wl.n_blocks, "token_pair": wl.token_pair,
                    "paired_blocks": list(wl.pair_blocks),
-                   "qkv": "int8" if wl.qkv_int8 else "bf16", "attention": "bf16",
+                   "qkv": "int8" if wl.qkv_int8 else "bf16", "wo": "bf16" if wl.wo_bf16 else "int8",
+                   "attention": "bf16",
                    "l2": "flushed between steps (512 MiB write outside the timed events)",
                    "parallelism": "replicas: one independent latent per GPU, no collective"},
         "roofline": roof, "kernel_share": shares, "kernel_roofline": all_roof,

@@ -76,13 +76,19 @@ typedef enum {
  *   [0,rope_t) rotate with t, the next rope_h with h, the rest with w; pair
  *   (2j, 2j+1) of a segment of length r has frequency rope_theta^(-2j/r)).
  *   ln_eps: LayerNorm epsilon (no affine, biased variance).
- *   qkv_int8: 1 = int8 QKV projection (default), 0 = bf16 QKV projection. */
+ *   qkv_int8: 1 = int8 QKV projection (default), 0 = bf16 QKV projection.
+ *   wo_bf16:  0 = int8 output projection on the quantized attention output
+ *             (default), 1 = bf16 output projection on the bf16 attention output
+ *             (the BF16 attention-output projection of the pages' tensor path,
+ *             "h3-metal: Apple Silicon을 위한 네이티브 MiniMax-H3 추론",
+ *             section "Metal 4 및 TensorOps"); the quant_o pass is skipped. */
 typedef struct {
   int B, T, H, W;
   int d, n_heads, head_dim, d_ff;
   int rope_t, rope_h, rope_w;
   float rope_theta, ln_eps;
   int qkv_int8;
+  int wo_bf16;
 } h3b_dims;
 
 /* Weights of one block (device pointers). int8 codes with one F32 scale per
@@ -96,15 +102,17 @@ typedef struct {
  *   wqkv_bf16 bf16 [3d][d]                    (qkv_int8 == 0)
  *   bqkv      fp32 [3d]; output channel o -> part o/d (Q, K, V),
  *             head (o % d)/head_dim, lane o % head_dim
- *   wo int8 [d][d]       + so fp32 [d],    bo fp32 [d]
+ *   wo int8 [d][d]       + so fp32 [d],    bo fp32 [d]   (wo/so when wo_bf16 == 0)
  *   w1 int8 [d_ff][d]    + s1 fp32 [d_ff], b1 fp32 [d_ff]
- *   w2 int8 [d][d_ff]    + s2 fp32 [d],    b2 fp32 [d] */
+ *   w2 int8 [d][d_ff]    + s2 fp32 [d],    b2 fp32 [d]
+ *   wo_bf16 bf16 [d][d]                                 (wo_bf16 == 1) */
 typedef struct {
   const void* w_ada; const float* b_ada;
   const int8_t* wqkv; const float* sqkv; const void* wqkv_bf16; const float* bqkv;
   const int8_t* wo; const float* so; const float* bo;
   const int8_t* w1; const float* s1; const float* b1;
   const int8_t* w2; const float* s2; const float* b2;
+  const void* wo_bf16;
 } h3b_block_weights;
 
 H3B_API const char* h3b_status_string(h3b_status s);
@@ -280,6 +288,16 @@ H3B_API h3b_status h3b_gemm_i8_gated_residual(const int8_t* A, const float* sA, 
                                       const float* sW, const float* bias, const float* gate,
                                       int rows_per_item, int gate_stride, void* x, int M, int N,
                                       int K, h3b_stream stream);
+
+/* bf16 GEMM with gated residual epilogue, in place on x bf16 [M][N]:
+ *   x[m][n] = bf16(x[m][n] + gate[m / rows_per_item][n] * (sum_k A[m][k] W[n][k] + bias[n]))
+ * A bf16 [M][K], W bf16 [N][K] (fp32 accumulation); gate as above. The output
+ * projection of the block when dims->wo_bf16 == 1. Same argument rules as
+ * h3b_gemm_i8_gated_residual (N, K positive multiples of 16; 16-byte aligned
+ * pointers). */
+H3B_API h3b_status h3b_gemm_bf16_gated_residual(const void* A, const void* W, const float* bias,
+                                                const float* gate, int rows_per_item, int gate_stride,
+                                                void* x, int M, int N, int K, h3b_stream stream);
 
 /* int8 GEMM with GELU epilogue: g bf16 [M][N] = bf16(GELU_tanh(C*sA[m]*sW[n] + bias[n]));
  * absmax fp32 [M] max-combined with each row's max |g| (zero it first). */

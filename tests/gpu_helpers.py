@@ -59,9 +59,11 @@ def oracle_weights(raw, qkv_int8=True):
         w[name], w[sname] = O.quantize_rows(raw[name])
     if not qkv_int8:
         w["wqkv_bf16"] = raw["wqkv_bf16"]
+    if "wo_bf16" in raw:
+        w["wo_bf16"] = raw["wo_bf16"]
     return w
 
 
 def oracle_dims(wl):
     return O.Dims(wl.B, wl.T, wl.H, wl.W, wl.d, wl.n_heads, wl.head_dim, wl.d_ff, wl.rope, wl.rope_theta,
-                  wl.ln_eps, wl.qkv_int8)
+                  wl.ln_eps, wl.qkv_int8, wl.wo_bf16)

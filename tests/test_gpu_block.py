@@ -110,7 +110,18 @@ def test_block_d2048_sampled():
     no_device_error()
 
 
-@pytest.mark.parametrize("name", ["d5120_L18432", "d5120_L18432_bf16qkv"])
+def test_block_d256_full_bf16_wo():
+    """The block with the bf16 output projection on the bf16 attention output."""
+    wl = synth.WORKLOADS["d256_L512"].with_(wo_bf16=True)
+    raw, c, x = synth.block_weights(wl), synth.cond(wl), synth.x_input(wl)
+    got, blk = _run_gpu_block(wl, raw, c, x)
+    ow = _weights_agree(raw, blk)
+    ref = O.block_forward(oracle_dims(wl), ow, c, x)
+    _compare(got, ref, x)
+    no_device_error()
+
+
+@pytest.mark.parametrize("name", ["d5120_L18432", "d5120_L18432_bf16qkv", "d5120_L18432_bf16wo"])
 def test_block_d5120_sampled(name):
     wl = synth.WORKLOADS[name]
     raw, c, x = synth.block_weights(wl), synth.cond(wl), synth.x_input(wl)

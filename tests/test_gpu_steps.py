@@ -217,6 +217,38 @@ def test_gemm_i8_gated_residual(M, N, K, items):
     no_device_error()
 
 
+@pytest.mark.parametrize("M,N,K,items", [(512, 256, 256, 1), (256, 2048, 2048, 2), (100, 512, 1040, 1)])
+def test_gemm_bf16_gated_residual(M, N, K, items):
+    """bf16 output projection (the block's Wo when wo_bf16 is set) with the gated residual."""
+    r = _rng(M + N + K)
+    a = synth.f32_to_bf16_bits((r.standard_normal((M, K)) * r.uniform(0.1, 3, (M, 1))).astype(np.float32))
+    w = synth.f32_to_bf16_bits((r.standard_normal((N, K)) / np.sqrt(K)).astype(np.float32))
+    bias = r.standard_normal(N).astype(np.float32) * 0.1
+    x = synth.f32_to_bf16_bits(r.standard_normal((M, N)).astype(np.float32))
+    gate = r.standard_normal((items, 2 * N)).astype(np.float32)
+    rpi = (M + items - 1) // items
+    xd = bf16_dev(x)
+    gd = to_dev(gate)
+    h3b.h3b_gemm_bf16_gated_residual(bf16_dev(a), bf16_dev(w), to_dev(bias), gd[:, N:], rpi, 2 * N, xd)
+    ad, wd = O.bf16_decode(a), O.bf16_decode(w)
+    y = O.gemm_f64(ad, wd) + bias
+    g = np.stack([gate[i // rpi, N:] for i in range(M)])
+    ref = O.bf16_decode(x) + g * y
+    got = O.bf16_decode(bf16_host(xd))
+    # one bf16 rounding of the result; fp32 accumulation over K (|error| <= K 2^-24 sum|a w|)
+    # and the fp32 error of x + gate*y relative to the terms' magnitude
+    absum = np.abs(ad) @ np.abs(wd).T + np.abs(bias)
+    terms = np.abs(O.bf16_decode(x)) + np.abs(g * y)
+    bound = 2.0 ** -8 * np.abs(ref) + 2.0 ** -20 * terms + K * 2.0 ** -24 * np.abs(g) * absum + 1e-30
+    assert np.all(np.abs(got - ref) <= bound)
+    # a zero gate leaves x bit-identical
+    xd2 = bf16_dev(x)
+    h3b.h3b_gemm_bf16_gated_residual(bf16_dev(a), bf16_dev(w), to_dev(bias), torch.zeros((items, N), device="cuda"),
+                                     rpi, N, xd2)
+    assert np.array_equal(bf16_host(xd2), x)
+    no_device_error()
+
+
 # ----------------------------------------------------------------------------- QKV + RoPE
 
 def _qkv_reference(wl, A_f32, sA, raw_w):

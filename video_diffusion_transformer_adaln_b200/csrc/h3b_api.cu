@@ -132,10 +132,17 @@ WsLayout ws_layout(const h3b_dims& d) {
 
 h3b_status check_weights(const h3b_dims& d, const h3b_block_weights* w) {
   if (!w) return fail(H3B_ERR_ARG, "weights is NULL");
-  const void* req[] = {w->w_ada, w->wo, w->so, w->w1, w->s1, w->w2, w->s2};
+  const void* req[] = {w->w_ada, w->w1, w->s1, w->w2, w->s2};
   for (const void* p : req) {
     if (!p) return fail(H3B_ERR_ARG, "a required weight pointer is NULL");
     if (!aligned16(p)) return fail(H3B_ERR_ALIGN, "weight pointer not 16-byte aligned");
+  }
+  if (d.wo_bf16) {
+    if (!w->wo_bf16) return fail(H3B_ERR_ARG, "wo_bf16 NULL");
+    if (!aligned16(w->wo_bf16)) return fail(H3B_ERR_ALIGN, "wo_bf16 alignment");
+  } else {
+    if (!w->wo || !w->so) return fail(H3B_ERR_ARG, "wo/so NULL");
+    if (!aligned16(w->wo) || !aligned16(w->so)) return fail(H3B_ERR_ALIGN, "wo/so alignment");
   }
   if (d.qkv_int8) {
     if (!w->wqkv || !w->sqkv) return fail(H3B_ERR_ARG, "wqkv/sqkv NULL");
@@ -252,13 +259,19 @@ h3b_status run_block(const h3b_dims& d, const h3b_block_weights& w, const float*
     AttnArgs a{d.B, L, d.n_heads, d.head_dim, qkv, o, absmax, di.err};
     H3B_CK(launch_attention(a, st), "attention");
   }
-  H3B_CK(launch_quant_rows_bf16(o, R, D, absmax, act, sA, st), "quant_o");
-  // a6: output projection + gated residual (gate_attn = chunk 2)
-  {
+  // a6: output projection + gated residual (gate_attn = chunk 2): int8 on the quantized
+  // attention output (a5), or bf16 directly on the bf16 attention output
+  if (!d.wo_bf16) {
+    H3B_CK(launch_quant_rows_bf16(o, R, D, absmax, act, sA, st), "quant_o");
     GemmArgs a = base_args(R, D, D, di.err);
     a.sA = sA; a.sW = w.so; a.bias = w.bo; a.out = x;
     a.gate = mod + 2 * D; a.rows_per_item = L; a.gate_stride = 6 * D;
     H3B_CK(launch_gemm(true, EPI_RESID, act, w.wo, a, di.sms, st), "gemm_wo");
+  } else {
+    GemmArgs a = base_args(R, D, D, di.err);
+    a.bias = w.bo; a.out = x;
+    a.gate = mod + 2 * D; a.rows_per_item = L; a.gate_stride = 6 * D;
+    H3B_CK(launch_gemm(false, EPI_RESID, o, w.wo_bf16, a, di.sms, st), "gemm_wo");
   }
   // a7: LN + modulation + quantization for the MLP (chunks 3, 4)
   H3B_CK(launch_ln_mod_quant(x, R, D, d.ln_eps, mod + 3 * D, mod + 4 * D, L, 6 * D, act, sA, nullptr, absmax, 1, di.err, di.sms, st), "ln_mod_quant_mlp");
@@ -650,6 +663,23 @@ h3b_status h3b_gemm_i8_gated_residual(const int8_t* A, const float* sA, const in
   a.sA = sA; a.sW = sW; a.bias = bias; a.out = x;
   a.gate = gate; a.rows_per_item = rows_per_item; a.gate_stride = gate_stride;
   H3B_CK(launch_gemm(true, EPI_RESID, A, W, a, di->sms, stream), "gemm_i8_gated_residual");
+  return H3B_OK;
+}
+
+h3b_status h3b_gemm_bf16_gated_residual(const void* A, const void* W, const float* bias, const float* gate,
+                                        int rows_per_item, int gate_stride, void* x, int M, int N, int K,
+                                        h3b_stream stream) {
+  cudaStream_t st = stream;
+  DeviceInfo* di = nullptr;
+  h3b_status s = gemm_common(A, W, x, M, N, K, &di);
+  if (s != H3B_OK) return s;
+  if (!gate) return fail(H3B_ERR_ARG, "gate NULL");
+  if (rows_per_item < 1 || gate_stride < 0 || gate_stride % 4 != 0) return fail(H3B_ERR_ARG, "rows_per_item/gate_stride");
+  if (!aligned16(gate) || (bias && !aligned16(bias))) return fail(H3B_ERR_ALIGN, "alignment");
+  GemmArgs a = base_args(M, N, K, di->err);
+  a.bias = bias; a.out = x;
+  a.gate = gate; a.rows_per_item = rows_per_item; a.gate_stride = gate_stride;
+  H3B_CK(launch_gemm(false, EPI_RESID, A, W, a, di->sms, stream), "gemm_bf16_gated_residual");
   return H3B_OK;
 }
 

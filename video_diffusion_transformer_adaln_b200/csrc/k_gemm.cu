@@ -483,6 +483,7 @@ cudaError_t launch_gemm(bool int8_operands, GemmEpilogue epi, const void* A, con
     switch (epi) {
       case EPI_DEQ: return launch_one<false, EPI_DEQ>(ta, tb, args, grid, st);
       case EPI_QKV: return launch_one<false, EPI_QKV>(ta, tb, args, grid, st);
+      case EPI_RESID: return launch_one<false, EPI_RESID>(ta, tb, args, grid, st);
       default: break;
     }
   }

@@ -31,7 +31,8 @@ class Dims(C.Structure):
     _fields_ = [("B", C.c_int), ("T", C.c_int), ("H", C.c_int), ("W", C.c_int),
                 ("d", C.c_int), ("n_heads", C.c_int), ("head_dim", C.c_int), ("d_ff", C.c_int),
                 ("rope_t", C.c_int), ("rope_h", C.c_int), ("rope_w", C.c_int),
-                ("rope_theta", C.c_float), ("ln_eps", C.c_float), ("qkv_int8", C.c_int)]
+                ("rope_theta", C.c_float), ("ln_eps", C.c_float), ("qkv_int8", C.c_int),
+                ("wo_bf16", C.c_int)]
 
     @property
     def L(self) -> int:
@@ -39,7 +40,7 @@ class Dims(C.Structure):
 
 
 WEIGHT_FIELDS = ("w_ada", "b_ada", "wqkv", "sqkv", "wqkv_bf16", "bqkv", "wo", "so", "bo",
-                 "w1", "s1", "b1", "w2", "s2", "b2")
+                 "w1", "s1", "b1", "w2", "s2", "b2", "wo_bf16")
 
 
 class BlockWeights(C.Structure):
@@ -89,6 +90,7 @@ def _declare(L):
         "h3b_qkv_projection": [vp, vp, vp, vp, vp, vp, vp],
         "h3b_attention": [vp, vp, vp, vp, vp],
         "h3b_gemm_i8_gated_residual": [vp, vp, vp, vp, vp, vp, i32, i32, vp, i32, i32, i32, vp],
+        "h3b_gemm_bf16_gated_residual": [vp, vp, vp, vp, i32, i32, vp, i32, i32, i32, vp],
         "h3b_gemm_i8_gelu": [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, vp],
     }
     for name, args in sigs.items():
@@ -132,9 +134,9 @@ def status_string(status: int) -> str:
 # --------------------------------------------------------------------------- block level
 
 def make_dims(B, T, H, W, d, n_heads, head_dim, d_ff, rope, rope_theta=10000.0, ln_eps=1e-6,
-              qkv_int8=True) -> Dims:
+              qkv_int8=True, wo_bf16=False) -> Dims:
     return Dims(B, T, H, W, d, n_heads, head_dim, d_ff, rope[0], rope[1], rope[2], rope_theta, ln_eps,
-                1 if qkv_int8 else 0)
+                1 if qkv_int8 else 0, 1 if wo_bf16 else 0)
 
 
 def make_weights(tensors: Dict[str, Optional[torch.Tensor]]) -> BlockWeights:
@@ -249,6 +251,13 @@ def h3b_gemm_i8_gated_residual(A, sA, W, sW, bias, gate, rows_per_item, gate_str
     N = W.shape[0]
     _check(lib().h3b_gemm_i8_gated_residual(_p(A), _p(sA), _p(W), _p(sW), _p(bias), _p(gate), rows_per_item,
                                             gate_stride, _p(x), M, N, K, _s(stream)), "h3b_gemm_i8_gated_residual")
+
+
+def h3b_gemm_bf16_gated_residual(A, W, bias, gate, rows_per_item, gate_stride, x, stream=None):
+    M, K = A.shape
+    N = W.shape[0]
+    _check(lib().h3b_gemm_bf16_gated_residual(_p(A), _p(W), _p(bias), _p(gate), rows_per_item, gate_stride,
+                                              _p(x), M, N, K, _s(stream)), "h3b_gemm_bf16_gated_residual")
 
 
 def h3b_gemm_i8_gelu(A, sA, W, sW, bias, g, absmax, stream=None):

@@ -16,7 +16,7 @@ from .synth import Workload
 
 def dims_of(wl: Workload) -> h3b.Dims:
     return h3b.make_dims(wl.B, wl.T, wl.H, wl.W, wl.d, wl.n_heads, wl.head_dim, wl.d_ff, wl.rope,
-                         wl.rope_theta, wl.ln_eps, wl.qkv_int8)
+                         wl.rope_theta, wl.ln_eps, wl.qkv_int8, wl.wo_bf16)
 
 
 def bf16_from_bits(bits: np.ndarray, device="cuda") -> torch.Tensor:
@@ -57,6 +57,8 @@ class DeviceBlock:
             del w32
         if not qkv_int8:
             t["wqkv_bf16"] = bf16_from_bits(raw["wqkv_bf16"], device)
+        if "wo_bf16" in raw:
+            t["wo_bf16"] = bf16_from_bits(raw["wo_bf16"], device)
         return cls(t)
 
     @classmethod
@@ -77,6 +79,8 @@ class DeviceBlock:
             w32 = torch.randn((n_out, n_in), generator=generator, device=device) / n_in ** 0.5
             if name == "wqkv" and not wl.qkv_int8:
                 t["wqkv_bf16"] = w32.to(torch.bfloat16)
+            elif name == "wo" and wl.wo_bf16:
+                t["wo_bf16"] = w32.to(torch.bfloat16)
             else:
                 t[name], t[sname] = quantize_weight(w32)
             del w32

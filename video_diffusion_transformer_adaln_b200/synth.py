@@ -14,6 +14,7 @@ Distributions (model dimensions are synthetic; the pages give none):
   Wqkv, Wo, W1, W2 ~ N(0, 1/d_in) fp32 ([out][in]); quantized per output channel
            by each side's own quantizer; biases are zero (passed as NULL)
   Wqkv_bf16 = the same Wqkv draws stored bf16 (for the bf16-QKV variant)
+  Wo_bf16   = the same Wo draws stored bf16 (for the bf16 output-projection variant)
 """
 from __future__ import annotations
 
@@ -42,6 +43,7 @@ class Workload:
     n_blocks: int = 1
     token_pair: bool = False
     qkv_int8: bool = True
+    wo_bf16: bool = False
     rope_theta: float = 10000.0
     ln_eps: float = 1e-6
     # multi-block pass: blocks [first, last) run on the paired grid (empty: none)
@@ -54,9 +56,7 @@ class Workload:
     def merged(self) -> "Workload":
         """The grid the block sees under token reduction (W halved)."""
         assert self.W % 2 == 0
-        return Workload(self.name + "/merged", self.T, self.H, self.W // 2, self.d, self.n_heads,
-                        self.head_dim, self.d_ff, self.rope, self.n_outliers, self.B, self.n_blocks,
-                        False, self.qkv_int8, self.rope_theta, self.ln_eps, (0, 0))
+        return self.with_(name=self.name + "/merged", W=self.W // 2, token_pair=False, pair_blocks=(0, 0))
 
     def with_(self, **kw) -> "Workload":
         args = dict(self.__dict__)
@@ -78,6 +78,8 @@ WORKLOADS: Dict[str, Workload] = {
     "d5120_L18432": _large(8, name="d5120_L18432"),
     # the same block with bf16 QKV (int8 MLP): the A/B of QKV quantization
     "d5120_L18432_bf16qkv": _large(8, name="d5120_L18432_bf16qkv", qkv_int8=False),
+    # the same block with a bf16 output projection on the bf16 attention output
+    "d5120_L18432_bf16wo": _large(8, name="d5120_L18432_bf16wo", wo_bf16=True),
     # token reduction around the d=5120 block: 8x48x48 -> 8x48x24 = 9216 merged tokens
     "d5120_L18432_pair": _large(8, name="d5120_L18432_pair", token_pair=True),
 }
@@ -149,6 +151,8 @@ def block_weights(wl: Workload, block: int = 0, seed: int = BASE_SEED) -> dict:
            "w1": lin("w1", F, d), "w2": lin("w2", d, F)}
     if not wl.qkv_int8:
         out["wqkv_bf16"] = f32_to_bf16_bits(out["wqkv"])
+    if wl.wo_bf16:
+        out["wo_bf16"] = f32_to_bf16_bits(out["wo"])
     return out
 
 
