@@ -57,6 +57,8 @@ def _declare(L):
     L.orc_gated_residual.argtypes = [vp, vp, vp, i64, i64, vp]
     L.orc_token_pair.argtypes = [vp, i64, i64, i64, i64, i64, vp]
     L.orc_token_unpair.argtypes = [vp, vp, vp, i64, i64, i64, i64, i64, vp]
+    L.orc_range_delta.argtypes = [vp, vp, i64, vp]
+    L.orc_range_apply.argtypes = [vp, vp, i64, vp]
     L.orc_threads.restype = i32
     L.orc_threads.argtypes = []
     L.orc_block_forward.restype = i32
@@ -208,6 +210,22 @@ def token_unpair(x_bf16, xm_bf16, ym, B, T, H, W, d):
     out = np.empty((B, T, H, W, d), np.float64)
     lib().orc_token_unpair(_p(_c(x_bf16, np.uint16)), _p(_c(xm_bf16, np.uint16)), _p(_c(ym, np.float64)),
                            B, T, H, W, d, _p(out))
+    return out
+
+
+def range_delta(before_bf16, after_bf16):
+    """delta = after - before (fp64 of bf16 values)."""
+    a, b = _c(before_bf16, np.uint16), _c(after_bf16, np.uint16)
+    out = np.empty(a.shape, np.float64)
+    lib().orc_range_delta(_p(a), _p(b), a.size, _p(out))
+    return out
+
+
+def range_apply(x_bf16, delta):
+    """bf16(x + delta)."""
+    x, d = _c(x_bf16, np.uint16), _c(delta, np.float64)
+    out = np.empty(x.shape, np.uint16)
+    lib().orc_range_apply(_p(x), _p(d), x.size, _p(out))
     return out
 
 

@@ -365,6 +365,21 @@ void orc_token_unpair(const uint16_t* x, const uint16_t* xm, const double* ym, i
 }
 
 // ---------------------------------------------------------------------------
+// Residual reuse across denoise steps ([README] "속도 및 품질 트레이드오프",
+// core-residual reuse): the delta a block range adds to the residual stream,
+// and its re-application to another step's stream.
+//   delta = after - before (fp64 of the bf16 values)
+//   out   = bf16(x + delta)
+// ---------------------------------------------------------------------------
+void orc_range_delta(const uint16_t* before, const uint16_t* after, int64_t n, double* delta) {
+  for (int64_t i = 0; i < n; ++i) delta[i] = orc_bf16_to_f64(after[i]) - orc_bf16_to_f64(before[i]);
+}
+
+void orc_range_apply(const uint16_t* x, const double* delta, int64_t n, uint16_t* out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = orc_f64_to_bf16(orc_bf16_to_f64(x[i]) + delta[i]);
+}
+
+// ---------------------------------------------------------------------------
 // One DiT block, forward.
 // ---------------------------------------------------------------------------
 typedef struct {

@@ -14,6 +14,7 @@ import pytest
 import torch
 
 import oracle as O
+from video_diffusion_transformer_adaln_b200 import synth
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
@@ -320,3 +321,23 @@ def test_token_pair_unpair_identities():
     z = np.zeros((B, T, H, W, d), np.uint16)
     out = O.token_unpair(z, np.zeros_like(xm), ym, B, T, H, W, d)
     assert np.array_equal(out[..., 0::2, :], ym) and np.array_equal(out[..., 1::2, :], ym)
+
+
+def test_range_delta_and_apply_closed_form():
+    """Residual reuse: delta = after - before exactly; re-applying it to the same stream
+    gives `after` back; applied to another stream it is the plain sum, rounded once."""
+    r = np.random.default_rng(31)
+    before = synth.f32_to_bf16_bits(r.standard_normal(4096).astype(np.float32))
+    after = synth.f32_to_bf16_bits((synth.bf16_bits_to_f32(before) + r.standard_normal(4096) * 0.3).astype(np.float32))
+    delta = O.range_delta(before, after)
+    assert np.array_equal(delta, synth.bf16_bits_to_f32(after).astype(np.float64)
+                          - synth.bf16_bits_to_f32(before).astype(np.float64))
+    assert np.array_equal(O.range_apply(before, delta), after)
+    other = synth.f32_to_bf16_bits(r.standard_normal(4096).astype(np.float32))
+    got = synth.bf16_bits_to_f32(O.range_apply(other, delta)).astype(np.float64)
+    exact = synth.bf16_bits_to_f32(other).astype(np.float64) + delta
+    # one rounding to bf16: within half a bf16 ulp of the exact sum
+    ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(exact), 1e-30))) - 7)
+    assert np.all(np.abs(got - exact) <= 0.5 * ulp)
+    # a zero delta is the identity
+    assert np.array_equal(O.range_apply(other, np.zeros(4096)), other)
