@@ -7,7 +7,16 @@ output projection with gated residual, fused LN+quantizer, int8 W1 + GELU,
 quantizer, int8 W2 with gated residual) over one synthetic latent of the
 chosen workload, through the library's C ABI. Token-reduction workloads add
 the pair/unpair kernels around the block; depth-50 workloads run 50 distinct
-blocks per step.
+blocks per step; residual-reuse workloads run a fresh and a reuse pass per
+step (two denoise steps).
+
+Timing: the pass is captured once as a CUDA graph (h3b_graph_capture_blocks)
+and each timed step replays it (`launch.mode` = "graph"); workloads with
+pairing or reuse launch on the stream ("stream"). K steps are timed with CUDA
+events, the input restored and L2 flushed between steps outside the events.
+The same K steps are then run with the library's per-launch profiler on; those
+per-kernel device times give kernel_share, kernel_roofline and the dominant
+kernel's roofline.
 
 Prints one JSON line (rank 0). Under torchrun each rank runs its own
 independent latent (replicas; no data-path collective): the value is the
@@ -101,6 +110,8 @@ def _block_kernel_work(name, wl, L):
         return R * (2.0 * d + d + 8), "byte", "hbm"
     if name == "quant_g":
         return R * (2.0 * F + F + 8), "byte", "hbm"
+    if name in ("range_delta", "range_apply"):  # 2 + 2 + 4 or 2 + 4 + 2 bytes per element
+        return 8.0 * R * d, "byte", "hbm"
     if name == "adaln_gemv":  # (its trailing blocks also fill the small RoPE table)
         return 12.0 * d * d + B * (4.0 * d + 24 * d), "byte", "hbm"
     return 0.0, "byte", "hbm"
@@ -187,7 +198,12 @@ class Workload:
             shp = (wl.B, wl.T, wl.H, wl.W // 2, wl.d)
             self.xm = torch.empty(shp, dtype=torch.bfloat16, device="cuda")
             self.ym = torch.empty_like(self.xm)
-        self.tokens = wl.B * wl.L
+        self.reuse = wl.reuse_blocks[0] < wl.reuse_blocks[1]
+        if self.reuse:
+            self.x_save = torch.empty_like(self.x)
+            self.delta = torch.empty(self.x.numel(), dtype=torch.float32, device="cuda")
+        # tokens per step: a reuse step is two denoise steps (one fresh pass, one reuse pass)
+        self.tokens = wl.B * wl.L * (2 if self.reuse else 1)
 
     def step(self, x=None, c=None):
         x = self.x if x is None else x
@@ -197,6 +213,11 @@ class Workload:
             h3b.h3b_token_pair(self.full, x, self.xm, self.ym)
             h3b.h3b_block_forward(self.dims, self.blocks[0].struct, c, self.ym, self.ws)
             h3b.h3b_token_unpair(self.full, x, self.xm, self.ym, x)
+        elif self.reuse:
+            structs = [b.struct for b in self.blocks]
+            f, l = wl.reuse_blocks
+            h3b.h3b_blocks_forward_cached(self.dims, structs, f, l, True, c, x, self.x_save, self.delta, self.ws)
+            h3b.h3b_blocks_forward_cached(self.dims, structs, f, l, False, c, x, None, self.delta, self.ws)
         elif wl.n_blocks > 1 and wl.pair_blocks[0] < wl.pair_blocks[1]:
             h3b.h3b_blocks_forward_reduced(self.full, [b.struct for b in self.blocks], wl.pair_blocks[0],
                                            wl.pair_blocks[1], c, x, self.xm, self.ym, self.ws)
@@ -322,22 +343,40 @@ def run_h3b(args, rank, world, local):
     torch.cuda.synchronize()
     barrier(world)
 
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    h3b.h3b_profile_read()  # drop anything recorded during warm-up
-    h3b.h3b_profile_enable(True)
-    torch.cuda.synchronize()
-    barrier(world)
-    for i in range(args.steps):
-        prep()  # restore the input and flush L2 outside the timed events
-        ev[i][0].record()
-        W.step()
-        ev[i][1].record()
-    torch.cuda.synchronize()
-    barrier(world)
-    h3b.h3b_profile_enable(False)
+    # The pass is captured once as a CUDA graph (h3b_graph_capture_blocks) where the workload
+    # is a plain multi-block pass; paired and residual-reuse steps launch on the stream.
+    graph = None
+    if not wl.token_pair and not wl.pair_blocks[0] < wl.pair_blocks[1] and not W.reuse:
+        graph = h3b.h3b_graph_capture_blocks(W.dims, [b.struct for b in W.blocks], W.c, W.x, W.ws)
+        for _ in range(2):
+            prep()
+            graph.launch()
+        torch.cuda.synchronize()
+    run_step = graph.launch if graph is not None else W.step
+
+    def timed(step_fn):
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        torch.cuda.synchronize()
+        barrier(world)
+        for i in range(args.steps):
+            prep()  # restore the input and flush L2 outside the timed events
+            ev[i][0].record()
+            step_fn()
+            ev[i][1].record()
+        torch.cuda.synchronize()
+        barrier(world)
+        return max_over_ranks(sum(a.elapsed_time(b) for a, b in ev), world)
+
+    # (1) the headline: K steps of the pass, nothing else on the stream
+    total_ms = timed(run_step)
+    stream_ms = timed(W.step) if graph is not None else total_ms
     clocks = sampler.stop() if sampler else None
-    step_ms = [a.elapsed_time(b) for a, b in ev]
-    total_ms = max_over_ranks(sum(step_ms), world)
+    # (2) per-kernel device times: the same K steps on the stream with the library's
+    #     profiler bracketing every launch with CUDA events
+    h3b.h3b_profile_read()  # drop anything recorded before
+    h3b.h3b_profile_enable(True)
+    prof_ms = timed(W.step)
+    h3b.h3b_profile_enable(False)
     prof = h3b.h3b_profile_read()
     err = h3b.h3b_device_error(clear=True)
     if err:
@@ -346,18 +385,17 @@ def run_h3b(args, rank, world, local):
     tokens_all = sum_over_ranks(W.tokens * args.steps, world)
     value = tokens_all / (total_ms / 1e3)
 
-    # ---- end to end: pinned host input -> device -> block -> host output, same API
+    # ---- end to end: pinned host input -> device -> pass -> host output, same API
     x_host = torch.empty(W.x.shape, dtype=torch.bfloat16, pin_memory=True)
     x_host.copy_(W.x_ref.cpu())
     c_host = torch.empty(W.c.shape, dtype=W.c.dtype, pin_memory=True)
     c_host.copy_(W.c.cpu())
     out_host = torch.empty_like(x_host, pin_memory=True)
-    c_dev = torch.empty_like(W.c)
     e2e_steps = max(3, min(args.steps, 20))
     for _ in range(2):
         W.x.copy_(x_host, non_blocking=True)
-        c_dev.copy_(c_host, non_blocking=True)
-        W.step(c=c_dev)
+        W.c.copy_(c_host, non_blocking=True)
+        run_step()
         out_host.copy_(W.x, non_blocking=True)
     torch.cuda.synchronize()
     barrier(world)
@@ -366,8 +404,8 @@ def run_h3b(args, rank, world, local):
         flush.zero_()
         eev[i][0].record()
         W.x.copy_(x_host, non_blocking=True)
-        c_dev.copy_(c_host, non_blocking=True)
-        W.step(c=c_dev)
+        W.c.copy_(c_host, non_blocking=True)  # the graph reads c from this buffer
+        run_step()
         out_host.copy_(W.x, non_blocking=True)
         eev[i][1].record()
     torch.cuda.synchronize()
@@ -376,6 +414,13 @@ def run_h3b(args, rank, world, local):
     e2e_value = sum_over_ranks(W.tokens * e2e_steps, world) / (e2e_ms / 1e3)
     h2d = x_host.numel() * x_host.element_size() + c_host.numel() * c_host.element_size()
     d2h = out_host.numel() * out_host.element_size()
+    launch = {"mode": "graph" if graph is not None else "stream",
+              "stream_ms_per_step": round(stream_ms / args.steps, 4),
+              "profiled_ms_per_step": round(prof_ms / args.steps, 4)}
+    if graph is not None:
+        launch["graph_ms_per_step"] = round(total_ms / args.steps, 4)
+        launch["kernels_per_step"] = graph.kernel_count
+        graph.destroy()
 
     # ---- roofline of the dominant kernel (live per-kernel device times)
     ktot = sum(ms for _, ms in prof.values()) or 1.0
@@ -411,7 +456,7 @@ def run_h3b(args, rank, world, local):
 
     gpu_launches = int(sum(n for n, _ in prof.values()))
     kernel_ms = {k: round(ms / args.steps, 4) for k, (n, ms) in prof.items()}
-    gap_ms = total_ms / args.steps - sum(ms for _, ms in prof.values()) / args.steps
+    gap_ms = prof_ms / args.steps - sum(ms for _, ms in prof.values()) / args.steps
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         orc = OracleRunner(wl)
@@ -426,13 +471,13 @@ def run_h3b(args, rank, world, local):
         "config": {"workload": args.workload, "batch": wl.B, "grid_THW": [wl.T, wl.H, wl.W], "tokens": wl.L,
                    "d": wl.d, "heads": wl.n_heads, "head_dim": wl.head_dim, "d_ff": wl.d_ff,
                    "blocks_per_step": wl.n_blocks, "token_pair": wl.token_pair,
-                   "paired_blocks": list(wl.pair_blocks),
+                   "paired_blocks": list(wl.pair_blocks), "reuse_blocks": list(wl.reuse_blocks),
                    "qkv": "int8" if wl.qkv_int8 else "bf16", "wo": "bf16" if wl.wo_bf16 else "int8",
                    "attention": "bf16",
                    "l2": "flushed between steps (512 MiB write outside the timed events)",
                    "parallelism": "replicas: one independent latent per GPU, no collective"},
         "roofline": roof, "kernel_share": shares, "kernel_roofline": all_roof,
-        "kernel_ms_per_step": kernel_ms, "launch_gap_ms_per_step": round(gap_ms, 4),
+        "kernel_ms_per_step": kernel_ms, "launch_gap_ms_per_step": round(gap_ms, 4), "launch": launch,
         "cpu_baseline": cpu,
         "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": e2e_steps},

@@ -183,6 +183,51 @@ H3B_API h3b_status h3b_blocks_forward_reduced(const h3b_dims* full, const h3b_bl
                                               int first, int last, const float* c, void* x, void* xm, void* ym,
                                               void* ws, size_t ws_bytes, h3b_stream stream);
 
+/* Residual reuse across denoise steps (the core-residual reuse of the pages'
+ * control table, "h3-metal: ...", section "속도 및 품질 트레이드오프"): the
+ * delta a block range [first, last) adds to the residual stream on a fresh
+ * denoise step is cached and re-applied on the following steps instead of
+ * running the range again.
+ *   h3b_blocks_forward_cached: blocks [0, first) and [last, n_blocks) run as in
+ *   h3b_blocks_forward. fresh != 0: x is copied to x_save (bf16, B*L*d), the
+ *   range runs, then delta = x - x_save (fp32, B*L*d). fresh == 0: the range is
+ *   skipped and x = bf16(x + delta). first == last: no range (x_save, delta unused).
+ *   Same workspace and argument rules as h3b_blocks_forward; x_save and delta
+ *   16-byte aligned, owned by the caller; delta must come from a fresh call
+ *   with the same dimensions.
+ *   h3b_range_delta / h3b_range_apply: the two steps alone, on n elements
+ *   (n % 8 == 0, 16-byte aligned). */
+H3B_API h3b_status h3b_blocks_forward_cached(const h3b_dims* dims, const h3b_block_weights* w, int n_blocks,
+                                             int first, int last, int fresh, const float* c, void* x,
+                                             void* x_save, float* delta, void* ws, size_t ws_bytes,
+                                             h3b_stream stream);
+H3B_API h3b_status h3b_range_delta(const void* before, const void* after, float* delta, long long n,
+                                   h3b_stream stream);
+H3B_API h3b_status h3b_range_apply(void* x, const float* delta, long long n, h3b_stream stream);
+
+/* CUDA Graph of a multi-block pass: h3b_graph_capture_blocks records
+ * h3b_blocks_forward(dims, w, n_blocks, c, x, ws, ws_bytes) (every launch, with
+ * its arguments) without running it; h3b_graph_launch replays the whole pass on
+ * `stream` as one graph launch. The result is that of h3b_blocks_forward with
+ * the same arguments (same kernels); only the per-launch host cost and the gaps
+ * between launches go away.
+ *   Ownership: the graph handle belongs to the caller (h3b_graph_destroy). The
+ *   graph refers to x, c, the weights and the workspace by address; they must
+ *   stay allocated and unmoved while the graph is used, and every replay reads
+ *   x as it is when the replay runs.
+ *   Errors: the same argument checks as h3b_blocks_forward (nothing is
+ *   captured then); H3B_ERR_ARG if profiling is on (h3b_profile_enable) or on
+ *   launch from another device than the capture's; H3B_ERR_CUDA on a failed
+ *   capture or instantiation. Run the pass once with the same dimensions before
+ *   capturing, so that every kernel is loaded.
+ *   h3b_graph_kernel_count: kernel launches in one replay (0 for NULL). */
+typedef struct h3b_graph_s* h3b_graph;
+H3B_API h3b_status h3b_graph_capture_blocks(const h3b_dims* dims, const h3b_block_weights* w, int n_blocks,
+                                            const float* c, void* x, void* ws, size_t ws_bytes, h3b_graph* out);
+H3B_API h3b_status h3b_graph_launch(h3b_graph g, h3b_stream stream);
+H3B_API int h3b_graph_kernel_count(h3b_graph g);
+H3B_API void h3b_graph_destroy(h3b_graph g);
+
 /* Token reduction ("Token Reduction" row of the control table): horizontally
  * adjacent tokens w = 2k, 2k+1 of each (t, h) row are merged by their mean.
  *   full: dims of the UNMERGED grid (W even).

@@ -12,7 +12,7 @@ import torch
 
 import oracle as O
 from gpu_helpers import (bf16_dev, bf16_host, no_device_error, oracle_dims, oracle_weights, rel_l2, require_gpu,
-                         to_dev)
+                         to_dev, bf16_ulp_diff)
 from video_diffusion_transformer_adaln_b200 import h3b, synth
 from video_diffusion_transformer_adaln_b200.runtime import (DeviceBlock, blocks_forward, block_forward, dims_of,
                                                             paired_block_forward, workspace)
@@ -201,6 +201,92 @@ def test_blocks_forward_three_blocks_d256():
     for b in range(3):
         block_forward(dims, blocks[b], to_dev(cs[b]), xd2, ws)
     assert np.array_equal(bf16_host(xd2), got)
+    no_device_error()
+
+
+def test_graph_replay_equals_stream_launches_d256():
+    """A captured three-block pass replays to the same bits as h3b_blocks_forward."""
+    wl = synth.WORKLOADS["d256_L512"].with_(n_blocks=3)
+    x = synth.x_input(wl)
+    raws = [synth.block_weights(wl, b) for b in range(3)]
+    cs = to_dev(np.stack([synth.cond(wl, b) for b in range(3)]))
+    dims = dims_of(wl)
+    blocks = [DeviceBlock.from_host(r) for r in raws]
+    ws = workspace(dims)
+    xd = bf16_dev(x)
+    blocks_forward(dims, blocks, cs, xd, ws)  # also loads every kernel before the capture
+    ref = bf16_host(xd)
+    xg = bf16_dev(x)
+    g = h3b.h3b_graph_capture_blocks(dims, [b.struct for b in blocks], cs, xg, ws)
+    torch.cuda.synchronize()
+    assert np.array_equal(bf16_host(xg), x)  # capturing runs nothing
+    assert g.kernel_count == 3 * 10
+    g.launch()
+    torch.cuda.synchronize()
+    assert np.array_equal(bf16_host(xg), ref)
+    xg.copy_(bf16_dev(x))  # a replay reads x as it is at launch time
+    g.launch()
+    torch.cuda.synchronize()
+    assert np.array_equal(bf16_host(xg), ref)
+    g.destroy()
+    # capturing with the profiler on is refused, and nothing is left captured
+    h3b.h3b_profile_enable(True)
+    try:
+        with pytest.raises(h3b.H3BError):
+            h3b.h3b_graph_capture_blocks(dims, [b.struct for b in blocks], cs, xg, ws)
+    finally:
+        h3b.h3b_profile_enable(False)
+        h3b.h3b_profile_read()
+    no_device_error()
+
+
+def test_blocks_forward_cached_range_d256():
+    """Residual reuse: a fresh pass caches the delta of blocks 1..3 (the last three of four);
+    a reuse pass skips them and re-applies the delta."""
+    wl = synth.WORKLOADS["d256_L512"].with_(n_blocks=4)
+    first, last = 1, 4
+    x = synth.x_input(wl)
+    raws = [synth.block_weights(wl, b) for b in range(4)]
+    cs = to_dev(np.stack([synth.cond(wl, b) for b in range(4)]))
+    dims = dims_of(wl)
+    blocks = [DeviceBlock.from_host(r) for r in raws]
+    structs = [b.struct for b in blocks]
+    ws = workspace(dims)
+    n = x.size
+    # reference: the plain pass, and block 0 alone
+    xr = bf16_dev(x)
+    blocks_forward(dims, blocks, cs, xr, ws)
+    ref = bf16_host(xr)
+    x0 = bf16_dev(x)
+    h3b.h3b_blocks_forward(dims, structs[:1], cs, x0, ws)
+    after0 = bf16_host(x0)
+    # fresh pass: the same result bit for bit; x_save is the range's input; delta = after - before
+    xf = bf16_dev(x)
+    x_save = torch.empty_like(xf)
+    delta = torch.empty(n, dtype=torch.float32, device="cuda")
+    h3b.h3b_blocks_forward_cached(dims, structs, first, last, True, cs, xf, x_save, delta, ws)
+    torch.cuda.synchronize()
+    assert np.array_equal(bf16_host(xf), ref)
+    assert np.array_equal(bf16_host(x_save), after0)
+    d_ref = O.range_delta(after0, ref)
+    d_got = delta.cpu().numpy().astype(np.float64).reshape(d_ref.shape)
+    assert np.all(np.abs(d_got - d_ref) <= 2.0 ** -24 * np.abs(d_ref))
+    # reuse pass on another step's stream: block 0 runs, the range is replaced by the delta
+    x2_bits = synth.f32_to_bf16_bits((synth.bf16_bits_to_f32(x) * 0.9).astype(np.float32))
+    x2 = bf16_dev(x2_bits)
+    h3b.h3b_blocks_forward_cached(dims, structs, first, last, False, cs, x2, None, delta, ws)
+    x2b = bf16_dev(x2_bits)
+    h3b.h3b_blocks_forward(dims, structs[:1], cs, x2b, ws)
+    want = O.range_apply(bf16_host(x2b), d_got)
+    got = bf16_host(x2)
+    assert bf16_ulp_diff(got, want).max() <= 1  # fp32 sum then bf16 vs one rounding of the exact sum
+    # the step entry points alone agree with the pass
+    d2 = torch.empty_like(delta)
+    h3b.h3b_range_delta(x_save, xf, d2)
+    assert torch.equal(d2, delta)
+    x3 = bf16_dev(after0)
+    h3b.h3b_range_apply(x3, delta)
+    assert bf16_ulp_diff(bf16_host(x3), O.range_apply(after0, d_got)).max() <= 1
     no_device_error()
 
 

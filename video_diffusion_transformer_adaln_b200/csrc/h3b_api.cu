@@ -169,6 +169,15 @@ bool g_prof_on = false;
 std::vector<ProfRec> g_prof_recs;
 std::vector<cudaEvent_t> g_prof_free;
 
+}  // namespace
+
+bool profiling_enabled() {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  return g_prof_on;
+}
+
+namespace {
+
 cudaEvent_t prof_event() {
   if (!g_prof_free.empty()) {
     cudaEvent_t e = g_prof_free.back();
@@ -419,6 +428,72 @@ h3b_status h3b_blocks_forward(const h3b_dims* dims, const h3b_block_weights* w, 
     s = run_block(*dims, w[i], c + i * c_stride, x, static_cast<uint8_t*>(ws), lay, i > 0, *di, stream);
     if (s != H3B_OK) return s;
   }
+  return H3B_OK;
+}
+
+h3b_status h3b_blocks_forward_cached(const h3b_dims* dims, const h3b_block_weights* w, int n_blocks, int first,
+                                     int last, int fresh, const float* c, void* x, void* x_save, float* delta,
+                                     void* ws, size_t ws_bytes, h3b_stream stream) {
+  WsLayout lay;
+  DeviceInfo* di = nullptr;
+  h3b_status s = block_common(dims, c, x, ws, ws_bytes, &lay, &di);
+  if (s != H3B_OK) return s;
+  if (n_blocks < 0 || (n_blocks > 0 && !w)) return fail(H3B_ERR_ARG, "n_blocks < 0 or weights NULL");
+  if (first < 0 || first > last || last > n_blocks) return fail(H3B_ERR_ARG, "need 0 <= first <= last <= n_blocks");
+  const bool range = first < last;
+  if (range && (!delta || !aligned16(delta))) return fail(H3B_ERR_ARG, "delta NULL or not 16-byte aligned");
+  if (range && fresh && (!x_save || !aligned16(x_save))) return fail(H3B_ERR_ARG, "x_save NULL or not 16-byte aligned");
+  for (int i = 0; i < n_blocks; ++i)
+    if ((s = check_weights(*dims, &w[i])) != H3B_OK) return s;
+  cudaStream_t st = stream;
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  const size_t c_stride = (size_t)dims->B * dims->d;
+  const long long n = (long long)dims->B * dims->T * dims->H * dims->W * dims->d;
+  bool rope_done = false;  // the first block that runs fills the RoPE table
+  auto run = [&](int i) {
+    const h3b_status r = run_block(*dims, w[i], c + i * c_stride, x, wsb, lay, rope_done, *di, st);
+    rope_done = true;
+    return r;
+  };
+  for (int i = 0; i < first; ++i)
+    if ((s = run(i)) != H3B_OK) return s;
+  if (range) {
+    if (fresh) {
+      const cudaError_t e = cudaMemcpyAsync(x_save, x, (size_t)n * 2, cudaMemcpyDeviceToDevice, st);
+      if (e != cudaSuccess) return cuda_fail(e, "save range input");
+      for (int i = first; i < last; ++i)
+        if ((s = run(i)) != H3B_OK) return s;
+      H3B_CK(launch_range_delta(x_save, x, delta, n, di->sms, st), "range_delta");
+    } else {
+      H3B_CK(launch_range_apply(x, delta, n, di->sms, st), "range_apply");
+    }
+  }
+  for (int i = last; i < n_blocks; ++i)
+    if ((s = run(i)) != H3B_OK) return s;
+  return H3B_OK;
+}
+
+h3b_status h3b_range_delta(const void* before, const void* after, float* delta, long long n, h3b_stream stream) {
+  cudaStream_t st = stream;
+  if (!before || !after || !delta) return fail(H3B_ERR_ARG, "NULL pointer");
+  if (n < 0 || n % 8 != 0) return fail(H3B_ERR_SHAPE, "n must be a non-negative multiple of 8");
+  if (!aligned16(before) || !aligned16(after) || !aligned16(delta)) return fail(H3B_ERR_ALIGN, "alignment");
+  DeviceInfo* di = nullptr;
+  h3b_status s = device_info(&di);
+  if (s != H3B_OK) return s;
+  H3B_CK(launch_range_delta(before, after, delta, n, di->sms, st), "range_delta");
+  return H3B_OK;
+}
+
+h3b_status h3b_range_apply(void* x, const float* delta, long long n, h3b_stream stream) {
+  cudaStream_t st = stream;
+  if (!x || !delta) return fail(H3B_ERR_ARG, "NULL pointer");
+  if (n < 0 || n % 8 != 0) return fail(H3B_ERR_SHAPE, "n must be a non-negative multiple of 8");
+  if (!aligned16(x) || !aligned16(delta)) return fail(H3B_ERR_ALIGN, "alignment");
+  DeviceInfo* di = nullptr;
+  h3b_status s = device_info(&di);
+  if (s != H3B_OK) return s;
+  H3B_CK(launch_range_apply(x, delta, n, di->sms, st), "range_apply");
   return H3B_OK;
 }
 

@@ -26,6 +26,10 @@ cudaError_t launch_quant_rows_f32(const float* w, int rows, int cols, int8_t* q,
                                   cudaStream_t st);
 cudaError_t launch_token_pair(const void* x, void* xm, void* xm2, long long lines, int W, int d,
                               int sms, cudaStream_t st);
+// delta fp32 [n] = after - before (bf16 [n]); x bf16 [n] = bf16(x + delta). n % 8 == 0.
+cudaError_t launch_range_delta(const void* before, const void* after, float* delta, long long n, int sms,
+                               cudaStream_t st);
+cudaError_t launch_range_apply(void* x, const float* delta, long long n, int sms, cudaStream_t st);
 cudaError_t launch_token_unpair(const void* x, const void* xm, const void* ym, void* out,
                                 long long lines, int W, int d, int sms, cudaStream_t st);
 cudaError_t launch_rope_table(float2* tab, int T, int H, int W, int rt, int rh, int rw,
@@ -75,6 +79,8 @@ cudaError_t launch_attention(const AttnArgs& a, cudaStream_t st);
 
 // ---- error detail reported by h3b_last_error_detail (h3b_api.cu)
 void set_error_detail(const std::string& why);
+// ---- whether h3b_profile_enable(1) is in effect (h3b_api.cu)
+bool profiling_enabled();
 
 // ---- TMA descriptor construction (h3b_api.cu)
 // Row-major 2D tensor of `rows` x `cols` elements of `elem_bytes` each,

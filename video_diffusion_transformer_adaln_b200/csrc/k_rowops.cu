@@ -534,6 +534,46 @@ __global__ void token_unpair_kernel(const __nv_bfloat16* __restrict__ x,
 }
 
 // ---------------------------------------------------------------------------
+// Residual reuse across denoise steps ([README] control table, core-residual
+// reuse): the delta of a block range, delta = x_after - x_before in fp32 (the
+// difference of two bf16 values), and its re-application x = bf16(x + delta).
+// Eight channels per thread: one 16-byte bf16 vector and two 16-byte fp32 ones.
+// ---------------------------------------------------------------------------
+__global__ void range_delta_kernel(const __nv_bfloat16* __restrict__ before, const __nv_bfloat16* __restrict__ after,
+                                   float* __restrict__ delta, long long n_vec) {
+  for (long long o = blockIdx.x * (long long)blockDim.x + threadIdx.x; o < n_vec;
+       o += (long long)gridDim.x * blockDim.x) {
+    const uint4 a = __ldcs(reinterpret_cast<const uint4*>(before) + o);
+    const uint4 b = __ldcs(reinterpret_cast<const uint4*>(after) + o);
+    const uint32_t ua[4] = {a.x, a.y, a.z, a.w}, ub[4] = {b.x, b.y, b.z, b.w};
+    float r[8];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      r[2 * e] = bf16_lo(ub[e]) - bf16_lo(ua[e]);
+      r[2 * e + 1] = bf16_hi(ub[e]) - bf16_hi(ua[e]);
+    }
+    float4* d4 = reinterpret_cast<float4*>(delta) + 2 * o;
+    __stcs(d4, make_float4(r[0], r[1], r[2], r[3]));
+    __stcs(d4 + 1, make_float4(r[4], r[5], r[6], r[7]));
+  }
+}
+
+__global__ void range_apply_kernel(__nv_bfloat16* __restrict__ x, const float* __restrict__ delta, long long n_vec) {
+  for (long long o = blockIdx.x * (long long)blockDim.x + threadIdx.x; o < n_vec;
+       o += (long long)gridDim.x * blockDim.x) {
+    const uint4 a = __ldcs(reinterpret_cast<const uint4*>(x) + o);
+    const float4 d0 = __ldcs(reinterpret_cast<const float4*>(delta) + 2 * o);
+    const float4 d1 = __ldcs(reinterpret_cast<const float4*>(delta) + 2 * o + 1);
+    const float dd[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
+    const uint32_t ua[4] = {a.x, a.y, a.z, a.w};
+    uint32_t r[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) r[e] = pack_bf16x2(bf16_lo(ua[e]) + dd[2 * e], bf16_hi(ua[e]) + dd[2 * e + 1]);
+    reinterpret_cast<uint4*>(x)[o] = make_uint4(r[0], r[1], r[2], r[3]);
+  }
+}
+
+// ---------------------------------------------------------------------------
 // RoPE table: for each axis (t, h, w) with n positions and segment length r,
 // entry [pos * (r/2) + j] = (cos, sin)(pos * theta^(-2j/r)), evaluated in fp64
 // and stored as fp32. Axis blocks are stored one after the other (t, h, w).
@@ -688,6 +728,22 @@ cudaError_t launch_token_pair(const void* x, void* xm, void* xm2, long long line
   token_pair_kernel<<<grid_for(n, sms), 256, 0, st>>>(
       static_cast<const __nv_bfloat16*>(x), static_cast<__nv_bfloat16*>(xm),
       static_cast<__nv_bfloat16*>(xm2), n, W / 2, d / 8);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_range_delta(const void* before, const void* after, float* delta, long long n, int sms,
+                               cudaStream_t st) {
+  if (n == 0) return cudaSuccess;
+  const long long nv = n / 8;
+  range_delta_kernel<<<grid_for(nv, sms), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(before),
+                                                        static_cast<const __nv_bfloat16*>(after), delta, nv);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_range_apply(void* x, const float* delta, long long n, int sms, cudaStream_t st) {
+  if (n == 0) return cudaSuccess;
+  const long long nv = n / 8;
+  range_apply_kernel<<<grid_for(nv, sms), 256, 0, st>>>(static_cast<__nv_bfloat16*>(x), delta, nv);
   return cudaGetLastError();
 }
 

@@ -91,6 +91,11 @@ def _declare(L):
         "h3b_attention": [vp, vp, vp, vp, vp],
         "h3b_gemm_i8_gated_residual": [vp, vp, vp, vp, vp, vp, i32, i32, vp, i32, i32, i32, vp],
         "h3b_gemm_bf16_gated_residual": [vp, vp, vp, vp, i32, i32, vp, i32, i32, i32, vp],
+        "h3b_graph_capture_blocks": [vp, vp, i32, vp, vp, vp, sz, vp],
+        "h3b_graph_launch": [vp, vp],
+        "h3b_blocks_forward_cached": [vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, sz, vp],
+        "h3b_range_delta": [vp, vp, vp, C.c_longlong, vp],
+        "h3b_range_apply": [vp, vp, C.c_longlong, vp],
         "h3b_gemm_i8_gelu": [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, vp],
     }
     for name, args in sigs.items():
@@ -103,6 +108,10 @@ def _declare(L):
     L.h3b_profile_enable.argtypes = [i32]
     L.h3b_profile_read.restype = i32
     L.h3b_profile_read.argtypes = [C.POINTER(KernelTime), i32]
+    L.h3b_graph_kernel_count.restype = i32
+    L.h3b_graph_kernel_count.argtypes = [vp]
+    L.h3b_graph_destroy.restype = None
+    L.h3b_graph_destroy.argtypes = [vp]
 
 
 def _p(t: Optional[torch.Tensor]):
@@ -170,6 +179,68 @@ def h3b_blocks_forward(dims: Dims, ws_list: Sequence[BlockWeights], c, x, ws, st
     arr = (BlockWeights * len(ws_list))(*ws_list)
     _check(lib().h3b_blocks_forward(C.byref(dims), arr, len(ws_list), _p(c), _p(x), _p(ws),
                                     ws.numel() * ws.element_size(), _s(stream)), "h3b_blocks_forward")
+
+
+def h3b_blocks_forward_cached(dims: Dims, ws_list: Sequence[BlockWeights], first: int, last: int, fresh: bool,
+                              c, x, x_save, delta, ws, stream=None):
+    arr = (BlockWeights * len(ws_list))(*ws_list)
+    _check(lib().h3b_blocks_forward_cached(C.byref(dims), arr, len(ws_list), first, last, 1 if fresh else 0, _p(c),
+                                           _p(x), _p(x_save), _p(delta), _p(ws), ws.numel() * ws.element_size(),
+                                           _s(stream)), "h3b_blocks_forward_cached")
+
+
+def h3b_range_delta(before, after, delta, stream=None):
+    _check(lib().h3b_range_delta(_p(before), _p(after), _p(delta), before.numel(), _s(stream)), "h3b_range_delta")
+
+
+def h3b_range_apply(x, delta, stream=None):
+    _check(lib().h3b_range_apply(_p(x), _p(delta), x.numel(), _s(stream)), "h3b_range_apply")
+
+
+class Graph:
+    """A captured multi-block pass (h3b_graph_capture_blocks); replay with launch()."""
+
+    def __init__(self, handle: int, keep):
+        self.handle = handle
+        self._keep = keep  # the argument structs the capture referenced
+
+    def launch(self, stream=None):
+        _check(lib().h3b_graph_launch(self.handle, _s(stream)), "h3b_graph_launch")
+
+    @property
+    def kernel_count(self) -> int:
+        return lib().h3b_graph_kernel_count(self.handle)
+
+    def destroy(self):
+        if self.handle:
+            lib().h3b_graph_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.destroy()
+        except Exception:
+            pass
+
+
+def h3b_graph_launch(g: Graph, stream=None):
+    g.launch(stream)
+
+
+def h3b_graph_kernel_count(g: Graph) -> int:
+    return g.kernel_count
+
+
+def h3b_graph_destroy(g: Graph):
+    g.destroy()
+
+
+def h3b_graph_capture_blocks(dims: Dims, blocks, c, x, ws) -> Graph:
+    arr = (BlockWeights * len(blocks))(*blocks)
+    h = C.c_void_p()
+    _check(lib().h3b_graph_capture_blocks(C.byref(dims), arr, len(blocks), _p(c), _p(x), _p(ws),
+                                          ws.numel() * ws.element_size(), C.byref(h)), "h3b_graph_capture_blocks")
+    return Graph(h.value, (dims, arr))
 
 
 def h3b_blocks_forward_reduced(full: Dims, ws_list: Sequence[BlockWeights], first: int, last: int, c, x, xm, ym,

@@ -48,6 +48,9 @@ class Workload:
     ln_eps: float = 1e-6
     # multi-block pass: blocks [first, last) run on the paired grid (empty: none)
     pair_blocks: Tuple[int, int] = (0, 0)
+    # residual reuse: a step is one fresh pass (blocks [first, last) run, their delta is
+    # cached) and one reuse pass (the range is replaced by the cached delta)
+    reuse_blocks: Tuple[int, int] = (0, 0)
 
     @property
     def L(self) -> int:
@@ -56,7 +59,8 @@ class Workload:
     def merged(self) -> "Workload":
         """The grid the block sees under token reduction (W halved)."""
         assert self.W % 2 == 0
-        return self.with_(name=self.name + "/merged", W=self.W // 2, token_pair=False, pair_blocks=(0, 0))
+        return self.with_(name=self.name + "/merged", W=self.W // 2, token_pair=False, pair_blocks=(0, 0),
+                          reuse_blocks=(0, 0))
 
     def with_(self, **kw) -> "Workload":
         args = dict(self.__dict__)
@@ -89,6 +93,9 @@ for _T in (2, 4, 8, 12, 16):
 # the same pass with token reduction over the middle half of the blocks (13..37)
 WORKLOADS["d5120_depth50_T8_pairmid"] = _large(8, name="d5120_depth50_T8_pairmid", n_blocks=50,
                                                pair_blocks=(13, 38))
+# two denoise steps of the pass: fresh (blocks 13..37 run, their delta cached), then reuse
+WORKLOADS["d5120_depth50_T8_reuse"] = _large(8, name="d5120_depth50_T8_reuse", n_blocks=50,
+                                             reuse_blocks=(13, 38))
 
 _TENSOR_IDS = {"x": 1, "outliers": 2, "c": 3, "w_ada": 4, "b_gate": 5, "wqkv": 6, "wo": 7,
                "w1": 8, "w2": 9}
