@@ -193,8 +193,9 @@ H3B_API h3b_status h3b_blocks_forward_reduced(const h3b_dims* full, const h3b_bl
  *   range runs, then delta = x - x_save (fp32, B*L*d). fresh == 0: the range is
  *   skipped and x = bf16(x + delta). first == last: no range (x_save, delta unused).
  *   Same workspace and argument rules as h3b_blocks_forward; x_save and delta
- *   16-byte aligned, owned by the caller; delta must come from a fresh call
- *   with the same dimensions.
+ *   16-byte aligned (H3B_ERR_ALIGN), owned by the caller; a bad range or a
+ *   NULL delta / x_save where needed is H3B_ERR_ARG, checked before anything
+ *   else. delta must come from a fresh call with the same dimensions.
  *   h3b_range_delta / h3b_range_apply: the two steps alone, on n elements
  *   (n % 8 == 0, 16-byte aligned). */
 H3B_API h3b_status h3b_blocks_forward_cached(const h3b_dims* dims, const h3b_block_weights* w, int n_blocks,

@@ -112,3 +112,32 @@ def test_valid_call_without_a_b200_launches_nothing(L):
     # On a host without a compute-capability-10.0 device the call stops at the
     # device query with ARCH or CUDA status; it never reports success.
     assert L.h3b_quantize_weights(0x1000, 4, 16, 0x2000, 0x3000, None) in (-5, -6)
+
+
+def test_reuse_and_graph_validation(L):
+    d = _dims()
+    w = h3b.BlockWeights()
+    for n in h3b.WEIGHT_FIELDS:
+        setattr(w, n, 0x10000)
+    arr = (h3b.BlockWeights * 4)(w, w, w, w)
+    x, c, ws, xs, dl = 0x20000, 0x30000, 0x40000, 0x50000, 0x60000
+    need = h3b.h3b_workspace_size(d)
+    f = L.h3b_blocks_forward_cached
+    # range outside [0, n_blocks] or reversed; a missing delta or x_save where the range needs it
+    assert f(C.byref(d), arr, 4, 3, 2, 1, c, x, xs, dl, ws, need, None) == -1
+    assert f(C.byref(d), arr, 4, 1, 5, 1, c, x, xs, dl, ws, need, None) == -1
+    assert f(C.byref(d), arr, 4, 1, 3, 0, c, x, None, None, ws, need, None) == -1
+    assert f(C.byref(d), arr, 4, 1, 3, 1, c, x, None, dl, ws, need, None) == -1
+    assert f(C.byref(d), arr, 4, 1, 3, 1, c, x, xs + 4, dl, ws, need, None) == -3
+    # the elementwise steps alone
+    assert L.h3b_range_delta(0x1000, 0x2000, 0x3000, 12, None) == -2
+    assert L.h3b_range_delta(None, 0x2000, 0x3000, 16, None) == -1
+    assert L.h3b_range_apply(0x1008, 0x3000, 16, None) == -3
+    # bf16 gated residual GEMM: gate and its stride are checked first
+    assert L.h3b_gemm_bf16_gated_residual(0x1000, 0x2000, None, None, 1, 256, 0x3000, 128, 256, 128, None) == -1
+    assert L.h3b_gemm_bf16_gated_residual(0x1000, 0x2000, None, 0x4000, 0, 256, 0x3000, 128, 256, 128, None) == -1
+    # graph handles
+    assert L.h3b_graph_capture_blocks(C.byref(d), arr, 4, c, x, ws, need, None) == -1
+    assert L.h3b_graph_launch(None, None) == -1
+    assert L.h3b_graph_kernel_count(None) == 0
+    L.h3b_graph_destroy(None)  # a no-op

@@ -434,15 +434,18 @@ h3b_status h3b_blocks_forward(const h3b_dims* dims, const h3b_block_weights* w, 
 h3b_status h3b_blocks_forward_cached(const h3b_dims* dims, const h3b_block_weights* w, int n_blocks, int first,
                                      int last, int fresh, const float* c, void* x, void* x_save, float* delta,
                                      void* ws, size_t ws_bytes, h3b_stream stream) {
+  // host-only checks of the range arguments first, then the common block checks
+  if (n_blocks < 0 || (n_blocks > 0 && !w)) return fail(H3B_ERR_ARG, "n_blocks < 0 or weights NULL");
+  if (first < 0 || first > last || last > n_blocks) return fail(H3B_ERR_ARG, "need 0 <= first <= last <= n_blocks");
+  const bool range = first < last;
+  if (range && !delta) return fail(H3B_ERR_ARG, "delta NULL");
+  if (range && fresh && !x_save) return fail(H3B_ERR_ARG, "x_save NULL");
+  if ((range && !aligned16(delta)) || (range && fresh && !aligned16(x_save)))
+    return fail(H3B_ERR_ALIGN, "delta / x_save not 16-byte aligned");
   WsLayout lay;
   DeviceInfo* di = nullptr;
   h3b_status s = block_common(dims, c, x, ws, ws_bytes, &lay, &di);
   if (s != H3B_OK) return s;
-  if (n_blocks < 0 || (n_blocks > 0 && !w)) return fail(H3B_ERR_ARG, "n_blocks < 0 or weights NULL");
-  if (first < 0 || first > last || last > n_blocks) return fail(H3B_ERR_ARG, "need 0 <= first <= last <= n_blocks");
-  const bool range = first < last;
-  if (range && (!delta || !aligned16(delta))) return fail(H3B_ERR_ARG, "delta NULL or not 16-byte aligned");
-  if (range && fresh && (!x_save || !aligned16(x_save))) return fail(H3B_ERR_ARG, "x_save NULL or not 16-byte aligned");
   for (int i = 0; i < n_blocks; ++i)
     if ((s = check_weights(*dims, &w[i])) != H3B_OK) return s;
   cudaStream_t st = stream;
@@ -745,12 +748,12 @@ h3b_status h3b_gemm_bf16_gated_residual(const void* A, const void* W, const floa
                                         int rows_per_item, int gate_stride, void* x, int M, int N, int K,
                                         h3b_stream stream) {
   cudaStream_t st = stream;
-  DeviceInfo* di = nullptr;
-  h3b_status s = gemm_common(A, W, x, M, N, K, &di);
-  if (s != H3B_OK) return s;
   if (!gate) return fail(H3B_ERR_ARG, "gate NULL");
   if (rows_per_item < 1 || gate_stride < 0 || gate_stride % 4 != 0) return fail(H3B_ERR_ARG, "rows_per_item/gate_stride");
   if (!aligned16(gate) || (bias && !aligned16(bias))) return fail(H3B_ERR_ALIGN, "alignment");
+  DeviceInfo* di = nullptr;
+  h3b_status s = gemm_common(A, W, x, M, N, K, &di);
+  if (s != H3B_OK) return s;
   GemmArgs a = base_args(M, N, K, di->err);
   a.bias = bias; a.out = x;
   a.gate = gate; a.rows_per_item = rows_per_item; a.gate_stride = gate_stride;
