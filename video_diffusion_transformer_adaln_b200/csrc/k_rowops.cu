@@ -650,16 +650,11 @@ static cudaError_t ln_dispatch(const void* x, int rows, int nv, float eps, const
   const int rpp_d = block / tpr;
   const size_t smem = (size_t)vpr * 4 * sizeof(float4) + (size_t)rpp_d * vpr * sizeof(uint4);
   auto kern = ln_mod_quant_kernel<VPT>;
-  static int attr_done = 0;
-  if (!attr_done) {
-    // the largest row (d = 8192, 1024 vectors): 64 KB of (1 + scale, shift) pairs + 16 KB staging
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)(32 * 32 * 4 * sizeof(float4) + 32 * 32 * sizeof(uint4)));
-    if (e != cudaSuccess) return e;
-    attr_done = 1;
-  }
+  // the attribute belongs to the current device, so it is set on every launch (a host-side call)
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
   int per_sm = 0;
-  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, block, smem);
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, block, smem);
   if (e != cudaSuccess) return e;
   if (per_sm < 1) per_sm = 1;
   const int rpp = block / tpr;
