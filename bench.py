@@ -25,7 +25,6 @@ total tokens/s of all ranks over the slowest rank's device time.
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl h3b|reference]
 """
 import argparse
-import datetime
 import json
 import os
 import statistics
@@ -41,7 +40,7 @@ import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
 from video_diffusion_transformer_adaln_b200 import build as cuda_build  # noqa: E402
-from video_diffusion_transformer_adaln_b200 import h3b, synth  # noqa: E402
+from video_diffusion_transformer_adaln_b200 import h3b, replicas, synth  # noqa: E402
 from video_diffusion_transformer_adaln_b200.runtime import (DeviceBlock, bf16_from_bits, dims_of,  # noqa: E402
                                                             workspace)
 
@@ -179,7 +178,7 @@ class Workload:
     def __init__(self, name, rank):
         self.wl = synth.WORKLOADS[name]
         wl = self.wl
-        seed = synth.BASE_SEED + rank  # one independent latent per rank
+        seed = replicas.latent_seed(rank)  # one independent latent per rank
         self.name = name
         x_bits = synth.x_input(wl, seed)
         self.x_ref = bf16_from_bits(x_bits, "cuda")
@@ -283,42 +282,11 @@ class OracleRunner:
 
 # ----------------------------------------------------------------------------- arms
 
-def dist_init():
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                device_id=torch.device("cuda", local))
-    else:
-        torch.cuda.set_device(0)
-    return rank, world, local
-
-
-def barrier(world):
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
-
-
-def max_over_ranks(v, world):
-    if world == 1:
-        return v
-    import torch.distributed as dist
-    t = torch.tensor([float(v)], device="cuda", dtype=torch.float64)
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
-
-
-def sum_over_ranks(v, world):
-    if world == 1:
-        return v
-    import torch.distributed as dist
-    t = torch.tensor([float(v)], device="cuda", dtype=torch.float64)
-    dist.all_reduce(t, op=dist.ReduceOp.SUM)
-    return float(t.item())
+# multi-GPU bookkeeping (replicas, no data-path collective): see replicas.py
+dist_init = lambda: replicas.init("nccl")  # noqa: E731
+barrier = replicas.barrier
+max_over_ranks = replicas.max_over_ranks
+sum_over_ranks = replicas.sum_over_ranks
 
 
 def run_h3b(args, rank, world, local):
