@@ -48,6 +48,7 @@ METRIC = "DiT block tokens/s (int8 MLP+QKV, bf16 attn); % of B200 INT8/BF16/HBM 
 UNIT = "tokens/s"
 DEFAULT_WORKLOAD = "d2048_L4096"
 L2_FLUSH_BYTES = 512 << 20
+E2E_FLUSH_BYTES = 160 << 20  # larger than the 126 MB L2
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # the recipe's nominal dense ratio of 8-bit to bf16 tensor throughput (4.5 / 2.25 PFLOP/s)
 INT8_OVER_BF16 = 2.0
@@ -353,35 +354,66 @@ def run_h3b(args, rank, world, local):
     tokens_all = sum_over_ranks(W.tokens * args.steps, world)
     value = tokens_all / (total_ms / 1e3)
 
-    # ---- end to end: pinned host input -> device -> pass -> host output, same API
+    # ---- end to end through the same API: every step copies its input (x, c) from pinned host
+    # memory, runs the pass and copies its result back into pinned host memory. Steps are
+    # pipelined over two device buffers and three streams: step i+1's input copy and step
+    # i-1's result copy overlap step i's pass. Before each pass the compute stream rewrites a
+    # buffer larger than L2 (inside the timed region).
     x_host = torch.empty(W.x.shape, dtype=torch.bfloat16, pin_memory=True)
     x_host.copy_(W.x_ref.cpu())
     c_host = torch.empty(W.c.shape, dtype=W.c.dtype, pin_memory=True)
     c_host.copy_(W.c.cpu())
-    out_host = torch.empty_like(x_host, pin_memory=True)
+    out_host = [torch.empty_like(x_host, pin_memory=True) for _ in range(2)]
+    xs = [W.x, torch.empty_like(W.x)]
+    cs = [W.c, torch.empty_like(W.c)]
+    graphs = None
+    if graph is not None:
+        graphs = [graph, h3b.h3b_graph_capture_blocks(W.dims, [b.struct for b in W.blocks], cs[1], xs[1], W.ws)]
+    e2e_flush = flush[:E2E_FLUSH_BYTES]
+    s_h2d, s_comp, s_d2h = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+
+    def e2e_run(n):
+        h2d_done = [torch.cuda.Event() for _ in range(n)]
+        comp_done = [torch.cuda.Event() for _ in range(n)]
+        d2h_done = [torch.cuda.Event() for _ in range(n)]
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        t0.record(s_h2d)
+        for i in range(n):
+            k = i % 2
+            with torch.cuda.stream(s_h2d):
+                if i >= 2:
+                    s_h2d.wait_event(d2h_done[i - 2])  # buffer k is free again
+                xs[k].copy_(x_host, non_blocking=True)
+                cs[k].copy_(c_host, non_blocking=True)
+                h2d_done[i].record(s_h2d)
+            with torch.cuda.stream(s_comp):
+                s_comp.wait_event(h2d_done[i])
+                e2e_flush.zero_()
+                if graphs is not None:
+                    graphs[k].launch(s_comp)
+                else:
+                    W.step(x=xs[k], c=cs[k])
+                comp_done[i].record(s_comp)
+            with torch.cuda.stream(s_d2h):
+                s_d2h.wait_event(comp_done[i])
+                out_host[k].copy_(xs[k], non_blocking=True)
+                d2h_done[i].record(s_d2h)
+        s_d2h.wait_event(d2h_done[n - 1])
+        t1.record(s_d2h)
+        torch.cuda.synchronize()
+        return t0.elapsed_time(t1)
+
     e2e_steps = max(3, min(args.steps, 20))
-    for _ in range(2):
-        W.x.copy_(x_host, non_blocking=True)
-        W.c.copy_(c_host, non_blocking=True)
-        run_step()
-        out_host.copy_(W.x, non_blocking=True)
-    torch.cuda.synchronize()
+    e2e_run(2)
     barrier(world)
-    eev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(e2e_steps)]
-    for i in range(e2e_steps):
-        flush.zero_()
-        eev[i][0].record()
-        W.x.copy_(x_host, non_blocking=True)
-        W.c.copy_(c_host, non_blocking=True)  # the graph reads c from this buffer
-        run_step()
-        out_host.copy_(W.x, non_blocking=True)
-        eev[i][1].record()
-    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e2e_run(e2e_steps), world)
     barrier(world)
-    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in eev), world)
+    if graphs is not None:
+        graphs[1].destroy()
     e2e_value = sum_over_ranks(W.tokens * e2e_steps, world) / (e2e_ms / 1e3)
     h2d = x_host.numel() * x_host.element_size() + c_host.numel() * c_host.element_size()
-    d2h = out_host.numel() * out_host.element_size()
+    d2h = out_host[0].numel() * out_host[0].element_size()
     launch = {"mode": "graph" if graph is not None else "stream",
               "stream_ms_per_step": round(stream_ms / args.steps, 4),
               "profiled_ms_per_step": round(prof_ms / args.steps, 4)}
@@ -448,7 +480,8 @@ def run_h3b(args, rank, world, local):
         "kernel_ms_per_step": kernel_ms, "launch_gap_ms_per_step": round(gap_ms, 4), "launch": launch,
         "cpu_baseline": cpu,
         "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "steps": e2e_steps},
+                "steps": e2e_steps, "pipelined": True,
+                "l2": f"a {E2E_FLUSH_BYTES >> 20} MiB write on the compute stream before each pass, inside the timed region"},
         "gpu_launches": gpu_launches, "clocks": clocks,
     }
     if rank == 0:
