@@ -20,8 +20,11 @@
 // 4-stage shared-memory ring; warp 1 issues tcgen05.mma from one thread into a
 // double-buffered TMEM accumulator (2 x 256 columns); warps 2-9 (two per
 // sub-partition, each half of the columns) drain the other accumulator
-// (tcgen05.ld) and run the epilogue while the next tile's MMAs proceed. Every
-// wait is bounded.
+// (tcgen05.ld) and run the epilogue while the next tile's MMAs proceed: each
+// warp stages its columns' weight scales, bias and gate in shared memory before
+// the accumulator wait, requests the next 32 accumulator columns before
+// processing the current ones, and (QKV) reads the RoPE table from shared
+// memory. Every wait is bounded.
 #include "h3b_common.cuh"
 #include "h3b_internal.h"
 

@@ -1,9 +1,13 @@
 // Memory-bound kernels of the block: AdaLN modulation GEMV, the fused
 // LayerNorm + modulation + per-row int8 quantizer, the quant-only pass, the
-// per-output-channel weight quantizer, token pairing and the RoPE table.
+// per-output-channel weight quantizer, token pairing, the residual-reuse delta
+// and its re-application, and the RoPE table.
 //
-// All of them stream rows with 16-byte vector accesses, one warp (or block)
-// per row, with warp-shuffle reductions; none keeps state between launches.
+// All of them stream with 16-byte vector accesses and keep no state between
+// launches. The GEMV gives a warp one output row; the LN quantizer spreads a
+// row over 1-8 warps (warp shuffles, then one shared slot per warp) and stages
+// its next rows with cp.async; the quant pass and the elementwise kernels
+// stream whole rows or flat ranges.
 //
 // Method references (web pages on the h3.c / h3-metal engine):
 //   "h3-metal: Apple Silicon을 위한 네이티브 MiniMax-H3 추론", section "Int8 양자화":
