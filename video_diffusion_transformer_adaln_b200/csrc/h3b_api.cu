@@ -245,7 +245,7 @@ h3b_status run_block(const h3b_dims& d, const h3b_block_weights& w, const float*
 
   // a1: AdaLN modulation vectors (the same launch fills the RoPE table when needed)
   H3B_CK(launch_adaln_gemv(w.w_ada, w.b_ada, c, d.B, D, mod, rope_ready ? nullptr : rope, d.T, d.H, d.W,
-                           d.rope_t, d.rope_h, d.rope_w, d.rope_theta, st), "adaln_gemv");
+                           d.rope_t, d.rope_h, d.rope_w, d.rope_theta, di.sms, st), "adaln_gemv");
   // a2: LN + modulation + quantization (or the bf16 activation for bf16 QKV)
   if (d.qkv_int8)
     H3B_CK(launch_ln_mod_quant(x, R, D, d.ln_eps, mod, mod + D, L, 6 * D, act, sA, nullptr, absmax, 1, di.err, di.sms, st), "ln_mod_quant");
@@ -271,7 +271,7 @@ h3b_status run_block(const h3b_dims& d, const h3b_block_weights& w, const float*
   // a6: output projection + gated residual (gate_attn = chunk 2): int8 on the quantized
   // attention output (a5), or bf16 directly on the bf16 attention output
   if (!d.wo_bf16) {
-    H3B_CK(launch_quant_rows_bf16(o, R, D, absmax, act, sA, st), "quant_o");
+    H3B_CK(launch_quant_rows_bf16(o, R, D, absmax, act, sA, di.sms, st), "quant_o");
     GemmArgs a = base_args(R, D, D, di.err);
     a.sA = sA; a.sW = w.so; a.bias = w.bo; a.out = x;
     a.gate = mod + 2 * D; a.rows_per_item = L; a.gate_stride = 6 * D;
@@ -290,7 +290,7 @@ h3b_status run_block(const h3b_dims& d, const h3b_block_weights& w, const float*
     a.sA = sA; a.sW = w.s1; a.bias = w.b1; a.out = g; a.absmax = absmax;
     H3B_CK(launch_gemm(true, EPI_GELU, act, w.w1, a, di.sms, st), "gemm_w1");
   }
-  H3B_CK(launch_quant_rows_bf16(g, R, F, absmax, act, sA, st), "quant_g");
+  H3B_CK(launch_quant_rows_bf16(g, R, F, absmax, act, sA, di.sms, st), "quant_g");
   // a9: W2 + gated residual (gate_mlp = chunk 5)
   {
     GemmArgs a = base_args(R, D, F, di.err);
@@ -612,7 +612,7 @@ h3b_status h3b_adaln_modulation(const h3b_dims* dims, const void* w_ada, const f
   if (!aligned16(w_ada) || !aligned16(c) || !aligned16(mod)) return fail(H3B_ERR_ALIGN, "alignment");
   DeviceInfo* di = nullptr;
   if ((s = device_info(&di)) != H3B_OK) return s;
-  H3B_CK(launch_adaln_gemv(w_ada, b_ada, c, dims->B, dims->d, mod, nullptr, 0, 0, 0, 0, 0, 0, 0.0, stream),
+  H3B_CK(launch_adaln_gemv(w_ada, b_ada, c, dims->B, dims->d, mod, nullptr, 0, 0, 0, 0, 0, 0, 0.0, di->sms, stream),
          "adaln_gemv");
   return H3B_OK;
 }
@@ -643,7 +643,7 @@ h3b_status h3b_quantize_rows(const void* h, int rows, int cols, const float* abs
   DeviceInfo* di = nullptr;
   h3b_status hs = device_info(&di);
   if (hs != H3B_OK) return hs;
-  H3B_CK(launch_quant_rows_bf16(h, rows, cols, absmax, q, s, stream), "quantize_rows");
+  H3B_CK(launch_quant_rows_bf16(h, rows, cols, absmax, q, s, di->sms, stream), "quantize_rows");
   return H3B_OK;
 }
 

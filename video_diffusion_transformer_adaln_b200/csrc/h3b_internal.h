@@ -15,13 +15,13 @@ namespace h3b {
 // rope_tab (optional): the same launch also fills the RoPE table (see launch_rope_table).
 cudaError_t launch_adaln_gemv(const void* W_ada, const float* bias, const float* c, int B, int d,
                               float* mod, float2* rope_tab, int T, int H, int W, int rt, int rh, int rw,
-                              double theta, cudaStream_t st);
+                              double theta, int sms, cudaStream_t st);
 cudaError_t launch_ln_mod_quant(const void* x, int rows, int d, float eps, const float* shift,
                                 const float* scale, int rows_per_item, int mod_stride, int8_t* q,
                                 float* s, void* h_out, float* absmax_zero, int write_codes, unsigned* err,
                                 int sms, cudaStream_t st);
 cudaError_t launch_quant_rows_bf16(const void* h, int rows, int cols, const float* absmax,
-                                   int8_t* q, float* s, cudaStream_t st);
+                                   int8_t* q, float* s, int sms, cudaStream_t st);
 cudaError_t launch_quant_rows_f32(const float* w, int rows, int cols, int8_t* q, float* s,
                                   cudaStream_t st);
 cudaError_t launch_token_pair(const void* x, void* xm, void* xm2, long long lines, int W, int d,

@@ -103,8 +103,10 @@ __device__ __forceinline__ uint32_t pack4_i8(int a, int b, int c, int d) {
 // ---------------------------------------------------------------------------
 constexpr int kGemvMaxB = 8;
 
-// One warp per output row j; the row's d/8 16-byte vectors (NV per lane) are
-// all requested before any is used, so each warp keeps its whole row in flight.
+// Persistent blocks: c is staged in shared memory once per block, then each
+// warp walks output rows j = (block * 8 + warp) + k * (blocks * 8). A row's d/8
+// 16-byte vectors (NV per lane) are all requested before any is used, so each
+// warp keeps a whole row in flight.
 struct RopeTableArgs {
   float2* tab;  // nullptr: no table this launch
   int T, H, W, rt, rh, rw;
@@ -127,40 +129,39 @@ __global__ void __launch_bounds__(256) adaln_gemv_kernel(const __nv_bfloat16* __
   }
   extern __shared__ float cs[];  // [B][d]
   for (int i = threadIdx.x; i < B * d; i += blockDim.x) cs[i] = c[i];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int j = blockIdx.x * 8 + warp;
-  const bool valid = j < 6 * d;
-  const uint4* wr = reinterpret_cast<const uint4*>(W + (size_t)(valid ? j : 0) * d);
-  uint4 w4[NV];
-#pragma unroll
-  for (int i = 0; i < NV; ++i) w4[i] = __ldcs(wr + lane + 32 * i);
   __syncthreads();
-  if (!valid) return;
-  float acc[kGemvMaxB];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int j = blockIdx.x * 8 + warp; j < 6 * d; j += gemv_blocks * 8) {  // warp-uniform
+    const uint4* wr = reinterpret_cast<const uint4*>(W + (size_t)j * d);
+    uint4 w4[NV];
 #pragma unroll
-  for (int b = 0; b < kGemvMaxB; ++b) acc[b] = 0.0f;
+    for (int i = 0; i < NV; ++i) w4[i] = __ldcs(wr + lane + 32 * i);
+    float acc[kGemvMaxB];
 #pragma unroll
-  for (int i = 0; i < NV; ++i) {
-    const uint32_t ww[4] = {w4[i].x, w4[i].y, w4[i].z, w4[i].w};
-    const int v = lane + 32 * i;
+    for (int b = 0; b < kGemvMaxB; ++b) acc[b] = 0.0f;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      const uint32_t ww[4] = {w4[i].x, w4[i].y, w4[i].z, w4[i].w};
+      const int v = lane + 32 * i;
+#pragma unroll
+      for (int b = 0; b < kGemvMaxB; ++b) {
+        if (b >= B) break;
+        const float4 c0 = *reinterpret_cast<const float4*>(cs + b * d + v * 8);
+        const float4 c1 = *reinterpret_cast<const float4*>(cs + b * d + v * 8 + 4);
+        float a = acc[b];
+        a = fmaf(bf16_lo(ww[0]), c0.x, a); a = fmaf(bf16_hi(ww[0]), c0.y, a);
+        a = fmaf(bf16_lo(ww[1]), c0.z, a); a = fmaf(bf16_hi(ww[1]), c0.w, a);
+        a = fmaf(bf16_lo(ww[2]), c1.x, a); a = fmaf(bf16_hi(ww[2]), c1.y, a);
+        a = fmaf(bf16_lo(ww[3]), c1.z, a); a = fmaf(bf16_hi(ww[3]), c1.w, a);
+        acc[b] = a;
+      }
+    }
 #pragma unroll
     for (int b = 0; b < kGemvMaxB; ++b) {
       if (b >= B) break;
-      const float4 c0 = *reinterpret_cast<const float4*>(cs + b * d + v * 8);
-      const float4 c1 = *reinterpret_cast<const float4*>(cs + b * d + v * 8 + 4);
-      float a = acc[b];
-      a = fmaf(bf16_lo(ww[0]), c0.x, a); a = fmaf(bf16_hi(ww[0]), c0.y, a);
-      a = fmaf(bf16_lo(ww[1]), c0.z, a); a = fmaf(bf16_hi(ww[1]), c0.w, a);
-      a = fmaf(bf16_lo(ww[2]), c1.x, a); a = fmaf(bf16_hi(ww[2]), c1.y, a);
-      a = fmaf(bf16_lo(ww[3]), c1.z, a); a = fmaf(bf16_hi(ww[3]), c1.w, a);
-      acc[b] = a;
+      const float r = warp_sum(acc[b]);
+      if (lane == 0) mod[(size_t)b * 6 * d + j] = r + (bias ? bias[j] : 0.0f);
     }
-  }
-#pragma unroll
-  for (int b = 0; b < kGemvMaxB; ++b) {
-    if (b >= B) break;
-    const float r = warp_sum(acc[b]);
-    if (lane == 0) mod[(size_t)b * 6 * d + j] = r + (bias ? bias[j] : 0.0f);
   }
 }
 
@@ -604,15 +605,18 @@ __global__ void rope_table_kernel(const RopeTableArgs r) {
 // ---------------------------------------------------------------------------
 template <int NV>
 static cudaError_t gemv_dispatch(const void* W, const float* bias, const float* c, int B, float* mod,
-                                 const RopeTableArgs& rope, cudaStream_t st) {
+                                 const RopeTableArgs& rope, int sms, cudaStream_t st) {
   constexpr int d = NV * 256;
   const size_t smem = (size_t)B * d * sizeof(float);
-  if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(adaln_gemv_kernel<NV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
-    if (e != cudaSuccess) return e;
-  }
-  const int gemv_blocks = (6 * d + 7) / 8;
+  cudaError_t e = cudaFuncSetAttribute(adaln_gemv_kernel<NV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, adaln_gemv_kernel<NV>, 256, smem);
+  if (e != cudaSuccess) return e;
+  per_sm = per_sm < 1 ? 1 : per_sm;
+  // persistent blocks, as many as are resident at once, at most one per 8 output rows
+  const int gemv_blocks = std::min((6 * d + 7) / 8, sms * per_sm);
   int rope_blocks = 0;
   if (rope.tab) {
     const int n = rope.T * (rope.rt / 2) + rope.H * (rope.rh / 2) + rope.W * (rope.rw / 2);
@@ -625,12 +629,12 @@ static cudaError_t gemv_dispatch(const void* W, const float* bias, const float* 
 
 cudaError_t launch_adaln_gemv(const void* W, const float* bias, const float* c, int B, int d,
                               float* mod, float2* rope_tab, int T, int H, int Wd, int rt, int rh, int rw,
-                              double theta, cudaStream_t st) {
+                              double theta, int sms, cudaStream_t st) {
   if (B > kGemvMaxB || d % 256 != 0) return cudaErrorInvalidValue;
   const RopeTableArgs rope{rope_tab, T, H, Wd, rt, rh, rw, theta};
 #define H3B_GV(nv) \
   case nv:         \
-    return gemv_dispatch<nv>(W, bias, c, B, mod, rope, st);
+    return gemv_dispatch<nv>(W, bias, c, B, mod, rope, sms, st);
   switch (d / 256) {
     H3B_GV(1) H3B_GV(2) H3B_GV(3) H3B_GV(4) H3B_GV(5) H3B_GV(6) H3B_GV(7) H3B_GV(8)
     H3B_GV(9) H3B_GV(10) H3B_GV(11) H3B_GV(12) H3B_GV(13) H3B_GV(14) H3B_GV(15) H3B_GV(16)
@@ -690,13 +694,14 @@ cudaError_t launch_ln_mod_quant(const void* x, int rows, int d, float eps, const
 }
 
 cudaError_t launch_quant_rows_bf16(const void* h, int rows, int cols, const float* absmax,
-                                   int8_t* q, float* s, cudaStream_t st) {
+                                   int8_t* q, float* s, int sms, cudaStream_t st) {
   if (rows == 0) return cudaSuccess;
   if (absmax) {
     const int vpr = cols / 8;
     // about 4096 vectors (64 KB of input) per block: each thread keeps four 16-byte loads in
     // flight over four rounds, and the per-block setup is amortized over several rows
     int rpb = 4096 / vpr;
+    rpb = std::min(rpb, rows / (4 * sms));  // but at least about four blocks per SM
     rpb = rpb < 1 ? 1 : (rpb > kQuantMaxRowsPerBlock ? kQuantMaxRowsPerBlock : rpb);
     quant_rows_known_absmax_kernel<<<(rows + rpb - 1) / rpb, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(h),
                                                                           rows, vpr, rpb, absmax, q, s);
