@@ -119,7 +119,7 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 }
 
 // ----------------------------------------------------------------------------
-// TMA tile loads (no multicast), completing on an mbarrier with a byte count.
+// TMA tile loads into this CTA's own shared memory, completing on an mbarrier with a byte count.
 // ----------------------------------------------------------------------------
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
