@@ -52,3 +52,23 @@ def test_bf16_encoding_of_draws():
 def test_sample_rows():
     r = synth.sample_rows(1000, 20)
     assert r[0] == 0 and r[-1] == 999 and len(set(r.tolist())) == 20 and np.all(np.diff(r) > 0)
+
+
+def test_variant_workloads():
+    W = synth.WORKLOADS
+    base = W["d5120_L18432"]
+    # the variants share the base block's draws (same sizes), differing only in flags
+    for name, flag in (("d5120_L18432_bf16wo", "wo_bf16"), ("d5120_L18432_bf16qkv", "qkv_int8")):
+        v = W[name]
+        assert (v.T, v.H, v.W, v.d, v.d_ff) == (base.T, base.H, base.W, base.d, base.d_ff)
+        assert getattr(v, flag) != getattr(base, flag)
+    small = synth.WORKLOADS["d256_L512"].with_(wo_bf16=True)
+    w = synth.block_weights(small)
+    assert np.array_equal(w["wo_bf16"], synth.f32_to_bf16_bits(w["wo"]))
+    # ranges of the multi-block variants lie inside the pass; merging clears them
+    for name, field in (("d5120_depth50_T8_pairmid", "pair_blocks"), ("d5120_depth50_T8_reuse", "reuse_blocks")):
+        v = W[name]
+        first, last = getattr(v, field)
+        assert 0 <= first < last <= v.n_blocks == 50
+        m = v.merged()
+        assert m.pair_blocks == (0, 0) and m.reuse_blocks == (0, 0) and m.W == v.W // 2
