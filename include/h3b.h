@@ -71,7 +71,9 @@ typedef enum {
  *   Latent grid T x H x W per batch item, flattened t-major, then h, then w:
  *   token l = (t*H + h)*W + w, L = T*H*W. B independent batch items.
  *   d = n_heads * head_dim; head_dim in {64, 128}; d % 256 == 0, d <= 8192;
- *   d_ff % 256 == 0, d_ff <= 32768.
+ *   d_ff % 256 == 0, d_ff <= 32768; 1 <= B <= 8; B*L < 2^31 tokens and
+ *   B*L*d_ff <= 2^40 (H3B_ERR_SHAPE otherwise, checked without overflow for
+ *   any int extents).
  *   RoPE: rope_t + rope_h + rope_w == head_dim, each even (3D RoPE; lanes
  *   [0,rope_t) rotate with t, the next rope_h with h, the rest with w; pair
  *   (2j, 2j+1) of a segment of length r has frequency rope_theta^(-2j/r)).
@@ -231,7 +233,8 @@ H3B_API void h3b_graph_destroy(h3b_graph g);
 
 /* Token reduction ("Token Reduction" row of the control table): horizontally
  * adjacent tokens w = 2k, 2k+1 of each (t, h) row are merged by their mean.
- *   full: dims of the UNMERGED grid (W even).
+ *   full: dims of the UNMERGED grid (W even); only B, T, H, W and d are read:
+ *   d % 8 == 0, d <= 65536, B*T*H*W < 2^31 (H3B_ERR_SHAPE otherwise).
  *   x  bf16 [B][T][H][W][d] -> xm bf16 [B][T][H][W/2][d], xm = bf16((a+b)/2).
  *   xm_copy: optional second destination receiving the same merged tokens
  *   (e.g. the buffer the block then updates in place), or NULL. */
@@ -323,7 +326,8 @@ H3B_API size_t h3b_rope_table_bytes(const h3b_dims* dims);
 
 /* Non-causal attention per batch item and head on the head-major qkv buffer.
  * o bf16 [B][L][d] (token-major, head h at columns [h*head_dim, (h+1)*head_dim));
- * absmax fp32 [B*L]: each row's max |o| is max-combined into it (zero it first). */
+ * absmax fp32 [B*L]: each row's max |o| is max-combined into it (zero it first).
+ * Reads B, T, H, W, n_heads and head_dim only: B*n_heads <= 65535, B*L < 2^31. */
 H3B_API h3b_status h3b_attention(const h3b_dims* dims, const void* qkv, void* o, float* absmax,
                          h3b_stream stream);
 

@@ -92,6 +92,30 @@ def test_block_forward_validation_order(L):
     assert st in (-1, -5, -6)  # weights are checked after the device query on a GPU-less host
 
 
+@pytest.mark.parametrize("T,H,W", [(2 ** 31 - 1, 2 ** 31 - 1, 2 ** 31 - 1), (65536, 65536, 2),
+                                   (2 ** 20, 2 ** 11, 1), (1, 2, 2 ** 30), (2 ** 16, 2 ** 16, 2 ** 16)])
+def test_grids_of_2_31_tokens_or_more_are_rejected_without_overflow(L, T, H, W):
+    # Extents whose product wraps a 64-bit integer, or lands exactly on 2^31, must
+    # not pass the size checks of any entry point that takes the grid.
+    d = _dims(T=T, H=H, W=W)
+    with pytest.raises(h3b.H3BError) as e:
+        h3b.h3b_workspace_size(d)
+    assert e.value.status == -2
+    full = _dims(T=T, H=H, W=W + (W & 1))
+    assert L.h3b_token_pair(C.byref(full), 0x1000, 0x2000, None, None) == -2
+    assert L.h3b_token_unpair(C.byref(full), 0x1000, 0x2000, 0x3000, 0x4000, None) == -2
+    assert L.h3b_attention(C.byref(d), 0x1000, 0x2000, 0x3000, None) == -2
+
+
+def test_batch_times_grid_limit(L):
+    # B * L must stay below 2^31 even when L alone is below it.
+    big = _dims(B=2, T=2 ** 15, H=2 ** 10, W=2 ** 5)  # L = 2^30, B*L = 2^31
+    with pytest.raises(h3b.H3BError):
+        h3b.h3b_workspace_size(big)
+    assert L.h3b_attention(C.byref(big), 0x1000, 0x2000, 0x3000, None) == -2
+    assert L.h3b_token_pair(C.byref(big), 0x1000, 0x2000, None, None) == -2
+
+
 def test_token_pair_validation(L):
     full = _dims(W=15)
     assert L.h3b_token_pair(C.byref(full), 0x1000, 0x2000, None, None) == -2

@@ -80,6 +80,17 @@ h3b_status device_info(DeviceInfo** out) {
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
+// Tokens of a T x H x W latent grid, or -1 when an extent is below 1 or the count
+// reaches 2^31. The product is formed one factor at a time, each step below 2^62,
+// so no extents a caller can pass make it overflow.
+long long grid_tokens(long long T, long long H, long long W) {
+  const long long lim = 1LL << 31;
+  if (T < 1 || H < 1 || W < 1 || T >= lim || H >= lim || W >= lim) return -1;
+  if (T * H >= lim) return -1;
+  const long long L = T * H * W;
+  return L >= lim ? -1 : L;
+}
+
 h3b_status check_dims(const h3b_dims* d) {
   if (!d) return fail(H3B_ERR_ARG, "dims is NULL");
   if (d->B < 1 || d->T < 1 || d->H < 1 || d->W < 1) return fail(H3B_ERR_SHAPE, "B, T, H, W must be >= 1");
@@ -93,9 +104,9 @@ h3b_status check_dims(const h3b_dims* d) {
       d->rope_t + d->rope_h + d->rope_w != d->head_dim)
     return fail(H3B_ERR_SHAPE, "rope split must be even parts summing to head_dim");
   if (!(d->rope_theta > 0.0f) || !(d->ln_eps >= 0.0f)) return fail(H3B_ERR_ARG, "rope_theta > 0 and ln_eps >= 0");
-  const long long L = (long long)d->T * d->H * d->W;
+  const long long L = grid_tokens(d->T, d->H, d->W);
+  if (L < 0 || L * d->B >= (1LL << 31)) return fail(H3B_ERR_SHAPE, "too many tokens");
   if (L * d->B * (long long)d->d_ff > (1LL << 40)) return fail(H3B_ERR_SHAPE, "problem too large");
-  if (L * d->B >= (1LL << 31)) return fail(H3B_ERR_SHAPE, "too many tokens");
   return H3B_OK;
 }
 
@@ -546,7 +557,10 @@ static h3b_status check_pair_dims(const h3b_dims* full) {
   if (!full) return fail(H3B_ERR_ARG, "dims is NULL");
   if (full->B < 1 || full->T < 1 || full->H < 1 || full->W < 2) return fail(H3B_ERR_SHAPE, "bad grid");
   if (full->W % 2 != 0) return fail(H3B_ERR_SHAPE, "W must be even for token pairing");
-  if (full->d < 8 || full->d % 8 != 0) return fail(H3B_ERR_SHAPE, "d must be a multiple of 8");
+  if (full->d < 8 || full->d % 8 != 0 || full->d > 65536)
+    return fail(H3B_ERR_SHAPE, "d must be a multiple of 8, <= 65536");
+  const long long L = grid_tokens(full->T, full->H, full->W);
+  if (L < 0 || L * full->B >= (1LL << 31)) return fail(H3B_ERR_SHAPE, "too many tokens");
   return H3B_OK;
 }
 
@@ -716,7 +730,8 @@ h3b_status h3b_attention(const h3b_dims* dims, const void* qkv, void* o, float* 
     return fail(H3B_ERR_SHAPE, "B, T, H, W, n_heads must be >= 1");
   if (dims->head_dim != 64 && dims->head_dim != 128) return fail(H3B_ERR_SHAPE, "head_dim must be 64 or 128");
   if ((long long)dims->B * dims->n_heads > 65535) return fail(H3B_ERR_SHAPE, "B * n_heads must be <= 65535");
-  if ((long long)dims->T * dims->H * dims->W >= (1LL << 31)) return fail(H3B_ERR_SHAPE, "too many tokens");
+  const long long L_tokens = grid_tokens(dims->T, dims->H, dims->W);
+  if (L_tokens < 0 || L_tokens * dims->B >= (1LL << 31)) return fail(H3B_ERR_SHAPE, "too many tokens");
   h3b_status s = H3B_OK;
   if (!qkv || !o || !absmax) return fail(H3B_ERR_ARG, "NULL pointer");
   if (!aligned16(qkv) || !aligned16(o)) return fail(H3B_ERR_ALIGN, "alignment");
