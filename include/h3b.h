@@ -34,6 +34,10 @@
  *     reported as H3B_ERR_CUDA. Kernel faults surface at the caller's next
  *     synchronization, as for any CUDA launch.
  *   - Every device pointer must be 16-byte aligned.
+ *   - A step entry point given an empty problem (M, rows or n equal to 0)
+ *     returns H3B_OK as soon as its sizes are checked: its pointers are not
+ *     inspected (NULL is accepted), the device is not queried and nothing is
+ *     launched.
  *   - Device-side waits are bounded. A wait that runs out records a nonzero code
  *     in the device error word and the kernel returns; read it with
  *     h3b_device_error after synchronizing.
@@ -305,7 +309,7 @@ H3B_API h3b_status h3b_quantize_rows(const void* h, int rows, int cols, const fl
                              float* s, h3b_stream stream);
 
 /* int8 GEMM on tensor cores, C[m][n] = sum_k A[m][k] W[n][k] (exact int32).
- * A int8 [M][K], W int8 [N][K], C int32 [M][N]; M >= 1, N % 16 == 0, K % 16 == 0. */
+ * A int8 [M][K], W int8 [N][K], C int32 [M][N]; M >= 0, N and K positive multiples of 16. */
 H3B_API h3b_status h3b_gemm_i8_s32(const int8_t* A, const int8_t* W, int32_t* C, int M, int N, int K,
                            h3b_stream stream);
 

@@ -131,6 +131,50 @@ def test_gemm_validation(L):
     assert L.h3b_gemm_i8_s32(None, 0x2000, 0x3000, 128, 256, 128, None) == -1
 
 
+def test_empty_problems_return_ok_after_their_size_checks(L):
+    # An empty problem returns OK once its sizes are checked: NULL pointers are
+    # accepted, the device is not queried (so this holds on a host without a GPU
+    # too) and nothing is launched.
+    assert L.h3b_gemm_i8_s32(None, None, None, 0, 256, 128, None) == 0
+    assert L.h3b_gemm_i8_dequant(None, None, None, None, None, None, 0, 256, 128, None) == 0
+    assert L.h3b_gemm_i8_gelu(None, None, None, None, None, None, None, 0, 256, 128, None) == 0
+    assert L.h3b_gemm_i8_gated_residual(None, None, None, None, None, None, 1, 0, None, 0, 256, 128, None) == 0
+    assert L.h3b_gemm_bf16_gated_residual(None, None, None, None, 1, 0, None, 0, 256, 128, None) == 0
+    assert L.h3b_quantize_rows(None, 0, 256, None, None, None, None) == 0
+    assert L.h3b_quantize_weights(None, 0, 256, None, None, None) == 0
+    assert L.h3b_ln_modulate_quantize(None, 0, 256, 1e-6, None, None, 1, 0, None, None, None, None, 1, None) == 0
+    assert L.h3b_range_delta(None, None, None, 0, None) == 0
+    assert L.h3b_range_apply(None, None, 0, None) == 0
+    # the sizes themselves are still checked
+    assert L.h3b_gemm_i8_s32(None, None, None, 0, 24, 128, None) == -2
+    assert L.h3b_gemm_i8_s32(None, None, None, -1, 256, 128, None) == -2
+    assert L.h3b_quantize_rows(None, 0, 17, None, None, None, None) == -2
+    assert L.h3b_ln_modulate_quantize(None, 0, 300, 1e-6, None, None, 1, 0, None, None, None, None, 1, None) == -2
+    assert L.h3b_ln_modulate_quantize(None, 0, 256, 1e-6, None, None, 0, 0, None, None, None, None, 1, None) == -1
+    assert L.h3b_range_apply(None, None, 4, None) == -2
+
+
+def test_step_arguments_are_checked_before_the_device_query(L):
+    # Every host check of a step entry point runs before the device is queried, so
+    # these are reported as argument errors even on a host without a GPU.
+    A, W, out = 0x10000, 0x20000, 0x30000
+    assert L.h3b_gemm_i8_dequant(A, None, W, 0x40000, None, out, 128, 256, 128, None) == -1      # sA NULL
+    assert L.h3b_gemm_i8_dequant(A, 0x40000, W, 0x40008, None, out, 128, 256, 128, None) == -3  # sW misaligned
+    assert L.h3b_gemm_i8_gelu(A, 0x40000, W, 0x40000, None, out, None, 128, 256, 128, None) == -1  # absmax NULL
+    assert L.h3b_gemm_i8_gated_residual(A, 0x40000, W, 0x40000, None, 0x50008, 1, 0, out,
+                                        128, 256, 128, None) == -3                                 # gate misaligned
+    assert L.h3b_gemm_i8_gated_residual(A, 0x40000, W, 0x40000, None, 0x50000, 0, 0, out,
+                                        128, 256, 128, None) == -1                                 # rows_per_item
+    assert L.h3b_gemm_bf16_gated_residual(A, W, None, None, 1, 0, out, 128, 256, 128, None) == -1  # gate NULL
+    assert L.h3b_gemm_bf16_gated_residual(A, W, None, 0x50000, 1, 6, out, 128, 256, 128, None) == -1  # stride % 4
+    assert L.h3b_ln_modulate_quantize(0x1000, 8, 256, 1e-6, None, 0x2000, 8, 0, 0x3000, 0x4000, None, None, 1,
+                                      None) == -1                                                  # shift NULL
+    assert L.h3b_ln_modulate_quantize(0x1000, 8, 256, 1e-6, 0x2000, 0x2000, 8, 0, 0x3000, 0x4000, 0x5008, None, 1,
+                                      None) == -3                                                  # h_out misaligned
+    assert L.h3b_quantize_rows(0x1000, 8, 256, None, None, 0x2000, None) == -1                     # q NULL
+    assert L.h3b_range_delta(0x1000, 0x2008, 0x3000, 64, None) == -3                                # after misaligned
+
+
 @pytest.mark.skipif(torch.cuda.is_available(), reason="would launch on the placeholder pointers")
 def test_valid_call_without_a_b200_launches_nothing(L):
     # On a host without a compute-capability-10.0 device the call stops at the

@@ -489,8 +489,9 @@ h3b_status h3b_blocks_forward_cached(const h3b_dims* dims, const h3b_block_weigh
 
 h3b_status h3b_range_delta(const void* before, const void* after, float* delta, long long n, h3b_stream stream) {
   cudaStream_t st = stream;
-  if (!before || !after || !delta) return fail(H3B_ERR_ARG, "NULL pointer");
   if (n < 0 || n % 8 != 0) return fail(H3B_ERR_SHAPE, "n must be a non-negative multiple of 8");
+  if (n == 0) return H3B_OK;  // empty problem: nothing to launch
+  if (!before || !after || !delta) return fail(H3B_ERR_ARG, "NULL pointer");
   if (!aligned16(before) || !aligned16(after) || !aligned16(delta)) return fail(H3B_ERR_ALIGN, "alignment");
   DeviceInfo* di = nullptr;
   h3b_status s = device_info(&di);
@@ -501,8 +502,9 @@ h3b_status h3b_range_delta(const void* before, const void* after, float* delta, 
 
 h3b_status h3b_range_apply(void* x, const float* delta, long long n, h3b_stream stream) {
   cudaStream_t st = stream;
-  if (!x || !delta) return fail(H3B_ERR_ARG, "NULL pointer");
   if (n < 0 || n % 8 != 0) return fail(H3B_ERR_SHAPE, "n must be a non-negative multiple of 8");
+  if (n == 0) return H3B_OK;  // empty problem: nothing to launch
+  if (!x || !delta) return fail(H3B_ERR_ARG, "NULL pointer");
   if (!aligned16(x) || !aligned16(delta)) return fail(H3B_ERR_ALIGN, "alignment");
   DeviceInfo* di = nullptr;
   h3b_status s = device_info(&di);
@@ -593,8 +595,9 @@ h3b_status h3b_token_unpair(const h3b_dims* full, const void* x, const void* xm,
 
 h3b_status h3b_quantize_weights(const float* w, int rows, int cols, int8_t* q, float* s, h3b_stream stream) {
   cudaStream_t st = stream;
-  if (!w || !q || !s) return fail(H3B_ERR_ARG, "NULL pointer");
   if (rows < 0 || cols < 16 || cols % 16 != 0) return fail(H3B_ERR_SHAPE, "cols must be a positive multiple of 16");
+  if (rows == 0) return H3B_OK;  // empty problem: nothing to launch
+  if (!w || !q || !s) return fail(H3B_ERR_ARG, "NULL pointer");
   if (!aligned16(w) || !aligned16(q)) return fail(H3B_ERR_ALIGN, "alignment");
   DeviceInfo* di = nullptr;
   h3b_status hs = device_info(&di);
@@ -635,9 +638,10 @@ h3b_status h3b_ln_modulate_quantize(const void* x, int rows, int d, float eps, c
                                     const float* scale, int rows_per_item, int mod_stride, int8_t* q, float* s,
                                     void* h_out, float* absmax_zero, int write_codes, h3b_stream stream) {
   cudaStream_t st = stream;
-  if (!x || !shift || !scale || (write_codes && (!q || !s))) return fail(H3B_ERR_ARG, "NULL pointer");
   if (rows < 0 || d < 256 || d % 256 != 0 || d > 8192) return fail(H3B_ERR_SHAPE, "d must be a multiple of 256, <= 8192");
   if (rows_per_item < 1 || mod_stride < 0 || mod_stride % 4 != 0) return fail(H3B_ERR_ARG, "rows_per_item/mod_stride");
+  if (rows == 0) return H3B_OK;  // empty problem: nothing to launch
+  if (!x || !shift || !scale || (write_codes && (!q || !s))) return fail(H3B_ERR_ARG, "NULL pointer");
   if (!aligned16(x) || !aligned16(shift) || !aligned16(scale) || (q && !aligned16(q)) || (h_out && !aligned16(h_out)))
     return fail(H3B_ERR_ALIGN, "alignment");
   DeviceInfo* di = nullptr;
@@ -651,8 +655,9 @@ h3b_status h3b_ln_modulate_quantize(const void* x, int rows, int d, float eps, c
 h3b_status h3b_quantize_rows(const void* h, int rows, int cols, const float* absmax, int8_t* q, float* s,
                              h3b_stream stream) {
   cudaStream_t st = stream;
-  if (!h || !q || !s) return fail(H3B_ERR_ARG, "NULL pointer");
   if (rows < 0 || cols < 16 || cols % 16 != 0) return fail(H3B_ERR_SHAPE, "cols must be a positive multiple of 16");
+  if (rows == 0) return H3B_OK;  // empty problem: nothing to launch
+  if (!h || !q || !s) return fail(H3B_ERR_ARG, "NULL pointer");
   if (!aligned16(h) || !aligned16(q)) return fail(H3B_ERR_ALIGN, "alignment");
   DeviceInfo* di = nullptr;
   h3b_status hs = device_info(&di);
@@ -661,20 +666,29 @@ h3b_status h3b_quantize_rows(const void* h, int rows, int cols, const float* abs
   return H3B_OK;
 }
 
-static h3b_status gemm_common(const void* A, const void* W, const void* out, int M, int N, int K,
-                              DeviceInfo** di) {
-  if (!A || !W || !out) return fail(H3B_ERR_ARG, "NULL pointer");
+// Host checks shared by the GEMM entry points (no device query). An empty problem
+// (M == 0) sets *empty and returns as soon as the sizes are checked: its pointers
+// are not inspected.
+static h3b_status gemm_checks(const void* A, const void* W, const void* out, int M, int N, int K, bool* empty) {
+  *empty = false;
   if (M < 0 || N < 16 || N % 16 != 0 || K < 16 || K % 16 != 0)
     return fail(H3B_ERR_SHAPE, "need M >= 0, N and K positive multiples of 16");
+  if (M == 0) {
+    *empty = true;
+    return H3B_OK;
+  }
+  if (!A || !W || !out) return fail(H3B_ERR_ARG, "NULL pointer");
   if (!aligned16(A) || !aligned16(W) || !aligned16(out)) return fail(H3B_ERR_ALIGN, "alignment");
-  return device_info(di);
+  return H3B_OK;
 }
 
 h3b_status h3b_gemm_i8_s32(const int8_t* A, const int8_t* W, int32_t* C, int M, int N, int K, h3b_stream stream) {
   cudaStream_t st = stream;
+  bool empty = false;
+  h3b_status s = gemm_checks(A, W, C, M, N, K, &empty);
+  if (s != H3B_OK || empty) return s;
   DeviceInfo* di = nullptr;
-  h3b_status s = gemm_common(A, W, C, M, N, K, &di);
-  if (s != H3B_OK) return s;
+  if ((s = device_info(&di)) != H3B_OK) return s;
   GemmArgs a = base_args(M, N, K, di->err);
   a.out = C;
   H3B_CK(launch_gemm(true, EPI_S32, A, W, a, di->sms, stream), "gemm_i8_s32");
@@ -684,11 +698,13 @@ h3b_status h3b_gemm_i8_s32(const int8_t* A, const int8_t* W, int32_t* C, int M, 
 h3b_status h3b_gemm_i8_dequant(const int8_t* A, const float* sA, const int8_t* W, const float* sW,
                                const float* bias, void* out, int M, int N, int K, h3b_stream stream) {
   cudaStream_t st = stream;
-  DeviceInfo* di = nullptr;
-  h3b_status s = gemm_common(A, W, out, M, N, K, &di);
-  if (s != H3B_OK) return s;
+  bool empty = false;
+  h3b_status s = gemm_checks(A, W, out, M, N, K, &empty);
+  if (s != H3B_OK || empty) return s;
   if (!sA || !sW) return fail(H3B_ERR_ARG, "scales NULL");
   if (!aligned16(sW) || (bias && !aligned16(bias))) return fail(H3B_ERR_ALIGN, "alignment");
+  DeviceInfo* di = nullptr;
+  if ((s = device_info(&di)) != H3B_OK) return s;
   GemmArgs a = base_args(M, N, K, di->err);
   a.sA = sA; a.sW = sW; a.bias = bias; a.out = out;
   H3B_CK(launch_gemm(true, EPI_DEQ, A, W, a, di->sms, stream), "gemm_i8_dequant");
@@ -746,12 +762,14 @@ h3b_status h3b_gemm_i8_gated_residual(const int8_t* A, const float* sA, const in
                                       const float* bias, const float* gate, int rows_per_item, int gate_stride,
                                       void* x, int M, int N, int K, h3b_stream stream) {
   cudaStream_t st = stream;
-  DeviceInfo* di = nullptr;
-  h3b_status s = gemm_common(A, W, x, M, N, K, &di);
-  if (s != H3B_OK) return s;
+  bool empty = false;
+  h3b_status s = gemm_checks(A, W, x, M, N, K, &empty);
+  if (s != H3B_OK || empty) return s;
   if (!sA || !sW || !gate) return fail(H3B_ERR_ARG, "scales/gate NULL");
   if (rows_per_item < 1 || gate_stride < 0 || gate_stride % 4 != 0) return fail(H3B_ERR_ARG, "rows_per_item/gate_stride");
   if (!aligned16(sW) || !aligned16(gate) || (bias && !aligned16(bias))) return fail(H3B_ERR_ALIGN, "alignment");
+  DeviceInfo* di = nullptr;
+  if ((s = device_info(&di)) != H3B_OK) return s;
   GemmArgs a = base_args(M, N, K, di->err);
   a.sA = sA; a.sW = sW; a.bias = bias; a.out = x;
   a.gate = gate; a.rows_per_item = rows_per_item; a.gate_stride = gate_stride;
@@ -763,12 +781,14 @@ h3b_status h3b_gemm_bf16_gated_residual(const void* A, const void* W, const floa
                                         int rows_per_item, int gate_stride, void* x, int M, int N, int K,
                                         h3b_stream stream) {
   cudaStream_t st = stream;
+  bool empty = false;
+  h3b_status s = gemm_checks(A, W, x, M, N, K, &empty);
+  if (s != H3B_OK || empty) return s;
   if (!gate) return fail(H3B_ERR_ARG, "gate NULL");
   if (rows_per_item < 1 || gate_stride < 0 || gate_stride % 4 != 0) return fail(H3B_ERR_ARG, "rows_per_item/gate_stride");
   if (!aligned16(gate) || (bias && !aligned16(bias))) return fail(H3B_ERR_ALIGN, "alignment");
   DeviceInfo* di = nullptr;
-  h3b_status s = gemm_common(A, W, x, M, N, K, &di);
-  if (s != H3B_OK) return s;
+  if ((s = device_info(&di)) != H3B_OK) return s;
   GemmArgs a = base_args(M, N, K, di->err);
   a.bias = bias; a.out = x;
   a.gate = gate; a.rows_per_item = rows_per_item; a.gate_stride = gate_stride;
@@ -779,11 +799,13 @@ h3b_status h3b_gemm_bf16_gated_residual(const void* A, const void* W, const floa
 h3b_status h3b_gemm_i8_gelu(const int8_t* A, const float* sA, const int8_t* W, const float* sW, const float* bias,
                             void* g, float* absmax, int M, int N, int K, h3b_stream stream) {
   cudaStream_t st = stream;
-  DeviceInfo* di = nullptr;
-  h3b_status s = gemm_common(A, W, g, M, N, K, &di);
-  if (s != H3B_OK) return s;
+  bool empty = false;
+  h3b_status s = gemm_checks(A, W, g, M, N, K, &empty);
+  if (s != H3B_OK || empty) return s;
   if (!sA || !sW || !absmax) return fail(H3B_ERR_ARG, "scales/absmax NULL");
   if (!aligned16(sW) || (bias && !aligned16(bias))) return fail(H3B_ERR_ALIGN, "alignment");
+  DeviceInfo* di = nullptr;
+  if ((s = device_info(&di)) != H3B_OK) return s;
   GemmArgs a = base_args(M, N, K, di->err);
   a.sA = sA; a.sW = sW; a.bias = bias; a.out = g; a.absmax = absmax;
   H3B_CK(launch_gemm(true, EPI_GELU, A, W, a, di->sms, stream), "gemm_i8_gelu");
