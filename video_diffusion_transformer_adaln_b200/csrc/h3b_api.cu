@@ -11,6 +11,7 @@
 //     section "性能上限" (AdaLN gating, RoPE and quantization folded into the
 //     preceding kernels; activation memory reused by lifetime).
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 #include <string>
 #include <vector>
@@ -176,16 +177,13 @@ struct ProfRec {
   cudaEvent_t a, b;
 };
 std::mutex g_prof_mu;
-bool g_prof_on = false;
+std::atomic<bool> g_prof_on{false};  // read by every launch without the lock
 std::vector<ProfRec> g_prof_recs;
 std::vector<cudaEvent_t> g_prof_free;
 
 }  // namespace
 
-bool profiling_enabled() {
-  std::lock_guard<std::mutex> lk(g_prof_mu);
-  return g_prof_on;
-}
+bool profiling_enabled() { return g_prof_on.load(); }
 
 namespace {
 
@@ -216,7 +214,10 @@ struct ProfScope {
     if (!a) return;
     std::lock_guard<std::mutex> lk(g_prof_mu);
     cudaEvent_t b = prof_event();
-    if (!b) return;
+    if (!b) {
+      g_prof_free.push_back(a);  // no end event: drop this launch's record, keep the event
+      return;
+    }
     cudaEventRecord(b, st);
     g_prof_recs.push_back({name, a, b});
   }
