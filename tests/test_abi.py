@@ -85,11 +85,41 @@ def test_block_forward_validation_order(L):
     # bad shape
     bad = _dims(d_ff=100)
     assert L.h3b_block_forward(C.byref(bad), C.byref(w), c, x, ws, need, None) == -2
-    # missing weight (placeholder pointers are never dereferenced: validation
-    # fails before any launch, on a GPU host as well)
+    # missing or misaligned weight (placeholder pointers are never dereferenced:
+    # every host check runs before the device query and any launch)
     w.w1 = None
-    st = L.h3b_block_forward(C.byref(d), C.byref(w), c, x, ws, need, None)
-    assert st in (-1, -5, -6)  # weights are checked after the device query on a GPU-less host
+    assert L.h3b_block_forward(C.byref(d), C.byref(w), c, x, ws, need, None) == -1
+    w.w1 = 0x10008
+    assert L.h3b_block_forward(C.byref(d), C.byref(w), c, x, ws, need, None) == -3
+
+
+def test_multi_block_entry_points_check_every_block_on_the_host(L):
+    d = _dims()
+    blocks = (h3b.BlockWeights * 3)()
+    for b in blocks:
+        for n in h3b.WEIGHT_FIELDS:
+            setattr(b, n, 0x10000)
+    blocks[2].s2 = None  # the last block's W2 scales are missing
+    x, c, ws, xm, ym = 0x20000, 0x30000, 0x40000, 0x50000, 0x60000
+    need = h3b.h3b_workspace_size(d)
+    assert L.h3b_blocks_forward(C.byref(d), blocks, 3, c, x, ws, need, None) == -1
+    assert L.h3b_blocks_forward(C.byref(d), blocks, -1, c, x, ws, need, None) == -1
+    assert L.h3b_blocks_forward(C.byref(d), None, 3, c, x, ws, need, None) == -1
+    # reduced pass: range, pairing shape and buffers
+    assert L.h3b_blocks_forward_reduced(C.byref(d), blocks, 3, 1, 2, c, x, xm, ym, ws, need, None) == -1
+    assert L.h3b_blocks_forward_reduced(C.byref(d), blocks, 3, 2, 1, c, x, xm, ym, ws, need, None) == -1
+    assert L.h3b_blocks_forward_reduced(C.byref(d), blocks, 3, 1, 2, c, x, None, ym, ws, need, None) == -1
+    assert L.h3b_blocks_forward_reduced(C.byref(d), blocks, 3, 1, 2, c, x, xm + 8, ym, ws, need, None) == -3
+    odd = _dims(W=15)
+    need_odd = h3b.h3b_workspace_size(odd)
+    assert L.h3b_blocks_forward_reduced(C.byref(odd), blocks, 3, 1, 2, c, x, xm, ym, ws, need_odd, None) == -2
+    # cached pass: range, buffers, and the same per-block weight check
+    assert L.h3b_blocks_forward_cached(C.byref(d), blocks, 3, 0, 4, 1, c, x, 0x70000, 0x80000, ws, need,
+                                       None) == -1
+    assert L.h3b_blocks_forward_cached(C.byref(d), blocks, 3, 0, 2, 1, c, x, None, 0x80000, ws, need,
+                                       None) == -1
+    assert L.h3b_blocks_forward_cached(C.byref(d), blocks, 3, 0, 2, 1, c, x, 0x70000, 0x80000, ws, need,
+                                       None) == -1
 
 
 @pytest.mark.parametrize("T,H,W", [(2 ** 31 - 1, 2 ** 31 - 1, 2 ** 31 - 1), (65536, 65536, 2),

@@ -404,8 +404,9 @@ size_t h3b_rope_table_bytes(const h3b_dims* dims) {
   return rope_bytes(*dims);
 }
 
+// Host checks shared by the block entry points (no device query).
 static h3b_status block_common(const h3b_dims* dims, const float* c, void* x, void* ws, size_t ws_bytes,
-                               WsLayout* lay, DeviceInfo** di) {
+                               WsLayout* lay) {
   h3b_status s = check_dims(dims);
   if (s != H3B_OK) return s;
   if (!c || !x || !ws) return fail(H3B_ERR_ARG, "c, x and ws must be non-NULL");
@@ -413,28 +414,30 @@ static h3b_status block_common(const h3b_dims* dims, const float* c, void* x, vo
   if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return fail(H3B_ERR_ALIGN, "workspace not 256-byte aligned");
   *lay = ws_layout(*dims);
   if (ws_bytes < lay->total) return fail(H3B_ERR_WORKSPACE, "workspace smaller than h3b_workspace_size");
-  return device_info(di);
+  return H3B_OK;
 }
 
 h3b_status h3b_block_forward(const h3b_dims* dims, const h3b_block_weights* w, const float* c, void* x,
                              void* ws, size_t ws_bytes, h3b_stream stream) {
   WsLayout lay;
-  DeviceInfo* di = nullptr;
-  h3b_status s = block_common(dims, c, x, ws, ws_bytes, &lay, &di);
+  h3b_status s = block_common(dims, c, x, ws, ws_bytes, &lay);
   if (s != H3B_OK) return s;
   if ((s = check_weights(*dims, w)) != H3B_OK) return s;
+  DeviceInfo* di = nullptr;
+  if ((s = device_info(&di)) != H3B_OK) return s;
   return run_block(*dims, *w, c, x, static_cast<uint8_t*>(ws), lay, false, *di, stream);
 }
 
 h3b_status h3b_blocks_forward(const h3b_dims* dims, const h3b_block_weights* w, int n_blocks, const float* c,
                               void* x, void* ws, size_t ws_bytes, h3b_stream stream) {
   WsLayout lay;
-  DeviceInfo* di = nullptr;
-  h3b_status s = block_common(dims, c, x, ws, ws_bytes, &lay, &di);
+  h3b_status s = block_common(dims, c, x, ws, ws_bytes, &lay);
   if (s != H3B_OK) return s;
   if (n_blocks < 0 || (n_blocks > 0 && !w)) return fail(H3B_ERR_ARG, "n_blocks < 0 or weights NULL");
   for (int i = 0; i < n_blocks; ++i)
     if ((s = check_weights(*dims, &w[i])) != H3B_OK) return s;
+  DeviceInfo* di = nullptr;
+  if ((s = device_info(&di)) != H3B_OK) return s;
   const size_t c_stride = (size_t)dims->B * dims->d;
   for (int i = 0; i < n_blocks; ++i) {
     s = run_block(*dims, w[i], c + i * c_stride, x, static_cast<uint8_t*>(ws), lay, i > 0, *di, stream);
@@ -455,11 +458,12 @@ h3b_status h3b_blocks_forward_cached(const h3b_dims* dims, const h3b_block_weigh
   if ((range && !aligned16(delta)) || (range && fresh && !aligned16(x_save)))
     return fail(H3B_ERR_ALIGN, "delta / x_save not 16-byte aligned");
   WsLayout lay;
-  DeviceInfo* di = nullptr;
-  h3b_status s = block_common(dims, c, x, ws, ws_bytes, &lay, &di);
+  h3b_status s = block_common(dims, c, x, ws, ws_bytes, &lay);
   if (s != H3B_OK) return s;
   for (int i = 0; i < n_blocks; ++i)
     if ((s = check_weights(*dims, &w[i])) != H3B_OK) return s;
+  DeviceInfo* di = nullptr;
+  if ((s = device_info(&di)) != H3B_OK) return s;
   cudaStream_t st = stream;
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   const size_t c_stride = (size_t)dims->B * dims->d;
@@ -518,8 +522,7 @@ h3b_status h3b_blocks_forward_reduced(const h3b_dims* full, const h3b_block_weig
                                       int first, int last, const float* c, void* x, void* xm, void* ym,
                                       void* ws, size_t ws_bytes, h3b_stream stream) {
   WsLayout lay_full;
-  DeviceInfo* di = nullptr;
-  h3b_status s = block_common(full, c, x, ws, ws_bytes, &lay_full, &di);
+  h3b_status s = block_common(full, c, x, ws, ws_bytes, &lay_full);
   if (s != H3B_OK) return s;
   if (n_blocks < 0 || (n_blocks > 0 && !w)) return fail(H3B_ERR_ARG, "n_blocks < 0 or weights NULL");
   if (first < 0 || first > last || last > n_blocks) return fail(H3B_ERR_ARG, "need 0 <= first <= last <= n_blocks");
@@ -536,6 +539,8 @@ h3b_status h3b_blocks_forward_reduced(const h3b_dims* full, const h3b_block_weig
   }
   for (int i = 0; i < n_blocks; ++i)
     if ((s = check_weights(*full, &w[i])) != H3B_OK) return s;
+  DeviceInfo* di = nullptr;
+  if ((s = device_info(&di)) != H3B_OK) return s;
   cudaStream_t st = stream;
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   const size_t c_stride = (size_t)full->B * full->d;
