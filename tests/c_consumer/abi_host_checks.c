@@ -5,6 +5,7 @@
  * Nothing here queries a device or launches a kernel, so it runs on a machine
  * without a GPU. Prints "OK" and exits 0 when every check holds.
  */
+#include <stddef.h>
 #include <stdio.h>
 #include <string.h>
 
@@ -21,6 +22,27 @@ static int failures = 0;
     }                                                                        \
   } while (0)
 
+/* Struct layouts as the C compiler sees them, one "struct field offset size" line
+   per field, for the binding's test to compare with its own mirror of the structs. */
+#define FIELD(S, F) printf("%s %s %zu %zu\n", #S, #F, offsetof(S, F), sizeof(((S*)0)->F))
+
+static void print_layouts(void) {
+  printf("sizeof h3b_dims %zu\n", sizeof(h3b_dims));
+  FIELD(h3b_dims, B); FIELD(h3b_dims, T); FIELD(h3b_dims, H); FIELD(h3b_dims, W);
+  FIELD(h3b_dims, d); FIELD(h3b_dims, n_heads); FIELD(h3b_dims, head_dim); FIELD(h3b_dims, d_ff);
+  FIELD(h3b_dims, rope_t); FIELD(h3b_dims, rope_h); FIELD(h3b_dims, rope_w);
+  FIELD(h3b_dims, rope_theta); FIELD(h3b_dims, ln_eps); FIELD(h3b_dims, qkv_int8); FIELD(h3b_dims, wo_bf16);
+  printf("sizeof h3b_block_weights %zu\n", sizeof(h3b_block_weights));
+  FIELD(h3b_block_weights, w_ada); FIELD(h3b_block_weights, b_ada); FIELD(h3b_block_weights, wqkv);
+  FIELD(h3b_block_weights, sqkv); FIELD(h3b_block_weights, wqkv_bf16); FIELD(h3b_block_weights, bqkv);
+  FIELD(h3b_block_weights, wo); FIELD(h3b_block_weights, so); FIELD(h3b_block_weights, bo);
+  FIELD(h3b_block_weights, w1); FIELD(h3b_block_weights, s1); FIELD(h3b_block_weights, b1);
+  FIELD(h3b_block_weights, w2); FIELD(h3b_block_weights, s2); FIELD(h3b_block_weights, b2);
+  FIELD(h3b_block_weights, wo_bf16);
+  printf("sizeof h3b_kernel_time %zu\n", sizeof(h3b_kernel_time));
+  FIELD(h3b_kernel_time, name); FIELD(h3b_kernel_time, launches); FIELD(h3b_kernel_time, total_ms);
+}
+
 /* 2 x 16 x 16 latent grid, d = 256 (4 heads of 64), d_ff = 1024. */
 static h3b_dims small_dims(void) {
   h3b_dims d;
@@ -35,6 +57,7 @@ static h3b_dims small_dims(void) {
 
 int main(void) {
   const h3b_dims d = small_dims();
+  print_layouts();
   size_t bytes = 0;
 
   /* workspace: at least the int8 activations (L x d_ff) and bf16 Q, K, V, O (8 L d bytes) */
