@@ -330,8 +330,11 @@ def test_blocks_forward_reduced_middle_range_d256():
 
 
 def test_depth50_pass_properties_d5120_T2():
-    """The 50-block pass at d=5120, L=4608: finite, deterministic, equal to 50
-    single-block calls; block 0's output matches the oracle on sampled rows."""
+    """The 50-block pass at d=5120, L=4608: finite, deterministic, and bit-identical
+    to 50 single-block calls. Each of those calls is the d=5120 block that
+    test_block_d5120_sampled checks against the oracle (with weights the oracle
+    quantizes itself); this pass's weights are drawn on the device, so its blocks
+    are not fed to the oracle."""
     wl = synth.WORKLOADS["d5120_depth50_T2"]
     dims = dims_of(wl)
     g = torch.Generator(device="cuda").manual_seed(synth.BASE_SEED)
