@@ -31,6 +31,12 @@ def bf16_host(t):
     return bits_from_bf16(t)
 
 
+def bf16_f64(bits):
+    """bf16 bit patterns as float64 (exact), decoded in numpy: GPU results are
+    compared without passing through the oracle."""
+    return synth.bf16_bits_to_f32(bits).astype(np.float64)
+
+
 def rel_l2(a, ref):
     a = np.asarray(a, np.float64)
     ref = np.asarray(ref, np.float64)

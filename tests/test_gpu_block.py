@@ -11,7 +11,7 @@ import pytest
 import torch
 
 import oracle as O
-from gpu_helpers import (bf16_dev, bf16_host, no_device_error, oracle_dims, oracle_weights, rel_l2, require_gpu,
+from gpu_helpers import (bf16_f64, bf16_dev, bf16_host, no_device_error, oracle_dims, oracle_weights, rel_l2, require_gpu,
                          to_dev, bf16_ulp_diff)
 from video_diffusion_transformer_adaln_b200 import h3b, synth
 from video_diffusion_transformer_adaln_b200.runtime import (DeviceBlock, blocks_forward, block_forward, dims_of,
@@ -41,8 +41,8 @@ def _run_gpu_block(wl, raw, c, x_bits):
 
 
 def _compare(got_bits, ref, x_bits, rows=None, n_blocks=1):
-    got = O.bf16_decode(got_bits).reshape(-1, ref.shape[-1])
-    xin = O.bf16_decode(x_bits).reshape(-1, ref.shape[-1])
+    got = bf16_f64(got_bits).reshape(-1, ref.shape[-1])
+    xin = bf16_f64(x_bits).reshape(-1, ref.shape[-1])
     if rows is not None:
         got, xin = got[rows], xin[rows]
     e = rel_l2(got, ref)
@@ -171,10 +171,10 @@ def test_token_reduction_d5120_sampled():
     assert np.array_equal(bf16_host(xm).reshape(xm_o.shape), xm_o)
     mrows = synth.sample_rows(m.L, 48)
     ym_o = O.block_forward(oracle_dims(m), ow, c, xm_o, rows=mrows)
-    xm_flat = O.bf16_decode(xm_o).reshape(-1, wl.d)
+    xm_flat = bf16_f64(xm_o).reshape(-1, wl.d)
     urows = np.concatenate([2 * mrows, 2 * mrows + 1])
-    ref = np.concatenate([O.bf16_decode(x).reshape(-1, wl.d)[2 * mrows] + ym_o - xm_flat[mrows],
-                          O.bf16_decode(x).reshape(-1, wl.d)[2 * mrows + 1] + ym_o - xm_flat[mrows]])
+    ref = np.concatenate([bf16_f64(x).reshape(-1, wl.d)[2 * mrows] + ym_o - xm_flat[mrows],
+                          bf16_f64(x).reshape(-1, wl.d)[2 * mrows + 1] + ym_o - xm_flat[mrows]])
     _compare(got, ref, x, urows)
     no_device_error()
 
@@ -268,25 +268,40 @@ def test_blocks_forward_cached_range_d256():
     torch.cuda.synchronize()
     assert np.array_equal(bf16_host(xf), ref)
     assert np.array_equal(bf16_host(x_save), after0)
-    d_ref = O.range_delta(after0, ref)
-    d_got = delta.cpu().numpy().astype(np.float64).reshape(d_ref.shape)
-    assert np.all(np.abs(d_got - d_ref) <= 2.0 ** -24 * np.abs(d_ref))
-    # reuse pass on another step's stream: block 0 runs, the range is replaced by the delta
+    # delta is the fp32 difference of the range's bf16 output and input (restated in numpy on
+    # the pass's own values; the oracle is held to seeded inputs below)
+    f32 = synth.bf16_bits_to_f32
+    d_got = delta.cpu().numpy()
+    assert np.array_equal(d_got, (f32(ref) - f32(after0)).reshape(-1))
+    # reuse pass on another step's stream: block 0 runs, the range is replaced by the delta,
+    # x = bf16(x + delta) with the sum in fp32
     x2_bits = synth.f32_to_bf16_bits((synth.bf16_bits_to_f32(x) * 0.9).astype(np.float32))
     x2 = bf16_dev(x2_bits)
     h3b.h3b_blocks_forward_cached(dims, structs, first, last, False, cs, x2, None, delta, ws)
     x2b = bf16_dev(x2_bits)
     h3b.h3b_blocks_forward(dims, structs[:1], cs, x2b, ws)
-    want = O.range_apply(bf16_host(x2b), d_got)
-    got = bf16_host(x2)
-    assert bf16_ulp_diff(got, want).max() <= 1  # fp32 sum then bf16 vs one rounding of the exact sum
+    want = synth.f32_to_bf16_bits(f32(bf16_host(x2b)).reshape(-1) + d_got).reshape(x.shape)
+    assert np.array_equal(bf16_host(x2), want)
     # the step entry points alone agree with the pass
     d2 = torch.empty_like(delta)
     h3b.h3b_range_delta(x_save, xf, d2)
     assert torch.equal(d2, delta)
     x3 = bf16_dev(after0)
     h3b.h3b_range_apply(x3, delta)
-    assert bf16_ulp_diff(bf16_host(x3), O.range_apply(after0, d_got)).max() <= 1
+    assert np.array_equal(bf16_host(x3).reshape(-1), synth.f32_to_bf16_bits(f32(after0).reshape(-1) + d_got))
+    # the two elementwise steps against the oracle, on seeded inputs
+    r = np.random.default_rng(11)
+    before = synth.f32_to_bf16_bits(r.standard_normal(n).astype(np.float32))
+    after = synth.f32_to_bf16_bits((f32(before) + 0.1 * r.standard_normal(n)).astype(np.float32))
+    d3 = torch.empty(n, dtype=torch.float32, device="cuda")
+    h3b.h3b_range_delta(bf16_dev(before), bf16_dev(after), d3)
+    d_ref = O.range_delta(before, after)
+    d_dev = d3.cpu().numpy().astype(np.float64)
+    assert np.all(np.abs(d_dev - d_ref) <= 2.0 ** -24 * np.abs(d_ref))
+    x5 = bf16_dev(before)
+    h3b.h3b_range_apply(x5, to_dev(d_ref.astype(np.float32)))
+    # fp32 sum then bf16 vs one rounding of the exact sum
+    assert bf16_ulp_diff(bf16_host(x5), O.range_apply(before, d_ref.astype(np.float32))).max() <= 1
     no_device_error()
 
 
@@ -315,7 +330,7 @@ def test_blocks_forward_reduced_middle_range_d256():
     yr = xmo
     for b in range(first, last):
         yr = O.bf16_round(O.block_forward(oracle_dims(m), oracle_weights(raws[b]), cs[b], yr)).reshape(xmo.shape)
-    xr = O.bf16_round(O.token_unpair(xr, xmo, O.bf16_decode(yr), wl.B, wl.T, wl.H, wl.W, wl.d))
+    xr = O.bf16_round(O.token_unpair(xr, xmo, bf16_f64(yr), wl.B, wl.T, wl.H, wl.W, wl.d))
     for b in range(last, 5):
         out = O.block_forward(oracle_dims(wl), oracle_weights(raws[b]), cs[b], xr)
         xr = O.bf16_round(out).reshape(x.shape)
@@ -351,5 +366,5 @@ def test_depth50_pass_properties_d5120_T2():
         block_forward(dims, blocks[i], c[i], xc, ws)
     a, b_, cc = bf16_host(xa), bf16_host(xb), bf16_host(xc)
     assert np.array_equal(a, b_) and np.array_equal(a, cc)
-    assert np.isfinite(O.bf16_decode(a)).all()
+    assert np.isfinite(bf16_f64(a)).all()
     no_device_error()

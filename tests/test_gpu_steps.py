@@ -10,7 +10,7 @@ import pytest
 import torch
 
 import oracle as O
-from gpu_helpers import (bf16_dev, bf16_host, bf16_ulp_diff, no_device_error, oracle_weights, rel_l2,
+from gpu_helpers import (bf16_f64, bf16_dev, bf16_host, bf16_ulp_diff, no_device_error, oracle_weights, rel_l2,
                          require_gpu, to_dev)
 from video_diffusion_transformer_adaln_b200 import h3b, synth
 from video_diffusion_transformer_adaln_b200.runtime import DeviceBlock, dims_of, quantize_weight
@@ -112,13 +112,13 @@ def test_ln_modulate_quantize(rows, d, items):
     # (1) the bf16 quantizer input matches the oracle's fp64 LN + modulation to one
     #     bf16 ulp of the value (at most 2^-7 |h|), plus the fp32 error of y*(1+scale)+shift when
     #     the two terms nearly cancel (bounded relative to the row's magnitude)
-    y = O.layernorm(O.bf16_decode(x), 1e-6)
+    y = O.layernorm(bf16_f64(x), 1e-6)
     ho = np.empty_like(hg)
     for i in range(rows):
         it = i // rpi
         ho[i] = O.modulate_bf16(y[i:i + 1], mod[it, 3 * d:4 * d].astype(np.float64),
                                 mod[it, 4 * d:5 * d].astype(np.float64))[0]
-    hgd, hod = O.bf16_decode(hg), O.bf16_decode(ho)
+    hgd, hod = bf16_f64(hg), bf16_f64(ho)
     bound = 2.0 ** -7 * np.abs(hod) + 2.0 ** -16 * np.abs(hod).max(axis=1, keepdims=True)
     assert np.all(np.abs(hgd - hod) <= bound)
     assert (hg != ho).mean() < 0.02
@@ -196,10 +196,10 @@ def test_gemm_i8_gelu(M, N, K):
     h3b.h3b_gemm_i8_gelu(to_dev(qa), to_dev(sa), to_dev(qw), to_dev(sw), to_dev(bias), g, am)
     gg = bf16_host(g)
     ref = O.gelu_tanh(O.dequant(O.gemm_i8(qa, qw), sa, sw, bias))
-    assert rel_l2(O.bf16_decode(gg), ref) < 4e-3
-    assert np.max(np.abs(O.bf16_decode(gg) - ref)) <= 2 ** -7 * np.max(np.abs(ref)) + 1e-3
+    assert rel_l2(bf16_f64(gg), ref) < 4e-3
+    assert np.max(np.abs(bf16_f64(gg) - ref)) <= 2 ** -7 * np.max(np.abs(ref)) + 1e-3
     # the reported absmax is exactly the max |g| of the written bf16 row
-    assert np.array_equal(am.cpu().numpy(), np.abs(O.bf16_decode(gg)).max(axis=1).astype(np.float32))
+    assert np.array_equal(am.cpu().numpy(), np.abs(bf16_f64(gg)).max(axis=1).astype(np.float32))
     no_device_error()
 
 
@@ -217,11 +217,11 @@ def test_gemm_i8_gated_residual(M, N, K, items):
     y = O.dequant(O.gemm_i8(qa, qw), sa, sw, bias)
     ref = np.empty((M, N))
     for i in range(M):
-        ref[i] = O.gated_residual(O.bf16_decode(x[i:i + 1]), y[i:i + 1], gate[i // rpi, N:2 * N])[0]
+        ref[i] = O.gated_residual(bf16_f64(x[i:i + 1]), y[i:i + 1], gate[i // rpi, N:2 * N])[0]
     # one bf16 rounding of the result, plus the fp32 error of x + gate*y when the
     # two terms nearly cancel (relative to the terms' magnitude)
-    got = O.bf16_decode(bf16_host(xd))
-    terms = np.abs(O.bf16_decode(x)) + np.abs(np.stack([gate[i // rpi, N:2 * N] for i in range(M)]) * y)
+    got = bf16_f64(bf16_host(xd))
+    terms = np.abs(bf16_f64(x)) + np.abs(np.stack([gate[i // rpi, N:2 * N] for i in range(M)]) * y)
     assert np.all(np.abs(got - ref) <= 2.0 ** -8 * np.abs(ref) + 2.0 ** -20 * terms + 1e-30)
     # a zero gate leaves x bit-identical
     xd2 = bf16_dev(x)
@@ -244,15 +244,15 @@ def test_gemm_bf16_gated_residual(M, N, K, items):
     xd = bf16_dev(x)
     gd = to_dev(gate)
     h3b.h3b_gemm_bf16_gated_residual(bf16_dev(a), bf16_dev(w), to_dev(bias), gd[:, N:], rpi, 2 * N, xd)
-    ad, wd = O.bf16_decode(a), O.bf16_decode(w)
+    ad, wd = bf16_f64(a), bf16_f64(w)
     y = O.gemm_f64(ad, wd) + bias
     g = np.stack([gate[i // rpi, N:] for i in range(M)])
-    ref = O.bf16_decode(x) + g * y
-    got = O.bf16_decode(bf16_host(xd))
+    ref = bf16_f64(x) + g * y
+    got = bf16_f64(bf16_host(xd))
     # one bf16 rounding of the result; fp32 accumulation over K (|error| <= K 2^-24 sum|a w|)
     # and the fp32 error of x + gate*y relative to the terms' magnitude
     absum = np.abs(ad) @ np.abs(wd).T + np.abs(bias)
-    terms = np.abs(O.bf16_decode(x)) + np.abs(g * y)
+    terms = np.abs(bf16_f64(x)) + np.abs(g * y)
     bound = 2.0 ** -8 * np.abs(ref) + 2.0 ** -20 * terms + K * 2.0 ** -24 * np.abs(g) * absum + 1e-30
     assert np.all(np.abs(got - ref) <= bound)
     # a zero gate leaves x bit-identical
@@ -274,7 +274,7 @@ def _qkv_reference(wl, A_f32, sA, raw_w):
         acc = O.gemm_i8(qa, w)
         qkv = O.dequant(acc, sA, s)
     else:
-        qkv = O.gemm_f64(O.bf16_decode(A_f32), O.bf16_decode(raw_w["wqkv_bf16"]))
+        qkv = O.gemm_f64(bf16_f64(A_f32), bf16_f64(raw_w["wqkv_bf16"]))
     t, h, w_ = O.grid_positions(wl.T, wl.H, wl.W)
     t, h, w_ = (np.tile(a, wl.B) for a in (t, h, w_))
     Q = O.rope_3d(qkv[:, :d], t, h, w_, wl.n_heads, wl.head_dim, wl.rope)
@@ -284,7 +284,7 @@ def _qkv_reference(wl, A_f32, sA, raw_w):
 
 def _head_major_to_token_major(qkv_dev, wl):
     B, H, L, dh = wl.B, wl.n_heads, wl.L, wl.head_dim
-    a = O.bf16_decode(bf16_host(qkv_dev)).reshape(3, B, H, L, dh)
+    a = bf16_f64(bf16_host(qkv_dev)).reshape(3, B, H, L, dh)
     return a.transpose(1, 3, 0, 2, 4).reshape(B * L, 3 * H * dh)
 
 
@@ -330,8 +330,8 @@ def test_attention(B, H, L, dh, n_q):
     o = torch.empty((B, L, H * dh), dtype=torch.bfloat16, device="cuda")
     am = torch.zeros(B * L, dtype=torch.float32, device="cuda")
     h3b.h3b_attention(dims, bf16_dev(qkv_bits), o, am)
-    og = O.bf16_decode(bf16_host(o))
-    q = O.bf16_decode(qkv_bits)
+    og = bf16_f64(bf16_host(o))
+    q = bf16_f64(qkv_bits)
     rows = synth.sample_rows(L, n_q)
     for b in range(B):
         tm = lambda part: q[part, b].transpose(1, 0, 2).reshape(L, H * dh)
@@ -359,11 +359,11 @@ def test_token_pair_unpair(B, T, H, W, d):
     ym_bits = synth.f32_to_bf16_bits(r.standard_normal((B, T, H, W // 2, d)).astype(np.float32))
     out = torch.empty_like(xd)
     h3b.h3b_token_unpair(full, xd, xm, bf16_dev(ym_bits), out)
-    ref = O.token_unpair(x, xo, O.bf16_decode(ym_bits), B, T, H, W, d)
+    ref = O.token_unpair(x, xo, bf16_f64(ym_bits), B, T, H, W, d)
     # one bf16 rounding of the result plus the fp32 error of x + (ym - xm) when
     # the terms nearly cancel (relative to the terms' magnitude)
-    got = O.bf16_decode(bf16_host(out))
-    terms = np.abs(O.bf16_decode(x)) + np.repeat(np.abs(O.bf16_decode(ym_bits)) + np.abs(O.bf16_decode(xo)), 2,
+    got = bf16_f64(bf16_host(out))
+    terms = np.abs(bf16_f64(x)) + np.repeat(np.abs(bf16_f64(ym_bits)) + np.abs(bf16_f64(xo)), 2,
                                                  axis=3)
     assert np.all(np.abs(got - ref) <= 2.0 ** -8 * np.abs(ref) + 2.0 ** -20 * terms)
     # identity block: unpair(x, xm, xm) == x exactly
