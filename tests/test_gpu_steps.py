@@ -123,12 +123,14 @@ def test_ln_modulate_quantize(rows, d, items):
     assert np.all(np.abs(hgd - hod) <= bound)
     assert (hg != ho).mean() < 0.02
     # (2) codes and scales against the oracle's quantization of its own h. Rows whose h equals
-    #     the oracle's match bit for bit. Elsewhere each h element and the row absmax differ by at
-    #     most 2^-7 relative (1), so v/s moves by at most 127 * 2 * 2^-7 < 2 and a code by at most 2.
+    #     the oracle's match bit for bit. Elsewhere each h element, and so the row absmax A,
+    #     differs by at most 2^-7 relative plus 2^-16 A (1); the scale then moves by at most
+    #     2^-7 + 2^-15 relative, v/s by at most 127 * (2^-6 + 2^-15 + 2^-16) / (1 - 2^-7) < 2.01,
+    #     and a rounded code by at most 3.
     qo, so = O.quantize_rows(hod.astype(np.float32))
     same = np.all(hg == ho, axis=1)
     assert np.array_equal(qg[same], qo[same]) and np.array_equal(sg[same], so[same])
-    assert np.all(np.abs(qg.astype(np.int32) - qo.astype(np.int32)) <= 2)
+    assert np.all(np.abs(qg.astype(np.int32) - qo.astype(np.int32)) <= 3)
     assert np.all(np.abs(sg.astype(np.float64) - so) <= (2.0 ** -7 + 2.0 ** -15) * so)
     # (3) the kernel's int8 decision on its own h is the binary32 rule, bit for bit: s = absmax/127
     #     and q = rint(h/s) in float32, restated here in numpy (the oracle only sees seeded inputs)
