@@ -10,7 +10,10 @@ Per block over R = B*L tokens, model width d, MLP width F:
   2n, write n, read the 4-byte absmax, write the 4-byte scale;
   token pairing: read 2d per original token, write d/2 tokens' worth (2 bytes
   each) to each of its two destinations; unpairing: read x (2d) and the merged
-  xm and ym (d each) per original token, write 2d."""
+  xm and ym (d each) per original token, write 2d.
+
+The reference arm (the CPU oracle) is also run here end to end: it needs no GPU,
+and its JSON line follows the same contract as the CUDA arm's."""
 import pytest
 
 import bench
@@ -78,3 +81,52 @@ def test_variant_precisions_pick_their_roofline():
     assert bench.kernel_work("gemm_qkv", synth.WORKLOADS["d5120_L18432_bf16qkv"])[2] == "tensor_bf16"
     assert bench.kernel_work("gemm_wo", synth.WORKLOADS["d5120_L18432_bf16wo"])[2] == "tensor_bf16"
     assert bench.kernel_work("gemm_wo", synth.WORKLOADS["d5120_L18432"])[2] == "tensor_i8"
+
+
+def _run_bench(args, env_extra=None, timeout=600):
+    import json
+    import os
+    import subprocess
+    import sys
+    env = dict(os.environ)
+    env.update(env_extra or {})
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py")] + args, capture_output=True, text=True,
+                       timeout=timeout, env=env, cwd=root)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.strip()]
+    return [json.loads(ln) for ln in lines]
+
+
+def test_reference_arm_prints_one_contract_line():
+    # The reference arm is the CPU oracle (no GPU needed): one JSON line with the same
+    # metric and unit as the CUDA arm, its own cpu_baseline and an e2e with no copies.
+    out = _run_bench(["--impl", "reference", "--workload", "d256_L512", "--steps", "3", "--warmup", "3",
+                      "--ref-rows", "4"])
+    assert len(out) == 1
+    line = out[0]
+    assert line["impl"] == "reference"
+    assert line["metric"] == bench.METRIC and line["unit"] == bench.UNIT
+    assert line["value"] > 0 and line["ms_per_step"] > 0
+    assert (line["n_gpus"], line["steps"], line["warmup"]) == (1, 3, 3)
+    assert line["higher_is_better"] is True and line["vs_baseline"] is None
+    assert line["config"]["workload"] == "d256_L512"
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == line["value"] and cb["sample"]
+    assert line["e2e"] == {"value": line["value"], "unit": line["unit"], "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
+
+
+def test_reference_arm_runs_on_rank_0_only():
+    assert _run_bench(["--impl", "reference", "--workload", "d256_L512", "--steps", "3", "--warmup", "3"],
+                      {"RANK": "1", "WORLD_SIZE": "2"}) == []
+
+
+def test_bench_rejects_fewer_than_three_warmup_steps():
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference", "--warmup", "2"],
+                       capture_output=True, text=True, timeout=300, cwd=root)
+    assert r.returncode != 0 and "--warmup must be >= 3" in r.stderr
