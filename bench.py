@@ -153,7 +153,14 @@ class ClockSampler:
         except Exception:
             self.proc.kill()
             return None
-        rows = [r.split(",") for r in out.strip().splitlines() if r.strip()]
+        return self.summarize(out)
+
+    @staticmethod
+    def summarize(csv_text):
+        """Median SM clock of the busy samples (above half the highest one), the max clock,
+        and every throttle reason seen active, from nvidia-smi's csv,noheader,nounits rows
+        of FIELDS; None when no row parses."""
+        rows = [r.split(",") for r in csv_text.strip().splitlines() if r.strip()]
         rows = [[c.strip() for c in r] for r in rows if len(r) >= 8]
         if not rows:
             return None
@@ -164,7 +171,7 @@ class ClockSampler:
             for n, v in zip(names, r[4:8]):
                 if v.lower().startswith("active"):
                     reasons.add(n)
-        busy = [m for m in mhz if m > 0.5 * max(mhz)] or mhz
+        busy = ([m for m in mhz if m > 0.5 * max(mhz)] or mhz) if mhz else []
         return {"sm_mhz": statistics.median(busy) if busy else None,
                 "sm_max_mhz": float(rows[0][1]) if rows[0][1].replace(".", "").isdigit() else None,
                 "reasons": sorted(reasons), "samples": len(rows),

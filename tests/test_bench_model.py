@@ -130,3 +130,23 @@ def test_bench_rejects_fewer_than_three_warmup_steps():
     r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference", "--warmup", "2"],
                        capture_output=True, text=True, timeout=300, cwd=root)
     assert r.returncode != 0 and "--warmup must be >= 3" in r.stderr
+
+
+def test_clock_summary_of_nvidia_smi_rows():
+    rows = "\n".join([
+        "1965, 1965, 310.5, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
+        "1920, 1965, 990.1, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "1890, 1965, 998.7, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "345, 1965, 120.0, 0x0000000000000001, Not Active, Not Active, Not Active, Not Active",  # idle
+        "[N/A], 1965, [N/A], [N/A], [N/A], [N/A], [N/A], [N/A]",
+        "garbage line",
+    ])
+    c = bench.ClockSampler.summarize(rows)
+    assert c["sm_mhz"] == 1920.0  # median of the busy samples 1965, 1920, 1890
+    assert c["sm_max_mhz"] == 1965.0
+    assert c["reasons"] == ["sw_power_cap"]
+    assert c["samples"] == 5
+    hot = bench.ClockSampler.summarize("1500, 1965, 700, 0x40, Not Active, Active, Not Active, Not Active")
+    assert hot["reasons"] == ["hw_thermal_slowdown"]
+    assert bench.ClockSampler.summarize("") is None
+    assert bench.ClockSampler.summarize("[N/A], [N/A], 1, 2, 3, 4, 5, 6")["sm_mhz"] is None
