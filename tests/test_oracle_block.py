@@ -127,3 +127,28 @@ def test_bf16_wo_projection_is_the_plain_product():
     xd = O.bf16_decode(x).reshape(-1, d)
     rel = np.linalg.norm((out - xd) - (out8 - xd)) / np.linalg.norm(out8 - xd)
     assert 0 < rel < 0.1
+
+
+def test_single_thread_run_gives_identical_results(tmp_path):
+    """No reduction crosses OpenMP threads, so one thread and all threads give the same
+    bytes (the block is run in a child process with OMP_NUM_THREADS=1)."""
+    import os
+    import subprocess
+    import sys
+    wl = WL.with_(B=2)
+    w = _weights(wl)
+    x, c = synth.x_input(wl), synth.cond(wl)
+    many = O.block_forward(_dims(wl), w, c, x)
+    out = tmp_path / "one.npy"
+    code = (
+        "import sys, numpy as np\n"
+        f"sys.path.insert(0, {os.path.dirname(os.path.dirname(os.path.abspath(__file__)))!r})\n"
+        f"sys.path.insert(0, {os.path.dirname(os.path.abspath(__file__))!r})\n"
+        "import oracle as O, test_oracle_block as T\n"
+        "assert O.threads() == 1\n"
+        "wl = T.WL.with_(B=2)\n"
+        "y = O.block_forward(T._dims(wl), T._weights(wl), T.synth.cond(wl), T.synth.x_input(wl))\n"
+        f"np.save({str(out)!r}, y)\n")
+    env = dict(os.environ, OMP_NUM_THREADS="1")
+    subprocess.run([sys.executable, "-c", code], check=True, env=env, timeout=300)
+    assert np.array_equal(np.load(out), many)
