@@ -132,6 +132,12 @@ H3B_API const char* h3b_last_error_detail(void);
 H3B_API h3b_status h3b_workspace_size(const h3b_dims* dims, size_t* bytes);
 
 /* One block forward, in place on the residual stream x (bf16 [B][L][d]).
+ * The block of "h3-metal: Apple Silicon을 위한 네이티브 MiniMax-H3 추론",
+ * section "Int8 양자화" (gated AdaLN; int8 QKV and MLP with per-token activation
+ * and per-output-channel weight scales; the quantizer fused into the AdaLN
+ * kernel), with the head-major Q/K/V of section "Metal 4 및 TensorOps" and the
+ * AdaLN/RoPE folding of "h3.c與MLX路線對比：MiniMax-H3在Apple Silicon上的兩種推理
+ * 實現工程取捨", section "性能上限":
  *   mod = AdaLN Linear(c)                                  c: fp32 [B][d]
  *   A1,s1 = quant(bf16(LN(x)(1+scale_attn)+shift_attn))    (fused kernel)
  *   Q,K,V = deq(A1 Wqkv^T)+bqkv, 3D RoPE on Q,K, written head-major
@@ -167,20 +173,23 @@ H3B_API h3b_status h3b_block_forward(const h3b_dims* dims, const h3b_block_weigh
 H3B_API h3b_status h3b_block_forward_noalloc(const h3b_dims* dims, const h3b_block_weights* w,
                                              const float* c, void* x, h3b_stream stream);
 
-/* n_blocks blocks in sequence on one residual stream x; block i uses w[i]
+/* n_blocks blocks in sequence on one residual stream x (the denoiser's stack of
+ * blocks; each block as in h3b_block_forward); block i uses w[i]
  * (HOST array of n_blocks weight structs holding device pointers) and
  * c + i*B*d (device, fp32 [n_blocks][B][d]). Same workspace as one block. */
 H3B_API h3b_status h3b_blocks_forward(const h3b_dims* dims, const h3b_block_weights* w, int n_blocks,
                               const float* c, void* x, void* ws, size_t ws_bytes,
                               h3b_stream stream);
 
-/* Multi-block pass with token reduction over a middle range of blocks
- * ("Token Reduction" row of the control table: horizontally adjacent video
- * tokens are paired in the middle blocks). Blocks [0, first) run on the full
- * grid `full`; then the tokens are paired once (h3b_token_pair into xm and ym),
- * blocks [first, last) run on the merged grid (W/2, in place on ym), the
- * block deltas are added back at both positions once (h3b_token_unpair into
- * x), and blocks [last, n_blocks) run on the full grid again.
+/* Multi-block pass with token reduction over a middle range of blocks (the
+ * Token Reduction row of the control table in "h3-metal: ...", section
+ * "속도 및 품질 트레이드오프": horizontally adjacent video tokens are paired in
+ * the middle blocks).
+ * Blocks [0, first) run on the full grid `full`; then the tokens are paired
+ * once (h3b_token_pair into xm and ym), blocks [first, last) run on the merged
+ * grid (W/2, in place on ym), the block deltas are added back at both
+ * positions once (h3b_token_unpair into x), and blocks [last, n_blocks) run on
+ * the full grid again.
  *   0 <= first <= last <= n_blocks; full->W even when first < last.
  *   xm, ym: bf16 [B][T][H][W/2][d] device buffers (unused when first == last).
  *   ws: at least h3b_workspace_size(full) bytes (that covers the merged grid).
@@ -235,8 +244,10 @@ H3B_API h3b_status h3b_graph_launch(h3b_graph g, h3b_stream stream);
 H3B_API int h3b_graph_kernel_count(h3b_graph g);
 H3B_API void h3b_graph_destroy(h3b_graph g);
 
-/* Token reduction ("Token Reduction" row of the control table): horizontally
- * adjacent tokens w = 2k, 2k+1 of each (t, h) row are merged by their mean.
+/* Token reduction ("h3-metal: Apple Silicon을 위한 네이티브 MiniMax-H3 추론",
+ * section "속도 및 품질 트레이드오프", the control table's Token Reduction row):
+ * horizontally adjacent tokens w = 2k, 2k+1 of each (t, h) row are merged by
+ * their mean.
  *   full: dims of the UNMERGED grid (W even); only B, T, H, W and d are read:
  *   d % 8 == 0, d <= 65536, B*T*H*W < 2^31 (H3B_ERR_SHAPE otherwise).
  *   x  bf16 [B][T][H][W][d] -> xm bf16 [B][T][H][W/2][d], xm = bf16((a+b)/2).
