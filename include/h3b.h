@@ -2,8 +2,9 @@
  * h3b — forward pass of one gated-AdaLN DiT block over video latent tokens, on
  * NVIDIA B200 (sm_100a). C ABI: plain pointers and sizes, no framework types.
  *
- * The method (web pages about the h3.c / h3-metal MiniMax-H3 engine):
- *   "h3-metal: Apple Silicon을 위한 네이티브 MiniMax-H3 추론"
+ * The method (web pages about the h3.c / h3-metal MiniMax-H3 engine; cited in
+ * the entry points below by the short names in brackets):
+ *   [README] "h3-metal: Apple Silicon을 위한 네이티브 MiniMax-H3 추론"
  *       section "Int8 양자화": int8 MLP and QKV with dynamic per-row activation
  *       quantization and per-output-channel weight scales; the activation
  *       quantizer is fused into the preceding gated-AdaLN kernel.
@@ -11,10 +12,10 @@
  *       attention input.
  *       section "속도 및 품질 트레이드오프" (Token Reduction row): horizontally
  *       adjacent video tokens are paired in the middle blocks.
- *   "h3.c與MLX路線對比：MiniMax-H3在Apple Silicon上的兩種推理實現工程取捨"
+ *   [MLX] "h3.c與MLX路線對比：MiniMax-H3在Apple Silicon上的兩種推理實現工程取捨"
  *       section "性能上限": AdaLN gating, RoPE and quantization folded into the
  *       kernel ahead of the projections.
- *   "맥북에서 AI 영상 생성 모델 돌리기 - MiniMax H3 로컬 실행과 30초 애니메이션 만들기"
+ *   [BLOG] "맥북에서 AI 영상 생성 모델 돌리기 - MiniMax H3 로컬 실행과 30초 애니메이션 만들기"
  *       section "int8 이 뭔가요": one F32 scale per output channel (weights),
  *       one F32 scale per row computed at run time (activations).
  * Dimensions, LayerNorm eps, GELU form and the RoPE split are parameters; the
@@ -262,7 +263,8 @@ H3B_API h3b_status h3b_token_pair(const h3b_dims* full, const void* x, void* xm,
 H3B_API h3b_status h3b_token_unpair(const h3b_dims* full, const void* x, const void* xm, const void* ym,
                             void* out, h3b_stream stream);
 
-/* Per-output-channel weight quantization (offline): w fp32 [rows][cols] ->
+/* Per-output-channel weight quantization (offline; [BLOG] "int8 이 뭔가요": one F32
+ * scale per output channel): w fp32 [rows][cols] ->
  * q int8 [rows][cols], s fp32 [rows]; s = absmax/127 (float),
  * q = clamp(round-half-even(w/s), -127, 127); an all-zero row gives s = 0,
  * q = 0. cols % 16 == 0. */
@@ -297,12 +299,14 @@ H3B_API int h3b_profile_read(h3b_kernel_time* out, int max_entries);
  * step can be checked on its own.
  * ------------------------------------------------------------------------- */
 
-/* AdaLN Linear: mod[b][j] = sum_k w_ada[j][k] c[b][k] + b_ada[j]; mod fp32 [B][6d]. */
+/* AdaLN Linear ([README] "Int8 양자화", gated AdaLN; [MLX] "性能上限"):
+ * mod[b][j] = sum_k w_ada[j][k] c[b][k] + b_ada[j]; mod fp32 [B][6d]. */
 H3B_API h3b_status h3b_adaln_modulation(const h3b_dims* dims, const void* w_ada, const float* b_ada,
                                 const float* c, float* mod, h3b_stream stream);
 
-/* Fused LayerNorm + modulation + per-row int8 quantization over rows of x
- * (bf16 [rows][d]); shift/scale fp32 [d] broadcast over rows_per_item rows,
+/* Fused LayerNorm + modulation + per-row int8 quantization ([README] "Int8 양자화":
+ * the activation quantizer fused into the AdaLN kernel; [BLOG] "int8 이 뭔가요": one
+ * F32 scale per row, computed at run time) over rows of x (bf16 [rows][d]); shift/scale fp32 [d] broadcast over rows_per_item rows,
  * then advance by mod_stride floats per batch item (rows_per_item = L,
  * mod_stride = 6d when reading a mod buffer; rows_per_item = rows for one set).
  *   h = bf16(LN(x)(1+scale)+shift); s = absmax(h)/127; q = rint(h/s)
@@ -313,13 +317,15 @@ H3B_API h3b_status h3b_ln_modulate_quantize(const void* x, int rows, int d, floa
                                     int8_t* q, float* s, void* h_out, float* absmax_zero,
                                     int write_codes, h3b_stream stream);
 
-/* Per-row int8 quantization of bf16 rows (h bf16 [rows][cols]). If absmax is
+/* Per-row int8 quantization of bf16 rows ([BLOG] "int8 이 뭔가요"; the same rule as
+ * the fused kernel) (h bf16 [rows][cols]). If absmax is
  * non-NULL it holds each row's max |h| (as produced by the attention and GELU
  * steps) and the row is read once; otherwise it is computed here. */
 H3B_API h3b_status h3b_quantize_rows(const void* h, int rows, int cols, const float* absmax, int8_t* q,
                              float* s, h3b_stream stream);
 
-/* int8 GEMM on tensor cores, C[m][n] = sum_k A[m][k] W[n][k] (exact int32).
+/* int8 GEMM on tensor cores ([README] "Int8 양자화": int8 projections),
+ * C[m][n] = sum_k A[m][k] W[n][k] (exact int32).
  * A int8 [M][K], W int8 [N][K], C int32 [M][N]; M >= 0, N and K positive multiples of 16. */
 H3B_API h3b_status h3b_gemm_i8_s32(const int8_t* A, const int8_t* W, int32_t* C, int M, int N, int K,
                            h3b_stream stream);
@@ -329,7 +335,8 @@ H3B_API h3b_status h3b_gemm_i8_dequant(const int8_t* A, const float* sA, const i
                                const float* bias, void* out, int M, int N, int K,
                                h3b_stream stream);
 
-/* QKV projection with 3D RoPE, written head-major:
+/* QKV projection with 3D RoPE ([MLX] "性能上限": RoPE folded ahead of the
+ * attention), written head-major ([README] "Metal 4 및 TensorOps"):
  *   qkv bf16 [3][B][n_heads][L][head_dim] (part, batch item, head, token, lane).
  * int8 (dims->qkv_int8 == 1): A int8 [B*L][d] + sA, w->wqkv + w->sqkv.
  * bf16 (dims->qkv_int8 == 0): A bf16 [B*L][d] (sA ignored), w->wqkv_bf16.
@@ -339,14 +346,17 @@ H3B_API h3b_status h3b_qkv_projection(const h3b_dims* dims, const void* A, const
                               h3b_stream stream);
 H3B_API size_t h3b_rope_table_bytes(const h3b_dims* dims);
 
-/* Non-causal attention per batch item and head on the head-major qkv buffer.
+/* Non-causal attention per batch item and head on the head-major qkv buffer
+ * (full attention over all latent tokens: [BLOG] "★ 긴 영상은 나눠 찍는 게 훨씬
+ * 쌉니다", step time growing about as frames^1.9).
  * o bf16 [B][L][d] (token-major, head h at columns [h*head_dim, (h+1)*head_dim));
  * absmax fp32 [B*L]: each row's max |o| is max-combined into it (zero it first).
  * Reads B, T, H, W, n_heads and head_dim only: B*n_heads <= 65535, B*L < 2^31. */
 H3B_API h3b_status h3b_attention(const h3b_dims* dims, const void* qkv, void* o, float* absmax,
                          h3b_stream stream);
 
-/* int8 GEMM with gated residual epilogue, in place on x bf16 [M][N]:
+/* int8 GEMM with gated residual epilogue ([README] "Int8 양자화", gated AdaLN),
+ * in place on x bf16 [M][N]:
  *   x[m][n] = bf16(x[m][n] + gate[m / rows_per_item][n] * (C*sA[m]*sW[n] + bias[n]))
  * gate fp32, rows of gate_stride floats per batch item. */
 H3B_API h3b_status h3b_gemm_i8_gated_residual(const int8_t* A, const float* sA, const int8_t* W,
@@ -354,7 +364,8 @@ H3B_API h3b_status h3b_gemm_i8_gated_residual(const int8_t* A, const float* sA, 
                                       int rows_per_item, int gate_stride, void* x, int M, int N,
                                       int K, h3b_stream stream);
 
-/* bf16 GEMM with gated residual epilogue, in place on x bf16 [M][N]:
+/* bf16 GEMM with gated residual epilogue ([README] "Metal 4 및 TensorOps": the BF16
+ * attention-output projection), in place on x bf16 [M][N]:
  *   x[m][n] = bf16(x[m][n] + gate[m / rows_per_item][n] * (sum_k A[m][k] W[n][k] + bias[n]))
  * A bf16 [M][K], W bf16 [N][K] (fp32 accumulation); gate as above. The output
  * projection of the block when dims->wo_bf16 == 1. Same argument rules as
@@ -364,7 +375,7 @@ H3B_API h3b_status h3b_gemm_bf16_gated_residual(const void* A, const void* W, co
                                                 const float* gate, int rows_per_item, int gate_stride,
                                                 void* x, int M, int N, int K, h3b_stream stream);
 
-/* int8 GEMM with GELU epilogue: g bf16 [M][N] = bf16(GELU_tanh(C*sA[m]*sW[n] + bias[n]));
+/* int8 GEMM with GELU epilogue ([README] "Int8 양자화": int8 MLP): g bf16 [M][N] = bf16(GELU_tanh(C*sA[m]*sW[n] + bias[n]));
  * absmax fp32 [M] max-combined with each row's max |g| (zero it first). */
 H3B_API h3b_status h3b_gemm_i8_gelu(const int8_t* A, const float* sA, const int8_t* W, const float* sW,
                             const float* bias, void* g, float* absmax, int M, int N, int K,
