@@ -288,6 +288,49 @@ class OracleRunner:
         return self.O.threads()
 
 
+def roofline_summary(prof, wl, peaks, peak_src):
+    """From the profiler's {kernel: (launches, total ms)}: each kernel's share of the device
+    time, every kernel's achieved rate and fraction of its roofline (algorithmic work per
+    launch / mean launch duration), and the dominant kernel's roofline object."""
+    ktot = sum(ms for _, ms in prof.values()) or 1.0
+    shares = {k: round(ms / ktot, 4) for k, (n, ms) in sorted(prof.items(), key=lambda kv: -kv[1][1])}
+
+    def peak_of(bound):
+        if bound == "hbm":
+            return peaks["hbm_gbs"]
+        return peaks["bf16_tflops"] * (INT8_OVER_BF16 if bound == "tensor_i8" else 1.0)
+
+    def rate(work, seconds, bound):  # GB/s for bytes, T(FL)OP/s for tensor work
+        return work / seconds / (1e9 if bound == "hbm" else 1e12)
+
+    dom = max(prof.items(), key=lambda kv: kv[1][1])[0] if prof else None
+    roof = None
+    if dom:
+        n_launch, ms = prof[dom]
+        per_launch_s = ms / n_launch / 1e3
+        work, unit, bound = kernel_work(dom, wl)
+        achieved, peak = rate(work, per_launch_s, bound), peak_of(bound)
+        runit = "GB/s" if bound == "hbm" else ("TOP/s" if bound == "tensor_i8" else "TFLOP/s")
+        source = {"tensor_i8": "bf16 burst x 2 nominal int8/bf16 ratio", "tensor_bf16": "bf16 burst"}.get(
+            bound, "copy bandwidth")
+        roof = {"bound": "hbm" if bound == "hbm" else "tensor", "kernel": dom, "achieved": round(achieved, 2),
+                "peak": round(peak, 1), "unit": runit, "frac": round(achieved / peak, 4),
+                "traffic": traffic_for(dom, wl, n_launch), "peak_source": f"{peak_src} ({source})",
+                "work_per_launch": work, "work_unit": unit, "launch_ms": round(per_launch_s * 1e3, 4)}
+    all_roof = {}
+    for k, (n, ms) in prof.items():
+        work, unit, bound = kernel_work(k, wl)
+        if work <= 0:
+            continue
+        r = rate(work, ms / n / 1e3, bound)
+        if bound == "hbm":
+            all_roof[k] = {"GB/s": round(r, 1), "frac": round(r / peak_of(bound), 3)}
+        else:
+            all_roof[k] = {("TOP/s" if bound == "tensor_i8" else "TFLOP/s"): round(r, 1),
+                           "frac": round(r / peak_of(bound), 3)}
+    return roof, shares, all_roof
+
+
 # ----------------------------------------------------------------------------- arms
 
 # multi-GPU bookkeeping (replicas, no data-path collective): see replicas.py
@@ -429,37 +472,7 @@ def run_h3b(args, rank, world, local):
         launch["kernels_per_step"] = graph.kernel_count
         graph.destroy()
 
-    # ---- roofline of the dominant kernel (live per-kernel device times)
-    ktot = sum(ms for _, ms in prof.values()) or 1.0
-    shares = {k: round(ms / ktot, 4) for k, (n, ms) in sorted(prof.items(), key=lambda kv: -kv[1][1])}
-    dom = max(prof.items(), key=lambda kv: kv[1][1])[0] if prof else None
-    roof = None
-    if dom:
-        n_launch, ms = prof[dom]
-        per_launch_s = ms / n_launch / 1e3
-        work, unit, bound = kernel_work(dom, wl)
-        if bound == "hbm":
-            achieved, peak, runit, rb = work / per_launch_s / 1e9, peaks["hbm_gbs"], "GB/s", "hbm"
-        else:
-            achieved = work / per_launch_s / 1e12
-            peak = peaks["bf16_tflops"] * (INT8_OVER_BF16 if bound == "tensor_i8" else 1.0)
-            runit, rb = ("TOP/s" if bound == "tensor_i8" else "TFLOP/s"), "tensor"
-        roof = {"bound": rb, "kernel": dom, "achieved": round(achieved, 2), "peak": round(peak, 1), "unit": runit,
-                "frac": round(achieved / peak, 4), "traffic": traffic_for(dom, wl, n_launch),
-                "peak_source": f"{peak_src} ({'bf16 burst x 2 nominal int8/bf16 ratio' if bound == 'tensor_i8' else 'bf16 burst' if bound == 'tensor_bf16' else 'copy bandwidth'})",
-                "work_per_launch": work, "work_unit": unit, "launch_ms": round(per_launch_s * 1e3, 4)}
-    all_roof = {}
-    for k, (n, ms) in prof.items():
-        work, unit, bound = kernel_work(k, wl)
-        if work <= 0:
-            continue
-        s = ms / n / 1e3
-        if bound == "hbm":
-            all_roof[k] = {"GB/s": round(work / s / 1e9, 1), "frac": round(work / s / 1e9 / peaks["hbm_gbs"], 3)}
-        else:
-            pk = peaks["bf16_tflops"] * (INT8_OVER_BF16 if bound == "tensor_i8" else 1.0)
-            all_roof[k] = {("TOP/s" if bound == "tensor_i8" else "TFLOP/s"): round(work / s / 1e12, 1),
-                           "frac": round(work / s / 1e12 / pk, 3)}
+    roof, shares, all_roof = roofline_summary(prof, wl, peaks, peak_src)
 
     gpu_launches = int(sum(n for n, _ in prof.values()))
     kernel_ms = {k: round(ms / args.steps, 4) for k, (n, ms) in prof.items()}

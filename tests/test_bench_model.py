@@ -150,3 +150,28 @@ def test_clock_summary_of_nvidia_smi_rows():
     assert hot["reasons"] == ["hw_thermal_slowdown"]
     assert bench.ClockSampler.summarize("") is None
     assert bench.ClockSampler.summarize("[N/A], [N/A], 1, 2, 3, 4, 5, 6")["sm_mhz"] is None
+
+
+def test_roofline_summary_of_a_profile():
+    # 10 steps of the d=2048 block: attention 1.50 ms over 10 launches (dominant), QKV 0.60 ms,
+    # the attention LN quantizer 0.20 ms
+    wl = synth.WORKLOADS["d2048_L4096"]
+    peaks = {"hbm_gbs": 6500.0, "bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0}
+    prof = {"attention": (10, 1.5), "gemm_qkv": (10, 0.6), "ln_mod_quant": (10, 0.2)}
+    roof, shares, all_roof = bench.roofline_summary(prof, wl, peaks, "measured")
+    assert list(shares) == ["attention", "gemm_qkv", "ln_mod_quant"]
+    assert shares["attention"] == pytest.approx(1.5 / 2.3, abs=1e-4)
+    flops = 4.0 * wl.L ** 2 * wl.d
+    assert roof["kernel"] == "attention" and roof["bound"] == "tensor" and roof["unit"] == "TFLOP/s"
+    assert roof["achieved"] == pytest.approx(flops / 150e-6 / 1e12, abs=0.01)
+    assert roof["peak"] == 1600.0 and roof["frac"] == pytest.approx(roof["achieved"] / 1600.0, abs=1e-4)
+    assert roof["launch_ms"] == 0.15 and roof["work_per_launch"] == flops
+    # the int8 GEMM against twice the bf16 peak, the LN quantizer against HBM
+    ops = 2.0 * wl.L * 3 * wl.d * wl.d
+    assert all_roof["gemm_qkv"]["TOP/s"] == pytest.approx(ops / 60e-6 / 1e12, abs=0.05)
+    assert all_roof["gemm_qkv"]["frac"] == pytest.approx(ops / 60e-6 / 1e12 / 3200.0, abs=1e-3)
+    byts = wl.L * (3 * wl.d + 8)
+    assert all_roof["ln_mod_quant"]["GB/s"] == pytest.approx(byts / 20e-6 / 1e9, abs=0.05)
+    assert all_roof["ln_mod_quant"]["frac"] == pytest.approx(byts / 20e-6 / 1e9 / 6500.0, abs=1e-3)
+    # an empty profile gives no roofline
+    assert bench.roofline_summary({}, wl, peaks, "measured") == (None, {}, {})
