@@ -242,6 +242,21 @@ def test_attention_matches_torch_sdpa():
     assert np.max(np.abs(out - ref)) < 1e-12
 
 
+def test_attention_matches_a_naive_loop_on_tiny_inputs():
+    """Scores, a max-free softmax and the weighted sum, written as plain Python loops."""
+    rng = np.random.default_rng(12)
+    nh, dh, L, nq = 2, 4, 5, 3
+    Q, K, V = (rng.standard_normal((n, nh * dh)) for n in (nq, L, L))
+    out = O.attention(Q, K, V, nh, dh)
+    for i in range(nq):
+        for h in range(nh):
+            cols = range(h * dh, (h + 1) * dh)
+            w = [math.exp(sum(Q[i, c] * K[j, c] for c in cols) / math.sqrt(dh)) for j in range(L)]
+            tot = sum(w)
+            for c in cols:
+                assert abs(out[i, c] - sum(w[j] / tot * V[j, c] for j in range(L))) < 1e-12
+
+
 def test_attention_special_cases():
     rng = np.random.default_rng(10)
     nh, dh, L = 2, 8, 9
