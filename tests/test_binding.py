@@ -138,3 +138,24 @@ def test_a_failing_status_raises_with_the_library_detail(monkeypatch):
         h3b.h3b_gemm_i8_s32(t(16, 16, dtype=torch.int8), t(24, 16, dtype=torch.int8), t(16, 24, dtype=torch.int32),
                             stream=0)
     assert e.value.status == -2 and "multiple of 16" in str(e.value) and "H3B_ERR_SHAPE" in str(e.value)
+
+
+def test_remaining_wrappers(rec):
+    dims = h3b.make_dims(2, 2, 16, 16, 256, 4, 64, 1024, (16, 24, 24))
+    w_ada, b_ada, c, mod = t(1536, 256, dtype=torch.bfloat16), t(1536), t(2, 256), t(2, 1536)
+    h3b.h3b_adaln_modulation(dims, w_ada, b_ada, c, mod, stream=9)
+    args = last(rec, "h3b_adaln_modulation")
+    assert args[0]._obj is dims and args[1:] == (ptr(w_ada), ptr(b_ada), ptr(c), ptr(mod), 9)
+    w = h3b.make_weights({"w1": t(4)})
+    assert w.w_ada is None and w.w1 is not None  # missing names are NULL
+    x = t(1024, 256, dtype=torch.bfloat16)
+    h3b.h3b_block_forward_noalloc(dims, w, c, x, stream=9)
+    args = last(rec, "h3b_block_forward_noalloc")
+    assert args[1]._obj is w and args[2:] == (ptr(c), ptr(x), 9)
+    ws = t(4096, dtype=torch.uint8)
+    g = h3b.h3b_graph_capture_blocks(dims, [w, w], c, x, ws)
+    args = last(rec, "h3b_graph_capture_blocks")
+    assert args[2:6] == (2, ptr(c), ptr(x), ptr(ws)) and args[6] == 4096
+    g.handle = None  # the stand-in returned no graph; nothing to destroy
+    assert h3b.h3b_device_error(clear=False) == 0
+    assert last(rec, "h3b_device_error")[1] == 0
