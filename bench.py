@@ -269,8 +269,9 @@ class OracleRunner:
         self.O.block_forward(self.dm, self.w, self.c, self.x, rows=rows)
         return time.perf_counter() - t0
 
-    def measure_kv(self):
-        self.t_kv = self.run(0)
+    def measure_kv(self, reps=1):
+        """Seconds of a1-a3 over all tokens (the median of `reps` runs)."""
+        self.t_kv = statistics.median(self.run(0) for _ in range(max(1, reps)))
         return self.t_kv
 
     def estimate(self, n_rows):
@@ -279,6 +280,18 @@ class OracleRunner:
             self.measure_kv()
         t = self.run(n_rows)
         return self.t_kv + max(t - self.t_kv, 0.0) / n_rows * self.R
+
+    def baseline(self, n_rows, budget_s=30.0):
+        """Median of up to three extrapolations, each against a median a1-a3 time, within
+        about `budget_s` seconds of host work (one of each when a single run is already long)."""
+        t0 = time.perf_counter()
+        first = self.run(0)
+        reps = 3 if 6 * first < budget_s else 1
+        self.t_kv = statistics.median([first] + [self.run(0) for _ in range(reps - 1)])
+        ests = []
+        while len(ests) < reps and (not ests or time.perf_counter() - t0 < budget_s):
+            ests.append(self.estimate(n_rows))
+        return statistics.median(ests), len(ests)
 
     def sample_text(self, n_rows):
         return (f"a1-a3 over all {self.R} tokens + a4-a9 on {n_rows} sampled tokens, "
@@ -480,9 +493,9 @@ def run_h3b(args, rank, world, local):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         orc = OracleRunner(wl)
-        est_s = orc.estimate(args.cpu_rows)
+        est_s, n_est = orc.baseline(args.cpu_rows)
         cpu = {"value": round(W.tokens / est_s, 2), "unit": UNIT, "cores": orc.threads(),
-               "kind": "oracle", "sample": orc.sample_text(args.cpu_rows)}
+               "kind": "oracle", "sample": orc.sample_text(args.cpu_rows) + f" (median of {n_est})"}
 
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
