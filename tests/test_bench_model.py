@@ -175,3 +175,15 @@ def test_roofline_summary_of_a_profile():
     assert all_roof["ln_mod_quant"]["frac"] == pytest.approx(byts / 20e-6 / 1e9 / 6500.0, abs=1e-3)
     # an empty profile gives no roofline
     assert bench.roofline_summary({}, wl, peaks, "measured") == (None, {}, {})
+
+
+def test_cpu_baseline_estimate_on_the_smallest_block():
+    orc = bench.OracleRunner(synth.WORKLOADS["d256_L512"])
+    est, n = orc.baseline(64, budget_s=30.0)
+    assert n == 3 and est > 0
+    # the extrapolation from 64 of 512 tokens stays within a small factor of a full run
+    import time
+    t0 = time.perf_counter()
+    orc.run(512)
+    full = time.perf_counter() - t0
+    assert 0.2 * full < est < 20 * full
