@@ -275,6 +275,14 @@ H3B_API h3b_status h3b_quantize_weights(const float* w, int rows, int cols, int8
  * Synchronizes the device. *code == 0 means no bounded wait ran out. */
 H3B_API h3b_status h3b_device_error(unsigned int* code, int clear);
 
+/* Test hook for failure detection without a GPU fault: one thread on the
+ * current device waits, with the bounded wait every pipeline of this library
+ * uses, on an mbarrier phase that nothing completes. The wait gives up after
+ * limit_ns (1 us to 1 s), ORs 1 << 5 into the device error word and the kernel
+ * returns normally; the context stays usable. Synchronous (legacy default
+ * stream). *waited_out = 1 when the wait ran out (the expected outcome). */
+H3B_API h3b_status h3b_test_bounded_wait(unsigned long long limit_ns, int* waited_out);
+
 /* ---------------------------------------------------------------------------
  * Kernel-level timing. While enabled (per process), every kernel launched by
  * the block entry points (h3b_block_forward, h3b_blocks_forward,

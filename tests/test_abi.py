@@ -239,3 +239,11 @@ def test_reuse_and_graph_validation(L):
     assert L.h3b_graph_launch(None, None) == -1
     assert L.h3b_graph_kernel_count(None) == 0
     L.h3b_graph_destroy(None)  # a no-op
+
+
+def test_bounded_wait_hook_validation(L):
+    out = C.c_int(-1)
+    assert L.h3b_test_bounded_wait(10, C.byref(out)) == -1  # below 1 us
+    assert L.h3b_test_bounded_wait(2_000_000_000, C.byref(out)) == -1  # above 1 s
+    assert L.h3b_test_bounded_wait(1_000_000, None) == -1
+    assert out.value == -1

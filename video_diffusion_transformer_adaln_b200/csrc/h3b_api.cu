@@ -24,6 +24,22 @@
 // runs out. Host code reaches it through its device address (per device).
 __device__ unsigned int g_h3b_error_word;
 
+// Test hook for the bounded waits: one thread waits, with the same bounded
+// mbarrier wait every pipeline uses, on a phase that nothing completes, so the
+// wait runs out after limit_ns, records ERR_WAIT_PROBE in the error word and
+// returns. Result: 1 when the wait ran out, 0 if the phase completed.
+__device__ int g_h3b_probe_result;
+
+static __global__ void bounded_wait_probe_kernel(unsigned* err, unsigned long long limit_ns) {
+  __shared__ __align__(8) unsigned long long bar;
+  if (threadIdx.x != 0) return;
+  const uint32_t b = h3b::smem_u32(&bar);
+  h3b::mbar_init(b, 1);
+  h3b::fence_barrier_init();
+  const bool completed = h3b::mbar_wait(b, 0, err, h3b::ERR_WAIT_PROBE, limit_ns);
+  g_h3b_probe_result = completed ? 0 : 1;
+}
+
 namespace h3b {
 namespace {
 
@@ -609,6 +625,20 @@ h3b_status h3b_quantize_weights(const float* w, int rows, int cols, int8_t* q, f
   h3b_status hs = device_info(&di);
   if (hs != H3B_OK) return hs;
   H3B_CK(launch_quant_rows_f32(w, rows, cols, q, s, stream), "quantize_weights");
+  return H3B_OK;
+}
+
+h3b_status h3b_test_bounded_wait(unsigned long long limit_ns, int* waited_out) {
+  if (!waited_out) return fail(H3B_ERR_ARG, "waited_out is NULL");
+  if (limit_ns < 1000ull || limit_ns > 1000000000ull) return fail(H3B_ERR_ARG, "limit_ns must be in [1 us, 1 s]");
+  DeviceInfo* di = nullptr;
+  h3b_status s = device_info(&di);
+  if (s != H3B_OK) return s;
+  cudaStream_t st = nullptr;
+  H3B_CK((bounded_wait_probe_kernel<<<1, 32>>>(di->err, limit_ns), cudaGetLastError()), "bounded_wait_probe");
+  int r = -1;
+  H3B_CK(cudaMemcpyFromSymbol(&r, g_h3b_probe_result, sizeof(int)), "read probe result");  // waits for the kernel
+  *waited_out = r;
   return H3B_OK;
 }
 

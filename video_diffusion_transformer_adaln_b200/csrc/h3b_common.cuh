@@ -19,6 +19,7 @@ enum : unsigned {
   ERR_WAIT_EPI = 1u << 2,       // a wait for the epilogue / softmax ran out
   ERR_WAIT_DRAIN = 1u << 3,     // a drain wait after an abort ran out
   ERR_BAD_LAUNCH = 1u << 4,     // a kernel saw launch parameters it cannot handle
+  ERR_WAIT_PROBE = 1u << 5,     // the test hook's wait ran out (h3b_test_bounded_wait)
 };
 
 // Upper bound on any single device-side wait. A healthy wait lasts micro- to

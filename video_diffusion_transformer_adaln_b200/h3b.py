@@ -82,6 +82,7 @@ def _declare(L):
         "h3b_token_unpair": [vp, vp, vp, vp, vp, vp],
         "h3b_quantize_weights": [vp, i32, i32, vp, vp, vp],
         "h3b_device_error": [C.POINTER(C.c_uint), i32],
+        "h3b_test_bounded_wait": [C.c_ulonglong, C.POINTER(C.c_int)],
         "h3b_adaln_modulation": [vp, vp, vp, vp, vp, vp],
         "h3b_ln_modulate_quantize": [vp, i32, i32, f32, vp, vp, i32, i32, vp, vp, vp, vp, i32, vp],
         "h3b_quantize_rows": [vp, i32, i32, vp, vp, vp, vp],
@@ -270,6 +271,13 @@ def h3b_device_error(clear: bool = True) -> int:
     if st not in (H3B_OK, -7):
         _check(st, "h3b_device_error")
     return code.value
+
+
+def h3b_test_bounded_wait(limit_ns: int) -> int:
+    """Run the library's bounded-wait test hook (see include/h3b.h); 1 when the wait ran out."""
+    out = C.c_int(-1)
+    _check(lib().h3b_test_bounded_wait(limit_ns, C.byref(out)), "h3b_test_bounded_wait")
+    return out.value
 
 
 # --------------------------------------------------------------------------- steps
