@@ -334,7 +334,8 @@ H3B_API h3b_status h3b_quantize_rows(const void* h, int rows, int cols, const fl
 
 /* int8 GEMM on tensor cores ([README] "Int8 양자화": int8 projections),
  * C[m][n] = sum_k A[m][k] W[n][k] (exact int32).
- * A int8 [M][K], W int8 [N][K], C int32 [M][N]; M >= 0, N and K positive multiples of 16. */
+ * A int8 [M][K], W int8 [N][K], C int32 [M][N]; M >= 0, N and K positive multiples of 16;
+ * M*N, M*K and N*K at most 2^40 (the same rules for every GEMM entry point). */
 H3B_API h3b_status h3b_gemm_i8_s32(const int8_t* A, const int8_t* W, int32_t* C, int M, int N, int K,
                            h3b_stream stream);
 

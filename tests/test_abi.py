@@ -247,3 +247,71 @@ def test_bounded_wait_hook_validation(L):
     assert L.h3b_test_bounded_wait(2_000_000_000, C.byref(out)) == -1  # above 1 s
     assert L.h3b_test_bounded_wait(1_000_000, None) == -1
     assert out.value == -1
+
+
+_I32 = (-2 ** 31, 2 ** 31 - 1)
+
+
+def _int_field(lo, hi):
+    from hypothesis import strategies as st
+    # mostly valid-looking values, plus edges and arbitrary int32
+    return st.one_of(st.integers(lo, hi), st.sampled_from([0, -1, 1, 2 ** 31 - 1, -2 ** 31, 2 ** 16, 2 ** 30]),
+                     st.integers(*_I32))
+
+
+def test_dims_checks_accept_exactly_the_documented_shapes(L):
+    """Property test of the host dims check (h3b_workspace_size): any int values either give
+    an error status, or satisfy every documented limit; nothing crashes or overflows."""
+    from hypothesis import HealthCheck, given, settings
+    from hypothesis import strategies as st
+
+    @settings(max_examples=400, deadline=None, suppress_health_check=list(HealthCheck))
+    @given(B=_int_field(1, 9), T=_int_field(1, 64), H=_int_field(1, 64), W=_int_field(1, 64),
+           heads=_int_field(1, 64), hd=st.sampled_from([64, 128, 96, 0, -64]), dff=_int_field(256, 40000),
+           split=st.sampled_from([(16, 24, 24), (32, 48, 48), (15, 25, 24), (0, 0, 64), (64, 64, 0)]))
+    def check(B, T, H, W, heads, hd, dff, split):
+        d = _dims(B=B, T=T, H=H, W=W, n_heads=heads, head_dim=hd, d=heads * hd if abs(heads * hd) < 2 ** 31 else 0,
+                  d_ff=dff, rope_t=split[0], rope_h=split[1], rope_w=split[2])
+        n = C.c_size_t(0)
+        st_ = L.h3b_workspace_size(C.byref(d), C.byref(n))
+        if st_ == 0:
+            Lt = d.T * d.H * d.W
+            assert 1 <= d.B <= 8 and min(d.T, d.H, d.W) >= 1 and d.B * Lt < 2 ** 31
+            assert d.head_dim in (64, 128) and d.d == d.n_heads * d.head_dim and d.d % 256 == 0 and d.d <= 8192
+            assert d.d_ff % 256 == 0 and 256 <= d.d_ff <= 32768 and d.B * Lt * d.d_ff <= 2 ** 40
+            assert d.rope_t + d.rope_h + d.rope_w == d.head_dim
+            assert n.value >= d.B * Lt * max(d.d, d.d_ff)
+        else:
+            assert st_ in (-1, -2)
+    check()
+
+
+def test_head_count_overflow_is_rejected(L):
+    # n_heads * head_dim wraps a 32-bit int to 0 here; d = 0 must not pass as "a multiple of 256"
+    d = _dims(n_heads=2 ** 30, head_dim=64, d=0)
+    with pytest.raises(h3b.H3BError):
+        h3b.h3b_workspace_size(d)
+    with pytest.raises(h3b.H3BError):
+        h3b.h3b_workspace_size(_dims(d=0, n_heads=0))
+
+
+def test_gemm_sizes_property(L):
+    """Any int M, N, K: either an error before any device query, or sizes within the
+    documented rules (here checked with NULL operands, so a passing size reports the
+    NULL pointer, or OK for M == 0)."""
+    from hypothesis import HealthCheck, given, settings
+    from hypothesis import strategies as st
+    ints = st.one_of(st.integers(-64, 4096), st.integers(*_I32),
+                     st.sampled_from([0, 16, 2 ** 31 - 16, 2 ** 20 * 16, 2 ** 24]))
+
+    @settings(max_examples=400, deadline=None, suppress_health_check=list(HealthCheck))
+    @given(M=ints, N=ints, K=ints)
+    def check(M, N, K):
+        st_ = L.h3b_gemm_i8_s32(None, None, None, M, N, K, None)
+        ok_sizes = M >= 0 and N >= 16 and N % 16 == 0 and K >= 16 and K % 16 == 0 and \
+            max(M * N, M * K, N * K) <= 2 ** 40
+        if not ok_sizes:
+            assert st_ == -2
+        else:
+            assert st_ == (0 if M == 0 else -1)
+    check()

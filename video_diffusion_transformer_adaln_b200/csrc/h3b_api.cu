@@ -113,8 +113,9 @@ h3b_status check_dims(const h3b_dims* d) {
   if (d->B < 1 || d->T < 1 || d->H < 1 || d->W < 1) return fail(H3B_ERR_SHAPE, "B, T, H, W must be >= 1");
   if (d->B > 8) return fail(H3B_ERR_SHAPE, "B must be <= 8");
   if (d->head_dim != 64 && d->head_dim != 128) return fail(H3B_ERR_SHAPE, "head_dim must be 64 or 128");
-  if (d->n_heads < 1 || d->d != d->n_heads * d->head_dim) return fail(H3B_ERR_SHAPE, "d != n_heads * head_dim");
-  if (d->d % 256 != 0 || d->d > 8192) return fail(H3B_ERR_SHAPE, "d must be a multiple of 256, <= 8192");
+  if (d->n_heads < 1 || (long long)d->d != (long long)d->n_heads * d->head_dim)
+    return fail(H3B_ERR_SHAPE, "d != n_heads * head_dim");
+  if (d->d < 256 || d->d % 256 != 0 || d->d > 8192) return fail(H3B_ERR_SHAPE, "d must be a multiple of 256 in [256, 8192]");
   if (d->d_ff < 256 || d->d_ff % 256 != 0 || d->d_ff > 32768)
     return fail(H3B_ERR_SHAPE, "d_ff must be a multiple of 256 in [256, 32768]");
   if (d->rope_t < 0 || d->rope_h < 0 || d->rope_w < 0 || (d->rope_t | d->rope_h | d->rope_w) & 1 ||
@@ -709,6 +710,9 @@ static h3b_status gemm_checks(const void* A, const void* W, const void* out, int
   *empty = false;
   if (M < 0 || N < 16 || N % 16 != 0 || K < 16 || K % 16 != 0)
     return fail(H3B_ERR_SHAPE, "need M >= 0, N and K positive multiples of 16");
+  const long long lim = 1LL << 40;  // elements of any operand or result; keeps every tile count in int
+  if ((long long)M * N > lim || (long long)M * K > lim || (long long)N * K > lim)
+    return fail(H3B_ERR_SHAPE, "problem too large (an operand or the result exceeds 2^40 elements)");
   if (M == 0) {
     *empty = true;
     return H3B_OK;
