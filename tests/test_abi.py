@@ -315,3 +315,54 @@ def test_gemm_sizes_property(L):
         else:
             assert st_ == (0 if M == 0 else -1)
     check()
+
+
+def test_step_size_checks_property(L):
+    """Arbitrary int32 sizes for the row, pairing and attention entry points, with NULL
+    pointers: a size outside the documented rules gives SHAPE (or ARG for the item
+    layout); a legal size gives OK when the problem is empty, else the NULL-pointer ARG."""
+    from hypothesis import HealthCheck, given, settings
+    from hypothesis import strategies as st
+    ints = st.one_of(st.integers(-4, 9000), st.integers(*_I32), st.sampled_from([0, 8, 16, 256, 2 ** 30, 2 ** 31 - 1]))
+    cfg = settings(max_examples=300, deadline=None, suppress_health_check=list(HealthCheck))
+
+    @cfg
+    @given(rows=ints, cols=ints)
+    def quant(rows, cols):
+        st_ = L.h3b_quantize_rows(None, rows, cols, None, None, None, None)
+        if rows < 0 or cols < 16 or cols % 16:
+            assert st_ == -2
+        else:
+            assert st_ == (0 if rows == 0 else -1)
+    quant()
+
+    @cfg
+    @given(rows=ints, d=ints, rpi=ints, ms=ints)
+    def ln(rows, d, rpi, ms):
+        st_ = L.h3b_ln_modulate_quantize(None, rows, d, 1e-6, None, None, rpi, ms, None, None, None, None, 1, None)
+        if rows < 0 or d < 256 or d % 256 or d > 8192:
+            assert st_ == -2
+        elif rpi < 1 or ms < 0 or ms % 4:
+            assert st_ == -1
+        else:
+            assert st_ == (0 if rows == 0 else -1)
+    ln()
+
+    @cfg
+    @given(B=ints, T=ints, H=ints, W=ints, d=ints)
+    def pair(B, T, H, W, d):
+        full = _dims(B=B, T=T, H=H, W=W, d=d)
+        st_ = L.h3b_token_pair(C.byref(full), None, None, None, None)
+        legal = B >= 1 and T >= 1 and H >= 1 and W >= 2 and W % 2 == 0 and 8 <= d <= 65536 and d % 8 == 0 and \
+            B * T * H * W < 2 ** 31
+        assert st_ == (-1 if legal else -2)
+    pair()
+
+    @cfg
+    @given(B=ints, T=ints, H=ints, W=ints, nh=ints, hd=st.sampled_from([64, 128, 32, 0]))
+    def attn(B, T, H, W, nh, hd):
+        dims = _dims(B=B, T=T, H=H, W=W, n_heads=nh, head_dim=hd)
+        st_ = L.h3b_attention(C.byref(dims), None, None, None, None)
+        legal = min(B, T, H, W, nh) >= 1 and hd in (64, 128) and B * nh <= 65535 and B * T * H * W < 2 ** 31
+        assert st_ == (-1 if legal else -2)
+    attn()
