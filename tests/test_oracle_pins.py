@@ -356,3 +356,23 @@ def test_range_delta_and_apply_closed_form():
     assert np.all(np.abs(got - exact) <= 0.5 * ulp)
     # a zero delta is the identity
     assert np.array_equal(O.range_apply(other, np.zeros(4096)), other)
+
+
+def test_bf16_rounding_is_one_rounding_of_the_double():
+    """Random doubles across the normal bf16 range, plus exact ties and values one float64
+    ulp either side of a tie (where rounding first to float32 would go wrong): the oracle's
+    rounding equals round-half-even applied once to the float64 bit pattern."""
+    rng = np.random.default_rng(14)
+    mant = rng.integers(0, 2 ** 52, 20000, dtype=np.uint64)
+    expo = rng.integers(1023 - 120, 1023 + 120, 20000, dtype=np.uint64)
+    sign = rng.integers(0, 2, 20000, dtype=np.uint64)
+    bits = (sign << np.uint64(63)) | (expo << np.uint64(52)) | mant
+    # ties: 7 kept fraction bits, then exactly half an ulp; and the neighbours of each tie
+    tie = (bits & ~np.uint64((1 << 45) - 1)) | np.uint64(1 << 44)
+    v = np.concatenate([bits.view(np.float64), tie.view(np.float64), (tie + np.uint64(1)).view(np.float64),
+                        (tie - np.uint64(1)).view(np.float64)])
+    u = v.view(np.uint64)
+    lsb = (u >> np.uint64(45)) & np.uint64(1)
+    r = (u + np.uint64((1 << 44) - 1) + lsb) & ~np.uint64((1 << 45) - 1)
+    want = (r.view(np.float64).astype(np.float32).view(np.uint32) >> np.uint32(16)).astype(np.uint16)
+    assert np.array_equal(O.bf16_round(v), want)
