@@ -36,6 +36,7 @@ MUTANTS = [
     ("bf16_ties_away", "step", "r = std::nearbyint(std::ldexp(a, -q));", "r = std::round(std::ldexp(a, -q));"),
     ("bf16_seven_bits", "step", "int q = e - 8;", "int q = e - 7;"),
     ("bf16_no_subnormals", "step", "if (q < -133) q = -133;", "if (q < -126) q = -126;"),
+    ("bf16_rounds_via_float", "step", "double a = std::fabs(v);", "double a = std::fabs((double)(float)v);"),
     # quantizer
     ("quant_scale_128", "step", "const float scale = absmax / 127.0f;", "const float scale = absmax / 128.0f;"),
     ("quant_truncates", "step", "float t = std::nearbyint(row[c] / scale);", "float t = std::trunc(row[c] / scale);"),
