@@ -115,6 +115,23 @@ int main(void) {
   EXPECT(h3b_range_apply(NULL, NULL, 0, NULL) == H3B_OK);
   EXPECT(h3b_range_apply(NULL, NULL, 4, NULL) == H3B_ERR_SHAPE);
 
+  /* the bounded-wait test hook checks its arguments on the host */
+  {
+    int waited = -1;
+    EXPECT(h3b_test_bounded_wait(10ull, &waited) == H3B_ERR_ARG);
+    EXPECT(h3b_test_bounded_wait(1000000ull, NULL) == H3B_ERR_ARG);
+    EXPECT(waited == -1);
+  }
+
+  /* the profiler's host side: nothing recorded yet */
+  {
+    h3b_kernel_time kt[4];
+    EXPECT(h3b_profile_enable(1) == H3B_OK);
+    EXPECT(h3b_profile_enable(0) == H3B_OK);
+    EXPECT(h3b_profile_read(kt, 4) == 0);
+    EXPECT(h3b_profile_read(NULL, 4) < 0);
+  }
+
   printf("%s\n", failures ? "FAILED" : "OK");
   return failures ? 1 : 0;
 }
