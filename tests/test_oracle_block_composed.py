@@ -216,3 +216,22 @@ def test_composition_helpers_against_known_values():
     r = rope(x, WL)
     assert np.array_equal(r[0], x[0])
     assert np.allclose(np.hypot(r[:, 0::2], r[:, 1::2]), np.hypot(x[:, 0::2], x[:, 1::2]), rtol=1e-12)
+
+
+def test_composition_holds_on_random_small_grids():
+    """The same comparison over random small grids, head shapes, RoPE splits and batch
+    sizes, including one-frame, one-row and one-column grids."""
+    from hypothesis import HealthCheck, given, settings
+    from hypothesis import strategies as st
+
+    @settings(max_examples=12, deadline=None, suppress_health_check=list(HealthCheck))
+    @given(T=st.integers(1, 3), H=st.integers(1, 4), W=st.integers(1, 5), B=st.integers(1, 2),
+           head=st.sampled_from([(4, 64, (16, 24, 24)), (2, 128, (32, 48, 48)), (4, 64, (0, 32, 32)),
+                                 (2, 128, (64, 0, 64))]),
+           qkv_int8=st.booleans(), wo_bf16=st.booleans())
+    def check(T, H, W, B, head, qkv_int8, wo_bf16):
+        nh, dh, rope = head
+        wl = synth.WORKLOADS["d256_L512"].with_(T=T, H=H, W=W, B=B, n_heads=nh, head_dim=dh, rope=rope,
+                                                 qkv_int8=qkv_int8, wo_bf16=wo_bf16)
+        _check(wl)
+    check()
