@@ -22,7 +22,11 @@ Prints one JSON line (rank 0). Under torchrun each rank runs its own
 independent latent (replicas; no data-path collective): the value is the
 total tokens/s of all ranks over the slowest rank's device time.
 
+The default workload is the largest single block: d=5120, 40 heads x 128,
+MLP 20480, an 8x48x48 latent grid (18432 tokens).
+
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl h3b|reference]
+  python bench.py --oracle-table   (host timings of the CPU oracle only)
 """
 import argparse
 import json
@@ -46,7 +50,7 @@ from video_diffusion_transformer_adaln_b200.runtime import (DeviceBlock, bf16_fr
 
 METRIC = "DiT block tokens/s (int8 MLP+QKV, bf16 attn); % of B200 INT8/BF16/HBM roofline"
 UNIT = "tokens/s"
-DEFAULT_WORKLOAD = "d2048_L4096"
+DEFAULT_WORKLOAD = "d5120_L18432"
 L2_FLUSH_BYTES = 512 << 20
 E2E_FLUSH_BYTES = 160 << 20  # larger than the 126 MB L2
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -236,20 +240,63 @@ class Workload:
 
 # ----------------------------------------------------------------------------- CPU oracle leg
 
+FULL_BLOCK_OPS = 1.0e12  # blocks up to this many ops are timed whole on the host
+
+
+def step_blocks(wl):
+    """The blocks one bench step runs: ([(tokens per batch item, count)], tokens per step).
+    Paired blocks run on the merged grid (L/2); a residual-reuse step is one fresh pass
+    over every block and one pass that skips the cached range (two denoise steps)."""
+    if wl.token_pair:
+        return [(wl.L // 2, 1)], wl.B * wl.L
+    f, l = wl.pair_blocks
+    if f < l:
+        return [(wl.L // 2, l - f), (wl.L, wl.n_blocks - (l - f))], wl.B * wl.L
+    f, l = wl.reuse_blocks
+    if f < l:
+        return [(wl.L, 2 * wl.n_blocks - (l - f))], 2 * wl.B * wl.L
+    return [(wl.L, wl.n_blocks)], wl.B * wl.L
+
+
+def block_ops(wl, L):
+    """Multiply-add ops x 2 of one block over L tokens per batch item: projections and attention."""
+    return 24.0 * wl.B * L * wl.d * wl.d + 4.0 * wl.B * L * L * wl.d
+
+
 class OracleRunner:
-    """The CPU oracle on a bounded sample of the workload: steps a1-a3 (AdaLN,
-    LN+quantizer, QKV projection with RoPE) for every token, then steps a4-a9
-    for n sampled tokens. The full-block time is extrapolated as
-    t(a1-a3, all tokens) + t(a4-a9 per token) x tokens."""
+    """The CPU oracle, as it stands, timed on the host cores.
+
+    full_block(): one whole block over every token of the workload's grid, timed
+    directly. Used when the step is that one block and it is small enough
+    (FULL_BLOCK_OPS).
+
+    sample(sub_tokens, n_q): a bounded sample for workloads whose block takes
+    minutes on the host. Three pieces of the oracle are timed:
+      t_sub  the whole block over every token of a slice of the grid (the first
+             frame, its first rows: about sub_tokens tokens), same dimensions and
+             weight distributions;
+      t_ada  the AdaLN Linear alone, a fixed cost per block and batch item;
+      t_att  the attention step for n_q query rows against L keys (seeded Q, K, V).
+    Attention costs c = t_att / (n_q L) per query-key pair; the slice's other work
+    grows linearly with its tokens. One block over L tokens per batch item is then
+        t(L) = B t_ada + (t_sub - B t_ada - c B L_sub^2) L / L_sub + c B L^2
+    and a step is the sum of t over the blocks it runs (step_blocks)."""
 
     def __init__(self, wl):
         import oracle as O  # the CPU oracle: benchmark baseline leg only
 
         self.O = O
-        if wl.n_blocks > 1 or wl.token_pair:
-            wl = wl.with_(n_blocks=1, token_pair=False)
         self.wl = wl
-        raw, self.c, self.x = synth.block_weights(wl), synth.cond(wl), synth.x_input(wl)
+        self.blocks, self.tokens = step_blocks(wl)
+        self.block_wl = wl.merged() if wl.token_pair else wl.with_(n_blocks=1, pair_blocks=(0, 0),
+                                                                   reuse_blocks=(0, 0))
+        self._sub = None
+        self._full = None
+        self._att = None
+
+    def _prepare(self, wl):
+        O = self.O
+        raw, c, x = synth.block_weights(wl), synth.cond(wl), synth.x_input(wl)
         w = {"w_ada": raw["w_ada"], "b_ada": raw["b_ada"]}
         for name, sname in (("wqkv", "sqkv"), ("wo", "so"), ("w1", "s1"), ("w2", "s2")):
             w[name], w[sname] = O.quantize_rows(raw[name])
@@ -257,45 +304,72 @@ class OracleRunner:
             w["wqkv_bf16"] = raw["wqkv_bf16"]
         if wl.wo_bf16:
             w["wo_bf16"] = raw["wo_bf16"]
-        self.w = w
-        self.dm = O.Dims(wl.B, wl.T, wl.H, wl.W, wl.d, wl.n_heads, wl.head_dim, wl.d_ff, wl.rope,
-                         wl.rope_theta, wl.ln_eps, wl.qkv_int8, wl.wo_bf16)
-        self.R = wl.B * wl.L
-        self.t_kv = None
+        dm = O.Dims(wl.B, wl.T, wl.H, wl.W, wl.d, wl.n_heads, wl.head_dim, wl.d_ff, wl.rope,
+                    wl.rope_theta, wl.ln_eps, wl.qkv_int8, wl.wo_bf16)
+        return dm, w, c, x
 
-    def run(self, n_rows):
-        rows = synth.sample_rows(self.R, n_rows) if n_rows else np.zeros(0, np.int64)
+    def can_time_full_block(self):
+        return self.blocks == [(self.wl.L, 1)] and block_ops(self.wl, self.wl.L) <= FULL_BLOCK_OPS
+
+    def full_block(self):
+        """Seconds of one whole block over every token (all rows)."""
+        if self._full is None:
+            self._full = self._prepare(self.block_wl)
+        dm, w, c, x = self._full
         t0 = time.perf_counter()
-        self.O.block_forward(self.dm, self.w, self.c, self.x, rows=rows)
+        self.O.block_forward(dm, w, c, x)
         return time.perf_counter() - t0
 
-    def measure_kv(self, reps=1):
-        """Seconds of a1-a3 over all tokens (the median of `reps` runs)."""
-        self.t_kv = statistics.median(self.run(0) for _ in range(max(1, reps)))
-        return self.t_kv
-
-    def estimate(self, n_rows):
-        """Extrapolated full-block seconds from one sampled run."""
-        if self.t_kv is None:
-            self.measure_kv()
-        t = self.run(n_rows)
-        return self.t_kv + max(t - self.t_kv, 0.0) / n_rows * self.R
-
-    def baseline(self, n_rows, budget_s=30.0):
-        """Median of up to three extrapolations, each against a median a1-a3 time, within
-        about `budget_s` seconds of host work (one of each when a single run is already long)."""
+    def sample(self, sub_tokens, n_q):
+        """Extrapolated seconds of one bench step and the sample's own wall seconds."""
+        bw = self.block_wl
+        if self._sub is None or self._sub[0] != sub_tokens:
+            h = max(1, min(bw.H, sub_tokens // bw.W))
+            self._sub = (sub_tokens, self._prepare(bw.with_(T=1, H=h)), bw.with_(T=1, H=h).L)
+        if self._att is None or self._att[0] != n_q:
+            r = np.random.default_rng(synth.BASE_SEED)
+            kv = [r.standard_normal((bw.L, bw.d)) for _ in range(2)]
+            self._att = (n_q, r.standard_normal((n_q, bw.d)), kv[0], kv[1])
+        _, (dm, w, c, x), L_sub = self._sub
+        _, q, k, v = self._att
+        O, B = self.O, bw.B
         t0 = time.perf_counter()
-        first = self.run(0)
-        reps = 3 if 6 * first < budget_s else 1
-        self.t_kv = statistics.median([first] + [self.run(0) for _ in range(reps - 1)])
-        ests = []
-        while len(ests) < reps and (not ests or time.perf_counter() - t0 < budget_s):
-            ests.append(self.estimate(n_rows))
-        return statistics.median(ests), len(ests)
+        O.adaln_linear(w["w_ada"], w["b_ada"], c[0])
+        t1 = time.perf_counter()
+        O.block_forward(dm, w, c, x)
+        t2 = time.perf_counter()
+        O.attention(q, k, v, bw.n_heads, bw.head_dim)
+        t3 = time.perf_counter()
+        t_ada, t_sub, t_att = t1 - t0, t2 - t1, t3 - t2
+        pair = t_att / (n_q * bw.L)
+        per_token = max(t_sub - B * t_ada - pair * B * L_sub * L_sub, 0.0) / (B * L_sub)
+        step = sum(n * (B * t_ada + per_token * B * L + pair * B * L * L) for L, n in self.blocks)
+        return step, t3 - t0
 
-    def sample_text(self, n_rows):
-        return (f"a1-a3 over all {self.R} tokens + a4-a9 on {n_rows} sampled tokens, "
-                f"extrapolated to {self.R} tokens")
+    def sample_text(self, sub_tokens, n_q):
+        bw = self.block_wl
+        h = max(1, min(bw.H, sub_tokens // bw.W))
+        blocks = " + ".join(f"{n} x {L}-token block" for L, n in self.blocks)
+        return (f"oracle pieces timed: the whole block over a 1x{h}x{bw.W} slice ({h * bw.W} tokens, all rows), "
+                f"the AdaLN Linear, and attention of {n_q} query rows against all {bw.L} keys; extrapolated "
+                f"to the step ({blocks}) as linear-in-tokens work plus attention per query-key pair")
+
+    def full_text(self):
+        return f"the whole block over all {self.tokens} tokens, timed directly (no extrapolation)"
+
+    def baseline(self, budget_s=30.0, sub_tokens=2304, n_q=32):
+        """(tokens/s, description, extrapolated): the median of up to three timings within
+        about budget_s of host work; the first of them also warms the oracle's buffers."""
+        t0 = time.perf_counter()
+        vals = []
+        if self.can_time_full_block():
+            while len(vals) < 3 and (not vals or time.perf_counter() - t0 + vals[-1] < budget_s):
+                vals.append(self.full_block())
+            return self.tokens / statistics.median(vals), self.full_text() + f" (median of {len(vals)})", False
+        while len(vals) < 3 and (not vals or time.perf_counter() - t0 < budget_s):
+            vals.append(self.sample(sub_tokens, n_q)[0])
+        return (self.tokens / statistics.median(vals),
+                self.sample_text(sub_tokens, n_q) + f" (median of {len(vals)})", True)
 
     def threads(self):
         return self.O.threads()
@@ -493,9 +567,9 @@ def run_h3b(args, rank, world, local):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         orc = OracleRunner(wl)
-        est_s, n_est = orc.baseline(args.cpu_rows)
-        cpu = {"value": round(W.tokens / est_s, 2), "unit": UNIT, "cores": orc.threads(),
-               "kind": "oracle", "sample": orc.sample_text(args.cpu_rows) + f" (median of {n_est})"}
+        v, text, extrap = orc.baseline(sub_tokens=args.cpu_sub_tokens, n_q=args.cpu_queries)
+        cpu = {"value": round(v, 2), "unit": UNIT, "cores": orc.threads(), "kind": "oracle", "sample": text,
+               "extrapolated": extrap}
 
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -522,30 +596,85 @@ def run_h3b(args, rank, world, local):
 
 
 def run_reference(args, rank, world, local):
-    """The CPU oracle as the reference arm (rank 0 only)."""
+    """The CPU oracle as the reference arm (rank 0 only). Each step is one bounded
+    timing of the oracle: the whole block when it is small (the step's tokens over
+    its measured seconds), else one OracleRunner.sample whose extrapolated step time
+    gives the value. ms_per_step is always the wall time the steps actually took."""
     if rank != 0:
         return
     wl = synth.WORKLOADS[args.workload]
     orc = OracleRunner(wl)
-    orc.measure_kv()
-    est = []
+    full = orc.can_time_full_block() and block_ops(wl, wl.L) <= args.ref_full_ops
+    walls, ests = [], []
     for i in range(args.warmup + args.steps):
-        e = orc.estimate(args.ref_rows)
+        if full:
+            wall = orc.full_block()
+            est = wall
+        else:
+            est, wall = orc.sample(args.ref_sub_tokens, args.ref_queries)
         if i >= args.warmup:
-            est.append(e)
-    sample, threads = orc.sample_text(args.ref_rows), orc.threads()
-    tokens = wl.B * wl.L
-    ms = 1e3 * sum(est) / len(est)
-    value = tokens / (ms / 1e3)
+            walls.append(wall)
+            ests.append(est)
+    threads = orc.threads()
+    ms = 1e3 * sum(walls) / len(walls)
+    est_ms = 1e3 * sum(ests) / len(ests)
+    value = orc.tokens / (est_ms / 1e3)
+    sample = orc.full_text() if full else orc.sample_text(args.ref_sub_tokens, args.ref_queries)
     line = {"metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms, 2), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64 (int8 decisions in f32)", "data": "synthetic", "impl": "reference",
             "config": {"workload": args.workload, "tokens": wl.L, "d": wl.d, "heads": wl.n_heads,
-                       "head_dim": wl.head_dim, "d_ff": wl.d_ff},
+                       "head_dim": wl.head_dim, "d_ff": wl.d_ff, "blocks_per_step": wl.n_blocks},
+            "extrapolated": not full,
+            "step_ms_extrapolated": None if full else round(est_ms, 1),
+            "step": ("one whole block per step" if full else
+                     "one bounded sample per step (ms_per_step is its wall time); value = the step's tokens over "
+                     "the step time extrapolated from the sample (step_ms_extrapolated)"),
             "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": threads, "kind": "oracle",
-                             "sample": sample},
+                             "sample": sample, "extrapolated": not full},
             "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
+
+
+ORACLE_TABLE = (("d256_L512", (1, None)), ("d2048_L4096", (1, None)), ("d5120_L18432", (None,)))
+
+
+def run_oracle_table(args):
+    """Host timings of the oracle for the baseline table: the whole block at 1 thread and
+    at every core for the small workloads, the bounded sample at every core for the
+    largest single block. Each entry runs in a child process (OMP_NUM_THREADS is read
+    when the oracle library loads) and prints one JSON object."""
+    rows = []
+    for name, thread_opts in ORACLE_TABLE:
+        for th in thread_opts:
+            env = dict(os.environ)
+            if th is not None:
+                env["OMP_NUM_THREADS"] = str(th)
+            else:
+                env.pop("OMP_NUM_THREADS", None)
+            r = subprocess.run([sys.executable, os.path.abspath(__file__), "--oracle-entry", name],
+                               capture_output=True, text=True, env=env, cwd=ROOT)
+            if r.returncode != 0:
+                rows.append({"workload": name, "threads": th, "error": r.stderr[-500:]})
+            else:
+                rows.append(json.loads(r.stdout.strip().splitlines()[-1]))
+            log(json.dumps(rows[-1]))
+    print(json.dumps({"oracle_table": rows, "nproc": os.cpu_count()}), flush=True)
+
+
+def run_oracle_entry(name):
+    wl = synth.WORKLOADS[name]
+    orc = OracleRunner(wl)
+    out = {"workload": name, "threads": orc.threads()}
+    if orc.can_time_full_block():
+        orc.full_block()  # load the library and touch the buffers once
+        t = orc.full_block()
+        out.update(block_s=round(t, 3), tokens_per_s=round(orc.tokens / t, 2), how=orc.full_text())
+    # the bounded sample the benchmark uses for large blocks, beside the whole block where both exist
+    est, wall = orc.sample(2304, 32)
+    out.update(sample_block_s=round(est, 3), sample_tokens_per_s=round(orc.tokens / est, 2),
+               sample_wall_s=round(wall, 2), sample_how=orc.sample_text(2304, 32))
+    print(json.dumps(out), flush=True)
 
 
 _TRAFFIC = None
@@ -583,16 +712,29 @@ def traffic_for(kernel, wl, n_launch):
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=100)
-    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
     ap.add_argument("--impl", default="h3b", choices=["h3b", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-rows", type=int, default=256, help="sampled tokens for the oracle baseline")
-    ap.add_argument("--ref-rows", type=int, default=128,
-                    help="sampled tokens per reference-arm step (fewer rows leave the oracle's row-parallel "
-                         "loops underused and bias the extrapolation upward: 16 rows read 2.4x slow at d=2048)")
+    ap.add_argument("--cpu-sub-tokens", type=int, default=2304,
+                    help="tokens of the grid slice the oracle baseline runs whole (large workloads)")
+    ap.add_argument("--cpu-queries", type=int, default=32, help="query rows of the baseline's attention piece")
+    ap.add_argument("--ref-sub-tokens", type=int, default=384,
+                    help="tokens of the grid slice each reference-arm step runs whole (large workloads)")
+    ap.add_argument("--ref-queries", type=int, default=16, help="query rows of each reference step's attention")
+    ap.add_argument("--ref-full-ops", type=float, default=1.0e11,
+                    help="reference steps run the whole block when it is at most this many ops")
+    ap.add_argument("--oracle-table", action="store_true",
+                    help="print host timings of the oracle (1 thread and all cores) and exit")
+    ap.add_argument("--oracle-entry", help=argparse.SUPPRESS)
     args = ap.parse_args()
+    if args.oracle_entry:
+        run_oracle_entry(args.oracle_entry)
+        return
+    if args.oracle_table:
+        run_oracle_table(args)
+        return
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":

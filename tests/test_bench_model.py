@@ -101,8 +101,7 @@ def _run_bench(args, env_extra=None, timeout=600):
 def test_reference_arm_prints_one_contract_line():
     # The reference arm is the CPU oracle (no GPU needed): one JSON line with the same
     # metric and unit as the CUDA arm, its own cpu_baseline and an e2e with no copies.
-    out = _run_bench(["--impl", "reference", "--workload", "d256_L512", "--steps", "3", "--warmup", "3",
-                      "--ref-rows", "4"])
+    out = _run_bench(["--impl", "reference", "--workload", "d256_L512", "--steps", "3", "--warmup", "3"])
     assert len(out) == 1
     line = out[0]
     assert line["impl"] == "reference"
@@ -113,6 +112,9 @@ def test_reference_arm_prints_one_contract_line():
     assert line["config"]["workload"] == "d256_L512"
     cb = line["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == line["value"] and cb["sample"]
+    # the smallest block runs whole each step: value is its tokens over the step time
+    assert line["extrapolated"] is False
+    assert line["value"] == pytest.approx(512 / (line["ms_per_step"] / 1e3), rel=1e-3)
     assert line["e2e"] == {"value": line["value"], "unit": line["unit"], "h2d_bytes_per_step": 0,
                            "d2h_bytes_per_step": 0}
 
@@ -177,13 +179,42 @@ def test_roofline_summary_of_a_profile():
     assert bench.roofline_summary({}, wl, peaks, "measured") == (None, {}, {})
 
 
-def test_cpu_baseline_estimate_on_the_smallest_block():
+def test_step_blocks_of_every_workload_kind():
+    wl = synth.WORKLOADS["d5120_L18432"]
+    assert bench.step_blocks(wl) == ([(18432, 1)], 18432)
+    assert bench.step_blocks(synth.WORKLOADS["d5120_L18432_pair"]) == ([(9216, 1)], 18432)
+    assert bench.step_blocks(synth.WORKLOADS["d5120_depth50_T16"]) == ([(36864, 50)], 36864)
+    # blocks 13..37 on the merged grid, the other 25 on the full grid
+    assert bench.step_blocks(synth.WORKLOADS["d5120_depth50_T8_pairmid"]) == ([(9216, 25), (18432, 25)], 18432)
+    # a fresh pass over 50 blocks and a reuse pass that skips 25: two denoise steps
+    assert bench.step_blocks(synth.WORKLOADS["d5120_depth50_T8_reuse"]) == ([(18432, 75)], 2 * 18432)
+    assert bench.block_ops(wl, wl.L) == 24 * wl.L * wl.d ** 2 + 4 * wl.L ** 2 * wl.d
+
+
+def test_cpu_baseline_times_the_small_block_whole():
     orc = bench.OracleRunner(synth.WORKLOADS["d256_L512"])
-    est, n = orc.baseline(64, budget_s=30.0)
-    assert n == 3 and est > 0
-    # the extrapolation from 64 of 512 tokens stays within a small factor of a full run
-    import time
-    t0 = time.perf_counter()
-    orc.run(512)
-    full = time.perf_counter() - t0
-    assert 0.2 * full < est < 20 * full
+    assert orc.can_time_full_block()
+    v, text, extrap = orc.baseline(budget_s=30.0)
+    assert v > 0 and not extrap and "no extrapolation" in text
+    assert not bench.OracleRunner(synth.WORKLOADS["d5120_L18432"]).can_time_full_block()
+
+
+def test_cpu_baseline_sample_extrapolates_near_the_whole_block():
+    # the bounded sample (a 1x4x16 slice run whole, plus attention of 16 queries against
+    # all 512 keys) against the whole block's own time, on the smallest block
+    orc = bench.OracleRunner(synth.WORKLOADS["d256_L512"])
+    full = min(orc.full_block() for _ in range(3))
+    est = min(orc.sample(64, 16)[0] for _ in range(3))
+    assert 0.2 * full < est < 5 * full, (est, full)
+    assert "1x4x16 slice" in orc.sample_text(64, 16)
+
+
+def test_reference_arm_sampled_steps_report_their_wall_time():
+    out = _run_bench(["--impl", "reference", "--workload", "d2048_L4096", "--steps", "3", "--warmup", "3",
+                      "--ref-full-ops", "0", "--ref-sub-tokens", "64", "--ref-queries", "4"])
+    line = out[0]
+    assert line["extrapolated"] is True and line["cpu_baseline"]["extrapolated"] is True
+    # value is the step's tokens over the extrapolated step time, which is longer than
+    # the bounded sample each step actually ran
+    assert line["value"] == pytest.approx(4096 / (line["step_ms_extrapolated"] / 1e3), rel=1e-3)
+    assert line["step_ms_extrapolated"] > line["ms_per_step"] > 0
