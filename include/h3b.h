@@ -23,9 +23,13 @@
  *
  * Conventions for every entry point
  *   - All tensor pointers are DEVICE pointers on the current CUDA device, owned
- *     by the caller; the library never allocates device memory for the block and
- *     keeps no state beyond per-device kernel attributes and one device-side
- *     error word (h3b_device_error).
+ *     by the caller; the library never allocates device memory for the block.
+ *     Its only device state is one error word per device (h3b_device_error) and
+ *     the fixed 32 MiB scratch array of h3b_block_forward_noalloc, which every
+ *     GPU that loads the library holds until the process exits. On the host it
+ *     keeps per-device attributes and device addresses, looked up once per
+ *     device index: use one CUDA context per device, and do not call
+ *     cudaDeviceReset between calls (the cached addresses would be stale).
  *   - Every call is asynchronous on `stream` (NULL = legacy default stream).
  *   - bf16 tensors are passed as `void*` (IEEE bfloat16 bit patterns).
  *   - Matrices are row-major. Weights are [out][in] (each output channel's input
@@ -164,9 +168,11 @@ H3B_API h3b_status h3b_block_forward(const h3b_dims* dims, const h3b_block_weigh
  *     H3B_ERR_WORKSPACE before any launch (use h3b_block_forward instead).
  *   - Every GPU that loads this library holds the 32 MiB array until the
  *     process exits.
- *   - The first call on a device looks up the array's device address on that
- *     device (cudaGetSymbolAddress); make that first call before any stream
- *     capture.
+ *   - The first call on a device checks the device (compute capability 10.0,
+ *     else H3B_ERR_ARCH) and looks up the array's device address on it
+ *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *     The address is cached per device index (one context per device; no
+ *     cudaDeviceReset between calls).
  *   - All calls on a device share the array: calls that overlap on the GPU
  *     (different streams or host threads) race on it; serialize them.
  *   - Nothing in the array needs to start at zero; the block's kernels zero

@@ -368,3 +368,52 @@ def test_depth50_pass_properties_d5120_T2():
     assert np.array_equal(a, b_) and np.array_equal(a, cc)
     assert np.isfinite(bf16_f64(a)).all()
     no_device_error()
+
+
+# ----------------------------------------------------------------------------- the 50-block pass's grids
+
+@pytest.mark.parametrize("T,block", [(4, 0), (12, 24), (16, 49)])
+def test_depth_pass_block_at_long_grids_sampled(T, block):
+    """One block of the 50-block pass (d=5120, 40x128 heads, MLP 20480, RoPE (32,48,48)) on
+    the T x 48 x 48 grids of the frame sweep, up to 36864 tokens: attention runs over up to
+    144 key tiles of 256 per query tile and RoPE reaches positions (T-1, 47, 47). The weights
+    and c of the pass's block index and a seeded x are generated on the host, so the oracle
+    sees seeded inputs only; 48 sampled rows (always the first and last token) are compared
+    at the block bar. The oracle projects Q, K and V for every token."""
+    wl = synth.WORKLOADS[f"d5120_depth50_T{T}"].with_(n_blocks=1)
+    raw, c, x = synth.block_weights(wl, block), synth.cond(wl, block), synth.x_input(wl)
+    got, blk = _run_gpu_block(wl, raw, c, x)
+    ow = _weights_agree(raw, blk)
+    del blk
+    torch.cuda.empty_cache()
+    rows = synth.sample_rows(wl.L, 48)
+    ref = O.block_forward(oracle_dims(wl), ow, c, x, rows=rows)
+    _compare(got, ref, x, rows)
+    no_device_error()
+
+
+def test_blocks_forward_three_blocks_d5120_T2():
+    """The pass's chaining at its real width: blocks 0, 1, 2 of the d=5120 pass on the 2x48x48
+    grid (4608 tokens) through h3b_blocks_forward, against the oracle chaining the same blocks
+    (full rows for blocks 0 and 1, since the next block's keys need every token; 64 sampled
+    rows of block 2). Between blocks the oracle's stream is bf16, as the library's is."""
+    wl = synth.WORKLOADS["d5120_depth50_T2"].with_(n_blocks=3)
+    x = synth.x_input(wl)
+    raws = [synth.block_weights(wl, b) for b in range(3)]
+    cs = np.stack([synth.cond(wl, b) for b in range(3)])
+    dims = dims_of(wl)
+    blocks = [DeviceBlock.from_host(r) for r in raws]
+    ows = [_weights_agree(r, b) for r, b in zip(raws, blocks)]
+    xd = bf16_dev(x)
+    blocks_forward(dims, blocks, to_dev(cs), xd, workspace(dims))
+    torch.cuda.synchronize()
+    got = bf16_host(xd)
+    del blocks
+    torch.cuda.empty_cache()
+    xr = x
+    for b in range(2):
+        xr = O.bf16_round(O.block_forward(oracle_dims(wl), ows[b], cs[b], xr)).reshape(x.shape)
+    rows = synth.sample_rows(wl.L, 64)
+    ref = O.block_forward(oracle_dims(wl), ows[2], cs[2], xr, rows=rows)
+    _compare(got, ref, x, rows, n_blocks=3)
+    no_device_error()

@@ -318,14 +318,48 @@ def test_qkv_projection_rope_head_major(name, B, qkv_int8):
     no_device_error()
 
 
+@pytest.mark.parametrize("T,qkv_int8", [(8, True), (16, True), (8, False)])
+def test_qkv_projection_rope_full_video_grids(T, qkv_int8):
+    """QKV + 3D RoPE on the full T x 48 x 48 grids of the d=5120 workloads (18432 and 36864
+    tokens), head_dim 128 with the (32, 48, 48) split, so every position up to (T-1, 47, 47)
+    is rotated and written head-major. The width is 512 (4 heads) to keep the oracle's GEMM
+    short: positions and the split, not the width, decide the rotation. All rows compared."""
+    wl = synth.WORKLOADS["d5120_L18432"].with_(T=T, d=512, n_heads=4, d_ff=2048, qkv_int8=qkv_int8)
+    raw = synth.block_weights(wl)
+    r = _rng(31 + T)
+    R, d = wl.B * wl.L, wl.d
+    dims = dims_of(wl)
+    qkv = torch.empty(3 * R * d, dtype=torch.bfloat16, device="cuda")
+    rope_ws = torch.empty(h3b.h3b_rope_table_bytes(dims), dtype=torch.uint8, device="cuda")
+    blk = DeviceBlock.from_host(raw, qkv_int8=qkv_int8)
+    if qkv_int8:
+        qa, sa = O.quantize_rows((r.standard_normal((R, d)) * 2).astype(np.float32))
+        h3b.h3b_qkv_projection(dims, to_dev(qa), to_dev(sa), blk.struct, qkv, rope_ws)
+        ref = _qkv_reference(wl, qa, sa, raw)
+    else:
+        a = synth.f32_to_bf16_bits((r.standard_normal((R, d)) * 2).astype(np.float32))
+        h3b.h3b_qkv_projection(dims, bf16_dev(a), None, blk.struct, qkv, rope_ws)
+        ref = _qkv_reference(wl, a, None, raw)
+    got = _head_major_to_token_major(qkv, wl)
+    assert np.max(np.abs(got - ref)) <= 2 ** -8 * np.max(np.abs(ref)) * 2
+    assert rel_l2(got, ref) < 4e-3
+    # per token: the last token (position (T-1, 47, 47)) and the first agree as closely
+    for row in (0, R - 1):
+        assert rel_l2(got[row], ref[row]) < 8e-3
+    no_device_error()
+
+
 # ----------------------------------------------------------------------------- attention
 
 @pytest.mark.parametrize("B,H,L,dh,n_q", [(1, 4, 512, 64, 512), (1, 2, 200, 128, 200), (2, 2, 777, 128, 128),
-                                          (1, 16, 4096, 128, 96), (1, 1, 128, 64, 128), (1, 1, 1, 128, 1)])
+                                          (1, 16, 4096, 128, 96), (1, 1, 128, 64, 128), (1, 1, 1, 128, 1),
+                                          (1, 40, 36864, 128, 48)])
 def test_attention(B, H, L, dh, n_q):
+    """The last case is the frame sweep's longest grid at its launch shape: 40 heads of 128
+    over 36864 tokens (144 key tiles per query tile)."""
     r = _rng(B * H * L * dh)
     # head-major bf16 Q, K, V with a spread of score magnitudes
-    qkv_bits = synth.f32_to_bf16_bits((r.standard_normal((3, B, H, L, dh)) *
+    qkv_bits = synth.f32_to_bf16_bits((r.standard_normal((3, B, H, L, dh), dtype=np.float32) *
                                        r.uniform(0.3, 2.0, (3, B, H, 1, 1))).astype(np.float32))
     wl = synth.Workload("attn", 1, 1, L, H * dh, H, dh, 256, (0, 0, dh), 0, B=B)
     dims = dims_of(wl)

@@ -336,6 +336,10 @@ h3b_status run_block(const h3b_dims& d, const h3b_block_weights& w, const float*
 // TMA descriptors (driver entry point fetched through the runtime).
 // ---------------------------------------------------------------------------
 void set_error_detail(const std::string& why) { g_detail = why; }
+int check_current_device() {
+  DeviceInfo* di = nullptr;
+  return device_info(&di);
+}
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,

@@ -79,6 +79,9 @@ cudaError_t launch_attention(const AttnArgs& a, cudaStream_t st);
 
 // ---- error detail reported by h3b_last_error_detail (h3b_api.cu)
 void set_error_detail(const std::string& why);
+// ---- H3B_OK when the current device is compute capability 10.0, else the status
+//      (H3B_ERR_ARCH, H3B_ERR_CUDA) the block entry points return (h3b_api.cu)
+int check_current_device();
 // ---- whether h3b_profile_enable(1) is in effect (h3b_api.cu)
 bool profiling_enabled();
 

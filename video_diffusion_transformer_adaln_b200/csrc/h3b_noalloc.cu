@@ -19,7 +19,8 @@
 // host-side stand-in. The device address is taken with cudaGetSymbolAddress,
 // once per device with that device current, on the first call on that device.
 // That first call therefore performs setup work and should happen before any
-// stream capture.
+// stream capture. The address is cached per device index, so it assumes one
+// CUDA context per device and no cudaDeviceReset between calls.
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -77,6 +78,9 @@ extern "C" h3b_status h3b_block_forward_noalloc(const h3b_dims* dims, const h3b_
                           std::to_string(kStaticScratchBytes) + " (use h3b_block_forward with a workspace)");
     return H3B_ERR_WORKSPACE;
   }
+  // The device check comes first: on a device without an sm_100a image the symbol
+  // lookup would fail with a CUDA error instead of the architecture status.
+  if ((s = static_cast<h3b_status>(h3b::check_current_device())) != H3B_OK) return s;
   void* scratch = nullptr;
   if ((s = scratch_address(&scratch)) != H3B_OK) return s;
   return h3b_block_forward(dims, w, c, x, scratch, kStaticScratchBytes, stream);

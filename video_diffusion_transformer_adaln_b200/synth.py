@@ -2,8 +2,9 @@
 
 Both the CUDA path and the CPU oracle are fed from here; this module computes
 nothing the block computes. Random draws use numpy's Philox counter-based
-generator, keyed per (base seed, workload, block, tensor), so any tensor of any
-block can be regenerated on its own.
+generator, keyed per (base seed, workload, block, tensor, row chunk), so any
+tensor of any block can be regenerated on its own, and large tensors are drawn
+by several host threads with the same values for any thread count.
 
 Distributions (model dimensions are synthetic; the pages give none):
   x        ~ N(0, 1), with a fixed set of outlier channels scaled by 16, stored bf16
@@ -101,12 +102,45 @@ _TENSOR_IDS = {"x": 1, "outliers": 2, "c": 3, "w_ada": 4, "b_gate": 5, "wqkv": 6
                "w1": 8, "w2": 9}
 
 
-def _rng(wl: Workload, seed: int, block: int, tensor: str) -> np.random.Generator:
+def _key(wl: Workload, seed: int, block: int, tensor: str) -> list:
     # The stream depends on the grid and model sizes, not on the variant flags, so
     # variants of one workload (bf16 QKV, token pairing) see identical draws.
     key = f"{wl.B}x{wl.T}x{wl.H}x{wl.W}|{wl.d}|{wl.n_heads}x{wl.head_dim}|{wl.d_ff}"
-    ss = np.random.SeedSequence([seed, zlib.crc32(key.encode()), block, _TENSOR_IDS[tensor]])
-    return np.random.Generator(np.random.Philox(ss))
+    return [seed, zlib.crc32(key.encode()), block, _TENSOR_IDS[tensor]]
+
+
+def _rng(wl: Workload, seed: int, block: int, tensor: str) -> np.random.Generator:
+    return np.random.Generator(np.random.Philox(np.random.SeedSequence(_key(wl, seed, block, tensor))))
+
+
+_CHUNK_ELEMS = 1 << 21
+
+
+def _normal(wl: Workload, seed: int, block: int, tensor: str, shape, part: int = 0) -> np.ndarray:
+    """N(0, 1) float32 draws of `shape`, in row chunks of about 2M values. Chunk j comes
+    from its own Philox stream keyed (tensor key, part, j), so the values do not depend
+    on how many host threads fill them; chunks are filled in parallel."""
+    shape = tuple(int(v) for v in shape)
+    cols = shape[-1]
+    rows = int(np.prod(shape[:-1], dtype=np.int64)) if len(shape) > 1 else 1
+    out = np.empty((rows, cols), np.float32)
+    step = max(1, _CHUNK_ELEMS // max(cols, 1))
+    starts = list(range(0, rows, step))
+    base = _key(wl, seed, block, tensor) + [part]
+
+    def fill(j):
+        r0 = starts[j]
+        g = np.random.Generator(np.random.Philox(np.random.SeedSequence(base + [j])))
+        g.standard_normal(out=out[r0:r0 + step], dtype=np.float32)
+
+    if len(starts) == 1:
+        fill(0)
+    else:
+        import os
+        from concurrent.futures import ThreadPoolExecutor
+        with ThreadPoolExecutor(max_workers=min(len(starts), os.cpu_count() or 1)) as ex:
+            list(ex.map(fill, range(len(starts))))
+    return out.reshape(shape)
 
 
 def f32_to_bf16_bits(a: np.ndarray) -> np.ndarray:
@@ -127,7 +161,7 @@ def outlier_channels(wl: Workload, seed: int = BASE_SEED) -> np.ndarray:
 
 def x_input(wl: Workload, seed: int = BASE_SEED) -> np.ndarray:
     """bf16 bits [B, L, d]."""
-    z = _rng(wl, seed, 0, "x").standard_normal((wl.B, wl.L, wl.d), dtype=np.float32)
+    z = _normal(wl, seed, 0, "x", (wl.B, wl.L, wl.d))
     z[..., outlier_channels(wl, seed)] *= np.float32(16.0)
     return f32_to_bf16_bits(z)
 
@@ -141,17 +175,17 @@ def block_weights(wl: Workload, block: int = 0, seed: int = BASE_SEED) -> dict:
     """Unquantized weights of one block: fp32 projections and bf16 AdaLN weights."""
     d, F = wl.d, wl.d_ff
     w_ada = np.zeros((6 * d, d), np.float32)
-    r = _rng(wl, seed, block, "w_ada")
     for k in (0, 1, 3, 4):  # shift/scale chunks; the gate chunks (2, 5) stay zero
-        w_ada[k * d:(k + 1) * d] = r.standard_normal((d, d), dtype=np.float32) * np.float32(1.0 / np.sqrt(d))
+        w_ada[k * d:(k + 1) * d] = _normal(wl, seed, block, "w_ada", (d, d), part=k) * np.float32(1.0 / np.sqrt(d))
     b_ada = np.zeros(6 * d, np.float32)
     g = _rng(wl, seed, block, "b_gate").standard_normal(2 * d, dtype=np.float32) * np.float32(np.sqrt(0.5))
     b_ada[2 * d:3 * d] = g[:d]
     b_ada[5 * d:6 * d] = g[d:]
 
     def lin(name, n_out, n_in):
-        return _rng(wl, seed, block, name).standard_normal((n_out, n_in), dtype=np.float32) * np.float32(
-            1.0 / np.sqrt(n_in))
+        w = _normal(wl, seed, block, name, (n_out, n_in))
+        w *= np.float32(1.0 / np.sqrt(n_in))
+        return w
 
     out = {"w_ada": f32_to_bf16_bits(w_ada), "b_ada": b_ada,
            "wqkv": lin("wqkv", 3 * d, d), "wo": lin("wo", d, d),
