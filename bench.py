@@ -80,10 +80,10 @@ def kernel_work(name, wl):
     bytes they must move (read once + write once). For passes that run some
     blocks on the paired grid, block kernels average over their launches."""
     full = wl.B * wl.L * wl.d
-    if name == "token_pair":
-        return 2.0 * full + 2 * 2.0 * full / 2, "byte", "hbm"
-    if name == "token_unpair":
-        return 2.0 * full + 2 * 2.0 * full / 2 + 2.0 * full, "byte", "hbm"
+    if name == "token_pair":  # read x, write the merged tokens once
+        return 2.0 * full + 2.0 * full / 2, "byte", "hbm"
+    if name == "token_unpair":  # read x and the block's merged output, write x (merged input recomputed)
+        return 2.0 * full + 2.0 * full / 2 + 2.0 * full, "byte", "hbm"
     if wl.token_pair:
         Ls = [wl.L // 2]
     elif wl.pair_blocks[0] < wl.pair_blocks[1]:
@@ -207,8 +207,7 @@ class Workload:
         self.ws = workspace(self.dims)
         if wl.token_pair or wl.pair_blocks[0] < wl.pair_blocks[1]:
             shp = (wl.B, wl.T, wl.H, wl.W // 2, wl.d)
-            self.xm = torch.empty(shp, dtype=torch.bfloat16, device="cuda")
-            self.ym = torch.empty_like(self.xm)
+            self.ym = torch.empty(shp, dtype=torch.bfloat16, device="cuda")
         self.reuse = wl.reuse_blocks[0] < wl.reuse_blocks[1]
         if self.reuse:
             self.x_save = torch.empty_like(self.x)
@@ -221,9 +220,9 @@ class Workload:
         c = self.c if c is None else c
         wl = self.wl
         if wl.token_pair:
-            h3b.h3b_token_pair(self.full, x, self.xm, self.ym)
+            h3b.h3b_token_pair(self.full, x, self.ym)
             h3b.h3b_block_forward(self.dims, self.blocks[0].struct, c, self.ym, self.ws)
-            h3b.h3b_token_unpair(self.full, x, self.xm, self.ym, x)
+            h3b.h3b_token_unpair(self.full, x, None, self.ym, x)
         elif self.reuse:
             structs = [b.struct for b in self.blocks]
             f, l = wl.reuse_blocks
@@ -231,7 +230,7 @@ class Workload:
             h3b.h3b_blocks_forward_cached(self.dims, structs, f, l, False, c, x, None, self.delta, self.ws)
         elif wl.n_blocks > 1 and wl.pair_blocks[0] < wl.pair_blocks[1]:
             h3b.h3b_blocks_forward_reduced(self.full, [b.struct for b in self.blocks], wl.pair_blocks[0],
-                                           wl.pair_blocks[1], c, x, self.xm, self.ym, self.ws)
+                                           wl.pair_blocks[1], c, x, None, self.ym, self.ws)
         elif wl.n_blocks > 1:
             h3b.h3b_blocks_forward(self.dims, [b.struct for b in self.blocks], c, x, self.ws)
         else:

@@ -193,12 +193,13 @@ H3B_API h3b_status h3b_blocks_forward(const h3b_dims* dims, const h3b_block_weig
  * "속도 및 품질 트레이드오프": horizontally adjacent video tokens are paired in
  * the middle blocks).
  * Blocks [0, first) run on the full grid `full`; then the tokens are paired
- * once (h3b_token_pair into xm and ym), blocks [first, last) run on the merged
- * grid (W/2, in place on ym), the block deltas are added back at both
- * positions once (h3b_token_unpair into x), and blocks [last, n_blocks) run on
- * the full grid again.
+ * once (h3b_token_pair into ym), blocks [first, last) run on the merged grid
+ * (W/2, in place on ym), the block deltas are added back at both positions
+ * once (h3b_token_unpair into x, which recomputes the merged input from x),
+ * and blocks [last, n_blocks) run on the full grid again.
  *   0 <= first <= last <= n_blocks; full->W even when first < last.
- *   xm, ym: bf16 [B][T][H][W/2][d] device buffers (unused when first == last).
+ *   ym: bf16 [B][T][H][W/2][d] device buffer (unused when first == last).
+ *   xm: not used (kept for the argument order); may be NULL.
  *   ws: at least h3b_workspace_size(full) bytes (that covers the merged grid).
  *   w, c: as for h3b_blocks_forward. */
 H3B_API h3b_status h3b_blocks_forward_reduced(const h3b_dims* full, const h3b_block_weights* w, int n_blocks,
@@ -265,7 +266,9 @@ H3B_API h3b_status h3b_token_pair(const h3b_dims* full, const void* x, void* xm,
 
 /* out[t,h,2k+j] = bf16(x[t,h,2k+j] + (ym[t,h,k] - xm[t,h,k])), j in {0,1}:
  * the block's delta on each merged token is added at both of its positions of
- * the unmerged residual. out may alias x. */
+ * the unmerged residual. out may alias x. xm may be NULL: the merged input is
+ * then recomputed from x by the rule of h3b_token_pair (the same bits), which
+ * saves reading it. */
 H3B_API h3b_status h3b_token_unpair(const h3b_dims* full, const void* x, const void* xm, const void* ym,
                             void* out, h3b_stream stream);
 

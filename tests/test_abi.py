@@ -108,8 +108,12 @@ def test_multi_block_entry_points_check_every_block_on_the_host(L):
     # reduced pass: range, pairing shape and buffers
     assert L.h3b_blocks_forward_reduced(C.byref(d), blocks, 3, 1, 2, c, x, xm, ym, ws, need, None) == -1
     assert L.h3b_blocks_forward_reduced(C.byref(d), blocks, 3, 2, 1, c, x, xm, ym, ws, need, None) == -1
+    assert L.h3b_blocks_forward_reduced(C.byref(d), blocks, 3, 1, 2, c, x, xm, None, ws, need, None) == -1
+    assert L.h3b_blocks_forward_reduced(C.byref(d), blocks, 3, 1, 2, c, x, xm, ym + 8, ws, need, None) == -3
+    # xm is not used (the unpairing recomputes the merged input): NULL or unaligned is accepted,
+    # and the call goes on to the per-block weight check
     assert L.h3b_blocks_forward_reduced(C.byref(d), blocks, 3, 1, 2, c, x, None, ym, ws, need, None) == -1
-    assert L.h3b_blocks_forward_reduced(C.byref(d), blocks, 3, 1, 2, c, x, xm + 8, ym, ws, need, None) == -3
+    assert L.h3b_blocks_forward_reduced(C.byref(d), blocks, 3, 1, 2, c, x, xm + 8, ym, ws, need, None) == -1
     odd = _dims(W=15)
     need_odd = h3b.h3b_workspace_size(odd)
     assert L.h3b_blocks_forward_reduced(C.byref(odd), blocks, 3, 1, 2, c, x, xm, ym, ws, need_odd, None) == -2

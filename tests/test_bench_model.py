@@ -8,9 +8,9 @@ Per block over R = B*L tokens, model width d, MLP width F:
   fused LN + modulation + quantizer: read 2d bytes, write d codes, a 4-byte
   scale and a 4-byte zeroed absmax per token; quantizer of a width-n row: read
   2n, write n, read the 4-byte absmax, write the 4-byte scale;
-  token pairing: read 2d per original token, write d/2 tokens' worth (2 bytes
-  each) to each of its two destinations; unpairing: read x (2d) and the merged
-  xm and ym (d each) per original token, write 2d.
+  token pairing: read 2d per original token, write the merged tokens once (d
+  per original token); unpairing: read x (2d) and the block's merged output
+  ym (d) per original token, write 2d (the merged input is recomputed from x).
 
 The reference arm (the CPU oracle) is also run here end to end: it needs no GPU,
 and its JSON line follows the same contract as the CUDA arm's."""
@@ -61,8 +61,8 @@ def test_memory_bound_bytes_per_token(name):
 def test_token_reduction_work():
     wl = synth.WORKLOADS["d5120_L18432_pair"]
     R, d = wl.B * wl.L, wl.d
-    assert work("token_pair", wl) == R * 4 * d
-    assert work("token_unpair", wl) == R * 6 * d
+    assert work("token_pair", wl) == R * 3 * d
+    assert work("token_unpair", wl) == R * 5 * d
     # the block between them runs on the merged grid of L/2 tokens
     assert work("gemm_qkv", wl) == 2 * (R // 2) * 3 * d * d
     assert work("attention", wl) == 4 * wl.B * (wl.L // 2) ** 2 * d

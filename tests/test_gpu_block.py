@@ -160,7 +160,9 @@ def test_token_reduction_d5120_sampled():
     blk = DeviceBlock.from_host(raw)
     full, merged = dims_of(wl), dims_of(wl.merged())
     xd = bf16_dev(x)
-    xm, ym = paired_block_forward(full, merged, blk, to_dev(c), xd, workspace(merged))
+    xm = torch.empty((wl.B, wl.T, wl.H, wl.W // 2, wl.d), dtype=torch.bfloat16, device="cuda")
+    h3b.h3b_token_pair(full, xd, xm)
+    paired_block_forward(full, merged, blk, to_dev(c), xd, workspace(merged))
     got = bf16_host(xd)
     ow = oracle_weights(raw)
     del blk
@@ -316,9 +318,8 @@ def test_blocks_forward_reduced_middle_range_d256():
     blocks = [DeviceBlock.from_host(r) for r in raws]
     xd = bf16_dev(x)
     shape = (wl.B, wl.T, wl.H, wl.W // 2, wl.d)
-    xm = torch.empty(shape, dtype=torch.bfloat16, device="cuda")
-    ym = torch.empty_like(xm)
-    h3b.h3b_blocks_forward_reduced(full, [b.struct for b in blocks], first, last, to_dev(cs), xd, xm, ym,
+    ym = torch.empty(shape, dtype=torch.bfloat16, device="cuda")
+    h3b.h3b_blocks_forward_reduced(full, [b.struct for b in blocks], first, last, to_dev(cs), xd, None, ym,
                                    workspace(full))
     got = bf16_host(xd)
     # the oracle composes the same pass; between blocks the stream is bf16

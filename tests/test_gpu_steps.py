@@ -402,6 +402,14 @@ def test_token_pair_unpair(B, T, H, W, d):
     terms = np.abs(bf16_f64(x)) + np.repeat(np.abs(bf16_f64(ym_bits)) + np.abs(bf16_f64(xo)), 2,
                                                  axis=3)
     assert np.all(np.abs(got - ref) <= 2.0 ** -8 * np.abs(ref) + 2.0 ** -20 * terms)
+    # without xm the merged input is recomputed from x: the same bits
+    out2 = torch.empty_like(xd)
+    h3b.h3b_token_unpair(full, xd, None, bf16_dev(ym_bits), out2)
+    assert torch.equal(out2, out)
+    # in place on x, as the token-reduction pass runs it
+    xd2 = bf16_dev(x)
+    h3b.h3b_token_unpair(full, xd2, None, bf16_dev(ym_bits), xd2)
+    assert torch.equal(xd2, out)
     # identity block: unpair(x, xm, xm) == x exactly
     h3b.h3b_token_unpair(full, xd, xm, xm, out)
     assert np.array_equal(bf16_host(out), x)

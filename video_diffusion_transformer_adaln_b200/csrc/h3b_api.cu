@@ -552,8 +552,9 @@ h3b_status h3b_blocks_forward_reduced(const h3b_dims* full, const h3b_block_weig
   WsLayout lay_merged = lay_full;
   if (reduced) {
     if (full->W % 2 != 0) return fail(H3B_ERR_SHAPE, "W must be even for token pairing");
-    if (!xm || !ym) return fail(H3B_ERR_ARG, "xm and ym must be non-NULL");
-    if (!aligned16(xm) || !aligned16(ym)) return fail(H3B_ERR_ALIGN, "xm/ym not 16-byte aligned");
+    if (!ym) return fail(H3B_ERR_ARG, "ym must be non-NULL");
+    if (!aligned16(ym)) return fail(H3B_ERR_ALIGN, "ym not 16-byte aligned");
+    (void)xm;  // the merged input is recomputed from x by the unpairing
     merged.W = full->W / 2;
     if ((s = check_dims(&merged)) != H3B_OK) return s;
     lay_merged = ws_layout(merged);
@@ -569,11 +570,11 @@ h3b_status h3b_blocks_forward_reduced(const h3b_dims* full, const h3b_block_weig
   for (int i = 0; i < first; ++i)
     if ((s = run_block(*full, w[i], c + i * c_stride, x, wsb, lay_full, i > 0, *di, st)) != H3B_OK) return s;
   if (reduced) {
-    H3B_CK(launch_token_pair(x, xm, ym, lines, full->W, full->d, di->sms, st), "token_pair");
+    H3B_CK(launch_token_pair(x, ym, nullptr, lines, full->W, full->d, di->sms, st), "token_pair");
     for (int i = first; i < last; ++i)
       if ((s = run_block(merged, w[i], c + i * c_stride, ym, wsb, lay_merged, i > first, *di, st)) != H3B_OK)
         return s;
-    H3B_CK(launch_token_unpair(x, xm, ym, x, lines, full->W, full->d, di->sms, st), "token_unpair");
+    H3B_CK(launch_token_unpair(x, nullptr, ym, x, lines, full->W, full->d, di->sms, st), "token_unpair");
   }
   for (int i = last; i < n_blocks; ++i)
     if ((s = run_block(*full, w[i], c + i * c_stride, x, wsb, lay_full, i > last || (!reduced && i > 0), *di, st)) !=
@@ -610,8 +611,9 @@ h3b_status h3b_token_unpair(const h3b_dims* full, const void* x, const void* xm,
                             h3b_stream stream) {
   h3b_status s = check_pair_dims(full);
   if (s != H3B_OK) return s;
-  if (!x || !xm || !ym || !out) return fail(H3B_ERR_ARG, "NULL pointer");
-  if (!aligned16(x) || !aligned16(xm) || !aligned16(ym) || !aligned16(out)) return fail(H3B_ERR_ALIGN, "alignment");
+  if (!x || !ym || !out) return fail(H3B_ERR_ARG, "NULL pointer");
+  if (!aligned16(x) || (xm && !aligned16(xm)) || !aligned16(ym) || !aligned16(out))
+    return fail(H3B_ERR_ALIGN, "alignment");
   DeviceInfo* di = nullptr;
   if ((s = device_info(&di)) != H3B_OK) return s;
   const long long lines = (long long)full->B * full->T * full->H;

@@ -30,6 +30,7 @@ cudaError_t launch_token_pair(const void* x, void* xm, void* xm2, long long line
 cudaError_t launch_range_delta(const void* before, const void* after, float* delta, long long n, int sms,
                                cudaStream_t st);
 cudaError_t launch_range_apply(void* x, const float* delta, long long n, int sms, cudaStream_t st);
+// xm may be nullptr: the merged input is then recomputed from x.
 cudaError_t launch_token_unpair(const void* x, const void* xm, const void* ym, void* out,
                                 long long lines, int W, int d, int sms, cudaStream_t st);
 cudaError_t launch_rope_table(float2* tab, int T, int H, int W, int rt, int rh, int rw,

@@ -167,17 +167,26 @@ __global__ void __launch_bounds__(256) adaln_gemv_kernel(const __nv_bfloat16* __
 
 // ---------------------------------------------------------------------------
 // Fused LayerNorm + modulation + per-row int8 quantization.
-//   y = (x - mean) * rsqrt(var + eps)          (fp32, two-pass variance)
+//   y = (x - mean) * rsqrt(var + eps)          (fp32; mean and variance merged
+//                                               from per-thread partial sums)
 //   h = bf16(y * (1 + scale) + shift)
 //   s = absmax(h) / 127, q = rint(h / s)       (binary32 decision)
 // A row of d = 256 NV channels (32 NV 16-byte vectors) is held in registers by
-// tpr = 32 NV / VPT threads, VPT vectors each; a block holds rpp = blockDim /
-// tpr rows at a time and walks its share of the rows in passes of rpp rows,
-// all of one batch item. The item's (1 + scale, shift) pairs sit in shared
-// memory, loaded when the item changes, laid out [4][vectors] so that a warp's
-// 16-byte reads of one channel pair per vector fall in distinct banks.
-// Reductions: warp shuffles, then one shared slot per warp and a barrier
-// (slots alternate between passes, so no barrier guards their reuse).
+// tpr = 32 NV / VPT threads, VPT vectors each (a row group of tpr / 32 warps);
+// a block holds rpp = blockDim / tpr row groups and walks its share of the rows
+// in passes of rpp rows, all of one batch item. The next pass's vectors are
+// loaded into registers while the current row is processed.
+// Statistics: each thread takes the mean and the centred sum of squares M2 of
+// its own 8 VPT values (two passes over registers), and these (mean, M2) pairs
+// are merged pairwise (Chan, Golub and LeVeque's update for equal counts:
+// mean = (m_a + m_b) / 2, M2 = M2_a + M2_b + (m_b - m_a)^2 n / 2), first across
+// the warp by shuffles, then across the row group's warps through shared
+// memory behind one named barrier of the row group. The symmetric form gives
+// every lane the same bits. The row absmax takes a second such barrier; the
+// absmax of the bf16-rounded h is the rounding of the fp32 absmax, since
+// rounding to nearest is monotone. The item's (1 + scale, shift) pairs sit in
+// shared memory, loaded when the item changes, laid out [4][vectors] so that a
+// warp's 16-byte reads of one channel pair per vector fall in distinct banks.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ float2 bf16x2_to_f2(uint32_t u) { return make_float2(bf16_lo(u), bf16_hi(u)); }
 __device__ __forceinline__ float max3f_row(float a, float b, float c) {
@@ -188,30 +197,29 @@ __device__ __forceinline__ float max3f_row(float a, float b, float c) {
 
 constexpr int kLnMaxWarps = 32;
 
-// 16-byte asynchronous copy global -> shared (L2 only), and the wait for all of
-// this thread's outstanding copies.
-__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src) : "memory");
+// Named barrier `id` over `count` threads (a multiple of 32).
+__device__ __forceinline__ void named_barrier(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
-// Lane-wise max of two bf16 pairs (both non-negative here).
-__device__ __forceinline__ uint32_t bf16x2_max(uint32_t a, uint32_t b) {
-  uint32_t r;
-  asm("max.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
-  return r;
+// Pairwise merge of two (mean, M2) summaries of n values each.
+__device__ __forceinline__ void chan_merge(float& mean, float& m2, float mean_b, float m2_b, float half_n) {
+  const float dlt = mean_b - mean;
+  m2 = (m2 + m2_b) + dlt * dlt * half_n;
+  mean = (mean + mean_b) * 0.5f;
 }
+
+// Largest block the launcher forms for a VPT (a row group of up to 992 threads at VPT 1).
+template <int VPT>
+constexpr int ln_max_threads() { return VPT == 1 ? 1024 : VPT == 2 ? 512 : VPT == 3 ? 320 : 256; }
 
 template <int VPT>
-__global__ void __launch_bounds__(1024, 1) ln_mod_quant_kernel(
+__global__ void __launch_bounds__(ln_max_threads<VPT>(), VPT >= 4 ? 2 : 1) ln_mod_quant_kernel(
     const __nv_bfloat16* __restrict__ x, int rows, int vpr, float eps, const float* __restrict__ shift,
     const float* __restrict__ scale, int rows_per_item, int mod_stride, int8_t* __restrict__ q,
     float* __restrict__ s, __nv_bfloat16* __restrict__ h_out, float* __restrict__ absmax_zero,
     int write_codes) {
   extern __shared__ float4 modp[];  // [4][vpr]: (1+sc[2c], 1+sc[2c+1], sh[2c], sh[2c+1]), c = 4 vec + e
-  // then the staging rows of the next pass: [rpp][vpr] 16-byte vectors, each written and read
-  // back by the same thread (cp.async), so no barrier guards them
   __shared__ float red[2][3][kLnMaxWarps];
   const int tpr = vpr / VPT;
   const int rpp = blockDim.x / tpr;
@@ -219,23 +227,28 @@ __global__ void __launch_bounds__(1024, 1) ln_mod_quant_kernel(
   const int t = threadIdx.x - sub * tpr;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int wpr = tpr >> 5, w0 = sub * wpr;
+  constexpr float kLocalN = 8.0f * VPT;
   const float inv_d = 1.0f / (float)(vpr * 8);
   const int items = (rows + rows_per_item - 1) / rows_per_item;
   const unsigned gpi = (unsigned)((rows_per_item + rpp - 1) / rpp);
   const unsigned total = (unsigned)items * gpi;  // passes; at most rows, so 32 bits suffice
   int cur = -1, par = 0;
   unsigned item = blockIdx.x / gpi, g_in = blockIdx.x % gpi;  // pass = (item, pass within item)
-  uint4* stage = reinterpret_cast<uint4*>(modp + 4 * vpr) + (size_t)sub * vpr;
-  // this thread's vectors of its row in pass (it, gi) -> staging, when that row exists
-  auto prefetch = [&](unsigned gg, unsigned it, unsigned gi) {
-    const int r = (int)gi * rpp + sub, rw = (int)it * rows_per_item + r;
-    if (gg >= total || r >= rows_per_item || rw >= rows) return;
-    const uint4* src = reinterpret_cast<const uint4*>(x) + (size_t)rw * vpr;
-#pragma unroll
-    for (int i = 0; i < VPT; ++i) cp_async16(stage + t + tpr * i, src + t + tpr * i);
+  // row-group barrier: a named barrier per group (ids 1..rpp), or the warp itself
+  auto group_sync = [&]() {
+    if (wpr > 1) named_barrier(1 + sub, tpr);
+    else __syncwarp();
   };
-  prefetch(blockIdx.x, item, g_in);
-  cp_async_commit();
+  // this thread's vectors of its row in pass (it, gi), zero when that row does not exist
+  auto load_row = [&](unsigned gg, unsigned it, unsigned gi, uint4 (&dst)[VPT]) {
+    const int r = (int)gi * rpp + sub, rw = (int)it * rows_per_item + r;
+    const bool ok = gg < total && r < rows_per_item && rw < rows;
+    const uint4* src = reinterpret_cast<const uint4*>(x) + (size_t)(ok ? rw : 0) * vpr;
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) dst[i] = ok ? __ldcs(src + t + tpr * i) : make_uint4(0, 0, 0, 0);
+  };
+  uint4 nxt[VPT];
+  load_row(blockIdx.x, item, g_in, nxt);
   for (unsigned g = blockIdx.x; g < total; g += gridDim.x) {
     if ((int)item != cur) {  // block-uniform
       __syncthreads();
@@ -251,14 +264,18 @@ __global__ void __launch_bounds__(1024, 1) ln_mod_quant_kernel(
     const int r_in = (int)g_in * rpp + sub;
     const int row = (int)item * rows_per_item + r_in;
     const bool valid = r_in < rows_per_item && row < rows;
-    cp_async_wait_all();
     uint4 v[VPT];
 #pragma unroll
-    for (int i = 0; i < VPT; ++i) v[i] = valid ? stage[t + tpr * i] : make_uint4(0, 0, 0, 0);
+    for (int i = 0; i < VPT; ++i) v[i] = nxt[i];
+    // start the next pass's loads
+    unsigned n_in = g_in + gridDim.x;
+    const unsigned n_item = item + n_in / gpi;
+    n_in %= gpi;
+    load_row(g + gridDim.x, n_item, n_in, nxt);
 
     float* rd = red[par][0];
     par ^= 1;
-    // the row in fp32 pairs, converted once
+    // the row in fp32 pairs, converted once; this thread's mean and M2
     float2 f[VPT * 4];
 #pragma unroll
     for (int i = 0; i < VPT; ++i) {
@@ -267,38 +284,47 @@ __global__ void __launch_bounds__(1024, 1) ln_mod_quant_kernel(
       f[4 * i + 2] = bf16x2_to_f2(v[i].z);
       f[4 * i + 3] = bf16x2_to_f2(v[i].w);
     }
-    // the staged vectors are in registers now: start the next pass's loads
-    unsigned n_in = g_in + gridDim.x;
-    const unsigned n_item = item + n_in / gpi;
-    n_in %= gpi;
-    prefetch(g + gridDim.x, n_item, n_in);
-    cp_async_commit();
     float2 acc = f[0];
 #pragma unroll
     for (int e = 1; e < VPT * 4; ++e) acc = __fadd2_rn(acc, f[e]);
-    float r = warp_sum(acc.x + acc.y);
-    if (lane == 0) rd[warp] = r;
-    __syncthreads();
-    r = 0.0f;
-    for (int k = 0; k < wpr; ++k) r += rd[w0 + k];
-    const float mean = r * inv_d;
-    const float2 nmean = make_float2(-mean, -mean);
-
+    const float lmean = (acc.x + acc.y) * (1.0f / kLocalN);
+    const float2 nl2 = make_float2(-lmean, -lmean);
 #pragma unroll
-    for (int e = 0; e < VPT * 4; ++e) f[e] = __fadd2_rn(f[e], nmean);  // x - mean
+    for (int e = 0; e < VPT * 4; ++e) f[e] = __fadd2_rn(f[e], nl2);  // x - local mean
     acc = __fmul2_rn(f[0], f[0]);
 #pragma unroll
     for (int e = 1; e < VPT * 4; ++e) acc = __ffma2_rn(f[e], f[e], acc);
-    r = warp_sum(acc.x + acc.y);
-    if (lane == 0) rd[kLnMaxWarps + warp] = r;
-    __syncthreads();
-    r = 0.0f;
-    for (int k = 0; k < wpr; ++k) r += rd[kLnMaxWarps + w0 + k];
-    const float rstd = 1.0f / sqrtf(r * inv_d + eps);
+    float mean = lmean, m2 = acc.x + acc.y, half_n = 0.5f * kLocalN;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const float mb = __shfl_xor_sync(0xFFFFFFFFu, mean, o), m2b = __shfl_xor_sync(0xFFFFFFFFu, m2, o);
+      chan_merge(mean, m2, mb, m2b, half_n);
+      half_n *= 2.0f;
+    }
+    if (wpr > 1) {
+      if (lane == 0) {
+        rd[warp] = mean;
+        rd[kLnMaxWarps + warp] = m2;
+      }
+      group_sync();
+      mean = rd[w0];
+      m2 = rd[kLnMaxWarps + w0];
+      for (int k = 1; k < wpr; ++k) {  // same order in every thread: identical bits
+        const float mb = rd[w0 + k], m2b = rd[kLnMaxWarps + w0 + k];
+        const float dlt = mb - mean;
+        // merge the first k warps' summary (32 k kLocalN values) with warp k's (32 kLocalN)
+        const float nk = (float)k;
+        m2 = (m2 + m2b) + dlt * dlt * (32.0f * kLocalN * nk / (nk + 1.0f));
+        mean = fmaf(dlt, 1.0f / (nk + 1.0f), mean);
+      }
+    }
+    const float rstd = 1.0f / sqrtf(m2 * inv_d + eps);
     const float2 rstd2 = make_float2(rstd, rstd);
+    const float ct = (lmean - mean) * rstd;  // (x - mean) rstd = (x - lmean) rstd + ct
+    const float2 ct2 = make_float2(ct, ct);
 
-    // h = bf16((x - mean) * rstd * (1 + scale) + shift); |h| max kept as a bf16 pair
-    uint32_t am2 = 0u;
+    // h = bf16((x - mean) * rstd * (1 + scale) + shift); max |h| in fp32 before the rounding
+    float am = 0.0f;
 #pragma unroll
     for (int i = 0; i < VPT; ++i) {
       const int vec = t + tpr * i;
@@ -306,19 +332,21 @@ __global__ void __launch_bounds__(1024, 1) ln_mod_quant_kernel(
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const float4 m = modp[e * vpr + vec];
-        const float2 y = __fmul2_rn(f[4 * i + e], rstd2);
+        const float2 y = __ffma2_rn(f[4 * i + e], rstd2, ct2);
         const float2 h = __ffma2_rn(y, make_float2(m.x, m.y), make_float2(m.z, m.w));
         u[e] = pack_bf16x2(h.x, h.y);
-        am2 = bf16x2_max(am2, u[e] & 0x7FFF7FFFu);
+        am = max3f_row(am, fabsf(h.x), fabsf(h.y));
       }
       v[i] = make_uint4(u[0], u[1], u[2], u[3]);
     }
-    float amax = fmaxf(bf16_lo(am2), bf16_hi(am2));
-    amax = warp_max(amax);
-    if (lane == 0) rd[2 * kLnMaxWarps + warp] = amax;
-    __syncthreads();
-    amax = 0.0f;
-    for (int k = 0; k < wpr; ++k) amax = fmaxf(amax, rd[2 * kLnMaxWarps + w0 + k]);
+    float amax = warp_max(am);
+    if (wpr > 1) {
+      if (lane == 0) rd[2 * kLnMaxWarps + warp] = amax;
+      group_sync();
+      amax = rd[2 * kLnMaxWarps + w0];
+      for (int k = 1; k < wpr; ++k) amax = fmaxf(amax, rd[2 * kLnMaxWarps + w0 + k]);
+    }
+    amax = round_bf16(amax);  // = the max of the rounded |h| (rounding is monotone)
     if (valid) {
       if (h_out) {
         uint4* hr = reinterpret_cast<uint4*>(h_out) + (size_t)row * vpr;
@@ -347,7 +375,6 @@ __global__ void __launch_bounds__(1024, 1) ln_mod_quant_kernel(
     item = n_item;
     g_in = n_in;
   }
-  cp_async_wait_all();
 }
 
 // Per-row quantization with each row's absmax already known: a block covers
@@ -513,28 +540,43 @@ __global__ void token_pair_kernel(const __nv_bfloat16* __restrict__ x, __nv_bflo
   }
 }
 
+// One thread per 16-byte vector of a merged token: it reads both unmerged
+// tokens of the pair and the block's merged output, and writes both positions,
+// so each byte is read and written once. Without xm the merged input is
+// recomputed from the pair by the same rounding token_pair_kernel applies.
 __global__ void token_unpair_kernel(const __nv_bfloat16* __restrict__ x,
                                     const __nv_bfloat16* __restrict__ xm,
                                     const __nv_bfloat16* __restrict__ ym, __nv_bfloat16* out,
-                                    long long n_vec, int W, int dvec) {
-  for (long long o = blockIdx.x * (long long)blockDim.x + threadIdx.x; o < n_vec;
+                                    long long n_out_vec, int Wm, int dvec) {
+  for (long long o = blockIdx.x * (long long)blockDim.x + threadIdx.x; o < n_out_vec;
        o += (long long)gridDim.x * blockDim.x) {
-    const long long tok = o / dvec;
-    const int cv = (int)(o - tok * dvec);
-    const long long line = tok / W;
-    const int w = (int)(tok - line * W);
-    const long long m = (line * (W / 2) + w / 2) * dvec + cv;
-    const uint4 a = __ldcs(reinterpret_cast<const uint4*>(x) + o);
-    const uint4 p = __ldg(reinterpret_cast<const uint4*>(xm) + m);
-    const uint4 y = __ldg(reinterpret_cast<const uint4*>(ym) + m);
-    const uint32_t ua[4] = {a.x, a.y, a.z, a.w}, up[4] = {p.x, p.y, p.z, p.w},
-                   uy[4] = {y.x, y.y, y.z, y.w};
-    uint32_t r[4];
+    const long long rp = o / dvec;
+    const int cv = (int)(o - rp * dvec);
+    const long long line = rp / Wm;
+    const int k = (int)(rp - line * Wm);
+    const long long in0 = ((line * (2LL * Wm) + 2 * k) * dvec + cv);
+    const uint4 a = __ldcs(reinterpret_cast<const uint4*>(x) + in0);
+    const uint4 b = __ldcs(reinterpret_cast<const uint4*>(x) + in0 + dvec);
+    const uint4 y = __ldcs(reinterpret_cast<const uint4*>(ym) + o);
+    const uint32_t ua[4] = {a.x, a.y, a.z, a.w}, ub[4] = {b.x, b.y, b.z, b.w}, uy[4] = {y.x, y.y, y.z, y.w};
+    uint32_t up[4];
+    if (xm) {
+      const uint4 p = __ldcs(reinterpret_cast<const uint4*>(xm) + o);
+      up[0] = p.x; up[1] = p.y; up[2] = p.z; up[3] = p.w;
+    } else {
 #pragma unroll
-    for (int e = 0; e < 4; ++e)
-      r[e] = pack_bf16x2(bf16_lo(ua[e]) + (bf16_lo(uy[e]) - bf16_lo(up[e])),
-                         bf16_hi(ua[e]) + (bf16_hi(uy[e]) - bf16_hi(up[e])));
-    reinterpret_cast<uint4*>(out)[o] = make_uint4(r[0], r[1], r[2], r[3]);
+      for (int e = 0; e < 4; ++e)
+        up[e] = pack_bf16x2((bf16_lo(ua[e]) + bf16_lo(ub[e])) * 0.5f, (bf16_hi(ua[e]) + bf16_hi(ub[e])) * 0.5f);
+    }
+    uint32_t ra[4], rb[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float dl = bf16_lo(uy[e]) - bf16_lo(up[e]), dh = bf16_hi(uy[e]) - bf16_hi(up[e]);
+      ra[e] = pack_bf16x2(bf16_lo(ua[e]) + dl, bf16_hi(ua[e]) + dh);
+      rb[e] = pack_bf16x2(bf16_lo(ub[e]) + dl, bf16_hi(ub[e]) + dh);
+    }
+    reinterpret_cast<uint4*>(out)[in0] = make_uint4(ra[0], ra[1], ra[2], ra[3]);
+    reinterpret_cast<uint4*>(out)[in0 + dvec] = make_uint4(rb[0], rb[1], rb[2], rb[3]);
   }
 }
 
@@ -656,7 +698,8 @@ static cudaError_t ln_dispatch(const void* x, int rows, int nv, float eps, const
   const int tpr = vpr / VPT;
   const int block = tpr * (tpr >= 256 ? 1 : 256 / tpr);
   const int rpp_d = block / tpr;
-  const size_t smem = (size_t)vpr * 4 * sizeof(float4) + (size_t)rpp_d * vpr * sizeof(uint4);
+  const size_t smem = (size_t)vpr * 4 * sizeof(float4);
+  (void)rpp_d;
   auto kern = ln_mod_quant_kernel<VPT>;
   // the attribute belongs to the current device, so it is set on every launch (a host-side call)
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -753,11 +796,11 @@ cudaError_t launch_range_apply(void* x, const float* delta, long long n, int sms
 
 cudaError_t launch_token_unpair(const void* x, const void* xm, const void* ym, void* out,
                                 long long lines, int W, int d, int sms, cudaStream_t st) {
-  const long long n = lines * W * (d / 8);
+  const long long n = lines * (W / 2) * (d / 8);
   if (n == 0) return cudaSuccess;
   token_unpair_kernel<<<grid_for(n, sms), 256, 0, st>>>(
       static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(xm),
-      static_cast<const __nv_bfloat16*>(ym), static_cast<__nv_bfloat16*>(out), n, W, d / 8);
+      static_cast<const __nv_bfloat16*>(ym), static_cast<__nv_bfloat16*>(out), n, W / 2, d / 8);
   return cudaGetLastError();
 }
 

@@ -102,12 +102,13 @@ def blocks_forward(dims: h3b.Dims, blocks: List[DeviceBlock], c: torch.Tensor, x
 
 
 def paired_block_forward(full: h3b.Dims, merged: h3b.Dims, blk: DeviceBlock, c: torch.Tensor, x: torch.Tensor,
-                         ws: torch.Tensor, xm: Optional[torch.Tensor] = None, ym: Optional[torch.Tensor] = None):
-    """Token reduction around one block: pair -> block on the merged grid -> unpair (in place on x)."""
+                         ws: torch.Tensor, ym: Optional[torch.Tensor] = None):
+    """Token reduction around one block: pair -> block on the merged grid -> unpair (in place
+    on x). The pairing writes the merged tokens once, into ym, where the block then runs; the
+    unpairing recomputes the merged input from x. Returns ym (the block's merged output)."""
     shape = (full.B, full.T, full.H, full.W // 2, full.d)
-    xm = xm if xm is not None else torch.empty(shape, dtype=torch.bfloat16, device=x.device)
     ym = ym if ym is not None else torch.empty(shape, dtype=torch.bfloat16, device=x.device)
-    h3b.h3b_token_pair(full, x, xm, ym)
+    h3b.h3b_token_pair(full, x, ym)
     h3b.h3b_block_forward(merged, blk.struct, c, ym, ws)
-    h3b.h3b_token_unpair(full, x, xm, ym, x)
-    return xm, ym
+    h3b.h3b_token_unpair(full, x, None, ym, x)
+    return ym
