@@ -166,12 +166,15 @@ def test_roofline_summary_of_a_profile():
     flops = 4.0 * wl.L ** 2 * wl.d
     assert roof["kernel"] == "attention" and roof["bound"] == "tensor" and roof["unit"] == "TFLOP/s"
     assert roof["achieved"] == pytest.approx(flops / 150e-6 / 1e12, abs=0.01)
-    assert roof["peak"] == 1600.0 and roof["frac"] == pytest.approx(roof["achieved"] / 1600.0, abs=1e-4)
+    # kernels timed inside the steps: the sustained figure, with the burst one beside it
+    assert roof["peak"] == 1400.0 and roof["frac"] == pytest.approx(roof["achieved"] / 1400.0, abs=1e-4)
+    assert roof["peak_burst"] == 1600.0 and roof["frac_burst"] == pytest.approx(roof["achieved"] / 1600.0, abs=1e-4)
     assert roof["launch_ms"] == 0.15 and roof["work_per_launch"] == flops
     # the int8 GEMM against twice the bf16 peak, the LN quantizer against HBM
     ops = 2.0 * wl.L * 3 * wl.d * wl.d
     assert all_roof["gemm_qkv"]["TOP/s"] == pytest.approx(ops / 60e-6 / 1e12, abs=0.05)
-    assert all_roof["gemm_qkv"]["frac"] == pytest.approx(ops / 60e-6 / 1e12 / 3200.0, abs=1e-3)
+    assert all_roof["gemm_qkv"]["frac"] == pytest.approx(ops / 60e-6 / 1e12 / 2800.0, abs=1e-3)
+    assert all_roof["gemm_qkv"]["frac_burst"] == pytest.approx(ops / 60e-6 / 1e12 / 3200.0, abs=1e-3)
     byts = wl.L * (3 * wl.d + 8)
     assert all_roof["ln_mod_quant"]["GB/s"] == pytest.approx(byts / 20e-6 / 1e9, abs=0.05)
     assert all_roof["ln_mod_quant"]["frac"] == pytest.approx(byts / 20e-6 / 1e9 / 6500.0, abs=1e-3)
