@@ -281,8 +281,19 @@ H3B_API h3b_status h3b_quantize_weights(const float* w, int rows, int cols, int8
                                 h3b_stream stream);
 
 /* Reads (and optionally clears) the device error word of the current device.
- * Synchronizes the device. *code == 0 means no bounded wait ran out. */
+ * Synchronizes the device. *code == 0 means no bounded wait ran out. Bits:
+ * 1 << 0..3 a bounded wait ran out (TMA tile, tensor-core commit, epilogue or
+ * softmax, drain after an abort), 1 << 4 bad launch parameters, 1 << 5 the
+ * test wait of h3b_test_bounded_wait, 1 << 6 (checked build only) an index fell
+ * outside its buffer and the access was skipped. */
 H3B_API h3b_status h3b_device_error(unsigned int* code, int clear);
+
+/* 1 when this library is the checked build (libh3b_checked.so): every kernel
+ * tests the global-memory indices it computes against its buffers' extents
+ * before the access, records a miss as 1 << 6 in the device error word and
+ * skips that access. It stands in for a memory checker where none can run;
+ * the normal build (0) compiles the tests out. */
+H3B_API int h3b_checked_build(void);
 
 /* Test hook for failure detection without a GPU fault: one thread on the
  * current device waits, with the bounded wait every pipeline of this library

@@ -658,7 +658,24 @@ h3b_status h3b_device_error(unsigned int* code, int clear) {
   H3B_CK(cudaDeviceSynchronize(), "cudaDeviceSynchronize");
   H3B_CK(cudaMemcpy(code, di->err, sizeof(unsigned), cudaMemcpyDeviceToHost), "read error word");
   if (clear) H3B_CK(cudaMemset(di->err, 0, sizeof(unsigned)), "clear error word");
+#ifdef H3B_CHECKED
+  // the row kernels' bounds word (they take no error-word argument)
+  if (unsigned* bw = rowops_bounds_word()) {
+    unsigned b = 0;
+    H3B_CK(cudaMemcpy(&b, bw, sizeof(unsigned), cudaMemcpyDeviceToHost), "read bounds word");
+    if (clear) H3B_CK(cudaMemset(bw, 0, sizeof(unsigned)), "clear bounds word");
+    *code |= b;
+  }
+#endif
   return *code ? H3B_ERR_DEVICE_CHECK : H3B_OK;
+}
+
+int h3b_checked_build(void) {
+#ifdef H3B_CHECKED
+  return 1;
+#else
+  return 0;
+#endif
 }
 
 // ---- step entry points ------------------------------------------------------

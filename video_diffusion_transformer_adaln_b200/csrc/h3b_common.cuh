@@ -20,7 +20,26 @@ enum : unsigned {
   ERR_WAIT_DRAIN = 1u << 3,     // a drain wait after an abort ran out
   ERR_BAD_LAUNCH = 1u << 4,     // a kernel saw launch parameters it cannot handle
   ERR_WAIT_PROBE = 1u << 5,     // the test hook's wait ran out (h3b_test_bounded_wait)
+  ERR_BOUNDS = 1u << 6,         // checked build: an index fell outside its buffer; the access was skipped
 };
+
+// ----------------------------------------------------------------------------
+// Checked build (compiled with -DH3B_CHECKED): every global-memory access whose
+// index the kernel computes is tested against the extent of its buffer first.
+// An index outside [0, n) ORs ERR_BOUNDS into the given word and the access is
+// skipped, so the kernel neither faults nor writes outside its buffers. In the
+// normal build the test compiles to `true`.
+// ----------------------------------------------------------------------------
+#ifdef H3B_CHECKED
+__device__ __forceinline__ bool index_ok(long long i, long long n, unsigned* word) {
+  if (i >= 0 && i < n) return true;
+  atomicOr(word, ERR_BOUNDS);
+  return false;
+}
+#define H3B_IDX_OK(i, n, word) (::h3b::index_ok((long long)(i), (long long)(n), (word)))
+#else
+#define H3B_IDX_OK(i, n, word) true
+#endif
 
 // Upper bound on any single device-side wait. A healthy wait lasts micro- to
 // milliseconds; this only ends a kernel whose pipeline can no longer progress.

@@ -35,6 +35,8 @@ cudaError_t launch_token_unpair(const void* x, const void* xm, const void* ym, v
                                 long long lines, int W, int d, int sms, cudaStream_t st);
 cudaError_t launch_rope_table(float2* tab, int T, int H, int W, int rt, int rh, int rw,
                               double theta, cudaStream_t st);
+// Device address of the row kernels' bounds word (checked build), or nullptr.
+unsigned* rowops_bounds_word();
 
 // ---- tensor-core GEMM (k_gemm.cu)
 enum GemmEpilogue : int {

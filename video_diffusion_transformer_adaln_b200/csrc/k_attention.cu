@@ -382,13 +382,14 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
           pk[e] = pack_bf16x2(v.x, v.y);
           amax = max3f(amax, fabsf(bf16_lo(pk[e])), fabsf(bf16_hi(pk[e])));
         }
-        if (q < L) {
+        if (q < L && H3B_IDX_OK(((long long)b * L + q) * dm + h * DH + c * 32 + 31, (long long)a.B * L * dm, a.err)) {
           uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
 #pragma unroll
           for (int gg = 0; gg < 4; ++gg) d4[gg] = make_uint4(pk[4 * gg], pk[4 * gg + 1], pk[4 * gg + 2], pk[4 * gg + 3]);
         }
       }
-      if (q < L) atomicMax(reinterpret_cast<unsigned*>(a.absmax) + (size_t)b * L + q, __float_as_uint(amax));
+      if (q < L && H3B_IDX_OK((long long)b * L + q, (long long)a.B * L, a.err))
+        atomicMax(reinterpret_cast<unsigned*>(a.absmax) + (size_t)b * L + q, __float_as_uint(amax));
     } else {
       *abort_flag = 1;
     }

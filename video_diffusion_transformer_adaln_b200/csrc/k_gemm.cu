@@ -105,7 +105,10 @@ __device__ __forceinline__ void prefetch_resid(const GemmArgs& p, int row, int c
   const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.out) + (size_t)row * p.N + col0);
 #pragma unroll
   for (int g = 0; g < kResidVecs; ++g)
-    xp[g] = (row_ok && col0 + 8 * g < p.N) ? src[g] : make_uint4(0, 0, 0, 0);
+    xp[g] = (row_ok && col0 + 8 * g < p.N &&
+             H3B_IDX_OK((long long)row * p.N + col0 + 8 * g + 7, (long long)p.M * p.N, p.err))
+                ? src[g]
+                : make_uint4(0, 0, 0, 0);
 }
 
 // Per-warp column constants of the current tile (the warp's 128 columns):
@@ -176,7 +179,8 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, uint32_t tbase,
         uint4* d4 = reinterpret_cast<uint4*>(static_cast<int32_t*>(p.out) + (size_t)row * p.N + col0);
 #pragma unroll
         for (int g = 0; g < 8; ++g)
-          if (g * 4 < valid) d4[g] = make_uint4(rc[4 * g], rc[4 * g + 1], rc[4 * g + 2], rc[4 * g + 3]);
+          if (g * 4 < valid && H3B_IDX_OK((long long)row * p.N + col0 + 4 * g + 3, (long long)p.M * p.N, p.err))
+            d4[g] = make_uint4(rc[4 * g], rc[4 * g + 1], rc[4 * g + 2], rc[4 * g + 3]);
       } else {
         float v[32];
         if (kInt8) {
@@ -201,8 +205,10 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, uint32_t tbase,
             v[4 * g] += b.x; v[4 * g + 1] += b.y; v[4 * g + 2] += b.z; v[4 * g + 3] += b.w;
           }
         }
+        // checked build: the last element this row's chunk writes lies inside the output
+        const bool out_ok = H3B_IDX_OK((long long)row * p.N + col0 + valid - 1, (long long)p.M * p.N, p.err);
         if (kEpi == EPI_DEQ) {
-          store_bf16x32(static_cast<__nv_bfloat16*>(p.out) + (size_t)row * p.N + col0, v, valid);
+          if (out_ok) store_bf16x32(static_cast<__nv_bfloat16*>(p.out) + (size_t)row * p.N + col0, v, valid);
         } else if (kEpi == EPI_GELU) {
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
@@ -211,7 +217,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, uint32_t tbase,
             v[e + 1] = round_bf16(gv.y);
             amax = fmaxf(amax, fmaxf(fabsf(v[e]), fabsf(v[e + 1])));
           }
-          store_bf16x32(static_cast<__nv_bfloat16*>(p.out) + (size_t)row * p.N + col0, v, valid);
+          if (out_ok) store_bf16x32(static_cast<__nv_bfloat16*>(p.out) + (size_t)row * p.N + col0, v, valid);
         } else if (kEpi == EPI_RESID) {
           __nv_bfloat16* xdst = static_cast<__nv_bfloat16*>(p.out) + (size_t)row * p.N + col0;
           const float* gsrc = gate_uniform ? &ec.gate[i * 32] : p.gate + (size_t)item * p.gate_stride + col0;
@@ -235,7 +241,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, uint32_t tbase,
               v[8 * g + 2 * e + 1] = fmaf(gg[2 * e + 1], v[8 * g + 2 * e + 1], bf16_hi(xu[e]));
             }
           }
-          store_bf16x32(xdst, v, valid);
+          if (out_ok) store_bf16x32(xdst, v, valid);
         } else if (kEpi == EPI_QKV) {
           const int part = col0 / p.d;
           const int rem = col0 - part * p.d;
@@ -255,9 +261,9 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, uint32_t tbase,
               v[2 * e + 1] = x0 * cs.y + x1 * cs.x;
             }
           }
-          __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.out) +
-                               ((((size_t)part * p.B + item) * p.n_heads + head) * p.L + l) * p.head_dim + lane0;
-          store_bf16x32(dst, v, 32);
+          const size_t off = ((((size_t)part * p.B + item) * p.n_heads + head) * p.L + l) * p.head_dim + lane0;
+          if (H3B_IDX_OK((long long)off + 31, (long long)p.M * p.N, p.err))
+            store_bf16x32(static_cast<__nv_bfloat16*>(p.out) + off, v, 32);
         }
       }
     }

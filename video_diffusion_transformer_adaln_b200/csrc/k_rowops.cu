@@ -22,6 +22,10 @@
 
 namespace h3b {
 
+// Bounds word of this file's kernels in the checked build (H3B_IDX_OK); the host
+// reads it together with the device error word.
+__device__ unsigned g_h3b_rowops_bounds;
+
 // ---------------------------------------------------------------------------
 // Warp / block reductions
 // ---------------------------------------------------------------------------
@@ -160,7 +164,8 @@ __global__ void __launch_bounds__(256) adaln_gemv_kernel(const __nv_bfloat16* __
     for (int b = 0; b < kGemvMaxB; ++b) {
       if (b >= B) break;
       const float r = warp_sum(acc[b]);
-      if (lane == 0) mod[(size_t)b * 6 * d + j] = r + (bias ? bias[j] : 0.0f);
+      if (lane == 0 && H3B_IDX_OK((long long)b * 6 * d + j, (long long)B * 6 * d, &g_h3b_rowops_bounds))
+        mod[(size_t)b * 6 * d + j] = r + (bias ? bias[j] : 0.0f);
     }
   }
 }
@@ -245,7 +250,10 @@ __global__ void __launch_bounds__(ln_max_threads<VPT>(), VPT >= 4 ? 2 : 1) ln_mo
     const bool ok = gg < total && r < rows_per_item && rw < rows;
     const uint4* src = reinterpret_cast<const uint4*>(x) + (size_t)(ok ? rw : 0) * vpr;
 #pragma unroll
-    for (int i = 0; i < VPT; ++i) dst[i] = ok ? __ldcs(src + t + tpr * i) : make_uint4(0, 0, 0, 0);
+    for (int i = 0; i < VPT; ++i)
+      dst[i] = ok && H3B_IDX_OK((long long)rw * vpr + t + tpr * i, (long long)rows * vpr, &g_h3b_rowops_bounds)
+                   ? __ldcs(src + t + tpr * i)
+                   : make_uint4(0, 0, 0, 0);
   };
   uint4 nxt[VPT];
   load_row(blockIdx.x, item, g_in, nxt);
@@ -351,13 +359,15 @@ __global__ void __launch_bounds__(ln_max_threads<VPT>(), VPT >= 4 ? 2 : 1) ln_mo
       if (h_out) {
         uint4* hr = reinterpret_cast<uint4*>(h_out) + (size_t)row * vpr;
 #pragma unroll
-        for (int i = 0; i < VPT; ++i) hr[t + tpr * i] = v[i];
+        for (int i = 0; i < VPT; ++i)
+          if (H3B_IDX_OK((long long)row * vpr + t + tpr * i, (long long)rows * vpr, &g_h3b_rowops_bounds))
+            hr[t + tpr * i] = v[i];
       }
-      if (absmax_zero && t == 0) absmax_zero[row] = 0.0f;
+      if (absmax_zero && t == 0 && H3B_IDX_OK(row, rows, &g_h3b_rowops_bounds)) absmax_zero[row] = 0.0f;
       if (write_codes) {
         const float sc = __fdiv_rn(amax, 127.0f);
         const float rcp = __frcp_rn(sc);
-        if (t == 0) s[row] = sc;
+        if (t == 0 && H3B_IDX_OK(row, rows, &g_h3b_rowops_bounds)) s[row] = sc;
         uint2* qr = reinterpret_cast<uint2*>(q) + (size_t)row * vpr;
 #pragma unroll
         for (int i = 0; i < VPT; ++i) {
@@ -368,7 +378,8 @@ __global__ void __launch_bounds__(ln_max_threads<VPT>(), VPT >= 4 ? 2 : 1) ln_mo
             code = quant8_fast(v[i], rcp, worst);
           }
           if (worst > kTieGuard) code = quant8_exact(v[i], sc, amax);  // near-tie, zero or subnormal scale
-          qr[t + tpr * i] = code;
+          if (H3B_IDX_OK((long long)row * vpr + t + tpr * i, (long long)rows * vpr, &g_h3b_rowops_bounds))
+            qr[t + tpr * i] = code;
         }
       }
     }
@@ -378,10 +389,12 @@ __global__ void __launch_bounds__(ln_max_threads<VPT>(), VPT >= 4 ? 2 : 1) ln_mo
 }
 
 // Per-row quantization with each row's absmax already known: a block covers
-// whole rows (rpb rows of vpr 16-byte vectors, rpb * vpr <= 4096 unless one row is longer,
-// rpb <= 32),
-// each thread keeps up to four vectors in flight; each row's scale and its
-// reciprocal are derived once, into shared memory.
+// whole rows (rpb rows of vpr 16-byte vectors, rpb * vpr <= 4096 unless one row
+// is longer, rpb <= 32). Each thread walks the block's vectors in rounds of
+// four, with the next round's loads issued before the current round is
+// quantized (the first round's before the scales are derived), so eight
+// vectors per thread are in flight. Each row's scale and its reciprocal are
+// derived once, into shared memory.
 constexpr int kQuantMaxRowsPerBlock = 32;
 __global__ void __launch_bounds__(256) quant_rows_known_absmax_kernel(const __nv_bfloat16* __restrict__ in,
                                                                       int rows, int vpr, int rpb,
@@ -393,25 +406,35 @@ __global__ void __launch_bounds__(256) quant_rows_known_absmax_kernel(const __nv
   __shared__ float samax[kQuantMaxRowsPerBlock];
   const unsigned row0 = blockIdx.x * (unsigned)rpb;
   const unsigned nr = min((unsigned)rpb, (unsigned)rows - row0);
+  const unsigned span = nr * (unsigned)vpr;  // vectors covered by this block
+  const size_t base = (size_t)row0 * vpr;
+  const uint4* src = reinterpret_cast<const uint4*>(in) + base;
+  uint4 nxt[U];
+  auto load_round = [&](unsigned k0) {
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const unsigned k = k0 + u * blockDim.x;
+      nxt[u] = k < span && H3B_IDX_OK(base + k, (long long)rows * vpr, &g_h3b_rowops_bounds)
+                   ? __ldcs(src + k)
+                   : make_uint4(0, 0, 0, 0);
+    }
+  };
+  load_round(threadIdx.x);
   if (threadIdx.x < nr) {
     const float amax = __ldg(absmax_in + row0 + threadIdx.x);
     const float sc = __fdiv_rn(amax, 127.0f);
     srow[threadIdx.x] = make_float2(sc, __frcp_rn(sc));
     samax[threadIdx.x] = amax;
-    s[row0 + threadIdx.x] = sc;
+    if (H3B_IDX_OK(row0 + threadIdx.x, rows, &g_h3b_rowops_bounds)) s[row0 + threadIdx.x] = sc;
   }
-  const unsigned span = nr * (unsigned)vpr;  // vectors covered by this block
-  const size_t base = (size_t)row0 * vpr;
   __syncthreads();
   // row of vector k, advanced incrementally (k only grows): r = k / vpr without a division
   unsigned r = 0, row_end = (unsigned)vpr;
   for (unsigned k0 = threadIdx.x; k0 < span; k0 += U * blockDim.x) {
     uint4 raw[U];
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const unsigned k = k0 + u * blockDim.x;
-      if (k < span) raw[u] = __ldcs(reinterpret_cast<const uint4*>(in) + base + k);
-    }
+    for (int u = 0; u < U; ++u) raw[u] = nxt[u];
+    load_round(k0 + U * blockDim.x);
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const unsigned k = k0 + u * blockDim.x;
@@ -428,7 +451,8 @@ __global__ void __launch_bounds__(256) quant_rows_known_absmax_kernel(const __nv
         code = quant8_fast(raw[u], sr.y, worst);
       }
       if (worst > kTieGuard) code = quant8_exact(raw[u], sr.x, samax[r]);  // near-tie, zero or subnormal scale
-      reinterpret_cast<uint2*>(q)[base + k] = code;
+      if (H3B_IDX_OK(base + k, (long long)rows * vpr, &g_h3b_rowops_bounds))
+        reinterpret_cast<uint2*>(q)[base + k] = code;
     }
   }
 }
@@ -526,6 +550,7 @@ __global__ void token_pair_kernel(const __nv_bfloat16* __restrict__ x, __nv_bflo
     const long long line = rp / Wm;
     const int k = (int)(rp - line * Wm);
     const long long in0 = ((line * (2LL * Wm) + 2 * k) * dvec + cv);
+    if (!H3B_IDX_OK(in0 + dvec, 2 * n_out_vec, &g_h3b_rowops_bounds)) continue;
     const uint4 a = __ldcs(reinterpret_cast<const uint4*>(x) + in0);
     const uint4 b = __ldcs(reinterpret_cast<const uint4*>(x) + in0 + dvec);
     const uint32_t ua[4] = {a.x, a.y, a.z, a.w}, ub[4] = {b.x, b.y, b.z, b.w};
@@ -555,6 +580,7 @@ __global__ void token_unpair_kernel(const __nv_bfloat16* __restrict__ x,
     const long long line = rp / Wm;
     const int k = (int)(rp - line * Wm);
     const long long in0 = ((line * (2LL * Wm) + 2 * k) * dvec + cv);
+    if (!H3B_IDX_OK(in0 + dvec, 2 * n_out_vec, &g_h3b_rowops_bounds)) continue;
     const uint4 a = __ldcs(reinterpret_cast<const uint4*>(x) + in0);
     const uint4 b = __ldcs(reinterpret_cast<const uint4*>(x) + in0 + dvec);
     const uint4 y = __ldcs(reinterpret_cast<const uint4*>(ym) + o);
@@ -802,6 +828,11 @@ cudaError_t launch_token_unpair(const void* x, const void* xm, const void* ym, v
       static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(xm),
       static_cast<const __nv_bfloat16*>(ym), static_cast<__nv_bfloat16*>(out), n, W / 2, d / 8);
   return cudaGetLastError();
+}
+
+unsigned* rowops_bounds_word() {
+  void* p = nullptr;
+  return cudaGetSymbolAddress(&p, g_h3b_rowops_bounds) == cudaSuccess ? static_cast<unsigned*>(p) : nullptr;
 }
 
 cudaError_t launch_rope_table(float2* tab, int T, int H, int W, int rt, int rh, int rw,

@@ -14,7 +14,8 @@ from typing import Dict, Optional, Sequence
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "_lib", "libh3b.so")
+# H3B_CHECKED=1 selects the checked build (indices tested against buffer extents in every kernel)
+LIB_PATH = os.path.join(_HERE, "_lib", "libh3b_checked.so" if os.environ.get("H3B_CHECKED") == "1" else "libh3b.so")
 
 H3B_OK = 0
 STATUS = {0: "H3B_OK", -1: "H3B_ERR_ARG", -2: "H3B_ERR_SHAPE", -3: "H3B_ERR_ALIGN",
@@ -59,7 +60,8 @@ def lib():
     if _LIB is None:
         if not os.path.exists(LIB_PATH):
             raise RuntimeError(f"h3b CUDA library not built ({LIB_PATH}); run "
-                               "video_diffusion_transformer_adaln_b200/build.py")
+                               "video_diffusion_transformer_adaln_b200/build.py"
+                               + (" --checked" if LIB_PATH.endswith("_checked.so") else ""))
         L = C.CDLL(LIB_PATH)
         _declare(L)
         _LIB = L
@@ -113,6 +115,8 @@ def _declare(L):
     L.h3b_graph_kernel_count.argtypes = [vp]
     L.h3b_graph_destroy.restype = None
     L.h3b_graph_destroy.argtypes = [vp]
+    L.h3b_checked_build.restype = i32
+    L.h3b_checked_build.argtypes = []
 
 
 def _p(t: Optional[torch.Tensor]):
@@ -263,6 +267,10 @@ def h3b_token_unpair(full: Dims, x, xm, ym, out, stream=None):
 def h3b_quantize_weights(w, q, s, stream=None):
     rows, cols = w.shape
     _check(lib().h3b_quantize_weights(_p(w), rows, cols, _p(q), _p(s), _s(stream)), "h3b_quantize_weights")
+
+
+def h3b_checked_build() -> bool:
+    return bool(lib().h3b_checked_build())
 
 
 def h3b_device_error(clear: bool = True) -> int:
