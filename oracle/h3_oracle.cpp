@@ -421,7 +421,8 @@ typedef struct {
 // "性能上限"):
 //   mod = AdaLN Linear(c)
 //   h1  = bf16(LN(x) * (1 + scale_a) + shift_a);  A1, s1 = quant(h1)
-//   QKV = deq(A1 Wqkv^T) + b;  RoPE(Q), RoPE(K)   (or bf16 h1 @ bf16 Wqkv^T)
+//   QKV = deq(A1 Wqkv^T) + b;  RoPE(Q), RoPE(K)   (or bf16 h1 @ bf16 Wqkv^T);
+//         Q, K, V rounded to bf16 (the attention's inputs)
 //   O   = attention(Q, K, V);  A2, s2 = quant(bf16(O))
 //   x1  = x + gate_a * (deq(A2 Wo^T) + bo)     (or bf16(O) @ bf16 Wo^T + bo: the
 //         BF16 attention-output projection of [README] "Metal 4 및 TensorOps")
@@ -484,6 +485,14 @@ int orc_block_forward(const orc_dims* dm, const orc_weights* wt, const float* c,
                 dm->rope_t, dm->rope_h, dm->rope_w, dm->rope_theta);
     orc_rope_3d(&K[(size_t)(b * L * d)], L, tp.data(), hp.data(), wp.data(), (int)nh, (int)dh,
                 dm->rope_t, dm->rope_h, dm->rope_w, dm->rope_theta);
+  }
+  // Q, K and V are the attention's bf16 inputs: the projections hand them to the
+  // attention in BF16, laid out head-major ([README] "Metal 4 및 TensorOps").
+  // Each is rounded once, after RoPE.
+  for (size_t i = 0; i < Q.size(); ++i) {
+    Q[i] = orc_bf16_to_f64(orc_f64_to_bf16(Q[i]));
+    K[i] = orc_bf16_to_f64(orc_f64_to_bf16(K[i]));
+    V[i] = orc_bf16_to_f64(orc_f64_to_bf16(V[i]));
   }
   if (tr && tr->mod) std::memcpy(tr->mod, mod.data(), mod.size() * sizeof(double));
   if (tr && tr->h1) std::memcpy(tr->h1, h1.data(), h1.size() * sizeof(uint16_t));

@@ -126,6 +126,8 @@ def composed_block(wl, w, c, x_bits):
             qkv = bf16_value(h1) @ bf16_value(w["wqkv_bf16"]).reshape(3 * d, d).T + bias("bqkv", 3 * d)
         Q, K, V = np.split(qkv, 3, axis=1)
         Q, K = rope(Q, wl), rope(K, wl)
+        # the attention's inputs are bf16
+        Q, K, V = (bf16_value(bf16_bits(a)) for a in (Q, K, V))
         o = attention(Q, K, V, wl)
         ob = bf16_value(bf16_bits(o))
         if wl.wo_bf16:

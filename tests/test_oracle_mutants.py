@@ -102,6 +102,7 @@ MUTANTS = [
     ("block_rows_ignored", "block", "sel[(size_t)i] = rows ? rows[i] : i;", "sel[(size_t)i] = i;"),
     ("block_bf16_qkv_no_bias", "block", "qkv[(size_t)(r * 3 * d + o)] += wt->bqkv[o];", "(void)0;"),
     ("block_bf16_wo_no_bias", "block", "yo[(size_t)(r * d + o)] += wt->bo[o];", "(void)0;"),
+    ("block_v_not_rounded", "block", "V[i] = orc_bf16_to_f64(orc_f64_to_bf16(V[i]));", "(void)0;"),
 ]
 
 

@@ -14,21 +14,19 @@
 //     frames^1.9, i.e. full attention over every latent token.
 //
 // Design (B200). One CTA per (256 queries, batch item x head): two query tiles
-// g = 0, 1 of 128 rows share every K/V tile of 64 keys.
-//   warp 0     TMA: Q0 and Q1 once, then K_j and V_j into 4-stage rings
-//   warp 1     tcgen05.mma from one thread. Each query tile has two score
-//              buffers in tensor memory, so S_g(j+2) is issued right behind
-//              P_g(j) V_j and is ready before the softmax of tile j+1 ends:
-//                S0(0) S1(0) S0(1) S1(1) | PV0(0) S0(2) PV1(0) S1(2) | PV0(1) ...
+// g = 0, 1 of 128 rows share every K/V tile.
+//   warp 0     TMA: Q0 and Q1 once, then K_j and V_j (128 keys) into 2-stage rings
+//   warp 1     tcgen05.mma from one thread, in the order
+//                S0(0) S1(0) | PV0(0) S0(1) PV1(0) S1(1) | PV0(1) S0(2) ...
+//              so the tensor core always has the other tile's work queued
 //   warps 2-5  softmax of tile 0, warps 6-9 softmax of tile 1 (thread = row)
-// Tensor memory (512 columns at head_dim 128): S0a S0b S1a S1b (64 each) | O0 | O1.
-// Each softmax thread reads its row of S_g(j) from buffer j mod 2, writes
-// P_g(j) = exp2(S*c - m) as bf16 pairs over the first 32 columns of that
-// buffer, and the P V product takes its A operand from tensor memory; the
-// tensor core runs one CTA's MMAs in issue order, so P_g(j) V_j reads the
-// buffer before S_g(j+2) overwrites it. The running max is kept until a row's
-// max grows by more than 2^8; then the softmax waits for P_g(j-1) V_{j-1} to
-// complete and rescales O_g and the row sum. The final division by the row sum
+// Tensor memory (512 columns): S0 | S1 | O0 | O1. Each softmax thread reads its
+// row of S_g, writes P_g = exp2(S*c - m) as bf16 pairs over the first 64
+// columns of S_g, and the P V product takes its A operand from tensor memory.
+// A commit tracks every earlier MMA of the issuing thread, so when S_g(j) is
+// complete, PV_g(j-1) is complete too: O_g can be rescaled then without another
+// barrier. The running max is kept until a row's max grows by more than 2^8
+// (then O_g and the row sum are rescaled); the final division by the row sum
 // is exact either way. Every wait is bounded and every decision guarding a
 // warp-collective TMEM access is warp-uniform.
 #include "h3b_common.cuh"
@@ -37,12 +35,9 @@
 
 namespace h3b {
 namespace attn {
-constexpr int BQ = 128, BKV = 64, kThreads = 320, KV_STAGES = 4;
+constexpr int BQ = 128, BKV = 128, kThreads = 320;
 constexpr uint32_t TMEM_COLS = 512;
-constexpr int BOX_ROWS = 64;                 // one TMA box: 64 rows x 128 bytes
-constexpr int BOX = BOX_ROWS * 128;          // 8 KB
-constexpr int QCHUNK = BQ * 128;             // 64 head lanes of a 128-row query tile
-constexpr int KVCHUNK = BKV * 128;           // 64 head lanes of a 64-key tile
+constexpr int BOX = 16384;  // one TMA box: 128 rows x 128 bytes
 }  // namespace attn
 
 __device__ __forceinline__ float fast_exp2(float x) {
@@ -85,20 +80,18 @@ __device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uin
 
 template <int DH>
 struct AttnLayout {
-  static constexpr int NBOX = DH / 64;                  // 64-lane chunks of a head row
-  static constexpr int QTILE = attn::BQ * DH * 2;       // bytes of one query tile
-  static constexpr int KVTILE = attn::BKV * DH * 2;     // bytes of one K or V tile
-  static constexpr int Q_OFF = 0;                       // Q0, Q1
-  static constexpr int K_OFF = Q_OFF + 2 * QTILE;       // K stages
-  static constexpr int V_OFF = K_OFF + attn::KV_STAGES * KVTILE;
-  static constexpr int BAR_OFF = V_OFF + attn::KV_STAGES * KVTILE;
-  static constexpr int NBARS = 28;
+  static constexpr int NBOX = DH / 64;             // TMA boxes per Q/K/V tile
+  static constexpr int TILE = attn::BKV * DH * 2;  // bytes of one Q/K/V tile
+  static constexpr int Q_OFF = 0;                  // Q0, Q1
+  static constexpr int K_OFF = Q_OFF + 2 * TILE;   // K stages 0, 1
+  static constexpr int V_OFF = K_OFF + 2 * TILE;   // V stages 0, 1
+  static constexpr int BAR_OFF = V_OFF + 2 * TILE;
+  static constexpr int NBARS = 16;
   static constexpr size_t SMEM_NEED = (size_t)BAR_OFF + NBARS * 8 + 16 + 1024;
   // At least 120 KB so two CTAs never share an SM: each holds all 512 TMEM columns.
   static constexpr size_t SMEM = SMEM_NEED > 120 * 1024 ? SMEM_NEED : 120 * 1024;
-  // tensor memory columns: score buffer b of tile g, output accumulator of tile g
-  static constexpr uint32_t s_col(int g, int b) { return (uint32_t)(g * 2 * attn::BKV + b * attn::BKV); }
-  static constexpr uint32_t o_col(int g) { return (uint32_t)(4 * attn::BKV + g * DH); }
+  // tensor memory columns: S0, S1, O0, O1
+  static constexpr uint32_t S_COL0 = 0, S_COL1 = 128, O_COL0 = 256, O_COL1 = 256 + DH;
 };
 
 // kPolyMod: every kPolyMod-th pair of exponentials goes to the FMA pipe (0: none).
@@ -107,7 +100,6 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
     attention_kernel(const __grid_constant__ CUtensorMap tm, const AttnArgs a, float scale_log2) {
   using namespace attn;
   using Lay = AttnLayout<DH>;
-  static_assert(4 * BKV + 2 * DH <= (int)TMEM_COLS, "tensor memory budget");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb0 = smem_u32(smem);
@@ -115,14 +107,13 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
   const uint32_t bar0 = smem_u32(bars);
   const uint32_t q_full = bar0;
   auto k_full = [&](int s) { return bar0 + 8u * (1 + s); };
-  auto k_empty = [&](int s) { return bar0 + 8u * (5 + s); };
-  auto v_full = [&](int s) { return bar0 + 8u * (9 + s); };
-  auto v_empty = [&](int s) { return bar0 + 8u * (13 + s); };
-  auto s_full = [&](int g, int b) { return bar0 + 8u * (17 + 2 * g + b); };
-  auto p_full = [&](int g) { return bar0 + 8u * (21 + g); };
-  auto pv_done = [&](int g) { return bar0 + 8u * (23 + g); };
-  auto fin = [&](int g) { return bar0 + 8u * (25 + g); };
-  const uint32_t drain = bar0 + 8u * 27;
+  auto k_empty = [&](int s) { return bar0 + 8u * (3 + s); };
+  auto v_full = [&](int s) { return bar0 + 8u * (5 + s); };
+  auto v_empty = [&](int s) { return bar0 + 8u * (7 + s); };
+  auto s_full = [&](int g) { return bar0 + 8u * (9 + g); };
+  auto p_full = [&](int g) { return bar0 + 8u * (11 + g); };
+  auto fin = [&](int g) { return bar0 + 8u * (13 + g); };
+  const uint32_t drain = bar0 + 8u * 15;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + Lay::NBARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -136,13 +127,10 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int s = 0; s < KV_STAGES; ++s) {
+    for (int s = 0; s < 2; ++s) {
       mbar_init(k_full(s), 1); mbar_init(k_empty(s), 1);
       mbar_init(v_full(s), 1); mbar_init(v_empty(s), 1);
-    }
-    for (int g = 0; g < 2; ++g) {
-      mbar_init(s_full(g, 0), 1); mbar_init(s_full(g, 1), 1);
-      mbar_init(p_full(g), 4); mbar_init(pv_done(g), 1); mbar_init(fin(g), 1);
+      mbar_init(s_full(s), 1); mbar_init(p_full(s), 4); mbar_init(fin(s), 1);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -162,44 +150,38 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
     if (lane == 0) {
       // ---------------- TMA producer
       bool ok = true;
-      // issued-but-unwaited bookkeeping for the drain: bit s (K stage s), bit 4+s (V stage s),
-      // and the parity of each stage's last fill
-      uint32_t filled = 0, fill_ph = 0;
-      mbar_arrive_expect_tx(q_full, 2 * Lay::QTILE);
+      uint32_t filled = 0, fill_ph = 0;  // bits s (K stage s) and 2+s (V stage s)
+      mbar_arrive_expect_tx(q_full, 2 * Lay::TILE);
       for (int g = 0; g < 2; ++g)
-        for (int c = 0; c < Lay::NBOX; ++c)
-          for (int h = 0; h < BQ / BOX_ROWS; ++h)
-            tma_load_3d(sb0 + Lay::Q_OFF + g * Lay::QTILE + c * QCHUNK + h * BOX, &tm, q_full, c * 64,
-                        qt * 2 * BQ + g * BQ + h * BOX_ROWS, bh);
+        for (int b = 0; b < Lay::NBOX; ++b)
+          tma_load_3d(sb0 + Lay::Q_OFF + g * Lay::TILE + b * BOX, &tm, q_full, b * 64, qt * 2 * BQ + g * BQ, bh);
       for (int j = 0; j < nkv && ok; ++j) {
-        const int s = j % KV_STAGES;
-        const uint32_t ph = (uint32_t)(j / KV_STAGES) & 1u;
+        const int s = j & 1;
+        const uint32_t ph = (j >> 1) & 1;
         if (!mbar_wait_or_abort(k_empty(s), ph ^ 1u, abort_flag, a.err, ERR_WAIT_MMA)) { ok = false; break; }
-        mbar_arrive_expect_tx(k_full(s), Lay::KVTILE);
-        for (int c = 0; c < Lay::NBOX; ++c)
-          tma_load_3d(sb0 + Lay::K_OFF + s * Lay::KVTILE + c * KVCHUNK, &tm, k_full(s), c * 64, j * BKV, BH + bh);
+        mbar_arrive_expect_tx(k_full(s), Lay::TILE);
+        for (int b = 0; b < Lay::NBOX; ++b)
+          tma_load_3d(sb0 + Lay::K_OFF + s * Lay::TILE + b * BOX, &tm, k_full(s), b * 64, j * BKV, BH + bh);
         filled |= 1u << s;
         fill_ph = (fill_ph & ~(1u << s)) | (ph << s);
         if (!mbar_wait_or_abort(v_empty(s), ph ^ 1u, abort_flag, a.err, ERR_WAIT_MMA)) { ok = false; break; }
-        mbar_arrive_expect_tx(v_full(s), Lay::KVTILE);
-        for (int c = 0; c < Lay::NBOX; ++c)
-          tma_load_3d(sb0 + Lay::V_OFF + s * Lay::KVTILE + c * KVCHUNK, &tm, v_full(s), c * 64, j * BKV,
-                      2 * BH + bh);
-        filled |= 16u << s;
-        fill_ph = (fill_ph & ~(16u << s)) | (ph << (4 + s));
+        mbar_arrive_expect_tx(v_full(s), Lay::TILE);
+        for (int b = 0; b < Lay::NBOX; ++b)
+          tma_load_3d(sb0 + Lay::V_OFF + s * Lay::TILE + b * BOX, &tm, v_full(s), b * 64, j * BKV, 2 * BH + bh);
+        filled |= 4u << s;
+        fill_ph = (fill_ph & ~(4u << s)) | (ph << (2 + s));
       }
       if (!ok) {
         *abort_flag = 1;
         mbar_wait(q_full, 0, a.err, ERR_WAIT_DRAIN, kDrainLimitNs);
-        for (int s = 0; s < KV_STAGES; ++s) {
+        for (int s = 0; s < 2; ++s) {
           if (filled & (1u << s)) mbar_wait(k_full(s), (fill_ph >> s) & 1u, a.err, ERR_WAIT_DRAIN, kDrainLimitNs);
-          if (filled & (16u << s))
-            mbar_wait(v_full(s), (fill_ph >> (4 + s)) & 1u, a.err, ERR_WAIT_DRAIN, kDrainLimitNs);
+          if (filled & (4u << s)) mbar_wait(v_full(s), (fill_ph >> (2 + s)) & 1u, a.err, ERR_WAIT_DRAIN, kDrainLimitNs);
         }
       } else {
-        for (int s = 0; s < KV_STAGES; ++s) {  // tail: every issued tile has been consumed
+        for (int s = 0; s < 2; ++s) {  // tail: every issued tile has been consumed
           if (filled & (1u << s)) mbar_wait(k_empty(s), (fill_ph >> s) & 1u, a.err, ERR_WAIT_MMA);
-          if (filled & (16u << s)) mbar_wait(v_empty(s), (fill_ph >> (4 + s)) & 1u, a.err, ERR_WAIT_MMA);
+          if (filled & (4u << s)) mbar_wait(v_empty(s), (fill_ph >> (2 + s)) & 1u, a.err, ERR_WAIT_MMA);
         }
       }
     }
@@ -207,51 +189,52 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
     if (lane == 0) {
       // ---------------- MMA issuer
       bool any = false;
-      auto issue_s = [&](int g, int j) -> bool {  // S_g(j) = Q_g K_j^T into score buffer j mod 2
-        const int s = j % KV_STAGES;
-        if (g == 0 && !mbar_wait_or_abort(k_full(s), (uint32_t)(j / KV_STAGES) & 1u, abort_flag, a.err,
-                                          ERR_WAIT_TMA))
-          return false;
+      auto issue_s = [&](int g, int j) -> bool {  // S_g(j) = Q_g K_j^T
+        const int s = j & 1;
+        if (g == 0 && !mbar_wait_or_abort(k_full(s), (j >> 1) & 1, abort_flag, a.err, ERR_WAIT_TMA)) return false;
         tc_fence_after();
-        const uint32_t q_addr = sb0 + Lay::Q_OFF + g * Lay::QTILE;
-        const uint32_t k_addr = sb0 + Lay::K_OFF + s * Lay::KVTILE;
+        const uint32_t q_addr = sb0 + Lay::Q_OFF + g * Lay::TILE;
+        const uint32_t k_addr = sb0 + Lay::K_OFF + s * Lay::TILE;
+        const uint32_t s_col = g == 0 ? Lay::S_COL0 : Lay::S_COL1;
 #pragma unroll
         for (int k = 0; k < DH / 16; ++k) {
-          const uint64_t ad = smem_desc_sw128(q_addr + (k >> 2) * QCHUNK + (k & 3) * 32, 16, 1024);
-          const uint64_t bd = smem_desc_sw128(k_addr + (k >> 2) * KVCHUNK + (k & 3) * 32, 16, 1024);
-          mma_f16(tmem + Lay::s_col(g, j & 1), ad, bd, IDESC_S, k > 0 ? 1u : 0u);
+          const uint64_t ad = smem_desc_sw128(q_addr + (k >> 2) * BOX + (k & 3) * 32, 16, 1024);
+          const uint64_t bd = smem_desc_sw128(k_addr + (k >> 2) * BOX + (k & 3) * 32, 16, 1024);
+          mma_f16(tmem + s_col, ad, bd, IDESC_S, k > 0 ? 1u : 0u);
         }
         any = true;
-        tc_commit(s_full(g, j & 1));
+        tc_commit(s_full(g));
         if (g == 1) tc_commit(k_empty(s));
         return true;
       };
       auto issue_pv = [&](int g, int j) -> bool {  // O_g += P_g(j) V_j
-        const int s = j % KV_STAGES;
-        if (!mbar_wait_or_abort(p_full(g), (uint32_t)j & 1u, abort_flag, a.err, ERR_WAIT_EPI)) return false;
-        if (g == 0 && !mbar_wait_or_abort(v_full(s), (uint32_t)(j / KV_STAGES) & 1u, abort_flag, a.err,
-                                          ERR_WAIT_TMA))
-          return false;
+        const int s = j & 1;
+        if (!mbar_wait_or_abort(p_full(g), j & 1, abort_flag, a.err, ERR_WAIT_EPI)) return false;
+        if (g == 0 && !mbar_wait_or_abort(v_full(s), (j >> 1) & 1, abort_flag, a.err, ERR_WAIT_TMA)) return false;
         tc_fence_after();
-        const uint32_t v_addr = sb0 + Lay::V_OFF + s * Lay::KVTILE;
+        const uint32_t v_addr = sb0 + Lay::V_OFF + s * Lay::TILE;
+        const uint32_t o_col = g == 0 ? Lay::O_COL0 : Lay::O_COL1;
+        const uint32_t s_col = g == 0 ? Lay::S_COL0 : Lay::S_COL1;
 #pragma unroll
         for (int k = 0; k < BKV / 16; ++k) {
-          const uint64_t bd = smem_desc_sw128(v_addr + k * 2048, KVCHUNK, 1024);
-          mma_f16_ts(tmem + Lay::o_col(g), tmem + Lay::s_col(g, j & 1) + k * 8, bd, IDESC_PV,
-                     (j > 0 || k > 0) ? 1u : 0u);
+          const uint64_t bd = smem_desc_sw128(v_addr + k * 2048, BOX, 1024);
+          mma_f16_ts(tmem + o_col, tmem + s_col + k * 8, bd, IDESC_PV, (j > 0 || k > 0) ? 1u : 0u);
         }
-        tc_commit(pv_done(g));
-        if (j == nkv - 1) tc_commit(fin(g));
         if (g == 1) tc_commit(v_empty(s));
         return true;
       };
       bool ok = mbar_wait(q_full, 0, a.err, ERR_WAIT_TMA);
-      for (int j = 0; j < 2 && j < nkv && ok; ++j) ok = issue_s(0, j) && issue_s(1, j);
+      ok = ok && issue_s(0, 0) && issue_s(1, 0);
       for (int j = 0; j < nkv && ok; ++j) {
         ok = issue_pv(0, j);
-        if (ok && j + 2 < nkv) ok = issue_s(0, j + 2);
-        if (ok) ok = issue_pv(1, j);
-        if (ok && j + 2 < nkv) ok = issue_s(1, j + 2);
+        if (!ok) break;
+        if (j + 1 < nkv) ok = issue_s(0, j + 1);
+        else tc_commit(fin(0));
+        if (!ok) break;
+        ok = issue_pv(1, j);
+        if (!ok) break;
+        if (j + 1 < nkv) ok = issue_s(1, j + 1);
+        else tc_commit(fin(1));
       }
       if (!ok) {
         *abort_flag = 1;
@@ -264,17 +247,16 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
   } else {
     // ---------------- softmax warps: 2-5 -> tile 0, 6-9 -> tile 1 (thread = query row)
     const int g = (warp - 2) >> 2;
-    const int quad = warp & 3;  // the TMEM lane quarter this warp may access
+    const int quad = warp & 3;
     const int row = quad * 32 + lane;
     const uint32_t t_lane = (uint32_t)(quad * 32) << 16;
-    const uint32_t o_col = Lay::o_col(g);
+    const uint32_t s_col = g == 0 ? Lay::S_COL0 : Lay::S_COL1;
+    const uint32_t o_col = g == 0 ? Lay::O_COL0 : Lay::O_COL1;
     const float2 c2 = make_float2(scale_log2, scale_log2);
     float m_run = -INFINITY, l_run = 0.0f;
     bool ok = true;
     for (int j = 0; j < nkv; ++j) {
-      const int b = j & 1;
-      const uint32_t s_col = Lay::s_col(g, b);
-      const bool s_ok = mbar_wait_or_abort(s_full(g, b), (uint32_t)(j >> 1) & 1u, abort_flag, a.err, ERR_WAIT_MMA);
+      const bool s_ok = mbar_wait_or_abort(s_full(g), j & 1, abort_flag, a.err, ERR_WAIT_MMA);
       if (!__all_sync(0xFFFFFFFFu, s_ok)) { ok = false; break; }
       tc_fence_after();
       uint32_t sr[BKV];
@@ -328,12 +310,8 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
       const float2 a03 = __fadd2_rn(a01, a23);
       l_run = fmaf(l_run, alpha, a03.x + a03.y);
 
-      // O_g holds the products up to key tile j-1 once P_g(j-1) V_{j-1} has completed
-      // (P_g(j) V_j waits for this warp's arrival below).
+      // S_g(j) complete => PV_g(j-1) complete: O_g is stable until P_g(j) is published.
       if (__any_sync(0xFFFFFFFFu, rescale)) {
-        const bool pv_ok = mbar_wait_or_abort(pv_done(g), (uint32_t)(j - 1) & 1u, abort_flag, a.err, ERR_WAIT_MMA);
-        if (!__all_sync(0xFFFFFFFFu, pv_ok)) { ok = false; break; }
-        tc_fence_after();
 #pragma unroll
         for (int c = 0; c < DH / 32; ++c) {
           uint32_t o[32];
@@ -350,10 +328,9 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
           tmem_st32(tmem + t_lane + o_col + c * 32, o);
         }
       }
-      // P_g(j) over the first BKV/2 columns of the buffer: column c holds keys 2c (low half) and 2c+1.
-#pragma unroll
-      for (int c = 0; c < BKV / 64; ++c)
-        tmem_st32(tmem + t_lane + s_col + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
+      // P_g(j) over the first 64 columns of S_g: column c holds keys 2c (low half) and 2c+1.
+      tmem_st32(tmem + t_lane + s_col, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+      tmem_st32(tmem + t_lane + s_col + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
@@ -407,7 +384,7 @@ static cudaError_t launch_attn(const AttnArgs& a, cudaStream_t st) {
   using Lay = AttnLayout<DH>;
   CUtensorMap tm;
   // qkv viewed as [3*B*H][L][DH]
-  if (!make_tmap_3d(&tm, a.qkv, 2, (uint64_t)DH, (uint64_t)a.L, (uint64_t)3 * a.B * a.n_heads, 64, attn::BOX_ROWS))
+  if (!make_tmap_3d(&tm, a.qkv, 2, (uint64_t)DH, (uint64_t)a.L, (uint64_t)3 * a.B * a.n_heads, 64, attn::BKV))
     return cudaErrorInvalidValue;
   auto k = attention_kernel<DH, kPolyMod>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Lay::SMEM);

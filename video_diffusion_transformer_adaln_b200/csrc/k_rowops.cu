@@ -172,26 +172,20 @@ __global__ void __launch_bounds__(256) adaln_gemv_kernel(const __nv_bfloat16* __
 
 // ---------------------------------------------------------------------------
 // Fused LayerNorm + modulation + per-row int8 quantization.
-//   y = (x - mean) * rsqrt(var + eps)          (fp32; mean and variance merged
-//                                               from per-thread partial sums)
+//   y = (x - mean) * rsqrt(var + eps)          (fp32, two-pass variance)
 //   h = bf16(y * (1 + scale) + shift)
 //   s = absmax(h) / 127, q = rint(h / s)       (binary32 decision)
 // A row of d = 256 NV channels (32 NV 16-byte vectors) is held in registers by
-// tpr = 32 NV / VPT threads, VPT vectors each (a row group of tpr / 32 warps);
-// a block holds rpp = blockDim / tpr row groups and walks its share of the rows
-// in passes of rpp rows, all of one batch item. The next pass's vectors are
-// loaded into registers while the current row is processed.
-// Statistics: each thread takes the mean and the centred sum of squares M2 of
-// its own 8 VPT values (two passes over registers), and these (mean, M2) pairs
-// are merged pairwise (Chan, Golub and LeVeque's update for equal counts:
-// mean = (m_a + m_b) / 2, M2 = M2_a + M2_b + (m_b - m_a)^2 n / 2), first across
-// the warp by shuffles, then across the row group's warps through shared
-// memory behind one named barrier of the row group. The symmetric form gives
-// every lane the same bits. The row absmax takes a second such barrier; the
-// absmax of the bf16-rounded h is the rounding of the fp32 absmax, since
-// rounding to nearest is monotone. The item's (1 + scale, shift) pairs sit in
-// shared memory, loaded when the item changes, laid out [4][vectors] so that a
-// warp's 16-byte reads of one channel pair per vector fall in distinct banks.
+// tpr = 32 NV / VPT threads, VPT vectors each; a block holds rpp = blockDim /
+// tpr rows at a time and walks its share of the rows in passes of rpp rows,
+// all of one batch item. The item's (1 + scale, shift) pairs sit in shared
+// memory, loaded when the item changes, laid out [4][vectors] so that a warp's
+// 16-byte reads of one channel pair per vector fall in distinct banks.
+// Reductions: warp shuffles, then one shared slot per warp and a named barrier
+// of the row group (slots alternate between passes, so no barrier guards their
+// reuse; a one-warp row needs only the warp's own sync). The row absmax is taken
+// in fp32 before the bf16 rounding: rounding to nearest is monotone, so the
+// rounded fp32 absmax is the absmax of the rounded h.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ float2 bf16x2_to_f2(uint32_t u) { return make_float2(bf16_lo(u), bf16_hi(u)); }
 __device__ __forceinline__ float max3f_row(float a, float b, float c) {
@@ -207,24 +201,30 @@ __device__ __forceinline__ void named_barrier(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
-// Pairwise merge of two (mean, M2) summaries of n values each.
-__device__ __forceinline__ void chan_merge(float& mean, float& m2, float mean_b, float m2_b, float half_n) {
-  const float dlt = mean_b - mean;
-  m2 = (m2 + m2_b) + dlt * dlt * half_n;
-  mean = (mean + mean_b) * 0.5f;
+// 16-byte asynchronous copy global -> shared (L2 only), and the wait for all of
+// this thread's outstanding copies.
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+// Lane-wise max of two bf16 pairs (both non-negative here).
+__device__ __forceinline__ uint32_t bf16x2_max(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
 }
 
-// Largest block the launcher forms for a VPT (a row group of up to 992 threads at VPT 1).
 template <int VPT>
-constexpr int ln_max_threads() { return VPT == 1 ? 1024 : VPT == 2 ? 512 : VPT == 3 ? 320 : 256; }
-
-template <int VPT>
-__global__ void __launch_bounds__(ln_max_threads<VPT>(), VPT >= 4 ? 2 : 1) ln_mod_quant_kernel(
+__global__ void __launch_bounds__(1024, 1) ln_mod_quant_kernel(
     const __nv_bfloat16* __restrict__ x, int rows, int vpr, float eps, const float* __restrict__ shift,
     const float* __restrict__ scale, int rows_per_item, int mod_stride, int8_t* __restrict__ q,
     float* __restrict__ s, __nv_bfloat16* __restrict__ h_out, float* __restrict__ absmax_zero,
     int write_codes) {
   extern __shared__ float4 modp[];  // [4][vpr]: (1+sc[2c], 1+sc[2c+1], sh[2c], sh[2c+1]), c = 4 vec + e
+  // then the staging rows of the next pass: [rpp][vpr] 16-byte vectors, each written and read
+  // back by the same thread (cp.async), so no barrier guards them
   __shared__ float red[2][3][kLnMaxWarps];
   const int tpr = vpr / VPT;
   const int rpp = blockDim.x / tpr;
@@ -232,31 +232,30 @@ __global__ void __launch_bounds__(ln_max_threads<VPT>(), VPT >= 4 ? 2 : 1) ln_mo
   const int t = threadIdx.x - sub * tpr;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int wpr = tpr >> 5, w0 = sub * wpr;
-  constexpr float kLocalN = 8.0f * VPT;
   const float inv_d = 1.0f / (float)(vpr * 8);
   const int items = (rows + rows_per_item - 1) / rows_per_item;
   const unsigned gpi = (unsigned)((rows_per_item + rpp - 1) / rpp);
   const unsigned total = (unsigned)items * gpi;  // passes; at most rows, so 32 bits suffice
   int cur = -1, par = 0;
   unsigned item = blockIdx.x / gpi, g_in = blockIdx.x % gpi;  // pass = (item, pass within item)
+  uint4* stage = reinterpret_cast<uint4*>(modp + 4 * vpr) + (size_t)sub * vpr;
   // row-group barrier: a named barrier per group (ids 1..rpp), or the warp itself
   auto group_sync = [&]() {
     if (wpr > 1) named_barrier(1 + sub, tpr);
     else __syncwarp();
   };
-  // this thread's vectors of its row in pass (it, gi), zero when that row does not exist
-  auto load_row = [&](unsigned gg, unsigned it, unsigned gi, uint4 (&dst)[VPT]) {
+  // this thread's vectors of its row in pass (it, gi) -> staging, when that row exists
+  auto prefetch = [&](unsigned gg, unsigned it, unsigned gi) {
     const int r = (int)gi * rpp + sub, rw = (int)it * rows_per_item + r;
-    const bool ok = gg < total && r < rows_per_item && rw < rows;
-    const uint4* src = reinterpret_cast<const uint4*>(x) + (size_t)(ok ? rw : 0) * vpr;
+    if (gg >= total || r >= rows_per_item || rw >= rows) return;
+    const uint4* src = reinterpret_cast<const uint4*>(x) + (size_t)rw * vpr;
 #pragma unroll
     for (int i = 0; i < VPT; ++i)
-      dst[i] = ok && H3B_IDX_OK((long long)rw * vpr + t + tpr * i, (long long)rows * vpr, &g_h3b_rowops_bounds)
-                   ? __ldcs(src + t + tpr * i)
-                   : make_uint4(0, 0, 0, 0);
+      if (H3B_IDX_OK((long long)rw * vpr + t + tpr * i, (long long)rows * vpr, &g_h3b_rowops_bounds))
+        cp_async16(stage + t + tpr * i, src + t + tpr * i);
   };
-  uint4 nxt[VPT];
-  load_row(blockIdx.x, item, g_in, nxt);
+  prefetch(blockIdx.x, item, g_in);
+  cp_async_commit();
   for (unsigned g = blockIdx.x; g < total; g += gridDim.x) {
     if ((int)item != cur) {  // block-uniform
       __syncthreads();
@@ -272,18 +271,14 @@ __global__ void __launch_bounds__(ln_max_threads<VPT>(), VPT >= 4 ? 2 : 1) ln_mo
     const int r_in = (int)g_in * rpp + sub;
     const int row = (int)item * rows_per_item + r_in;
     const bool valid = r_in < rows_per_item && row < rows;
+    cp_async_wait_all();
     uint4 v[VPT];
 #pragma unroll
-    for (int i = 0; i < VPT; ++i) v[i] = nxt[i];
-    // start the next pass's loads
-    unsigned n_in = g_in + gridDim.x;
-    const unsigned n_item = item + n_in / gpi;
-    n_in %= gpi;
-    load_row(g + gridDim.x, n_item, n_in, nxt);
+    for (int i = 0; i < VPT; ++i) v[i] = valid ? stage[t + tpr * i] : make_uint4(0, 0, 0, 0);
 
     float* rd = red[par][0];
     par ^= 1;
-    // the row in fp32 pairs, converted once; this thread's mean and M2
+    // the row in fp32 pairs, converted once
     float2 f[VPT * 4];
 #pragma unroll
     for (int i = 0; i < VPT; ++i) {
@@ -292,44 +287,35 @@ __global__ void __launch_bounds__(ln_max_threads<VPT>(), VPT >= 4 ? 2 : 1) ln_mo
       f[4 * i + 2] = bf16x2_to_f2(v[i].z);
       f[4 * i + 3] = bf16x2_to_f2(v[i].w);
     }
+    // the staged vectors are in registers now: start the next pass's loads
+    unsigned n_in = g_in + gridDim.x;
+    const unsigned n_item = item + n_in / gpi;
+    n_in %= gpi;
+    prefetch(g + gridDim.x, n_item, n_in);
+    cp_async_commit();
     float2 acc = f[0];
 #pragma unroll
     for (int e = 1; e < VPT * 4; ++e) acc = __fadd2_rn(acc, f[e]);
-    const float lmean = (acc.x + acc.y) * (1.0f / kLocalN);
-    const float2 nl2 = make_float2(-lmean, -lmean);
+    float r = warp_sum(acc.x + acc.y);
+    if (lane == 0) rd[warp] = r;
+    group_sync();
+    r = 0.0f;
+    for (int k = 0; k < wpr; ++k) r += rd[w0 + k];
+    const float mean = r * inv_d;
+    const float2 nmean = make_float2(-mean, -mean);
+
 #pragma unroll
-    for (int e = 0; e < VPT * 4; ++e) f[e] = __fadd2_rn(f[e], nl2);  // x - local mean
+    for (int e = 0; e < VPT * 4; ++e) f[e] = __fadd2_rn(f[e], nmean);  // x - mean
     acc = __fmul2_rn(f[0], f[0]);
 #pragma unroll
     for (int e = 1; e < VPT * 4; ++e) acc = __ffma2_rn(f[e], f[e], acc);
-    float mean = lmean, m2 = acc.x + acc.y, half_n = 0.5f * kLocalN;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const float mb = __shfl_xor_sync(0xFFFFFFFFu, mean, o), m2b = __shfl_xor_sync(0xFFFFFFFFu, m2, o);
-      chan_merge(mean, m2, mb, m2b, half_n);
-      half_n *= 2.0f;
-    }
-    if (wpr > 1) {
-      if (lane == 0) {
-        rd[warp] = mean;
-        rd[kLnMaxWarps + warp] = m2;
-      }
-      group_sync();
-      mean = rd[w0];
-      m2 = rd[kLnMaxWarps + w0];
-      for (int k = 1; k < wpr; ++k) {  // same order in every thread: identical bits
-        const float mb = rd[w0 + k], m2b = rd[kLnMaxWarps + w0 + k];
-        const float dlt = mb - mean;
-        // merge the first k warps' summary (32 k kLocalN values) with warp k's (32 kLocalN)
-        const float nk = (float)k;
-        m2 = (m2 + m2b) + dlt * dlt * (32.0f * kLocalN * nk / (nk + 1.0f));
-        mean = fmaf(dlt, 1.0f / (nk + 1.0f), mean);
-      }
-    }
-    const float rstd = 1.0f / sqrtf(m2 * inv_d + eps);
+    r = warp_sum(acc.x + acc.y);
+    if (lane == 0) rd[kLnMaxWarps + warp] = r;
+    group_sync();
+    r = 0.0f;
+    for (int k = 0; k < wpr; ++k) r += rd[kLnMaxWarps + w0 + k];
+    const float rstd = 1.0f / sqrtf(r * inv_d + eps);
     const float2 rstd2 = make_float2(rstd, rstd);
-    const float ct = (lmean - mean) * rstd;  // (x - mean) rstd = (x - lmean) rstd + ct
-    const float2 ct2 = make_float2(ct, ct);
 
     // h = bf16((x - mean) * rstd * (1 + scale) + shift); max |h| in fp32 before the rounding
     float am = 0.0f;
@@ -340,7 +326,7 @@ __global__ void __launch_bounds__(ln_max_threads<VPT>(), VPT >= 4 ? 2 : 1) ln_mo
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const float4 m = modp[e * vpr + vec];
-        const float2 y = __ffma2_rn(f[4 * i + e], rstd2, ct2);
+        const float2 y = __fmul2_rn(f[4 * i + e], rstd2);
         const float2 h = __ffma2_rn(y, make_float2(m.x, m.y), make_float2(m.z, m.w));
         u[e] = pack_bf16x2(h.x, h.y);
         am = max3f_row(am, fabsf(h.x), fabsf(h.y));
@@ -348,13 +334,11 @@ __global__ void __launch_bounds__(ln_max_threads<VPT>(), VPT >= 4 ? 2 : 1) ln_mo
       v[i] = make_uint4(u[0], u[1], u[2], u[3]);
     }
     float amax = warp_max(am);
-    if (wpr > 1) {
-      if (lane == 0) rd[2 * kLnMaxWarps + warp] = amax;
-      group_sync();
-      amax = rd[2 * kLnMaxWarps + w0];
-      for (int k = 1; k < wpr; ++k) amax = fmaxf(amax, rd[2 * kLnMaxWarps + w0 + k]);
-    }
-    amax = round_bf16(amax);  // = the max of the rounded |h| (rounding is monotone)
+    if (lane == 0) rd[2 * kLnMaxWarps + warp] = amax;
+    group_sync();
+    amax = 0.0f;
+    for (int k = 0; k < wpr; ++k) amax = fmaxf(amax, rd[2 * kLnMaxWarps + w0 + k]);
+    amax = round_bf16(amax);  // = the max of the rounded |h|
     if (valid) {
       if (h_out) {
         uint4* hr = reinterpret_cast<uint4*>(h_out) + (size_t)row * vpr;
@@ -386,6 +370,7 @@ __global__ void __launch_bounds__(ln_max_threads<VPT>(), VPT >= 4 ? 2 : 1) ln_mo
     item = n_item;
     g_in = n_in;
   }
+  cp_async_wait_all();
 }
 
 // Per-row quantization with each row's absmax already known: a block covers
@@ -715,17 +700,17 @@ cudaError_t launch_adaln_gemv(const void* W, const float* bias, const float* c, 
 }
 
 // Threads per row: the fewest warps w dividing NV with NV / w <= 6 vectors per
-// thread; the block holds as many rows as fit in 256 threads (at least one).
+// thread; the block holds as many rows as fit in 512 threads (at least one), so
+// one copy of the modulation table serves more rows.
 template <int VPT>
 static cudaError_t ln_dispatch(const void* x, int rows, int nv, float eps, const float* shift,
                                const float* scale, int rpi, int ms, int8_t* q, float* s, void* h,
                                float* az, int wc, int sms, cudaStream_t st) {
   const int vpr = 32 * nv;
   const int tpr = vpr / VPT;
-  const int block = tpr * (tpr >= 256 ? 1 : 256 / tpr);
+  const int block = tpr * (tpr >= 512 ? 1 : 512 / tpr);
   const int rpp_d = block / tpr;
-  const size_t smem = (size_t)vpr * 4 * sizeof(float4);
-  (void)rpp_d;
+  const size_t smem = (size_t)vpr * 4 * sizeof(float4) + (size_t)rpp_d * vpr * sizeof(uint4);
   auto kern = ln_mod_quant_kernel<VPT>;
   // the attribute belongs to the current device, so it is set on every launch (a host-side call)
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
