@@ -27,6 +27,7 @@ MLP 20480, an 8x48x48 latent grid (18432 tokens).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl h3b|reference]
   python bench.py --oracle-table   (host timings of the CPU oracle only)
+  python bench.py --profile-kernel attention   (one kernel alone, for ncu captures)
 """
 import argparse
 import json
@@ -645,6 +646,57 @@ def run_reference(args, rank, world, local):
     print(json.dumps(line), flush=True)
 
 
+PROFILE_KERNELS = ("attention", "ln_mod_quant", "quant_o", "adaln_gemv", "token_pair", "token_unpair")
+
+
+def run_profile_kernel(name, workload):
+    """One step kernel alone at the workload's shape, three launches (for ncu captures of a
+    single kernel: `ncu -k regex:<kernel> -s 2 -c 1 python bench.py --profile-kernel NAME`)."""
+    cuda_build.build()
+    h3b.lib()
+    wl = synth.WORKLOADS[workload]
+    B, L, d, H, dh = wl.B, wl.L, wl.d, wl.n_heads, wl.head_dim
+    g = torch.Generator(device="cuda").manual_seed(synth.BASE_SEED)
+    dims = dims_of(wl)
+    if name == "attention":
+        qkv = (torch.randn(3 * B * H * L * dh, generator=g, device="cuda") * 0.8).to(torch.bfloat16)
+        o = torch.empty((B, L, d), dtype=torch.bfloat16, device="cuda")
+        am = torch.zeros(B * L, dtype=torch.float32, device="cuda")
+        fn = lambda: h3b.h3b_attention(dims, qkv, o, am)  # noqa: E731
+    elif name in ("ln_mod_quant", "quant_o"):
+        x = torch.randn((B * L, d), generator=g, device="cuda").to(torch.bfloat16)
+        q = torch.empty((B * L, d), dtype=torch.int8, device="cuda")
+        s = torch.empty(B * L, dtype=torch.float32, device="cuda")
+        if name == "ln_mod_quant":
+            sh = torch.randn(d, generator=g, device="cuda") * 0.1
+            sc = torch.randn(d, generator=g, device="cuda") * 0.1
+            fn = lambda: h3b.h3b_ln_modulate_quantize(x, B * L, d, wl.ln_eps, sh, sc, L, d, q, s)  # noqa: E731
+        else:
+            am = x.float().abs().amax(dim=1).contiguous()
+            fn = lambda: h3b.h3b_quantize_rows(x, q, s, absmax=am)  # noqa: E731
+    elif name == "adaln_gemv":
+        w = (torch.randn((6 * d, d), generator=g, device="cuda") * d ** -0.5).to(torch.bfloat16)
+        c = torch.randn((B, d), generator=g, device="cuda")
+        mod = torch.empty((B, 6 * d), device="cuda")
+        fn = lambda: h3b.h3b_adaln_modulation(dims, w, None, c, mod)  # noqa: E731
+    else:
+        x = torch.randn((B, wl.T, wl.H, wl.W, d), generator=g, device="cuda").to(torch.bfloat16)
+        ym = torch.empty((B, wl.T, wl.H, wl.W // 2, d), dtype=torch.bfloat16, device="cuda")
+        h3b.h3b_token_pair(dims, x, ym)
+        out = torch.empty_like(x)
+        fn = ((lambda: h3b.h3b_token_pair(dims, x, ym)) if name == "token_pair" else
+              (lambda: h3b.h3b_token_unpair(dims, x, None, ym, out)))
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    for _ in range(3):
+        flush.zero_()
+        fn()
+    torch.cuda.synchronize()
+    err = h3b.h3b_device_error(clear=True)
+    log(f"{name} at {workload}: 3 launches, device error word {err:#x}")
+    if err:
+        raise SystemExit(1)
+
+
 ORACLE_TABLE = (("d256_L512", (1, None)), ("d2048_L4096", (1, None)), ("d5120_L18432", (None,)))
 
 
@@ -737,7 +789,12 @@ def main():
     ap.add_argument("--oracle-table", action="store_true",
                     help="print host timings of the oracle (1 thread and all cores) and exit")
     ap.add_argument("--oracle-entry", help=argparse.SUPPRESS)
+    ap.add_argument("--profile-kernel", choices=PROFILE_KERNELS,
+                    help="run one step kernel alone at the workload's shape (three launches) and exit")
     args = ap.parse_args()
+    if args.profile_kernel:
+        run_profile_kernel(args.profile_kernel, args.workload)
+        return
     if args.oracle_entry:
         run_oracle_entry(args.oracle_entry)
         return

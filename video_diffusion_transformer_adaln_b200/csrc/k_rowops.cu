@@ -108,9 +108,11 @@ __device__ __forceinline__ uint32_t pack4_i8(int a, int b, int c, int d) {
 constexpr int kGemvMaxB = 8;
 
 // Persistent blocks: c is staged in shared memory once per block, then each
-// warp walks output rows j = (block * 8 + warp) + k * (blocks * 8). A row's d/8
-// 16-byte vectors (NV per lane) are all requested before any is used, so each
-// warp keeps a whole row in flight.
+// warp walks groups of kGemvRows consecutive output rows, j0 = (block * 8 +
+// warp) * kGemvRows + k * (blocks * 8 * kGemvRows). A group is read in chunks of
+// kGemvChunk 16-byte vectors per lane and row, all requested before any is used;
+// each c vector read from shared memory then serves all rows of the group, so
+// shared-memory traffic is a quarter of one row at a time.
 struct RopeTableArgs {
   float2* tab;  // nullptr: no table this launch
   int T, H, W, rt, rh, rw;
@@ -119,13 +121,18 @@ struct RopeTableArgs {
 
 __device__ void rope_table_entries(const RopeTableArgs& r, int first, int stride);
 
-template <int NV>
+constexpr int kGemvRows = 4;
+constexpr int kGemvChunk = 4;
+
+// MB: the largest batch the instance handles (1, or kGemvMaxB), so one latent keeps few accumulators.
+template <int NV, int MB>
 __global__ void __launch_bounds__(256) adaln_gemv_kernel(const __nv_bfloat16* __restrict__ W,
                                                          const float* __restrict__ bias,
                                                          const float* __restrict__ c, int B,
                                                          float* __restrict__ mod, const RopeTableArgs rope,
                                                          int gemv_blocks) {
   constexpr int d = NV * 256;
+  constexpr int R = kGemvRows, CH = kGemvChunk;
   if ((int)blockIdx.x >= gemv_blocks) {  // trailing blocks fill the RoPE table
     rope_table_entries(rope, ((int)blockIdx.x - gemv_blocks) * blockDim.x + threadIdx.x,
                        ((int)gridDim.x - gemv_blocks) * blockDim.x);
@@ -135,38 +142,54 @@ __global__ void __launch_bounds__(256) adaln_gemv_kernel(const __nv_bfloat16* __
   for (int i = threadIdx.x; i < B * d; i += blockDim.x) cs[i] = c[i];
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int j = blockIdx.x * 8 + warp; j < 6 * d; j += gemv_blocks * 8) {  // warp-uniform
-    const uint4* wr = reinterpret_cast<const uint4*>(W + (size_t)j * d);
-    uint4 w4[NV];
+  for (int j0 = (blockIdx.x * 8 + warp) * R; j0 < 6 * d; j0 += gemv_blocks * 8 * R) {  // warp-uniform
+    float acc[R][MB];
 #pragma unroll
-    for (int i = 0; i < NV; ++i) w4[i] = __ldcs(wr + lane + 32 * i);
-    float acc[kGemvMaxB];
+    for (int r = 0; r < R; ++r)
 #pragma unroll
-    for (int b = 0; b < kGemvMaxB; ++b) acc[b] = 0.0f;
+      for (int b = 0; b < MB; ++b) acc[r][b] = 0.0f;
+#pragma unroll 1
+    for (int i0 = 0; i0 < NV; i0 += CH) {
+      uint4 w4[R][CH];
 #pragma unroll
-    for (int i = 0; i < NV; ++i) {
-      const uint32_t ww[4] = {w4[i].x, w4[i].y, w4[i].z, w4[i].w};
-      const int v = lane + 32 * i;
+      for (int r = 0; r < R; ++r) {
+        const uint4* wr = reinterpret_cast<const uint4*>(W + (size_t)(j0 + r) * d);
 #pragma unroll
-      for (int b = 0; b < kGemvMaxB; ++b) {
-        if (b >= B) break;
-        const float4 c0 = *reinterpret_cast<const float4*>(cs + b * d + v * 8);
-        const float4 c1 = *reinterpret_cast<const float4*>(cs + b * d + v * 8 + 4);
-        float a = acc[b];
-        a = fmaf(bf16_lo(ww[0]), c0.x, a); a = fmaf(bf16_hi(ww[0]), c0.y, a);
-        a = fmaf(bf16_lo(ww[1]), c0.z, a); a = fmaf(bf16_hi(ww[1]), c0.w, a);
-        a = fmaf(bf16_lo(ww[2]), c1.x, a); a = fmaf(bf16_hi(ww[2]), c1.y, a);
-        a = fmaf(bf16_lo(ww[3]), c1.z, a); a = fmaf(bf16_hi(ww[3]), c1.w, a);
-        acc[b] = a;
+        for (int i = 0; i < CH; ++i)
+          if (i0 + i < NV) w4[r][i] = __ldcs(wr + lane + 32 * (i0 + i));
+      }
+#pragma unroll
+      for (int i = 0; i < CH; ++i) {
+        if (i0 + i >= NV) break;
+        const int v = lane + 32 * (i0 + i);
+#pragma unroll
+        for (int b = 0; b < MB; ++b) {
+          if (b >= B) break;
+          const float4 c0 = *reinterpret_cast<const float4*>(cs + b * d + v * 8);
+          const float4 c1 = *reinterpret_cast<const float4*>(cs + b * d + v * 8 + 4);
+#pragma unroll
+          for (int r = 0; r < R; ++r) {
+            const uint32_t ww[4] = {w4[r][i].x, w4[r][i].y, w4[r][i].z, w4[r][i].w};
+            float a = acc[r][b];
+            a = fmaf(bf16_lo(ww[0]), c0.x, a); a = fmaf(bf16_hi(ww[0]), c0.y, a);
+            a = fmaf(bf16_lo(ww[1]), c0.z, a); a = fmaf(bf16_hi(ww[1]), c0.w, a);
+            a = fmaf(bf16_lo(ww[2]), c1.x, a); a = fmaf(bf16_hi(ww[2]), c1.y, a);
+            a = fmaf(bf16_lo(ww[3]), c1.z, a); a = fmaf(bf16_hi(ww[3]), c1.w, a);
+            acc[r][b] = a;
+          }
+        }
       }
     }
 #pragma unroll
-    for (int b = 0; b < kGemvMaxB; ++b) {
-      if (b >= B) break;
-      const float r = warp_sum(acc[b]);
-      if (lane == 0 && H3B_IDX_OK((long long)b * 6 * d + j, (long long)B * 6 * d, &g_h3b_rowops_bounds))
-        mod[(size_t)b * 6 * d + j] = r + (bias ? bias[j] : 0.0f);
-    }
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+      for (int b = 0; b < MB; ++b) {
+        if (b >= B) break;
+        const float sum = warp_sum(acc[r][b]);
+        const int j = j0 + r;
+        if (lane == 0 && H3B_IDX_OK((long long)b * 6 * d + j, (long long)B * 6 * d, &g_h3b_rowops_bounds))
+          mod[(size_t)b * 6 * d + j] = sum + (bias ? bias[j] : 0.0f);
+      }
   }
 }
 
@@ -656,28 +679,35 @@ __global__ void rope_table_kernel(const RopeTableArgs r) {
 // ---------------------------------------------------------------------------
 // Launchers
 // ---------------------------------------------------------------------------
-template <int NV>
-static cudaError_t gemv_dispatch(const void* W, const float* bias, const float* c, int B, float* mod,
-                                 const RopeTableArgs& rope, int sms, cudaStream_t st) {
+template <int NV, int MB>
+static cudaError_t gemv_launch(const void* W, const float* bias, const float* c, int B, float* mod,
+                               const RopeTableArgs& rope, int sms, cudaStream_t st) {
   constexpr int d = NV * 256;
+  auto kern = adaln_gemv_kernel<NV, MB>;
   const size_t smem = (size_t)B * d * sizeof(float);
-  cudaError_t e = cudaFuncSetAttribute(adaln_gemv_kernel<NV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   int per_sm = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, adaln_gemv_kernel<NV>, 256, smem);
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 256, smem);
   if (e != cudaSuccess) return e;
   per_sm = per_sm < 1 ? 1 : per_sm;
-  // persistent blocks, as many as are resident at once, at most one per 8 output rows
-  const int gemv_blocks = std::min((6 * d + 7) / 8, sms * per_sm);
+  // persistent blocks, as many as are resident at once, at most one per 8 row groups
+  const int gemv_blocks = std::min((6 * d + 8 * kGemvRows - 1) / (8 * kGemvRows), sms * per_sm);
   int rope_blocks = 0;
   if (rope.tab) {
     const int n = rope.T * (rope.rt / 2) + rope.H * (rope.rh / 2) + rope.W * (rope.rw / 2);
     rope_blocks = (n + 255) / 256;
   }
-  adaln_gemv_kernel<NV><<<gemv_blocks + rope_blocks, 256, smem, st>>>(static_cast<const __nv_bfloat16*>(W), bias,
-                                                                      c, B, mod, rope, gemv_blocks);
+  kern<<<gemv_blocks + rope_blocks, 256, smem, st>>>(static_cast<const __nv_bfloat16*>(W), bias, c, B, mod, rope,
+                                                      gemv_blocks);
   return cudaGetLastError();
+}
+
+template <int NV>
+static cudaError_t gemv_dispatch(const void* W, const float* bias, const float* c, int B, float* mod,
+                                 const RopeTableArgs& rope, int sms, cudaStream_t st) {
+  return B == 1 ? gemv_launch<NV, 1>(W, bias, c, B, mod, rope, sms, st)
+                : gemv_launch<NV, kGemvMaxB>(W, bias, c, B, mod, rope, sms, st);
 }
 
 cudaError_t launch_adaln_gemv(const void* W, const float* bias, const float* c, int B, int d,
