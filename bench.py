@@ -646,7 +646,8 @@ def run_reference(args, rank, world, local):
     print(json.dumps(line), flush=True)
 
 
-PROFILE_KERNELS = ("attention", "ln_mod_quant", "quant_o", "adaln_gemv", "token_pair", "token_unpair")
+PROFILE_KERNELS = ("attention", "ln_mod_quant", "quant_o", "adaln_gemv", "token_pair", "token_unpair",
+                   "gemm_w1", "gemm_w2")
 
 
 def run_profile_kernel(name, workload):
@@ -674,6 +675,21 @@ def run_profile_kernel(name, workload):
         else:
             am = x.float().abs().amax(dim=1).contiguous()
             fn = lambda: h3b.h3b_quantize_rows(x, q, s, absmax=am)  # noqa: E731
+    elif name in ("gemm_w1", "gemm_w2"):
+        # the MLP projections at the workload's shape: int8 codes of a random activation and weight
+        K, N = (d, wl.d_ff) if name == "gemm_w1" else (wl.d_ff, d)
+        A = torch.randint(-127, 128, (B * L, K), generator=g, device="cuda", dtype=torch.int8)
+        Wq = torch.randint(-127, 128, (N, K), generator=g, device="cuda", dtype=torch.int8)
+        sA = torch.rand(B * L, generator=g, device="cuda") * 0.01
+        sW = torch.rand(N, generator=g, device="cuda") * 0.01
+        if name == "gemm_w1":
+            out = torch.empty((B * L, N), dtype=torch.bfloat16, device="cuda")
+            am = torch.zeros(B * L, dtype=torch.float32, device="cuda")
+            fn = lambda: h3b.h3b_gemm_i8_gelu(A, sA, Wq, sW, None, out, am)  # noqa: E731
+        else:
+            x = torch.randn((B * L, N), generator=g, device="cuda").to(torch.bfloat16)
+            gate = torch.randn((B, N), generator=g, device="cuda") * 0.5
+            fn = lambda: h3b.h3b_gemm_i8_gated_residual(A, sA, Wq, sW, None, gate, L, N, x)  # noqa: E731
     elif name == "adaln_gemv":
         w = (torch.randn((6 * d, d), generator=g, device="cuda") * d ** -0.5).to(torch.bfloat16)
         c = torch.randn((B, d), generator=g, device="cuda")
