@@ -62,10 +62,12 @@ def test_row_quantizer_bit_exact(rows, cols, with_absmax):
     no_device_error()
 
 
-def test_row_quantizer_every_bf16_value():
+@pytest.mark.parametrize("with_absmax", [False, True])
+def test_row_quantizer_every_bf16_value(with_absmax):
     """Every finite bf16 value up to a row's absmax, for 64 random scales and for
     scale 1 (absmax 127: exact half-integer ties): the int8 decision matches the
-    oracle's binary32 division bit for bit."""
+    oracle's binary32 division bit for bit, with the absmax found by the kernel
+    and with it given (the pass that requantizes O and G)."""
     allb = np.arange(0, 0x7F80, dtype=np.uint16)  # non-negative finite bf16 bit patterns
     pos = synth.bf16_bits_to_f32(allb)
     r = _rng(77)
@@ -84,14 +86,17 @@ def test_row_quantizer_every_bf16_value():
     hb = synth.f32_to_bf16_bits(h)
     q = torch.empty((len(rows), cols), dtype=torch.int8, device="cuda")
     s = torch.empty(len(rows), dtype=torch.float32, device="cuda")
-    h3b.h3b_quantize_rows(bf16_dev(hb), q, s)
-    qo, so = O.quantize_rows(synth.bf16_bits_to_f32(hb))
+    hf = synth.bf16_bits_to_f32(hb)
+    am = to_dev(np.abs(hf).max(axis=1).astype(np.float32)) if with_absmax else None
+    h3b.h3b_quantize_rows(bf16_dev(hb), q, s, absmax=am)
+    qo, so = O.quantize_rows(hf)
     assert np.array_equal(s.cpu().numpy(), so)
     assert np.array_equal(q.cpu().numpy(), qo)
     no_device_error()
 
 
-@pytest.mark.parametrize("rows,d,items", [(512, 256, 1), (37, 2048, 1), (64, 5120, 1), (96, 256, 3), (8, 8192, 2)])
+@pytest.mark.parametrize("rows,d,items", [(512, 256, 1), (37, 2048, 1), (64, 5120, 1), (96, 256, 3), (8, 8192, 2),
+                                           (40, 768, 2), (19, 3072, 1), (16, 5376, 1), (23, 7936, 1)])
 def test_ln_modulate_quantize(rows, d, items):
     r = _rng(rows * d)
     wl = synth.WORKLOADS["d256_L512"].with_(d=d, n_heads=d // 64)

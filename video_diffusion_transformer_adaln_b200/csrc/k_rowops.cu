@@ -64,8 +64,8 @@ __device__ __forceinline__ int quant_code_fast(float v, float scale, float rcp) 
 // t = v * RN(1/scale); adding 1.5 * 2^23 rounds t to the nearest integer
 // (ties to even) in the low mantissa bits, whose low byte is the int8 code
 // (|t| <= 127.5 never yields -128). |t - rint(t)| is tracked; if any element
-// lies within 2^-14 of a half-integer the caller recomputes the vector with the
-// exact division (quant_code), so the result equals the binary32 decision.
+// lies within 2^-14 of a half-integer the caller patches those elements with
+// quant8_slow, so the result equals the binary32 decision.
 __device__ __forceinline__ uint2 quant8_fast(uint4 v, float rcp, float& worst) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
   const float2 r2 = make_float2(rcp, rcp), M2 = make_float2(12582912.0f, 12582912.0f);
@@ -84,20 +84,62 @@ __device__ __forceinline__ uint2 quant8_fast(uint4 v, float rcp, float& worst) {
   const uint32_t hi = __byte_perm(__byte_perm(b[4], b[5], 0x0040), __byte_perm(b[6], b[7], 0x0040), 0x5410);
   return make_uint2(lo, hi);
 }
-__device__ __forceinline__ uint32_t pack4_i8(int a, int b, int c, int d);
-__device__ __noinline__ uint2 quant8_exact(uint4 v, float scale, float absmax) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-  int c[8];
-#pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    c[2 * e] = quant_code(__uint_as_float(w[e] << 16), scale, absmax);
-    c[2 * e + 1] = quant_code(__uint_as_float(w[e] & 0xFFFF0000u), scale, absmax);
-  }
-  return make_uint2(pack4_i8(c[0], c[1], c[2], c[3]), pack4_i8(c[4], c[5], c[6], c[7]));
-}
 __device__ __forceinline__ uint32_t pack4_i8(int a, int b, int c, int d) {
   return (uint32_t)(a & 0xFF) | ((uint32_t)(b & 0xFF) << 8) | ((uint32_t)(c & 0xFF) << 16) |
          ((uint32_t)(d & 0xFF) << 24);
+}
+// Scales below this take the division for every element (quant8_slow); at or
+// above it RN(1/scale) is finite and every quantity below is a normal number.
+constexpr float kMinFastScale = 0x1p-100f;
+// The codes of a vector whose fast path saw a near tie, patched element by
+// element. On bf16 rows a few elements in a thousand have v * RN(1/scale) within
+// 2^-14 of a half-integer (bf16 values over a bf16 absmax put many quotients on
+// or next to one), so only those elements are decided again, without a
+// division: with h the half-integer next to t and r = v - h * scale,
+//   r is exact in binary32 (one fma): v and h * scale are multiples of
+//     ulp(scale) / 2, and |r| < 2^-13 scale needs fewer than 13 bits of them;
+//   RN(v / scale) == h exactly when |r| <= scale * ulp(h) / 2 (h has at most 9
+//     significant bits, so a quotient midway to h's neighbour rounds to h; the
+//     smaller spacing just below |h| = 0.5 changes no code), and then the code
+//     is the even integer next to h (rint(h));
+//   otherwise the code is h + 0.5 when r > 0 and h - 0.5 when r < 0.
+// A zero, subnormal or tiny scale (the whole row) takes the division itself.
+__device__ __noinline__ uint2 quant8_slow(uint4 v, float scale, float rcp, float absmax, uint2 code) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  if (!(scale >= kMinFastScale)) {
+    int c[8];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      c[2 * e] = quant_code(bf16_lo(w[e]), scale, absmax);
+      c[2 * e + 1] = quant_code(bf16_hi(w[e]), scale, absmax);
+    }
+    return make_uint2(pack4_i8(c[0], c[1], c[2], c[3]), pack4_i8(c[4], c[5], c[6], c[7]));
+  }
+  uint32_t word[2] = {code.x, code.y};
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const float x = (e & 1) ? bf16_hi(w[e >> 1]) : bf16_lo(w[e >> 1]);
+    const float t = x * rcp;
+    const float c0 = rintf(t);
+    const float dd = t - c0;
+    if (fabsf(dd) > kTieGuard) {
+      const float h = c0 + copysignf(0.5f, dd);
+      const float r = fmaf(-h, scale, x);
+      const float us = __uint_as_float((__float_as_uint(h) & 0x7F800000u) - (24u << 23)) * scale;
+      const float c = fabsf(r) <= us ? rintf(h) : (r > 0.0f ? h + 0.5f : h - 0.5f);
+      const uint32_t byte = (uint32_t)max(-127, min(127, (int)c)) & 0xFFu;
+      const int k = e >> 2, sh = 8 * (e & 3);
+      word[k] = (word[k] & ~(0xFFu << sh)) | (byte << sh);
+    }
+  }
+  return make_uint2(word[0], word[1]);
+}
+// Eight codes of one bf16 vector, bit-identical to quant_code on each element.
+__device__ __forceinline__ uint2 quant8(uint4 v, float scale, float rcp, float absmax) {
+  float worst = scale >= kMinFastScale ? 0.0f : 1.0f;  // zero, tiny or NaN scale: the slow path decides
+  uint2 code = quant8_fast(v, rcp, worst);
+  if (worst > kTieGuard) code = quant8_slow(v, scale, rcp, absmax, code);
+  return code;
 }
 
 // ---------------------------------------------------------------------------
@@ -378,13 +420,7 @@ __global__ void __launch_bounds__(1024, 1) ln_mod_quant_kernel(
         uint2* qr = reinterpret_cast<uint2*>(q) + (size_t)row * vpr;
 #pragma unroll
         for (int i = 0; i < VPT; ++i) {
-          uint2 code;
-          float worst = 1.0f;
-          if (rcp < INFINITY) {
-            worst = 0.0f;
-            code = quant8_fast(v[i], rcp, worst);
-          }
-          if (worst > kTieGuard) code = quant8_exact(v[i], sc, amax);  // near-tie, zero or subnormal scale
+          const uint2 code = quant8(v[i], sc, rcp, amax);
           if (H3B_IDX_OK((long long)row * vpr + t + tpr * i, (long long)rows * vpr, &g_h3b_rowops_bounds))
             qr[t + tpr * i] = code;
         }
@@ -452,13 +488,7 @@ __global__ void __launch_bounds__(256) quant_rows_known_absmax_kernel(const __nv
         row_end += (unsigned)vpr;
       }
       const float2 sr = srow[r];
-      uint2 code;
-      float worst = 1.0f;
-      if (sr.y < INFINITY) {
-        worst = 0.0f;
-        code = quant8_fast(raw[u], sr.y, worst);
-      }
-      if (worst > kTieGuard) code = quant8_exact(raw[u], sr.x, samax[r]);  // near-tie, zero or subnormal scale
+      const uint2 code = quant8(raw[u], sr.x, sr.y, samax[r]);
       if (H3B_IDX_OK(base + k, (long long)rows * vpr, &g_h3b_rowops_bounds))
         reinterpret_cast<uint2*>(q)[base + k] = code;
     }
