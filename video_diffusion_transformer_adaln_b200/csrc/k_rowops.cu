@@ -61,11 +61,14 @@ __device__ __forceinline__ int quant_code_fast(float v, float scale, float rcp) 
   return max(-127, min(127, (int)c));
 }
 // Eight codes of one 16-byte bf16 vector without a branch per element:
-// t = v * RN(1/scale); adding 1.5 * 2^23 rounds t to the nearest integer
-// (ties to even) in the low mantissa bits, whose low byte is the int8 code
-// (|t| <= 127.5 never yields -128). |t - rint(t)| is tracked; if any element
-// lies within 2^-14 of a half-integer the caller patches those elements with
-// quant8_slow, so the result equals the binary32 decision.
+// a = fma(v, RN(1/scale), 1.5 * 2^23) rounds the exact product p = v * RN(1/scale)
+// to the nearest integer c (ties to even) in the low mantissa bits, whose low
+// byte is the int8 code (|p| <= 127.5 never yields -128), and
+// dd = fma(v, RN(1/scale), -c) is p - c to within 2^-25. p differs from v / scale
+// by at most 127.5 * 2^-24 = 2^-17 and RN(v / scale) from v / scale by at most
+// 2^-18, so where |dd| <= 0.5 - 2^-14 the binary32 decision rint(RN(v / scale))
+// is c. The largest |dd| is tracked; if an element lies closer to a half-integer
+// the caller patches those elements with quant8_slow.
 __device__ __forceinline__ uint2 quant8_fast(uint4 v, float rcp, float& worst) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
   const float2 r2 = make_float2(rcp, rcp), M2 = make_float2(12582912.0f, 12582912.0f);
@@ -73,9 +76,10 @@ __device__ __forceinline__ uint2 quant8_fast(uint4 v, float rcp, float& worst) {
   uint32_t b[8];
 #pragma unroll
   for (int e = 0; e < 4; ++e) {
-    const float2 t = __fmul2_rn(make_float2(__uint_as_float(w[e] << 16), __uint_as_float(w[e] & 0xFFFF0000u)), r2);
-    const float2 a = __fadd2_rn(t, M2);
-    const float2 dd = __ffma2_rn(__fadd2_rn(a, nM2), make_float2(-1.0f, -1.0f), t);  // t - rint(t), exact
+    const float2 x = make_float2(__uint_as_float(w[e] << 16), __uint_as_float(w[e] & 0xFFFF0000u));
+    const float2 a = __ffma2_rn(x, r2, M2);
+    const float2 c = __fadd2_rn(a, nM2);  // exact
+    const float2 dd = __ffma2_rn(x, r2, make_float2(-c.x, -c.y));
     worst = fmaxf(worst, fmaxf(fabsf(dd.x), fabsf(dd.y)));
     b[2 * e] = __float_as_uint(a.x);
     b[2 * e + 1] = __float_as_uint(a.y);
@@ -97,7 +101,8 @@ constexpr float kMinFastScale = 0x1p-100f;
 // or next to one), so only those elements are decided again, without a
 // division: with h the half-integer next to t and r = v - h * scale,
 //   r is exact in binary32 (one fma): v and h * scale are multiples of
-//     ulp(scale) / 2, and |r| < 2^-13 scale needs fewer than 13 bits of them;
+//     ulp(scale) / 2, and |r| < 2^-13 scale (|v / scale - h| < 2^-14 + 2^-17)
+//     needs fewer than 13 bits of them;
 //   RN(v / scale) == h exactly when |r| <= scale * ulp(h) / 2 (h has at most 9
 //     significant bits, so a quotient midway to h's neighbour rounds to h; the
 //     smaller spacing just below |h| = 0.5 changes no code), and then the code
@@ -119,9 +124,8 @@ __device__ __noinline__ uint2 quant8_slow(uint4 v, float scale, float rcp, float
 #pragma unroll
   for (int e = 0; e < 8; ++e) {
     const float x = (e & 1) ? bf16_hi(w[e >> 1]) : bf16_lo(w[e >> 1]);
-    const float t = x * rcp;
-    const float c0 = rintf(t);
-    const float dd = t - c0;
+    const float c0 = fmaf(x, rcp, 12582912.0f) - 12582912.0f;  // as quant8_fast
+    const float dd = fmaf(x, rcp, -c0);
     if (fabsf(dd) > kTieGuard) {
       const float h = c0 + copysignf(0.5f, dd);
       const float r = fmaf(-h, scale, x);
@@ -281,9 +285,18 @@ __device__ __forceinline__ uint32_t bf16x2_max(uint32_t a, uint32_t b) {
   return r;
 }
 
-template <int VPT>
+// Threads per block of the LN quantizer: the row's tpr threads, times as many
+// rows as fit in 512 threads (or one row of up to 1024 threads).
+__host__ __device__ constexpr int ln_block(int vpr, int vpt) {
+  return vpr / vpt >= 512 ? vpr / vpt : (512 / (vpr / vpt)) * (vpr / vpt);
+}
+
+// VPT vectors per thread; NV > 0 fixes the row at 32 NV vectors (d = 256 NV) at
+// compile time, so that strides and the block shape are constants; NV = 0 takes
+// the row length from vpr_arg.
+template <int VPT, int NV>
 __global__ void __launch_bounds__(1024, 1) ln_mod_quant_kernel(
-    const __nv_bfloat16* __restrict__ x, int rows, int vpr, float eps, const float* __restrict__ shift,
+    const __nv_bfloat16* __restrict__ x, int rows, int vpr_arg, float eps, const float* __restrict__ shift,
     const float* __restrict__ scale, int rows_per_item, int mod_stride, int8_t* __restrict__ q,
     float* __restrict__ s, __nv_bfloat16* __restrict__ h_out, float* __restrict__ absmax_zero,
     int write_codes) {
@@ -291,8 +304,10 @@ __global__ void __launch_bounds__(1024, 1) ln_mod_quant_kernel(
   // then the staging rows of the next pass: [rpp][vpr] 16-byte vectors, each written and read
   // back by the same thread (cp.async), so no barrier guards them
   __shared__ float red[2][3][kLnMaxWarps];
+  const int vpr = NV ? 32 * NV : vpr_arg;
+  const int nthreads = NV ? ln_block(32 * NV, VPT) : (int)blockDim.x;
   const int tpr = vpr / VPT;
-  const int rpp = blockDim.x / tpr;
+  const int rpp = nthreads / tpr;
   const int sub = threadIdx.x / tpr;
   const int t = threadIdx.x - sub * tpr;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -326,7 +341,7 @@ __global__ void __launch_bounds__(1024, 1) ln_mod_quant_kernel(
       __syncthreads();
       const float2* sc2 = reinterpret_cast<const float2*>(scale + (size_t)item * mod_stride);
       const float2* sh2 = reinterpret_cast<const float2*>(shift + (size_t)item * mod_stride);
-      for (int c = threadIdx.x; c < 4 * vpr; c += blockDim.x) {
+      for (int c = threadIdx.x; c < 4 * vpr; c += nthreads) {
         const float2 a = __ldg(sc2 + c), b = __ldg(sh2 + c);
         modp[(c & 3) * vpr + (c >> 2)] = make_float4(1.0f + a.x, 1.0f + a.y, b.x, b.y);
       }
@@ -353,9 +368,11 @@ __global__ void __launch_bounds__(1024, 1) ln_mod_quant_kernel(
       f[4 * i + 3] = bf16x2_to_f2(v[i].w);
     }
     // the staged vectors are in registers now: start the next pass's loads
-    unsigned n_in = g_in + gridDim.x;
-    const unsigned n_item = item + n_in / gpi;
-    n_in %= gpi;
+    unsigned n_in = g_in + gridDim.x, n_item = item;
+    while (n_in >= gpi) {  // (item, pass within item) of the next pass, without a division
+      n_in -= gpi;
+      ++n_item;
+    }
     prefetch(g + gridDim.x, n_item, n_in);
     cp_async_commit();
     float2 acc = f[0];
@@ -435,17 +452,18 @@ __global__ void __launch_bounds__(1024, 1) ln_mod_quant_kernel(
 // Per-row quantization with each row's absmax already known: a block covers
 // whole rows (rpb rows of vpr 16-byte vectors, rpb * vpr <= 4096 unless one row
 // is longer, rpb <= 32). Each thread walks the block's vectors in rounds of
-// four, with the next round's loads issued before the current round is
-// quantized (the first round's before the scales are derived), so eight
-// vectors per thread are in flight. Each row's scale and its reciprocal are
-// derived once, into shared memory.
+// four, loading the next round into the other of two register sets before it
+// quantizes the current one (the first round's loads are issued before the
+// scales are derived), so eight vectors per thread are in flight. Each row's
+// scale and its reciprocal are derived once, into shared memory.
 constexpr int kQuantMaxRowsPerBlock = 32;
-__global__ void __launch_bounds__(256) quant_rows_known_absmax_kernel(const __nv_bfloat16* __restrict__ in,
-                                                                      int rows, int vpr, int rpb,
-                                                                      const float* __restrict__ absmax_in,
-                                                                      int8_t* __restrict__ q,
-                                                                      float* __restrict__ s) {
-  constexpr int U = 4;
+constexpr int kQuantThreads = 256;
+__global__ void __launch_bounds__(kQuantThreads, 4) quant_rows_known_absmax_kernel(const __nv_bfloat16* __restrict__ in,
+                                                                               int rows, int vpr, int rpb,
+                                                                               const float* __restrict__ absmax_in,
+                                                                               int8_t* __restrict__ q,
+                                                                               float* __restrict__ s) {
+  constexpr int U = 4, T = kQuantThreads;
   __shared__ float2 srow[kQuantMaxRowsPerBlock];  // (scale, RN(1/scale)) of the block's rows
   __shared__ float samax[kQuantMaxRowsPerBlock];
   const unsigned row0 = blockIdx.x * (unsigned)rpb;
@@ -453,17 +471,18 @@ __global__ void __launch_bounds__(256) quant_rows_known_absmax_kernel(const __nv
   const unsigned span = nr * (unsigned)vpr;  // vectors covered by this block
   const size_t base = (size_t)row0 * vpr;
   const uint4* src = reinterpret_cast<const uint4*>(in) + base;
-  uint4 nxt[U];
-  auto load_round = [&](unsigned k0) {
+  uint2* dst = reinterpret_cast<uint2*>(q) + base;
+  auto load_round = [&](unsigned k0, uint4(&buf)[U]) {
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      const unsigned k = k0 + u * blockDim.x;
-      nxt[u] = k < span && H3B_IDX_OK(base + k, (long long)rows * vpr, &g_h3b_rowops_bounds)
+      const unsigned k = k0 + u * T;
+      buf[u] = k < span && H3B_IDX_OK(base + k, (long long)rows * vpr, &g_h3b_rowops_bounds)
                    ? __ldcs(src + k)
                    : make_uint4(0, 0, 0, 0);
     }
   };
-  load_round(threadIdx.x);
+  uint4 ra[U], rb[U];
+  load_round(threadIdx.x, ra);
   if (threadIdx.x < nr) {
     const float amax = __ldg(absmax_in + row0 + threadIdx.x);
     const float sc = __fdiv_rn(amax, 127.0f);
@@ -474,24 +493,26 @@ __global__ void __launch_bounds__(256) quant_rows_known_absmax_kernel(const __nv
   __syncthreads();
   // row of vector k, advanced incrementally (k only grows): r = k / vpr without a division
   unsigned r = 0, row_end = (unsigned)vpr;
-  for (unsigned k0 = threadIdx.x; k0 < span; k0 += U * blockDim.x) {
-    uint4 raw[U];
-#pragma unroll
-    for (int u = 0; u < U; ++u) raw[u] = nxt[u];
-    load_round(k0 + U * blockDim.x);
+  auto quant_round = [&](unsigned k0, const uint4(&buf)[U]) {
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      const unsigned k = k0 + u * blockDim.x;
+      const unsigned k = k0 + u * T;
       if (k >= span) break;
       while (k >= row_end) {
         ++r;
         row_end += (unsigned)vpr;
       }
       const float2 sr = srow[r];
-      const uint2 code = quant8(raw[u], sr.x, sr.y, samax[r]);
-      if (H3B_IDX_OK(base + k, (long long)rows * vpr, &g_h3b_rowops_bounds))
-        reinterpret_cast<uint2*>(q)[base + k] = code;
+      const uint2 code = quant8(buf[u], sr.x, sr.y, samax[r]);
+      if (H3B_IDX_OK(base + k, (long long)rows * vpr, &g_h3b_rowops_bounds)) dst[k] = code;
     }
+  };
+  for (unsigned k0 = threadIdx.x; k0 < span; k0 += 2 * U * T) {
+    load_round(k0 + U * T, rb);
+    quant_round(k0, ra);
+    if (k0 + U * T >= span) break;
+    load_round(k0 + 2 * U * T, ra);
+    quant_round(k0 + U * T, rb);
   }
 }
 
@@ -762,16 +783,16 @@ cudaError_t launch_adaln_gemv(const void* W, const float* bias, const float* c, 
 // Threads per row: the fewest warps w dividing NV with NV / w <= 6 vectors per
 // thread; the block holds as many rows as fit in 512 threads (at least one), so
 // one copy of the modulation table serves more rows.
-template <int VPT>
+template <int VPT, int NV>
 static cudaError_t ln_dispatch(const void* x, int rows, int nv, float eps, const float* shift,
                                const float* scale, int rpi, int ms, int8_t* q, float* s, void* h,
                                float* az, int wc, int sms, cudaStream_t st) {
   const int vpr = 32 * nv;
   const int tpr = vpr / VPT;
-  const int block = tpr * (tpr >= 512 ? 1 : 512 / tpr);
+  const int block = ln_block(vpr, VPT);
   const int rpp_d = block / tpr;
   const size_t smem = (size_t)vpr * 4 * sizeof(float4) + (size_t)rpp_d * vpr * sizeof(uint4);
-  auto kern = ln_mod_quant_kernel<VPT>;
+  auto kern = ln_mod_quant_kernel<VPT, NV>;
   // the attribute belongs to the current device, so it is set on every launch (a host-side call)
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -794,15 +815,19 @@ cudaError_t launch_ln_mod_quant(const void* x, int rows, int d, float eps, const
   if (rows == 0) return cudaSuccess;
   const int nv = d / 256;
   if (nv < 1 || nv > 32 || d % 256) return cudaErrorInvalidValue;
+  // the widths of the workloads get kernels with the row length built in
+  if (nv == 20) return ln_dispatch<5, 20>(x, rows, nv, eps, shift, scale, rows_per_item, mod_stride, q, s, h_out, absmax_zero, write_codes, sms, st);
+  if (nv == 8) return ln_dispatch<4, 8>(x, rows, nv, eps, shift, scale, rows_per_item, mod_stride, q, s, h_out, absmax_zero, write_codes, sms, st);
+  if (nv == 1) return ln_dispatch<1, 1>(x, rows, nv, eps, shift, scale, rows_per_item, mod_stride, q, s, h_out, absmax_zero, write_codes, sms, st);
   int w = 1;
   while (nv % w || nv / w > 6) ++w;
   switch (nv / w) {
-    case 1: return ln_dispatch<1>(x, rows, nv, eps, shift, scale, rows_per_item, mod_stride, q, s, h_out, absmax_zero, write_codes, sms, st);
-    case 2: return ln_dispatch<2>(x, rows, nv, eps, shift, scale, rows_per_item, mod_stride, q, s, h_out, absmax_zero, write_codes, sms, st);
-    case 3: return ln_dispatch<3>(x, rows, nv, eps, shift, scale, rows_per_item, mod_stride, q, s, h_out, absmax_zero, write_codes, sms, st);
-    case 4: return ln_dispatch<4>(x, rows, nv, eps, shift, scale, rows_per_item, mod_stride, q, s, h_out, absmax_zero, write_codes, sms, st);
-    case 5: return ln_dispatch<5>(x, rows, nv, eps, shift, scale, rows_per_item, mod_stride, q, s, h_out, absmax_zero, write_codes, sms, st);
-    case 6: return ln_dispatch<6>(x, rows, nv, eps, shift, scale, rows_per_item, mod_stride, q, s, h_out, absmax_zero, write_codes, sms, st);
+    case 1: return ln_dispatch<1, 0>(x, rows, nv, eps, shift, scale, rows_per_item, mod_stride, q, s, h_out, absmax_zero, write_codes, sms, st);
+    case 2: return ln_dispatch<2, 0>(x, rows, nv, eps, shift, scale, rows_per_item, mod_stride, q, s, h_out, absmax_zero, write_codes, sms, st);
+    case 3: return ln_dispatch<3, 0>(x, rows, nv, eps, shift, scale, rows_per_item, mod_stride, q, s, h_out, absmax_zero, write_codes, sms, st);
+    case 4: return ln_dispatch<4, 0>(x, rows, nv, eps, shift, scale, rows_per_item, mod_stride, q, s, h_out, absmax_zero, write_codes, sms, st);
+    case 5: return ln_dispatch<5, 0>(x, rows, nv, eps, shift, scale, rows_per_item, mod_stride, q, s, h_out, absmax_zero, write_codes, sms, st);
+    case 6: return ln_dispatch<6, 0>(x, rows, nv, eps, shift, scale, rows_per_item, mod_stride, q, s, h_out, absmax_zero, write_codes, sms, st);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -817,7 +842,7 @@ cudaError_t launch_quant_rows_bf16(const void* h, int rows, int cols, const floa
     int rpb = 4096 / vpr;
     rpb = std::min(rpb, rows / (4 * sms));  // but at least about four blocks per SM
     rpb = rpb < 1 ? 1 : (rpb > kQuantMaxRowsPerBlock ? kQuantMaxRowsPerBlock : rpb);
-    quant_rows_known_absmax_kernel<<<(rows + rpb - 1) / rpb, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(h),
+    quant_rows_known_absmax_kernel<<<(rows + rpb - 1) / rpb, kQuantThreads, 0, st>>>(static_cast<const __nv_bfloat16*>(h),
                                                                           rows, vpr, rpb, absmax, q, s);
     return cudaGetLastError();
   }
