@@ -647,7 +647,7 @@ def run_reference(args, rank, world, local):
 
 
 PROFILE_KERNELS = ("attention", "ln_mod_quant", "quant_o", "adaln_gemv", "token_pair", "token_unpair",
-                   "gemm_w1", "gemm_w2")
+                   "gemm_qkv", "gemm_wo", "gemm_w1", "gemm_w2")
 
 
 def run_profile_kernel(name, workload):
@@ -675,9 +675,18 @@ def run_profile_kernel(name, workload):
         else:
             am = x.float().abs().amax(dim=1).contiguous()
             fn = lambda: h3b.h3b_quantize_rows(x, q, s, absmax=am)  # noqa: E731
-    elif name in ("gemm_w1", "gemm_w2"):
-        # the MLP projections at the workload's shape: int8 codes of a random activation and weight
-        K, N = (d, wl.d_ff) if name == "gemm_w1" else (wl.d_ff, d)
+    elif name == "gemm_qkv":
+        # QKV + 3D RoPE, written head-major, from int8 codes of a random activation
+        blk = DeviceBlock.random_on_device(wl, g)
+        A = torch.randint(-127, 128, (B * L, d), generator=g, device="cuda", dtype=torch.int8)
+        sA = torch.rand(B * L, generator=g, device="cuda") * 0.01
+        qkv = torch.empty(3 * B * L * d, dtype=torch.bfloat16, device="cuda")
+        rope_ws = torch.empty(h3b.h3b_rope_table_bytes(dims), dtype=torch.uint8, device="cuda")
+        fn = lambda: h3b.h3b_qkv_projection(dims, A, sA, blk.struct, qkv, rope_ws)  # noqa: E731
+    elif name in ("gemm_wo", "gemm_w1", "gemm_w2"):
+        # the output and MLP projections at the workload's shape: int8 codes of a random
+        # activation and weight
+        K, N = {"gemm_wo": (d, d), "gemm_w1": (d, wl.d_ff), "gemm_w2": (wl.d_ff, d)}[name]
         A = torch.randint(-127, 128, (B * L, K), generator=g, device="cuda", dtype=torch.int8)
         Wq = torch.randint(-127, 128, (N, K), generator=g, device="cuda", dtype=torch.int8)
         sA = torch.rand(B * L, generator=g, device="cuda") * 0.01

@@ -67,9 +67,9 @@ __device__ __forceinline__ int quant_code_fast(float v, float scale, float rcp) 
 // dd = fma(v, RN(1/scale), -c) is p - c to within 2^-25. p differs from v / scale
 // by at most 127.5 * 2^-24 = 2^-17 and RN(v / scale) from v / scale by at most
 // 2^-18, so where |dd| <= 0.5 - 2^-14 the binary32 decision rint(RN(v / scale))
-// is c. The largest |dd| is tracked; if an element lies closer to a half-integer
-// the caller patches those elements with quant8_slow.
-__device__ __forceinline__ uint2 quant8_fast(uint4 v, float rcp, float& worst) {
+// is c. The largest |dd| is tracked and the dd are returned; if an element lies
+// closer to a half-integer the caller patches those elements with quant8_slow.
+__device__ __forceinline__ uint2 quant8_fast(uint4 v, float rcp, float& worst, float2 (&dds)[4]) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
   const float2 r2 = make_float2(rcp, rcp), M2 = make_float2(12582912.0f, 12582912.0f);
   const float2 nM2 = make_float2(-12582912.0f, -12582912.0f);
@@ -81,6 +81,7 @@ __device__ __forceinline__ uint2 quant8_fast(uint4 v, float rcp, float& worst) {
     const float2 c = __fadd2_rn(a, nM2);  // exact
     const float2 dd = __ffma2_rn(x, r2, make_float2(-c.x, -c.y));
     worst = fmaxf(worst, fmaxf(fabsf(dd.x), fabsf(dd.y)));
+    dds[e] = dd;
     b[2 * e] = __float_as_uint(a.x);
     b[2 * e + 1] = __float_as_uint(a.y);
   }
@@ -98,8 +99,9 @@ constexpr float kMinFastScale = 0x1p-100f;
 // The codes of a vector whose fast path saw a near tie, patched element by
 // element. On bf16 rows a few elements in a thousand have v * RN(1/scale) within
 // 2^-14 of a half-integer (bf16 values over a bf16 absmax put many quotients on
-// or next to one), so only those elements are decided again, without a
-// division: with h the half-integer next to t and r = v - h * scale,
+// or next to one, most of them exactly), so only those elements, found from the
+// fast path's distances dd, are decided again, without a division: with h the
+// half-integer next to the product and r = v - h * scale,
 //   r is exact in binary32 (one fma): v and h * scale are multiples of
 //     ulp(scale) / 2, and |r| < 2^-13 scale (|v / scale - h| < 2^-14 + 2^-17)
 //     needs fewer than 13 bits of them;
@@ -109,7 +111,11 @@ constexpr float kMinFastScale = 0x1p-100f;
 //     is the even integer next to h (rint(h));
 //   otherwise the code is h + 0.5 when r > 0 and h - 0.5 when r < 0.
 // A zero, subnormal or tiny scale (the whole row) takes the division itself.
-__device__ __noinline__ uint2 quant8_slow(uint4 v, float scale, float rcp, float absmax, uint2 code) {
+// kGivenDd: the fast path's dd are passed in (d0..d3); otherwise they are
+// recomputed here, which keeps the caller's live registers down.
+template <bool kGivenDd>
+__device__ __noinline__ uint2 quant8_slow(uint4 v, float scale, float rcp, float absmax, uint2 code, float2 d0,
+                                         float2 d1, float2 d2, float2 d3) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
   if (!(scale >= kMinFastScale)) {
     int c[8];
@@ -121,11 +127,12 @@ __device__ __noinline__ uint2 quant8_slow(uint4 v, float scale, float rcp, float
     return make_uint2(pack4_i8(c[0], c[1], c[2], c[3]), pack4_i8(c[4], c[5], c[6], c[7]));
   }
   uint32_t word[2] = {code.x, code.y};
+  const float given[8] = {d0.x, d0.y, d1.x, d1.y, d2.x, d2.y, d3.x, d3.y};
 #pragma unroll
   for (int e = 0; e < 8; ++e) {
     const float x = (e & 1) ? bf16_hi(w[e >> 1]) : bf16_lo(w[e >> 1]);
     const float c0 = fmaf(x, rcp, 12582912.0f) - 12582912.0f;  // as quant8_fast
-    const float dd = fmaf(x, rcp, -c0);
+    const float dd = kGivenDd ? given[e] : fmaf(x, rcp, -c0);
     if (fabsf(dd) > kTieGuard) {
       const float h = c0 + copysignf(0.5f, dd);
       const float r = fmaf(-h, scale, x);
@@ -139,10 +146,12 @@ __device__ __noinline__ uint2 quant8_slow(uint4 v, float scale, float rcp, float
   return make_uint2(word[0], word[1]);
 }
 // Eight codes of one bf16 vector, bit-identical to quant_code on each element.
+template <bool kGivenDd>
 __device__ __forceinline__ uint2 quant8(uint4 v, float scale, float rcp, float absmax) {
   float worst = scale >= kMinFastScale ? 0.0f : 1.0f;  // zero, tiny or NaN scale: the slow path decides
-  uint2 code = quant8_fast(v, rcp, worst);
-  if (worst > kTieGuard) code = quant8_slow(v, scale, rcp, absmax, code);
+  float2 dd[4];
+  uint2 code = quant8_fast(v, rcp, worst, dd);
+  if (worst > kTieGuard) code = quant8_slow<kGivenDd>(v, scale, rcp, absmax, code, dd[0], dd[1], dd[2], dd[3]);
   return code;
 }
 
@@ -437,7 +446,7 @@ __global__ void __launch_bounds__(1024, 1) ln_mod_quant_kernel(
         uint2* qr = reinterpret_cast<uint2*>(q) + (size_t)row * vpr;
 #pragma unroll
         for (int i = 0; i < VPT; ++i) {
-          const uint2 code = quant8(v[i], sc, rcp, amax);
+          const uint2 code = quant8<true>(v[i], sc, rcp, amax);
           if (H3B_IDX_OK((long long)row * vpr + t + tpr * i, (long long)rows * vpr, &g_h3b_rowops_bounds))
             qr[t + tpr * i] = code;
         }
@@ -503,7 +512,7 @@ __global__ void __launch_bounds__(kQuantThreads, 4) quant_rows_known_absmax_kern
         row_end += (unsigned)vpr;
       }
       const float2 sr = srow[r];
-      const uint2 code = quant8(buf[u], sr.x, sr.y, samax[r]);
+      const uint2 code = quant8<false>(buf[u], sr.x, sr.y, samax[r]);
       if (H3B_IDX_OK(base + k, (long long)rows * vpr, &g_h3b_rowops_bounds)) dst[k] = code;
     }
   };
