@@ -34,11 +34,16 @@ constexpr int BM = 128, BN = 256, BKB = 128, STAGES = 4;
 constexpr int A_BYTES = BM * BKB;
 constexpr int B_BYTES = BN * BKB;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+// CTA pairs: per CTA and stage its 128 rows of A and its 128 of the tile's 256 B
+// rows, six stages in the same shared memory as the single-CTA ring
+constexpr int PAIR_STAGES = 6;
+constexpr int PAIR_STAGE_BYTES = 2 * BM * BKB;
+static_assert(PAIR_STAGES * PAIR_STAGE_BYTES == STAGES * STAGE_BYTES, "same shared-memory layout");
 constexpr int kEpiWarps = 8;  // two per sub-partition, each half of the tile's columns
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr size_t kL2Budget = 48ull << 20;  // operand bytes the raster keeps resident in L2
 constexpr uint32_t TMEM_COLS = 512;
-constexpr int kBars = 2 * STAGES + 4 + 1;
+constexpr int kBars = 2 * PAIR_STAGES + 4 + 1;  // enough for either ring
 constexpr size_t CONST_OFF = (size_t)STAGES * STAGE_BYTES + 256;     // per-warp epilogue constants
 constexpr size_t ROPE_OFF = CONST_OFF + kEpiWarps * 3 * 128 * 4;     // RoPE table, when it fits
 constexpr size_t SMEM_BASE = ROPE_OFF + 1024;                         // + 1024 for the alignment slack
@@ -277,14 +282,24 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, uint32_t tbase,
     atomicMax(reinterpret_cast<unsigned*>(p.absmax) + row, __float_as_uint(amax));
 }
 
-template <bool kInt8, int kEpi>
+// kPair: the CTA is one of a pair (cluster of two) that computes 256 x 256
+// tiles: rank r takes rows [256 mb + 128 r, +128) of A and rows [256 nb + 128 r,
+// +128) of W into its shared memory, the even CTA issues every MMA for both
+// (M = 256, cta_group::2) and commits to both CTAs' barriers, and each CTA's
+// epilogue drains its own 128 x 256 accumulator. The stage's bytes of both CTAs
+// complete on the even CTA's full barrier; both CTAs' epilogues release an
+// accumulator on the even CTA's tempty barrier.
+template <bool kInt8, int kEpi, bool kPair>
 __global__ void __launch_bounds__(gemm::kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const GemmArgs p) {
   using namespace gemm;
+  constexpr int NS = kPair ? PAIR_STAGES : STAGES;
+  constexpr int SB = kPair ? PAIR_STAGE_BYTES : STAGE_BYTES;
+  constexpr int MT = kPair ? 2 * BM : BM;  // tile rows
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + NS * SB);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kBars);
   EpiConst* epi_const = reinterpret_cast<EpiConst*>(smem + CONST_OFF);
   float2* rope_smem = reinterpret_cast<float2*>(smem + ROPE_OFF);
@@ -292,21 +307,34 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
   const uint32_t sbase = smem_u32(smem);
   const uint32_t bar0 = smem_u32(bars);
   auto full = [&](int s) { return bar0 + 8u * s; };
-  auto empty = [&](int s) { return bar0 + 8u * (STAGES + s); };
-  auto tfull = [&](int a) { return bar0 + 8u * (2 * STAGES + a); };
-  auto tempty = [&](int a) { return bar0 + 8u * (2 * STAGES + 2 + a); };
-  const uint32_t drain = bar0 + 8u * (2 * STAGES + 4);
+  auto empty = [&](int s) { return bar0 + 8u * (NS + s); };
+  auto tfull = [&](int a) { return bar0 + 8u * (2 * NS + a); };
+  auto tempty = [&](int a) { return bar0 + 8u * (2 * NS + 2 + a); };
+  const uint32_t drain = bar0 + 8u * (2 * NS + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n_m = (p.M + BM - 1) / BM, n_n = (p.N + BN - 1) / BN;
+  const uint32_t rank = kPair ? cluster_ctarank() : 0u;
+  const bool leader = rank == 0;
+  // an abort in either CTA of a pair ends the waits of both
+  auto set_abort = [&]() {
+    *abort_flag = 1;
+    if (kPair) {
+      const uint32_t peer = mapa_shared(smem_u32((const void*)abort_flag), rank ^ 1u);
+      asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(peer), "r"(1) : "memory");
+    }
+  };
+  const int unit = kPair ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;  // pair or CTA
+  const int units = kPair ? (int)(gridDim.x >> 1) : (int)gridDim.x;
+  const int n_m = (p.M + MT - 1) / MT, n_n = (p.N + BN - 1) / BN;
   const int n_tiles = n_m * n_n;
   constexpr int BKE = kInt8 ? BKB : BKB / 2;  // K elements per stage
   const int nk = (p.K + BKE - 1) / BKE;
-  constexpr uint32_t IDESC = kInt8 ? instr_desc(2, 1, 0, 0, BM, BN) : instr_desc(1, 1, 0, 0, BM, BN);
+  constexpr uint32_t IDESC = kInt8 ? instr_desc(2, 1, 0, 0, MT, BN) : instr_desc(1, 1, 0, 0, MT, BN);
+  constexpr uint32_t B_ROWS = kPair ? BN / 2 : BN;  // W rows of a stage in this CTA
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) { mbar_init(full(s), 1); mbar_init(empty(s), 1); }
-    for (int a = 0; a < 2; ++a) { mbar_init(tfull(a), 1); mbar_init(tempty(a), kEpiWarps); }
+    for (int s = 0; s < NS; ++s) { mbar_init(full(s), 1); mbar_init(empty(s), 1); }
+    for (int a = 0; a < 2; ++a) { mbar_init(tfull(a), 1); mbar_init(tempty(a), (kPair ? 2 : 1) * kEpiWarps); }
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -315,54 +343,68 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
   if (kEpi == EPI_QKV)  // the whole RoPE table, once per CTA, when the launcher reserved room for it
     for (int i = threadIdx.x; i < p.rope_smem_entries; i += blockDim.x) rope_smem[i] = __ldg(p.rope + i);
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
-    tmem_relinquish();
+    if (kPair) {
+      tmem_alloc_pair(smem_u32(tmem_slot), TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+      tmem_relinquish();
+    }
     tc_fence_before();
   }
   __syncthreads();
+  if (kPair) cluster_sync_all();  // both CTAs' barriers exist before any remote arrival
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
   if (warp == 0) {
     if (lane == 0) {
-      // ---------------- TMA producer
+      // ---------------- TMA producer (in both CTAs of a pair)
       int s = 0;
       uint32_t ph = 0;
       uint32_t issued = 0, issued_ph = 0;  // per-stage bitmask of the last issued phase
       bool ok = true;
-      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
+      for (int t = unit; t < n_tiles && ok; t += units) {
         int mb, nb;
         tile_coords(t, n_m, n_n, p.raster_n, p.group, mb, nb);
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait_or_abort(empty(s), ph ^ 1u, abort_flag, p.err, ERR_WAIT_MMA)) { ok = false; break; }
-          mbar_arrive_expect_tx(full(s), STAGE_BYTES);
-          const uint32_t a_dst = sbase + s * STAGE_BYTES;
-          tma_load_2d(a_dst, &tmA, full(s), kb * BKE, mb * BM);
-          tma_load_2d(a_dst + A_BYTES, &tmB, full(s), kb * BKE, nb * BN);
+          const uint32_t a_dst = sbase + s * SB;
+          if (kPair) {
+            if (leader) mbar_arrive_expect_tx(full(s), 2 * SB);
+            const uint32_t fb = mapa_shared(full(s), 0);
+            tma_load_2d_pair(a_dst, &tmA, fb, kb * BKE, mb * MT + (int)rank * BM);
+            tma_load_2d_pair(a_dst + A_BYTES, &tmB, fb, kb * BKE, nb * BN + (int)rank * (int)B_ROWS);
+          } else {
+            mbar_arrive_expect_tx(full(s), SB);
+            tma_load_2d(a_dst, &tmA, full(s), kb * BKE, mb * MT);
+            tma_load_2d(a_dst + A_BYTES, &tmB, full(s), kb * BKE, nb * BN);
+          }
           issued |= 1u << s;
           issued_ph = (issued_ph & ~(1u << s)) | (ph << s);
-          if (++s == STAGES) { s = 0; ph ^= 1u; }
+          if (++s == NS) { s = 0; ph ^= 1u; }
         }
       }
       if (!ok) {
-        *abort_flag = 1;
-        for (int i = 0; i < STAGES; ++i)  // let in-flight tiles land before the CTA exits
-          if (issued & (1u << i)) mbar_wait(full(i), (issued_ph >> i) & 1u, p.err, ERR_WAIT_DRAIN, kDrainLimitNs);
+        set_abort();
+        if (leader)  // let in-flight tiles land before the CTA exits (a pair's full barriers count both CTAs)
+          for (int i = 0; i < NS; ++i)
+            if (issued & (1u << i)) mbar_wait(full(i), (issued_ph >> i) & 1u, p.err, ERR_WAIT_DRAIN, kDrainLimitNs);
       } else {
         // tail: every filled stage has been consumed (its commit has arrived)
-        for (int i = 0; i < STAGES; ++i)
+        for (int i = 0; i < NS; ++i)
           if (issued & (1u << i)) mbar_wait(empty(i), (issued_ph >> i) & 1u, p.err, ERR_WAIT_MMA);
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      // ---------------- MMA issuer
+    if (lane == 0 && leader) {
+      // ---------------- MMA issuer (the even CTA of a pair issues for both)
       int s = 0;
       uint32_t ph = 0;
       int tl = 0;
       bool ok = true;
       bool any = false;
-      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++tl) {
+      for (int t = unit; t < n_tiles && ok; t += units, ++tl) {
         const int acc = tl & 1;
         const uint32_t aph = (tl >> 1) & 1;
         if (!mbar_wait_or_abort(tempty(acc), aph ^ 1u, abort_flag, p.err, ERR_WAIT_EPI)) { ok = false; break; }
@@ -371,25 +413,34 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait_or_abort(full(s), ph, abort_flag, p.err, ERR_WAIT_TMA)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t a_addr = sbase + s * STAGE_BYTES;
+          const uint32_t a_addr = sbase + s * SB;
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
             const uint64_t ad = smem_desc_sw128(a_addr + k * 32, 16, 1024);
             const uint64_t bd = smem_desc_sw128(a_addr + A_BYTES + k * 32, 16, 1024);
-            if (kInt8) mma_i8(d_tmem, ad, bd, IDESC, (kb | k) != 0);
-            else mma_f16(d_tmem, ad, bd, IDESC, (kb | k) != 0);
+            const uint32_t accum = (kb | k) != 0;
+            if (kPair) {
+              if (kInt8) mma_i8_pair(d_tmem, ad, bd, IDESC, accum);
+              else mma_f16_pair(d_tmem, ad, bd, IDESC, accum);
+            } else {
+              if (kInt8) mma_i8(d_tmem, ad, bd, IDESC, accum);
+              else mma_f16(d_tmem, ad, bd, IDESC, accum);
+            }
           }
           any = true;
-          tc_commit(empty(s));
-          if (++s == STAGES) { s = 0; ph ^= 1u; }
+          if (kPair) tc_commit_pair(empty(s));
+          else tc_commit(empty(s));
+          if (++s == NS) { s = 0; ph ^= 1u; }
         }
         if (!ok) break;
-        tc_commit(tfull(acc));
+        if (kPair) tc_commit_pair(tfull(acc));
+        else tc_commit(tfull(acc));
       }
       if (!ok) {
-        *abort_flag = 1;
+        set_abort();
         if (any) {  // wait for the MMAs already issued before TMEM is released
-          tc_commit(drain);
+          if (kPair) tc_commit_pair_local(drain);
+          else tc_commit(drain);
           mbar_wait(drain, 0, p.err, ERR_WAIT_DRAIN, kDrainLimitNs);
         }
       }
@@ -399,25 +450,31 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
     // 2-5 take columns [0, 128) of the tile, warps 6-9 columns [128, 256)
     const int quad = warp & 3;
     const int half = (warp - 2) >> 2;
+    const uint32_t tempty_leader0 = kPair ? mapa_shared(tempty(0), 0) : tempty(0);
+    const uint32_t tempty_leader1 = kPair ? mapa_shared(tempty(1), 0) : tempty(1);
     int tl = 0;
-    for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++tl) {
+    for (int t = unit; t < n_tiles; t += units, ++tl) {
       int mb, nb;
       tile_coords(t, n_m, n_n, p.raster_n, p.group, mb, nb);
       const int acc = tl & 1;
       const uint32_t aph = (tl >> 1) & 1;
-      const int row = mb * BM + quad * 32 + lane;
+      const int r0 = mb * MT + (int)rank * BM + quad * 32;  // this warp's first row
+      const int row = r0 + lane;
       const int n0 = nb * BN + half * (BN / 2);
       EpiConst& ec = epi_const[warp - 2];
       // this warp finished its previous tile, so its constants buffer is free
-      stage_constants<kInt8, kEpi>(p, ec, n0, mb * BM + quad * 32, lane);
-      const int first_row = min(mb * BM + quad * 32, p.M - 1), last_row = min(mb * BM + quad * 32 + 31, p.M - 1);
+      stage_constants<kInt8, kEpi>(p, ec, n0, r0, lane);
+      const int first_row = min(r0, p.M - 1), last_row = min(r0 + 31, p.M - 1);
       const bool gate_uniform = kEpi == EPI_RESID && first_row / p.rows_per_item == last_row / p.rows_per_item;
       uint4 xp[kResidVecs];
       if (kEpi == EPI_RESID) prefetch_resid(p, row, n0, xp);
       __syncwarp();
       // tcgen05.ld is warp-collective: the wait outcome is made warp-uniform.
       const bool t_ok = mbar_wait_or_abort(tfull(acc), aph, abort_flag, p.err, ERR_WAIT_MMA);
-      if (!__all_sync(0xFFFFFFFFu, t_ok)) { *abort_flag = 1; break; }
+      if (!__all_sync(0xFFFFFFFFu, t_ok)) {
+        if (lane == 0) set_abort();
+        break;
+      }
       tc_fence_after();
       // this warp's 32 lanes and 128 columns of the accumulator
       const uint32_t tbase = tmem_base + ((uint32_t)(quad * 32) << 16) + acc * BN + half * (BN / 2);
@@ -425,42 +482,81 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
                                  p.rope_smem_entries > 0 ? rope_smem : p.rope, xp);
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(tempty(acc));
+      if (lane == 0) {
+        if (kPair) mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);
+        else mbar_arrive(tempty(acc));
+      }
     }
   }
   __syncthreads();
+  if (kPair) cluster_sync_all();  // the pair's MMAs and remote arrivals are over before TMEM goes
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_base, TMEM_COLS);
+    if (kPair) tmem_dealloc_pair(tmem_base, TMEM_COLS);
+    else tmem_dealloc(tmem_base, TMEM_COLS);
   }
 }
 
-template <bool kInt8, int kEpi>
+template <bool kInt8, int kEpi, bool kPair>
 static cudaError_t launch_one(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& a,
                               int grid, cudaStream_t st) {
-  auto k = gemm_kernel<kInt8, kEpi>;
+  auto k = gemm_kernel<kInt8, kEpi, kPair>;
   const size_t smem = gemm::SMEM_BASE + (size_t)a.rope_smem_entries * sizeof(float2);
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gemm::kSmemMax);
   if (e != cudaSuccess) return e;
-  k<<<grid, gemm::kThreads, smem, st>>>(ta, tb, a);
-  return cudaGetLastError();
+  if (!kPair) {
+    k<<<grid, gemm::kThreads, smem, st>>>(ta, tb, a);
+    return cudaGetLastError();
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid, 1, 1);
+  cfg.blockDim = dim3(gemm::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  // persistent pairs: no more than can be resident at once
+  int clusters = 0;
+  e = cudaOccupancyMaxActiveClusters(&clusters, k, &cfg);
+  if (e != cudaSuccess) return e;
+  if (clusters < 1) return cudaErrorInvalidConfiguration;
+  if ((int)cfg.gridDim.x > 2 * clusters) cfg.gridDim.x = 2u * (unsigned)clusters;
+  return cudaLaunchKernelEx(&cfg, k, ta, tb, a);
+}
+
+// The GEMMs run on CTA pairs (256 x 256 tiles, half of every W tile per SM) when
+// the GPU has at least two SMs and the problem at least one pair tile.
+constexpr bool kUsePairs = true;
+
+template <bool kInt8, int kEpi>
+static cudaError_t launch_epi(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& a, bool pair,
+                              int grid, cudaStream_t st) {
+  return pair ? launch_one<kInt8, kEpi, true>(ta, tb, a, grid, st) : launch_one<kInt8, kEpi, false>(ta, tb, a, grid, st);
 }
 
 cudaError_t launch_gemm(bool int8_operands, GemmEpilogue epi, const void* A, const void* W,
                         const GemmArgs& a, int sms, cudaStream_t st) {
   using namespace gemm;
   if (a.M == 0) return cudaSuccess;
+  const bool pair = kUsePairs && sms >= 2;
+  const int MT = pair ? 2 * BM : BM;
   const int eb = int8_operands ? 1 : 2;
   const uint32_t bke = int8_operands ? BKB : BKB / 2;
   CUtensorMap ta, tb;
   if (!make_tmap_2d(&ta, A, eb, (uint64_t)a.K, (uint64_t)a.M, (uint64_t)a.K * eb, bke, BM))
     return cudaErrorInvalidValue;
-  if (!make_tmap_2d(&tb, W, eb, (uint64_t)a.K, (uint64_t)a.N, (uint64_t)a.K * eb, bke, BN))
+  if (!make_tmap_2d(&tb, W, eb, (uint64_t)a.K, (uint64_t)a.N, (uint64_t)a.K * eb, bke, pair ? BN / 2 : BN))
     return cudaErrorInvalidValue;
-  const int n_m = (a.M + BM - 1) / BM, n_n = (a.N + BN - 1) / BN;
+  const int n_m = (a.M + MT - 1) / MT, n_n = (a.N + BN - 1) / BN;
   const int n_tiles = n_m * n_n;
-  const int grid = n_tiles < sms ? n_tiles : sms;
+  const int units = pair ? sms / 2 : sms;  // persistent pairs or CTAs
+  const int grid = (n_tiles < units ? n_tiles : units) * (pair ? 2 : 1);
   // Raster: keep either a band of A stripes or a band of W slices resident in L2,
   // whichever makes the other operand's repeated streaming cheaper.
   GemmArgs args = a;
@@ -470,7 +566,7 @@ cudaError_t launch_gemm(bool int8_operands, GemmEpilogue epi, const void* A, con
     if (entries <= kRopeSmemMaxEntries) args.rope_smem_entries = entries;
   }
   {
-    const double stripe_a = (double)BM * a.K * eb, slice_w = (double)BN * a.K * eb;
+    const double stripe_a = (double)MT * a.K * eb, slice_w = (double)BN * a.K * eb;
     const double bytes_a = (double)a.M * a.K * eb, bytes_w = (double)a.N * a.K * eb;
     int gm = (int)(kL2Budget / stripe_a), gn = (int)(kL2Budget / slice_w);
     gm = gm < 1 ? 1 : (gm > n_m ? n_m : gm);
@@ -482,17 +578,17 @@ cudaError_t launch_gemm(bool int8_operands, GemmEpilogue epi, const void* A, con
   }
   if (int8_operands) {
     switch (epi) {
-      case EPI_S32: return launch_one<true, EPI_S32>(ta, tb, args, grid, st);
-      case EPI_DEQ: return launch_one<true, EPI_DEQ>(ta, tb, args, grid, st);
-      case EPI_QKV: return launch_one<true, EPI_QKV>(ta, tb, args, grid, st);
-      case EPI_RESID: return launch_one<true, EPI_RESID>(ta, tb, args, grid, st);
-      case EPI_GELU: return launch_one<true, EPI_GELU>(ta, tb, args, grid, st);
+      case EPI_S32: return launch_epi<true, EPI_S32>(ta, tb, args, pair, grid, st);
+      case EPI_DEQ: return launch_epi<true, EPI_DEQ>(ta, tb, args, pair, grid, st);
+      case EPI_QKV: return launch_epi<true, EPI_QKV>(ta, tb, args, pair, grid, st);
+      case EPI_RESID: return launch_epi<true, EPI_RESID>(ta, tb, args, pair, grid, st);
+      case EPI_GELU: return launch_epi<true, EPI_GELU>(ta, tb, args, pair, grid, st);
     }
   } else {
     switch (epi) {
-      case EPI_DEQ: return launch_one<false, EPI_DEQ>(ta, tb, args, grid, st);
-      case EPI_QKV: return launch_one<false, EPI_QKV>(ta, tb, args, grid, st);
-      case EPI_RESID: return launch_one<false, EPI_RESID>(ta, tb, args, grid, st);
+      case EPI_DEQ: return launch_epi<false, EPI_DEQ>(ta, tb, args, pair, grid, st);
+      case EPI_QKV: return launch_epi<false, EPI_QKV>(ta, tb, args, pair, grid, st);
+      case EPI_RESID: return launch_epi<false, EPI_RESID>(ta, tb, args, pair, grid, st);
       default: break;
     }
   }
