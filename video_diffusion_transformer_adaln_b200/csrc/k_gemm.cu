@@ -14,10 +14,14 @@
 //   "h3.c與MLX路線對比：MiniMax-H3在Apple Silicon上的兩種推理實現工程取捨",
 //     section "性能上限" (RoPE folded into the kernel of the projections).
 //
-// Design (B200): persistent kernel, one 128x256 output tile at a time per CTA,
-// tiles rastered in L2-sized groups (a band of A stripes or of W slices stays
-// resident). Warp 0 streams A/B tiles with TMA (128-byte swizzle) into a
-// 4-stage shared-memory ring; warp 1 issues tcgen05.mma from one thread into a
+// Design (B200): persistent kernel on CTA pairs (clusters of two), one 256x256
+// output tile at a time per pair, tiles rastered in L2-sized groups (a band of
+// A stripes or of W slices stays resident). In each CTA warp 0 streams its 128
+// rows of A and its 128 of the tile's 256 W rows with TMA (128-byte swizzle)
+// into a 6-stage shared-memory ring, so that an SM pulls 32 KB per K step
+// instead of the 48 KB of a one-CTA 128x256 tile (the L2-to-shared-memory feed
+// bounded that one near 78% of the MMA rate); warp 1 of the even CTA issues
+// tcgen05.mma (cta_group::2, M = 256) from one thread into each CTA's
 // double-buffered TMEM accumulator (2 x 256 columns); warps 2-9 (two per
 // sub-partition, each half of the columns) drain the other accumulator
 // (tcgen05.ld) and run the epilogue while the next tile's MMAs proceed: each
