@@ -45,7 +45,7 @@ constexpr int PAIR_STAGE_BYTES = 2 * BM * BKB;
 static_assert(PAIR_STAGES * PAIR_STAGE_BYTES == STAGES * STAGE_BYTES, "same shared-memory layout");
 constexpr int kEpiWarps = 8;  // two per sub-partition, each half of the tile's columns
 constexpr int kThreads = 64 + 32 * kEpiWarps;
-constexpr size_t kL2Budget = 48ull << 20;  // operand bytes the raster keeps resident in L2
+constexpr size_t kL2Budget = 32ull << 20;  // operand bytes the raster keeps resident in L2
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int kBars = 2 * PAIR_STAGES + 4 + 1;  // enough for either ring
 constexpr size_t CONST_OFF = (size_t)STAGES * STAGE_BYTES + 256;     // per-warp epilogue constants
