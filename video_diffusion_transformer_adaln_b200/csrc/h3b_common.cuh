@@ -271,7 +271,7 @@ __device__ __forceinline__ void mma_f16_pair(uint32_t d_tmem, uint64_t adesc, ui
       : "memory");
 }
 // TMA tile load into this CTA's shared memory whose byte count completes on
-// `bar_cluster`, a barrier of either CTA of the pair (no multicast).
+// `bar_cluster`, a barrier of either CTA of the pair (the data lands in this CTA only).
 __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, uint32_t bar_cluster, int c0,
                                                  int c1) {
   asm volatile(
