@@ -29,6 +29,8 @@
 // the accumulator wait, requests the next 32 accumulator columns before
 // processing the current ones, and (QKV) reads the RoPE table from shared
 // memory. Every wait is bounded.
+#include <atomic>
+
 #include "h3b_common.cuh"
 #include "h3b_internal.h"
 
@@ -525,11 +527,22 @@ static cudaError_t launch_one(const CUtensorMap& ta, const CUtensorMap& tb, cons
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  // persistent pairs: no more than can be resident at once
-  int clusters = 0;
-  e = cudaOccupancyMaxActiveClusters(&clusters, k, &cfg);
+  // persistent pairs: no more than can be resident at once (looked up once per device;
+  // the shared-memory size the launcher asks for does not change the answer)
+  constexpr int kMaxDevices = 64;
+  static std::atomic<int> resident[kMaxDevices];
+  int dev = 0;
+  e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (clusters < 1) return cudaErrorInvalidConfiguration;
+  int clusters = dev >= 0 && dev < kMaxDevices ? resident[dev].load(std::memory_order_relaxed) : 0;
+  if (clusters < 1) {
+    cfg.dynamicSmemBytes = gemm::kSmemMax;  // the most the kernel asks for
+    e = cudaOccupancyMaxActiveClusters(&clusters, k, &cfg);
+    cfg.dynamicSmemBytes = smem;
+    if (e != cudaSuccess) return e;
+    if (clusters < 1) return cudaErrorInvalidConfiguration;
+    if (dev >= 0 && dev < kMaxDevices) resident[dev].store(clusters, std::memory_order_relaxed);
+  }
   if ((int)cfg.gridDim.x > 2 * clusters) cfg.gridDim.x = 2u * (unsigned)clusters;
   return cudaLaunchKernelEx(&cfg, k, ta, tb, a);
 }
