@@ -19,7 +19,12 @@
 //   warp 1     tcgen05.mma from one thread, in the order
 //                S0(0) S1(0) | PV0(0) S0(1) PV1(0) S1(1) | PV0(1) S0(2) ...
 //              so the tensor core always has the other tile's work queued
-//   warps 2-5  softmax of tile 0, warps 6-9 softmax of tile 1 (thread = row)
+//   warps 2-3  idle (they complete warpgroup 0 for the register split)
+//   warps 4-7  softmax of tile 0, warps 8-11 softmax of tile 1 (thread = row)
+// Registers: launched at 168 per thread (384 threads), warpgroup 0 gives up all
+// but 56 (setmaxnreg.dec) and the two softmax warpgroups take 224 (setmaxnreg.inc),
+// so that a thread's 128 scores, the exponential pipeline and the O rescale fit
+// without spilling.
 // Tensor memory (512 columns): S0 | S1 | O0 | O1. Each softmax thread reads its
 // row of S_g, writes P_g = exp2(S*c - m) as bf16 pairs over the first 64
 // columns of S_g, and the P V product takes its A operand from tensor memory.
@@ -35,7 +40,11 @@
 
 namespace h3b {
 namespace attn {
-constexpr int BQ = 128, BKV = 128, kThreads = 320;
+constexpr int BQ = 128, BKV = 128, kThreads = 384;
+// registers per thread after the split: warpgroup 0 (TMA, MMA, two idle warps) gives
+// up registers, the two softmax warpgroups take them (launch: 384 x 168 = 64512;
+// 128 x 56 + 256 x 224 = 64512; per sub-partition 56 + 224 + 224 <= 512)
+constexpr uint32_t kRegsControl = 56, kRegsSoftmax = 224;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int BOX = 16384;  // one TMA box: 128 rows x 128 bytes
 }  // namespace attn
@@ -146,7 +155,9 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  // each role changes its register budget at its start (all four warps of a warpgroup)
   if (warp == 0) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsControl));
     if (lane == 0) {
       // ---------------- TMA producer
       bool ok = true;
@@ -186,6 +197,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
       }
     }
   } else if (warp == 1) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsControl));
     if (lane == 0) {
       // ---------------- MMA issuer
       bool any = false;
@@ -244,9 +256,12 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         }
       }
     }
+  } else if (warp < 4) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsControl));
   } else {
-    // ---------------- softmax warps: 2-5 -> tile 0, 6-9 -> tile 1 (thread = query row)
-    const int g = (warp - 2) >> 2;
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
+    // ---------------- softmax warps: 4-7 -> tile 0, 8-11 -> tile 1 (thread = query row)
+    const int g = (warp - 4) >> 2;
     const int quad = warp & 3;
     const int row = quad * 32 + lane;
     const uint32_t t_lane = (uint32_t)(quad * 32) << 16;
