@@ -256,7 +256,8 @@ __global__ void __launch_bounds__(256) adaln_gemv_kernel(const __nv_bfloat16* __
 // A row of d = 256 NV channels (32 NV 16-byte vectors) is held in registers by
 // tpr = 32 NV / VPT threads, VPT vectors each; a block holds rpp = blockDim /
 // tpr rows at a time and walks its share of the rows in passes of rpp rows,
-// all of one batch item. The item's (1 + scale, shift) pairs sit in shared
+// all of one batch item, staging the next pass's rows in shared memory with
+// cp.async while it works on the current ones. The item's (1 + scale, shift) pairs sit in shared
 // memory, loaded when the item changes, laid out [4][vectors] so that a warp's
 // 16-byte reads of one channel pair per vector fall in distinct banks.
 // Reductions: warp shuffles, then one shared slot per warp and a named barrier
@@ -286,13 +287,6 @@ __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src)
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
-
-// Lane-wise max of two bf16 pairs (both non-negative here).
-__device__ __forceinline__ uint32_t bf16x2_max(uint32_t a, uint32_t b) {
-  uint32_t r;
-  asm("max.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
-  return r;
-}
 
 // Threads per block of the LN quantizer: the row's tpr threads, times as many
 // rows as fit in 512 threads (or one row of up to 1024 threads).
