@@ -100,8 +100,12 @@ def test_row_quantizer_every_bf16_value(with_absmax):
 def test_ln_modulate_quantize(rows, d, items):
     r = _rng(rows * d)
     wl = synth.WORKLOADS["d256_L512"].with_(d=d, n_heads=d // 64)
-    x = synth.f32_to_bf16_bits(r.standard_normal((rows, d)).astype(np.float32) *
-                               np.where(np.isin(np.arange(d), synth.outlier_channels(wl)), 16, 1).astype(np.float32))
+    xf = (r.standard_normal((rows, d)).astype(np.float32) *
+          np.where(np.isin(np.arange(d), synth.outlier_channels(wl)), 16, 1).astype(np.float32))
+    if rows > 2:  # rows with zero variance: a constant row and an all-zero row (h = shift)
+        xf[rows // 2] = 3.0
+        xf[rows - 1] = 0.0
+    x = synth.f32_to_bf16_bits(xf)
     mod = r.standard_normal((items, 6 * d)).astype(np.float32)
     rpi = (rows + items - 1) // items
     q = torch.empty((rows, d), dtype=torch.int8, device="cuda")
