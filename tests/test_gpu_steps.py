@@ -49,7 +49,11 @@ def test_weight_quantizer_bit_exact(rows, cols):
                                                    (129, 20480, True), (5, 16, False)])
 def test_row_quantizer_bit_exact(rows, cols, with_absmax):
     r = _rng(rows + cols)
-    h = synth.f32_to_bf16_bits((r.standard_normal((rows, cols)) * r.uniform(0.01, 30, (rows, 1))).astype(np.float32))
+    hf0 = (r.standard_normal((rows, cols)) * r.uniform(0.01, 30, (rows, 1))).astype(np.float32)
+    if rows > 3:  # tiny rows: scale below 2^-100 (the division for every element), then subnormal
+        hf0[2] *= np.float32(1e-33)
+        hf0[3] *= np.float32(1e-37)
+    h = synth.f32_to_bf16_bits(hf0)
     h[1] = 0  # an all-zero row
     hf = synth.bf16_bits_to_f32(h)
     q = torch.empty((rows, cols), dtype=torch.int8, device="cuda")
