@@ -392,6 +392,36 @@ def test_attention(B, H, L, dh, n_q):
     no_device_error()
 
 
+def test_attention_running_max_jumps():
+    """Key tiles whose scores grow from one 128-key tile to the next by far more than 2^8 (head
+    0: keys scaled 1, 4, 7, 10, 13 by tile), so that the kernel's lazily kept running max moves
+    and O and the row sum are rescaled at every tile, and shrink the same way (head 1: the
+    first tile holds the max throughout)."""
+    B, H, L, dh = 1, 2, 640, 128
+    r = _rng(4242)
+    q = r.standard_normal((B, H, L, dh)).astype(np.float32)
+    k = r.standard_normal((B, H, L, dh)).astype(np.float32)
+    v = r.standard_normal((B, H, L, dh)).astype(np.float32)
+    tile = np.arange(L) // 128
+    k[:, 0] *= (1.0 + 3.0 * tile).astype(np.float32)[None, :, None]
+    k[:, 1] *= (1.0 + 3.0 * (tile.max() - tile)).astype(np.float32)[None, :, None]
+    qkv_bits = synth.f32_to_bf16_bits(np.stack([q, k, v]))
+    wl = synth.Workload("attn", 1, 1, L, H * dh, H, dh, 256, (0, 0, dh), 0, B=B)
+    dims = dims_of(wl)
+    o = torch.empty((B, L, H * dh), dtype=torch.bfloat16, device="cuda")
+    am = torch.zeros(B * L, dtype=torch.float32, device="cuda")
+    h3b.h3b_attention(dims, bf16_dev(qkv_bits), o, am)
+    og = bf16_f64(bf16_host(o))
+    qb = bf16_f64(qkv_bits)
+    rows = synth.sample_rows(L, 128)
+    tm = lambda part: qb[part, 0].transpose(1, 0, 2).reshape(L, H * dh)  # noqa: E731
+    ref = O.attention(tm(0)[rows], tm(1), tm(2), H, dh)
+    got = og[0, rows]
+    assert rel_l2(got, ref) < 1e-2
+    assert np.max(np.abs(got - ref)) < 2e-2 * np.max(np.abs(ref)) + 1e-3
+    no_device_error()
+
+
 # ----------------------------------------------------------------------------- token pairing
 
 @pytest.mark.parametrize("B,T,H,W,d", [(1, 2, 16, 16, 256), (2, 1, 3, 6, 8), (1, 8, 48, 48, 5120)])
