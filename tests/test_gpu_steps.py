@@ -331,13 +331,15 @@ def test_qkv_projection_rope_head_major(name, B, qkv_int8):
     no_device_error()
 
 
-@pytest.mark.parametrize("T,qkv_int8", [(8, True), (16, True), (8, False)])
-def test_qkv_projection_rope_full_video_grids(T, qkv_int8):
+@pytest.mark.parametrize("T,HW,qkv_int8", [(8, 48, True), (16, 48, True), (8, 48, False), (2, 64, True)])
+def test_qkv_projection_rope_full_video_grids(T, HW, qkv_int8):
     """QKV + 3D RoPE on the full T x 48 x 48 grids of the d=5120 workloads (18432 and 36864
     tokens), head_dim 128 with the (32, 48, 48) split, so every position up to (T-1, 47, 47)
     is rotated and written head-major. The width is 512 (4 heads) to keep the oracle's GEMM
-    short: positions and the split, not the width, decide the rotation. All rows compared."""
-    wl = synth.WORKLOADS["d5120_L18432"].with_(T=T, d=512, n_heads=4, d_ff=2048, qkv_int8=qkv_int8)
+    short: positions and the split, not the width, decide the rotation. All rows compared.
+    The 2 x 64 x 64 grid's RoPE table (3104 cos/sin entries) is larger than the shared memory
+    the GEMM has left for it, so the epilogue reads it from global memory instead."""
+    wl = synth.WORKLOADS["d5120_L18432"].with_(T=T, H=HW, W=HW, d=512, n_heads=4, d_ff=2048, qkv_int8=qkv_int8)
     raw = synth.block_weights(wl)
     r = _rng(31 + T)
     R, d = wl.B * wl.L, wl.d
@@ -356,7 +358,7 @@ def test_qkv_projection_rope_full_video_grids(T, qkv_int8):
     got = _head_major_to_token_major(qkv, wl)
     assert np.max(np.abs(got - ref)) <= 2 ** -8 * np.max(np.abs(ref)) * 2
     assert rel_l2(got, ref) < 4e-3
-    # per token: the last token (position (T-1, 47, 47)) and the first agree as closely
+    # per token: the last token (position (T-1, H-1, W-1)) and the first agree as closely
     for row in (0, R - 1):
         assert rel_l2(got[row], ref[row]) < 8e-3
     no_device_error()
