@@ -218,8 +218,11 @@ def test_gemm_i8_gelu(M, N, K):
     no_device_error()
 
 
-@pytest.mark.parametrize("M,N,K,items", [(512, 256, 256, 1), (256, 2048, 8192, 2), (100, 512, 1024, 1)])
+@pytest.mark.parametrize("M,N,K,items", [(512, 256, 256, 1), (256, 2048, 8192, 2), (100, 512, 1024, 1),
+                                         (100, 512, 1024, 3)])
 def test_gemm_i8_gated_residual(M, N, K, items):
+    """items=3 over 100 rows gives 34 rows per item, so some warps' 32 rows straddle two
+    items and read their gates row by row instead of from the staged per-item copy."""
     qa, sa, qw, sw, bias = _quant_operands(M, N, K, 13)
     r = _rng(14)
     x = synth.f32_to_bf16_bits(r.standard_normal((M, N)).astype(np.float32))
@@ -246,7 +249,8 @@ def test_gemm_i8_gated_residual(M, N, K, items):
     no_device_error()
 
 
-@pytest.mark.parametrize("M,N,K,items", [(512, 256, 256, 1), (256, 2048, 2048, 2), (100, 512, 1040, 1)])
+@pytest.mark.parametrize("M,N,K,items", [(512, 256, 256, 1), (256, 2048, 2048, 2), (100, 512, 1040, 1),
+                                         (100, 512, 1040, 3)])
 def test_gemm_bf16_gated_residual(M, N, K, items):
     """bf16 output projection (the block's Wo when wo_bf16 is set) with the gated residual."""
     r = _rng(M + N + K)
