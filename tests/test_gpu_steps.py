@@ -46,7 +46,7 @@ def test_weight_quantizer_bit_exact(rows, cols):
 
 
 @pytest.mark.parametrize("rows,cols,with_absmax", [(33, 1024, False), (33, 1024, True), (512, 256, False),
-                                                   (129, 20480, True), (5, 16, False)])
+                                                   (129, 20480, True), (5, 16, False), (37, 5120, True)])
 def test_row_quantizer_bit_exact(rows, cols, with_absmax):
     r = _rng(rows + cols)
     hf0 = (r.standard_normal((rows, cols)) * r.uniform(0.01, 30, (rows, 1))).astype(np.float32)

@@ -461,17 +461,21 @@ __global__ void __launch_bounds__(1024, 1) ln_mod_quant_kernel(
 // scale and its reciprocal are derived once, into shared memory.
 constexpr int kQuantMaxRowsPerBlock = 32;
 constexpr int kQuantThreads = 256;
+// VPR > 0 fixes the row at VPR vectors at compile time (the widths of the block's O and
+// G rows); VPR = 0 takes it from vpr_arg.
+template <int VPR>
 __global__ void __launch_bounds__(kQuantThreads, 4) quant_rows_known_absmax_kernel(const __nv_bfloat16* __restrict__ in,
-                                                                               int rows, int vpr, int rpb,
+                                                                               int rows, int vpr_arg, int rpb,
                                                                                const float* __restrict__ absmax_in,
                                                                                int8_t* __restrict__ q,
                                                                                float* __restrict__ s) {
   constexpr int U = 4, T = kQuantThreads;
+  const unsigned vpr = VPR ? (unsigned)VPR : (unsigned)vpr_arg;
   __shared__ float2 srow[kQuantMaxRowsPerBlock];  // (scale, RN(1/scale)) of the block's rows
   __shared__ float samax[kQuantMaxRowsPerBlock];
   const unsigned row0 = blockIdx.x * (unsigned)rpb;
   const unsigned nr = min((unsigned)rpb, (unsigned)rows - row0);
-  const unsigned span = nr * (unsigned)vpr;  // vectors covered by this block
+  const unsigned span = nr * vpr;  // vectors covered by this block
   const size_t base = (size_t)row0 * vpr;
   const uint4* src = reinterpret_cast<const uint4*>(in) + base;
   uint2* dst = reinterpret_cast<uint2*>(q) + base;
@@ -494,16 +498,21 @@ __global__ void __launch_bounds__(kQuantThreads, 4) quant_rows_known_absmax_kern
     if (H3B_IDX_OK(row0 + threadIdx.x, rows, &g_h3b_rowops_bounds)) s[row0 + threadIdx.x] = sc;
   }
   __syncthreads();
-  // row of vector k, advanced incrementally (k only grows): r = k / vpr without a division
-  unsigned r = 0, row_end = (unsigned)vpr;
+  // row of vector k: a division by the constant row length, or advanced incrementally
+  // (k only grows) when the length is known only at run time
+  unsigned r = 0, row_end = vpr;
   auto quant_round = [&](unsigned k0, const uint4(&buf)[U]) {
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const unsigned k = k0 + u * T;
       if (k >= span) break;
-      while (k >= row_end) {
-        ++r;
-        row_end += (unsigned)vpr;
+      if (VPR) {
+        r = k / (unsigned)(VPR ? VPR : 1);
+      } else {
+        while (k >= row_end) {
+          ++r;
+          row_end += vpr;
+        }
       }
       const float2 sr = srow[r];
       const uint2 code = quant8<false>(buf[u], sr.x, sr.y, samax[r]);
@@ -845,8 +854,12 @@ cudaError_t launch_quant_rows_bf16(const void* h, int rows, int cols, const floa
     int rpb = 4096 / vpr;
     rpb = std::min(rpb, rows / (4 * sms));  // but at least about four blocks per SM
     rpb = rpb < 1 ? 1 : (rpb > kQuantMaxRowsPerBlock ? kQuantMaxRowsPerBlock : rpb);
-    quant_rows_known_absmax_kernel<<<(rows + rpb - 1) / rpb, kQuantThreads, 0, st>>>(static_cast<const __nv_bfloat16*>(h),
-                                                                          rows, vpr, rpb, absmax, q, s);
+    const int grid = (rows + rpb - 1) / rpb;
+    const auto* in = static_cast<const __nv_bfloat16*>(h);
+    if (vpr == 640) quant_rows_known_absmax_kernel<640><<<grid, kQuantThreads, 0, st>>>(in, rows, vpr, rpb, absmax, q, s);
+    else if (vpr == 2560)
+      quant_rows_known_absmax_kernel<2560><<<grid, kQuantThreads, 0, st>>>(in, rows, vpr, rpb, absmax, q, s);
+    else quant_rows_known_absmax_kernel<0><<<grid, kQuantThreads, 0, st>>>(in, rows, vpr, rpb, absmax, q, s);
     return cudaGetLastError();
   }
   quant_rows_kernel<__nv_bfloat16><<<rows, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(h), cols,
