@@ -90,9 +90,11 @@ bool profiling_enabled();
 
 // ---- TMA descriptor construction (h3b_api.cu)
 // Row-major 2D tensor of `rows` x `cols` elements of `elem_bytes` each,
-// `row_stride_bytes` apart; box of box_cols x box_rows with 128-byte swizzle.
+// `row_stride_bytes` apart; box of box_cols x box_rows with a 128-, 64- or 32-byte
+// swizzle (0: none).
 bool make_tmap_2d(CUtensorMap* map, const void* base, int elem_bytes, uint64_t cols,
-                  uint64_t rows, uint64_t row_stride_bytes, uint32_t box_cols, uint32_t box_rows);
+                  uint64_t rows, uint64_t row_stride_bytes, uint32_t box_cols, uint32_t box_rows,
+                  int swizzle_bytes = 128);
 // 3D tensor [d2][d1][d0] (d0 innermost), box of box0 x box1 x 1, 128-byte swizzle.
 bool make_tmap_3d(CUtensorMap* map, const void* base, int elem_bytes, uint64_t d0, uint64_t d1,
                   uint64_t d2, uint32_t box0, uint32_t box1);

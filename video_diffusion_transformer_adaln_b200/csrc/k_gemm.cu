@@ -53,7 +53,13 @@ constexpr int kBars = 2 * PAIR_STAGES + 4 + 1;  // enough for either ring
 constexpr size_t CONST_OFF = (size_t)STAGES * STAGE_BYTES + 256;     // per-warp epilogue constants
 constexpr size_t ROPE_OFF = CONST_OFF + kEpiWarps * 3 * 128 * 4;     // RoPE table, when it fits
 constexpr size_t SMEM_BASE = ROPE_OFF + 1024;                         // + 1024 for the alignment slack
+// bf16 row-major epilogues: per epilogue warp one 32-row x 32-column staging box
+// (64-byte swizzle) that a TMA store writes out; in place of the RoPE table
+constexpr int STG_BYTES = 32 * 32 * 2;
+constexpr size_t STG_OFF = (ROPE_OFF + 1023) & ~size_t(1023);
+constexpr size_t SMEM_STG = STG_OFF + kEpiWarps * STG_BYTES + 1024;
 constexpr size_t kSmemMax = 227 * 1024;
+static_assert(SMEM_STG <= kSmemMax, "staging boxes fit");
 constexpr int kRopeSmemMaxEntries = (int)((kSmemMax - SMEM_BASE) / 8);
 }  // namespace gemm
 
@@ -150,14 +156,45 @@ __device__ __forceinline__ void stage_constants(const GemmArgs& p, EpiConst& ec,
   }
 }
 
+// The bf16 row-major outputs (dequant, GELU, gated residual) leave through TMA
+// stores: a warp's 32 rows x 32 columns go to its staging box, thread = row, the
+// 16-byte chunk c of row r at chunk c ^ ((r >> 1) & 3) (the 64-byte swizzle,
+// which also spreads a quarter-warp's eight 16-byte writes over all banks), and
+// one lane stores the box. The hardware clips rows >= M and columns >= N.
+template <int kEpi>
+constexpr bool tma_store_epi() { return kEpi == EPI_DEQ || kEpi == EPI_GELU || kEpi == EPI_RESID; }
+
+__device__ __forceinline__ void stage_and_store(const CUtensorMap* tmC, uint32_t stg, const uint32_t (&pk)[16],
+                                                int lane, int col0, int r0, bool rows_in) {
+  // the previous box of this warp has been read out of the staging buffer
+  if (lane == 0) bulk_wait_group_read0();
+  __syncwarp();
+  const uint32_t rowaddr = stg + (uint32_t)lane * 64u;
+  const uint32_t sw = ((uint32_t)lane >> 1) & 3u;
+#pragma unroll
+  for (int c = 0; c < 4; ++c)
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(rowaddr + 16u * ((uint32_t)c ^ sw)),
+                 "r"(pk[4 * c]), "r"(pk[4 * c + 1]), "r"(pk[4 * c + 2]), "r"(pk[4 * c + 3])
+                 : "memory");
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0 && rows_in) {
+    tma_store_2d(tmC, stg, col0, r0);
+    bulk_commit_group();
+  }
+}
+
 // Epilogue of the warp's 32 rows x 128 columns of one 128x256 tile; the thread
 // owns TMEM lane = tile row. TMEM loads are double-buffered: chunk i+1 (32
 // columns) is requested before chunk i is processed. `rope_s` is the RoPE
-// table in shared memory (or the global table when it did not fit).
+// table in shared memory (or the global table when it did not fit). `r0` is
+// the warp's first row; `stg` its staging box for the TMA-stored outputs.
 template <bool kInt8, int kEpi>
 __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, uint32_t tbase, int row, bool row_ok, int n0,
                                               const EpiConst& ec, bool gate_uniform, const float2* rope_s,
-                                              const uint4 (&xp)[kResidVecs]) {
+                                              const uint4 (&xp)[kResidVecs], const CUtensorMap* tmC,
+                                              uint32_t stg, int r0) {
+  constexpr bool kTmaStore = tma_store_epi<kEpi>();
   float sa = 1.0f;
   if (kInt8 && kEpi != EPI_S32 && row_ok) sa = __ldg(p.sA + row);
   int item = 0, l = 0, pt = 0, ph = 0, pw = 0;
@@ -184,6 +221,11 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, uint32_t tbase,
     const bool next = i + 1 < 4 && col0 + 32 < p.N;
     if (kDoubleBuffer && next) tmem_ld32(tbase + (i + 1) * 32, r[(i + 1) & 1]);
     const uint32_t (&rc)[32] = r[kDoubleBuffer ? (i & 1) : 0];
+    uint32_t pk[16];  // the chunk as bf16 pairs, for the TMA store (zero in rows past M)
+    if (kTmaStore) {
+#pragma unroll
+      for (int e = 0; e < 16; ++e) pk[e] = 0u;
+    }
     if (row_ok) {
       const int valid = min(32, p.N - col0);
       if (kEpi == EPI_S32) {
@@ -219,7 +261,8 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, uint32_t tbase,
         // checked build: the last element this row's chunk writes lies inside the output
         const bool out_ok = H3B_IDX_OK((long long)row * p.N + col0 + valid - 1, (long long)p.M * p.N, p.err);
         if (kEpi == EPI_DEQ) {
-          if (out_ok) store_bf16x32(static_cast<__nv_bfloat16*>(p.out) + (size_t)row * p.N + col0, v, valid);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
         } else if (kEpi == EPI_GELU) {
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
@@ -228,9 +271,9 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, uint32_t tbase,
             v[e + 1] = round_bf16(gv.y);
             amax = fmaxf(amax, fmaxf(fabsf(v[e]), fabsf(v[e + 1])));
           }
-          if (out_ok) store_bf16x32(static_cast<__nv_bfloat16*>(p.out) + (size_t)row * p.N + col0, v, valid);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
         } else if (kEpi == EPI_RESID) {
-          __nv_bfloat16* xdst = static_cast<__nv_bfloat16*>(p.out) + (size_t)row * p.N + col0;
           const float* gsrc = gate_uniform ? &ec.gate[i * 32] : p.gate + (size_t)item * p.gate_stride + col0;
 #pragma unroll
           for (int g = 0; g < 4; ++g) {
@@ -252,7 +295,8 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, uint32_t tbase,
               v[8 * g + 2 * e + 1] = fmaf(gg[2 * e + 1], v[8 * g + 2 * e + 1], bf16_hi(xu[e]));
             }
           }
-          if (out_ok) store_bf16x32(xdst, v, valid);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
         } else if (kEpi == EPI_QKV) {
           const int part = col0 / p.d;
           const int rem = col0 - part * p.d;
@@ -276,8 +320,10 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, uint32_t tbase,
           if (H3B_IDX_OK((long long)off + 31, (long long)p.M * p.N, p.err))
             store_bf16x32(static_cast<__nv_bfloat16*>(p.out) + off, v, 32);
         }
+        (void)out_ok;
       }
     }
+    if (kTmaStore) stage_and_store(tmC, stg, pk, threadIdx.x & 31, col0, r0, r0 < p.M);
     if (next) {
       if (!kDoubleBuffer) tmem_ld32(tbase + (i + 1) * 32, r[0]);
       tmem_ld_wait();
@@ -298,7 +344,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, uint32_t tbase,
 template <bool kInt8, int kEpi, bool kPair>
 __global__ void __launch_bounds__(gemm::kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                const GemmArgs p) {
+                const __grid_constant__ CUtensorMap tmC, const GemmArgs p) {
   using namespace gemm;
   constexpr int NS = kPair ? PAIR_STAGES : STAGES;
   constexpr int SB = kPair ? PAIR_STAGE_BYTES : STAGE_BYTES;
@@ -345,7 +391,11 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 0 && lane == 0) { tma_prefetch_desc(&tmA); tma_prefetch_desc(&tmB); }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+    if (tma_store_epi<kEpi>()) tma_prefetch_desc(&tmC);
+  }
   if (kEpi == EPI_QKV)  // the whole RoPE table, once per CTA, when the launcher reserved room for it
     for (int i = threadIdx.x; i < p.rope_smem_entries; i += blockDim.x) rope_smem[i] = __ldg(p.rope + i);
   if (warp == 1) {
@@ -485,7 +535,8 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
       // this warp's 32 lanes and 128 columns of the accumulator
       const uint32_t tbase = tmem_base + ((uint32_t)(quad * 32) << 16) + acc * BN + half * (BN / 2);
       epilogue_tile<kInt8, kEpi>(p, tbase, row, row < p.M, n0, ec, gate_uniform,
-                                 p.rope_smem_entries > 0 ? rope_smem : p.rope, xp);
+                                 p.rope_smem_entries > 0 ? rope_smem : p.rope, xp, &tmC,
+                                 sbase + (uint32_t)STG_OFF + (uint32_t)(warp - 2) * STG_BYTES, r0);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
@@ -493,6 +544,8 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
         else mbar_arrive(tempty(acc));
       }
     }
+    // the staging boxes are read and the stores written before the CTA exits
+    if (tma_store_epi<kEpi>() && lane == 0) bulk_wait_group0();
   }
   __syncthreads();
   if (kPair) cluster_sync_all();  // the pair's MMAs and remote arrivals are over before TMEM goes
@@ -505,14 +558,15 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
 }
 
 template <bool kInt8, int kEpi, bool kPair>
-static cudaError_t launch_one(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& a,
-                              int grid, cudaStream_t st) {
+static cudaError_t launch_one(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc,
+                              const GemmArgs& a, int grid, cudaStream_t st) {
   auto k = gemm_kernel<kInt8, kEpi, kPair>;
-  const size_t smem = gemm::SMEM_BASE + (size_t)a.rope_smem_entries * sizeof(float2);
+  const size_t smem = tma_store_epi<kEpi>() ? gemm::SMEM_STG
+                                            : gemm::SMEM_BASE + (size_t)a.rope_smem_entries * sizeof(float2);
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gemm::kSmemMax);
   if (e != cudaSuccess) return e;
   if (!kPair) {
-    k<<<grid, gemm::kThreads, smem, st>>>(ta, tb, a);
+    k<<<grid, gemm::kThreads, smem, st>>>(ta, tb, tc, a);
     return cudaGetLastError();
   }
   cudaLaunchConfig_t cfg = {};
@@ -544,7 +598,7 @@ static cudaError_t launch_one(const CUtensorMap& ta, const CUtensorMap& tb, cons
     if (dev >= 0 && dev < kMaxDevices) resident[dev].store(clusters, std::memory_order_relaxed);
   }
   if ((int)cfg.gridDim.x > 2 * clusters) cfg.gridDim.x = 2u * (unsigned)clusters;
-  return cudaLaunchKernelEx(&cfg, k, ta, tb, a);
+  return cudaLaunchKernelEx(&cfg, k, ta, tb, tc, a);
 }
 
 // The GEMMs run on CTA pairs (256 x 256 tiles, half of every W tile per SM) when
@@ -552,9 +606,10 @@ static cudaError_t launch_one(const CUtensorMap& ta, const CUtensorMap& tb, cons
 constexpr bool kUsePairs = true;
 
 template <bool kInt8, int kEpi>
-static cudaError_t launch_epi(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& a, bool pair,
-                              int grid, cudaStream_t st) {
-  return pair ? launch_one<kInt8, kEpi, true>(ta, tb, a, grid, st) : launch_one<kInt8, kEpi, false>(ta, tb, a, grid, st);
+static cudaError_t launch_epi(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc,
+                              const GemmArgs& a, bool pair, int grid, cudaStream_t st) {
+  return pair ? launch_one<kInt8, kEpi, true>(ta, tb, tc, a, grid, st)
+              : launch_one<kInt8, kEpi, false>(ta, tb, tc, a, grid, st);
 }
 
 cudaError_t launch_gemm(bool int8_operands, GemmEpilogue epi, const void* A, const void* W,
@@ -569,6 +624,11 @@ cudaError_t launch_gemm(bool int8_operands, GemmEpilogue epi, const void* A, con
   if (!make_tmap_2d(&ta, A, eb, (uint64_t)a.K, (uint64_t)a.M, (uint64_t)a.K * eb, bke, BM))
     return cudaErrorInvalidValue;
   if (!make_tmap_2d(&tb, W, eb, (uint64_t)a.K, (uint64_t)a.N, (uint64_t)a.K * eb, bke, pair ? BN / 2 : BN))
+    return cudaErrorInvalidValue;
+  // the bf16 [M][N] output of the TMA-stored epilogues: 32 x 32 boxes, 64-byte swizzle
+  CUtensorMap tc = tb;
+  if ((epi == EPI_DEQ || epi == EPI_GELU || epi == EPI_RESID) &&
+      !make_tmap_2d(&tc, a.out, 2, (uint64_t)a.N, (uint64_t)a.M, (uint64_t)a.N * 2, 32, 32, 64))
     return cudaErrorInvalidValue;
   const int n_m = (a.M + MT - 1) / MT, n_n = (a.N + BN - 1) / BN;
   const int n_tiles = n_m * n_n;
@@ -595,17 +655,17 @@ cudaError_t launch_gemm(bool int8_operands, GemmEpilogue epi, const void* A, con
   }
   if (int8_operands) {
     switch (epi) {
-      case EPI_S32: return launch_epi<true, EPI_S32>(ta, tb, args, pair, grid, st);
-      case EPI_DEQ: return launch_epi<true, EPI_DEQ>(ta, tb, args, pair, grid, st);
-      case EPI_QKV: return launch_epi<true, EPI_QKV>(ta, tb, args, pair, grid, st);
-      case EPI_RESID: return launch_epi<true, EPI_RESID>(ta, tb, args, pair, grid, st);
-      case EPI_GELU: return launch_epi<true, EPI_GELU>(ta, tb, args, pair, grid, st);
+      case EPI_S32: return launch_epi<true, EPI_S32>(ta, tb, tc, args, pair, grid, st);
+      case EPI_DEQ: return launch_epi<true, EPI_DEQ>(ta, tb, tc, args, pair, grid, st);
+      case EPI_QKV: return launch_epi<true, EPI_QKV>(ta, tb, tc, args, pair, grid, st);
+      case EPI_RESID: return launch_epi<true, EPI_RESID>(ta, tb, tc, args, pair, grid, st);
+      case EPI_GELU: return launch_epi<true, EPI_GELU>(ta, tb, tc, args, pair, grid, st);
     }
   } else {
     switch (epi) {
-      case EPI_DEQ: return launch_epi<false, EPI_DEQ>(ta, tb, args, pair, grid, st);
-      case EPI_QKV: return launch_epi<false, EPI_QKV>(ta, tb, args, pair, grid, st);
-      case EPI_RESID: return launch_epi<false, EPI_RESID>(ta, tb, args, pair, grid, st);
+      case EPI_DEQ: return launch_epi<false, EPI_DEQ>(ta, tb, tc, args, pair, grid, st);
+      case EPI_QKV: return launch_epi<false, EPI_QKV>(ta, tb, tc, args, pair, grid, st);
+      case EPI_RESID: return launch_epi<false, EPI_RESID>(ta, tb, tc, args, pair, grid, st);
       default: break;
     }
   }
