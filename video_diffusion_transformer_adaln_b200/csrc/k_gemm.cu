@@ -113,19 +113,26 @@ __device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const float (&
   }
 }
 
-// Epilogue of one 128x256 tile for the thread owning TMEM lane = tile row.
-// Residual rows this thread updates: its 128 columns of x, loaded before the
-// accumulator is ready so the global-memory latency overlaps the K loop.
-constexpr int kResidVecs = 16;  // 128 bf16 columns = 16 x 16 bytes
-__device__ __forceinline__ void prefetch_resid(const GemmArgs& p, int row, int col0, uint4 (&xp)[kResidVecs]) {
-  const bool row_ok = row < p.M;
-  const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.out) + (size_t)row * p.N + col0);
+// The residual x of a warp's 32 rows x 128 columns, loaded before the accumulator
+// is ready so the global-memory latency overlaps the K loop. The loads are
+// coalesced: for chunk i (32 columns) and row group j, lane l reads row
+// r0 + 8 j + l / 4, columns 32 i + 8 (l % 4) .. + 7 (eight rows of 64 bytes per
+// instruction); the epilogue turns them into one row per thread through the
+// warp's staging box.
+constexpr int kResidVecs = 16;  // 4 chunks x 4 row groups of 16 bytes
+__device__ __forceinline__ void prefetch_resid(const GemmArgs& p, int r0, int n0, int lane, uint4 (&xp)[kResidVecs]) {
+  const __nv_bfloat16* x = static_cast<const __nv_bfloat16*>(p.out);
 #pragma unroll
-  for (int g = 0; g < kResidVecs; ++g)
-    xp[g] = (row_ok && col0 + 8 * g < p.N &&
-             H3B_IDX_OK((long long)row * p.N + col0 + 8 * g + 7, (long long)p.M * p.N, p.err))
-                ? src[g]
-                : make_uint4(0, 0, 0, 0);
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int row = r0 + 8 * j + (lane >> 2);
+      const int col = n0 + 32 * i + 8 * (lane & 3);
+      xp[4 * i + j] = (row < p.M && col < p.N &&
+                       H3B_IDX_OK((long long)row * p.N + col + 7, (long long)p.M * p.N, p.err))
+                          ? *reinterpret_cast<const uint4*>(x + (size_t)row * p.N + col)
+                          : make_uint4(0, 0, 0, 0);
+    }
 }
 
 // Per-warp column constants of the current tile (the warp's 128 columns):
@@ -164,11 +171,40 @@ __device__ __forceinline__ void stage_constants(const GemmArgs& p, EpiConst& ec,
 template <int kEpi>
 constexpr bool tma_store_epi() { return kEpi == EPI_DEQ || kEpi == EPI_GELU || kEpi == EPI_RESID; }
 
-__device__ __forceinline__ void stage_and_store(const CUtensorMap* tmC, uint32_t stg, const uint32_t (&pk)[16],
-                                                int lane, int col0, int r0, bool rows_in) {
-  // the previous box of this warp has been read out of the staging buffer
+// Byte offset of the 16-byte chunk c of row r in a staging box.
+__device__ __forceinline__ uint32_t stg_off(uint32_t r, uint32_t c) { return r * 64u + 16u * (c ^ ((r >> 1) & 3u)); }
+
+// The previous box of this warp has been read out of the staging buffer.
+__device__ __forceinline__ void stage_acquire(int lane) {
   if (lane == 0) bulk_wait_group_read0();
   __syncwarp();
+}
+
+// Chunk i of the coalesced residual prefetch into the staging box, then this
+// thread's row of it (the box must have been acquired).
+__device__ __forceinline__ void stage_resid_row(uint32_t stg, const uint4 (&xp)[kResidVecs], int i, int lane,
+                                                uint4 (&xr)[4]) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint4 v = xp[4 * i + j];
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(stg + stg_off(8u * j + ((uint32_t)lane >> 2), lane & 3u)),
+                 "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+  }
+  __syncwarp();
+#pragma unroll
+  for (int c = 0; c < 4; ++c)
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(xr[c].x), "=r"(xr[c].y), "=r"(xr[c].z), "=r"(xr[c].w)
+                 : "r"(stg + stg_off((uint32_t)lane, (uint32_t)c))
+                 : "memory");
+}
+
+// This thread's row of the chunk into the staging box and one lane's TMA store
+// of the box (the box must have been acquired; a thread overwrites only the
+// positions of its own row).
+__device__ __forceinline__ void stage_and_store(const CUtensorMap* tmC, uint32_t stg, const uint32_t (&pk)[16],
+                                                int lane, int col0, int r0, bool rows_in) {
   const uint32_t rowaddr = stg + (uint32_t)lane * 64u;
   const uint32_t sw = ((uint32_t)lane >> 1) & 3u;
 #pragma unroll
@@ -222,9 +258,14 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, uint32_t tbase,
     if (kDoubleBuffer && next) tmem_ld32(tbase + (i + 1) * 32, r[(i + 1) & 1]);
     const uint32_t (&rc)[32] = r[kDoubleBuffer ? (i & 1) : 0];
     uint32_t pk[16];  // the chunk as bf16 pairs, for the TMA store (zero in rows past M)
+    uint4 xr[4];      // gated residual: this row's 32 columns of x
     if (kTmaStore) {
 #pragma unroll
       for (int e = 0; e < 16; ++e) pk[e] = 0u;
+      if (kEpi == EPI_RESID) {
+        stage_acquire(threadIdx.x & 31);
+        stage_resid_row(stg, xp, i, threadIdx.x & 31, xr);
+      }
     }
     if (row_ok) {
       const int valid = min(32, p.N - col0);
@@ -278,7 +319,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, uint32_t tbase,
 #pragma unroll
           for (int g = 0; g < 4; ++g) {
             if (g * 8 >= valid) break;
-            const uint4 xv = xp[i * 4 + g];
+            const uint4 xv = xr[g];
             float4 ga, gb;
             if (gate_uniform) {
               ga = *reinterpret_cast<const float4*>(gsrc + 8 * g);
@@ -323,7 +364,10 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, uint32_t tbase,
         (void)out_ok;
       }
     }
-    if (kTmaStore) stage_and_store(tmC, stg, pk, threadIdx.x & 31, col0, r0, r0 < p.M);
+    if (kTmaStore) {
+      if (kEpi != EPI_RESID) stage_acquire(threadIdx.x & 31);
+      stage_and_store(tmC, stg, pk, threadIdx.x & 31, col0, r0, r0 < p.M);
+    }
     if (next) {
       if (!kDoubleBuffer) tmem_ld32(tbase + (i + 1) * 32, r[0]);
       tmem_ld_wait();
@@ -523,7 +567,7 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
       const int first_row = min(r0, p.M - 1), last_row = min(r0 + 31, p.M - 1);
       const bool gate_uniform = kEpi == EPI_RESID && first_row / p.rows_per_item == last_row / p.rows_per_item;
       uint4 xp[kResidVecs];
-      if (kEpi == EPI_RESID) prefetch_resid(p, row, n0, xp);
+      if (kEpi == EPI_RESID) prefetch_resid(p, r0, n0, lane, xp);
       __syncwarp();
       // tcgen05.ld is warp-collective: the wait outcome is made warp-uniform.
       const bool t_ok = mbar_wait_or_abort(tfull(acc), aph, abort_flag, p.err, ERR_WAIT_MMA);
