@@ -12,6 +12,7 @@
 //     preceding kernels; activation memory reused by lifetime).
 #include <algorithm>
 #include <atomic>
+#include <cstdlib>
 #include <mutex>
 #include <string>
 #include <vector>
@@ -201,6 +202,14 @@ std::vector<cudaEvent_t> g_prof_free;
 }  // namespace
 
 bool profiling_enabled() { return g_prof_on.load(); }
+
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* v = std::getenv("H3B_PDL");
+    return !(v && v[0] == '0');
+  }();
+  return on;
+}
 
 namespace {
 

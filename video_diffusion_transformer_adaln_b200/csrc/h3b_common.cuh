@@ -161,6 +161,18 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
+// Programmatic dependent launch. Every kernel of this library waits for the
+// grid before it in the stream (its completion and memory flush) before its
+// first access to global data, and only then lets the next grid start; so when
+// a grid starts, every grid before its immediate predecessor has completed, and
+// the work before the wait (barrier init, TMEM allocation, descriptor prefetch)
+// overlaps the predecessor's tail. Without the launch attribute the wait returns
+// at once.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // TMA tile store from this CTA's shared memory into global memory. Elements of the
 // box that fall outside the tensor are not written. Completion is tracked per
 // thread in bulk groups: commit after the stores, then wait until the source

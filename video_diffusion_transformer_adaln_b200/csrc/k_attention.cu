@@ -154,6 +154,8 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  griddep_wait();  // Q, K, V are the previous grid's output
+  griddep_launch_dependents();
 
   // each role changes its register budget at its start (all four warps of a warpgroup)
   if (warp == 0) {
@@ -406,8 +408,7 @@ static cudaError_t launch_attn(const AttnArgs& a, cudaStream_t st) {
   if (e != cudaSuccess) return e;
   const dim3 grid((a.L + 2 * attn::BQ - 1) / (2 * attn::BQ), a.B * a.n_heads);
   const float scale_log2 = 1.4426950408889634f / sqrtf((float)DH);
-  k<<<grid, attn::kThreads, Lay::SMEM, st>>>(tm, a, scale_log2);
-  return cudaGetLastError();
+  return launch_pdl(k, grid, dim3(attn::kThreads), Lay::SMEM, st, tm, a, scale_log2);
 }
 
 cudaError_t launch_attention(const AttnArgs& a, cudaStream_t st) {

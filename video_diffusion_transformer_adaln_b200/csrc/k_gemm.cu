@@ -440,8 +440,6 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
     tma_prefetch_desc(&tmB);
     if (tma_store_epi<kEpi>()) tma_prefetch_desc(&tmC);
   }
-  if (kEpi == EPI_QKV)  // the whole RoPE table, once per CTA, when the launcher reserved room for it
-    for (int i = threadIdx.x; i < p.rope_smem_entries; i += blockDim.x) rope_smem[i] = __ldg(p.rope + i);
   if (warp == 1) {
     if (kPair) {
       tmem_alloc_pair(smem_u32(tmem_slot), TMEM_COLS);
@@ -456,6 +454,12 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
   if (kPair) cluster_sync_all();  // both CTAs' barriers exist before any remote arrival
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  griddep_wait();  // A (and the residual x) come from earlier grids
+  griddep_launch_dependents();
+  if (kEpi == EPI_QKV && p.rope_smem_entries > 0) {  // the whole RoPE table, once per CTA
+    for (int i = threadIdx.x; i < p.rope_smem_entries; i += blockDim.x) rope_smem[i] = __ldg(p.rope + i);
+    __syncthreads();
+  }
 
   if (warp == 0) {
     if (lane == 0) {
@@ -609,22 +613,21 @@ static cudaError_t launch_one(const CUtensorMap& ta, const CUtensorMap& tb, cons
                                             : gemm::SMEM_BASE + (size_t)a.rope_smem_entries * sizeof(float2);
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gemm::kSmemMax);
   if (e != cudaSuccess) return e;
-  if (!kPair) {
-    k<<<grid, gemm::kThreads, smem, st>>>(ta, tb, tc, a);
-    return cudaGetLastError();
-  }
+  if (!kPair) return launch_pdl(k, dim3(grid), dim3(gemm::kThreads), smem, st, ta, tb, tc, a);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)grid, 1, 1);
   cfg.blockDim = dim3(gemm::kThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 1;  // the occupancy query below sees the cluster shape only
   // persistent pairs: no more than can be resident at once (looked up once per device;
   // the shared-memory size the launcher asks for does not change the answer)
   constexpr int kMaxDevices = 64;
@@ -642,6 +645,7 @@ static cudaError_t launch_one(const CUtensorMap& ta, const CUtensorMap& tb, cons
     if (dev >= 0 && dev < kMaxDevices) resident[dev].store(clusters, std::memory_order_relaxed);
   }
   if ((int)cfg.gridDim.x > 2 * clusters) cfg.gridDim.x = 2u * (unsigned)clusters;
+  cfg.numAttrs = pdl_enabled() ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, k, ta, tb, tc, a);
 }
 

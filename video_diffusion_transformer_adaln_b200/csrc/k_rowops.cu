@@ -186,6 +186,8 @@ __global__ void __launch_bounds__(256) adaln_gemv_kernel(const __nv_bfloat16* __
                                                          const float* __restrict__ c, int B,
                                                          float* __restrict__ mod, const RopeTableArgs rope,
                                                          int gemv_blocks) {
+  griddep_wait();
+  griddep_launch_dependents();
   constexpr int d = NV * 256;
   constexpr int R = kGemvRows, CH = kGemvChunk;
   if ((int)blockIdx.x >= gemv_blocks) {  // trailing blocks fill the RoPE table
@@ -303,6 +305,8 @@ __global__ void __launch_bounds__(1024, 1) ln_mod_quant_kernel(
     const float* __restrict__ scale, int rows_per_item, int mod_stride, int8_t* __restrict__ q,
     float* __restrict__ s, __nv_bfloat16* __restrict__ h_out, float* __restrict__ absmax_zero,
     int write_codes) {
+  griddep_wait();
+  griddep_launch_dependents();
   extern __shared__ float4 modp[];  // [4][vpr]: (1+sc[2c], 1+sc[2c+1], sh[2c], sh[2c+1]), c = 4 vec + e
   // then the staging rows of the next pass: [rpp][vpr] 16-byte vectors, each written and read
   // back by the same thread (cp.async), so no barrier guards them
@@ -469,6 +473,8 @@ __global__ void __launch_bounds__(kQuantThreads, 4) quant_rows_known_absmax_kern
                                                                                const float* __restrict__ absmax_in,
                                                                                int8_t* __restrict__ q,
                                                                                float* __restrict__ s) {
+  griddep_wait();
+  griddep_launch_dependents();
   constexpr int U = 4, T = kQuantThreads;
   const unsigned vpr = VPR ? (unsigned)VPR : (unsigned)vpr_arg;
   __shared__ float2 srow[kQuantMaxRowsPerBlock];  // (scale, RN(1/scale)) of the block's rows
@@ -557,6 +563,8 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(const T* __restrict__ i
                                                          const float* __restrict__ absmax_in,
                                                          int8_t* __restrict__ q,
                                                          float* __restrict__ s) {
+  griddep_wait();
+  griddep_launch_dependents();
   __shared__ float red[8];
   const int row = blockIdx.x;
   const T* r = in + (size_t)row * cols;
@@ -614,6 +622,8 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(const T* __restrict__ i
 __global__ void token_pair_kernel(const __nv_bfloat16* __restrict__ x, __nv_bfloat16* __restrict__ xm,
                                   __nv_bfloat16* __restrict__ xm2, long long n_out_vec, int Wm,
                                   int dvec) {
+  griddep_wait();
+  griddep_launch_dependents();
   for (long long o = blockIdx.x * (long long)blockDim.x + threadIdx.x; o < n_out_vec;
        o += (long long)gridDim.x * blockDim.x) {
     const long long rp = o / dvec;
@@ -644,6 +654,8 @@ __global__ void token_unpair_kernel(const __nv_bfloat16* __restrict__ x,
                                     const __nv_bfloat16* __restrict__ xm,
                                     const __nv_bfloat16* __restrict__ ym, __nv_bfloat16* out,
                                     long long n_out_vec, int Wm, int dvec) {
+  griddep_wait();
+  griddep_launch_dependents();
   for (long long o = blockIdx.x * (long long)blockDim.x + threadIdx.x; o < n_out_vec;
        o += (long long)gridDim.x * blockDim.x) {
     const long long rp = o / dvec;
@@ -685,6 +697,8 @@ __global__ void token_unpair_kernel(const __nv_bfloat16* __restrict__ x,
 // ---------------------------------------------------------------------------
 __global__ void range_delta_kernel(const __nv_bfloat16* __restrict__ before, const __nv_bfloat16* __restrict__ after,
                                    float* __restrict__ delta, long long n_vec) {
+  griddep_wait();
+  griddep_launch_dependents();
   for (long long o = blockIdx.x * (long long)blockDim.x + threadIdx.x; o < n_vec;
        o += (long long)gridDim.x * blockDim.x) {
     const uint4 a = __ldcs(reinterpret_cast<const uint4*>(before) + o);
@@ -703,6 +717,8 @@ __global__ void range_delta_kernel(const __nv_bfloat16* __restrict__ before, con
 }
 
 __global__ void range_apply_kernel(__nv_bfloat16* __restrict__ x, const float* __restrict__ delta, long long n_vec) {
+  griddep_wait();
+  griddep_launch_dependents();
   for (long long o = blockIdx.x * (long long)blockDim.x + threadIdx.x; o < n_vec;
        o += (long long)gridDim.x * blockDim.x) {
     const uint4 a = __ldcs(reinterpret_cast<const uint4*>(x) + o);
@@ -736,6 +752,8 @@ __device__ void rope_table_entries(const RopeTableArgs& r, int first, int stride
 }
 
 __global__ void rope_table_kernel(const RopeTableArgs r) {
+  griddep_wait();
+  griddep_launch_dependents();
   rope_table_entries(r, blockIdx.x * blockDim.x + threadIdx.x, gridDim.x * blockDim.x);
 }
 
@@ -761,9 +779,8 @@ static cudaError_t gemv_launch(const void* W, const float* bias, const float* c,
     const int n = rope.T * (rope.rt / 2) + rope.H * (rope.rh / 2) + rope.W * (rope.rw / 2);
     rope_blocks = (n + 255) / 256;
   }
-  kern<<<gemv_blocks + rope_blocks, 256, smem, st>>>(static_cast<const __nv_bfloat16*>(W), bias, c, B, mod, rope,
-                                                      gemv_blocks);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(gemv_blocks + rope_blocks), dim3(256), smem, st,
+                    static_cast<const __nv_bfloat16*>(W), bias, c, B, mod, rope, gemv_blocks);
 }
 
 template <int NV>
@@ -815,9 +832,8 @@ static cudaError_t ln_dispatch(const void* x, int rows, int nv, float eps, const
   const int rpp = block / tpr;
   const long long passes = (long long)((rows + rpi - 1) / rpi) * ((rpi + rpp - 1) / rpp);
   const long long grid = std::min<long long>(passes, (long long)sms * per_sm);
-  kern<<<(int)grid, block, smem, st>>>(static_cast<const __nv_bfloat16*>(x), rows, vpr, eps, shift, scale, rpi, ms,
-                                        q, s, static_cast<__nv_bfloat16*>(h), az, wc);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3((unsigned)grid), dim3(block), smem, st, static_cast<const __nv_bfloat16*>(x), rows,
+                    vpr, eps, shift, scale, rpi, ms, q, s, static_cast<__nv_bfloat16*>(h), az, wc);
 }
 
 cudaError_t launch_ln_mod_quant(const void* x, int rows, int d, float eps, const float* shift,
@@ -856,22 +872,19 @@ cudaError_t launch_quant_rows_bf16(const void* h, int rows, int cols, const floa
     rpb = rpb < 1 ? 1 : (rpb > kQuantMaxRowsPerBlock ? kQuantMaxRowsPerBlock : rpb);
     const int grid = (rows + rpb - 1) / rpb;
     const auto* in = static_cast<const __nv_bfloat16*>(h);
-    if (vpr == 640) quant_rows_known_absmax_kernel<640><<<grid, kQuantThreads, 0, st>>>(in, rows, vpr, rpb, absmax, q, s);
-    else if (vpr == 2560)
-      quant_rows_known_absmax_kernel<2560><<<grid, kQuantThreads, 0, st>>>(in, rows, vpr, rpb, absmax, q, s);
-    else quant_rows_known_absmax_kernel<0><<<grid, kQuantThreads, 0, st>>>(in, rows, vpr, rpb, absmax, q, s);
-    return cudaGetLastError();
+    auto kern = vpr == 640    ? quant_rows_known_absmax_kernel<640>
+                : vpr == 2560 ? quant_rows_known_absmax_kernel<2560>
+                              : quant_rows_known_absmax_kernel<0>;
+    return launch_pdl(kern, dim3(grid), dim3(kQuantThreads), 0, st, in, rows, vpr, rpb, absmax, q, s);
   }
-  quant_rows_kernel<__nv_bfloat16><<<rows, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(h), cols,
-                                                        absmax, q, s);
-  return cudaGetLastError();
+  return launch_pdl(quant_rows_kernel<__nv_bfloat16>, dim3(rows), dim3(256), 0, st,
+                    static_cast<const __nv_bfloat16*>(h), cols, absmax, q, s);
 }
 
 cudaError_t launch_quant_rows_f32(const float* w, int rows, int cols, int8_t* q, float* s,
                                   cudaStream_t st) {
   if (rows == 0) return cudaSuccess;
-  quant_rows_kernel<float><<<rows, 256, 0, st>>>(w, cols, nullptr, q, s);
-  return cudaGetLastError();
+  return launch_pdl(quant_rows_kernel<float>, dim3(rows), dim3(256), 0, st, w, cols, (const float*)nullptr, q, s);
 }
 
 static int grid_for(long long n, int sms) {
@@ -884,36 +897,32 @@ cudaError_t launch_token_pair(const void* x, void* xm, void* xm2, long long line
                               int sms, cudaStream_t st) {
   const long long n = lines * (W / 2) * (d / 8);
   if (n == 0) return cudaSuccess;
-  token_pair_kernel<<<grid_for(n, sms), 256, 0, st>>>(
-      static_cast<const __nv_bfloat16*>(x), static_cast<__nv_bfloat16*>(xm),
-      static_cast<__nv_bfloat16*>(xm2), n, W / 2, d / 8);
-  return cudaGetLastError();
+  return launch_pdl(token_pair_kernel, dim3(grid_for(n, sms)), dim3(256), 0, st, static_cast<const __nv_bfloat16*>(x),
+                    static_cast<__nv_bfloat16*>(xm), static_cast<__nv_bfloat16*>(xm2), n, W / 2, d / 8);
 }
 
 cudaError_t launch_range_delta(const void* before, const void* after, float* delta, long long n, int sms,
                                cudaStream_t st) {
   if (n == 0) return cudaSuccess;
   const long long nv = n / 8;
-  range_delta_kernel<<<grid_for(nv, sms), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(before),
-                                                        static_cast<const __nv_bfloat16*>(after), delta, nv);
-  return cudaGetLastError();
+  return launch_pdl(range_delta_kernel, dim3(grid_for(nv, sms)), dim3(256), 0, st,
+                    static_cast<const __nv_bfloat16*>(before), static_cast<const __nv_bfloat16*>(after), delta, nv);
 }
 
 cudaError_t launch_range_apply(void* x, const float* delta, long long n, int sms, cudaStream_t st) {
   if (n == 0) return cudaSuccess;
   const long long nv = n / 8;
-  range_apply_kernel<<<grid_for(nv, sms), 256, 0, st>>>(static_cast<__nv_bfloat16*>(x), delta, nv);
-  return cudaGetLastError();
+  return launch_pdl(range_apply_kernel, dim3(grid_for(nv, sms)), dim3(256), 0, st, static_cast<__nv_bfloat16*>(x),
+                    delta, nv);
 }
 
 cudaError_t launch_token_unpair(const void* x, const void* xm, const void* ym, void* out,
                                 long long lines, int W, int d, int sms, cudaStream_t st) {
   const long long n = lines * (W / 2) * (d / 8);
   if (n == 0) return cudaSuccess;
-  token_unpair_kernel<<<grid_for(n, sms), 256, 0, st>>>(
-      static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(xm),
-      static_cast<const __nv_bfloat16*>(ym), static_cast<__nv_bfloat16*>(out), n, W / 2, d / 8);
-  return cudaGetLastError();
+  return launch_pdl(token_unpair_kernel, dim3(grid_for(n, sms)), dim3(256), 0, st, static_cast<const __nv_bfloat16*>(x),
+                    static_cast<const __nv_bfloat16*>(xm), static_cast<const __nv_bfloat16*>(ym),
+                    static_cast<__nv_bfloat16*>(out), n, W / 2, d / 8);
 }
 
 unsigned* rowops_bounds_word() {
@@ -924,8 +933,7 @@ unsigned* rowops_bounds_word() {
 cudaError_t launch_rope_table(float2* tab, int T, int H, int W, int rt, int rh, int rw,
                               double theta, cudaStream_t st) {
   const int n = T * (rt / 2) + H * (rh / 2) + W * (rw / 2);
-  rope_table_kernel<<<(n + 255) / 256, 256, 0, st>>>(RopeTableArgs{tab, T, H, W, rt, rh, rw, theta});
-  return cudaGetLastError();
+  return launch_pdl(rope_table_kernel, dim3((n + 255) / 256), dim3(256), 0, st, RopeTableArgs{tab, T, H, W, rt, rh, rw, theta});
 }
 
 }  // namespace h3b
