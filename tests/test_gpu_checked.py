@@ -1,4 +1,5 @@
-"""The checked build of the library (libh3b_checked.so) on the block and its steps.
+"""The checked build of the library (libh3b_checked.so), and launches without
+programmatic dependent launch, on the block and its steps.
 
 In the checked build every kernel tests each global-memory index it computes
 against the extent of its buffer before the access; an index outside records
@@ -10,7 +11,13 @@ raw int8 GEMM at ragged sizes and the QKV projection, first with the normal
 library in this process and then with the checked library in a child process
 (the binding picks the library when it is first loaded). The checked run must
 leave the error word clear, and its outputs must equal the normal build's bit
-for bit: the checks change no arithmetic."""
+for bit: the checks change no arithmetic.
+
+The same cases (with the bf16-output GEMM epilogues at ragged sizes, whose TMA
+stores the hardware clips at M and N, and a two-block pass) run once more in a
+child process with H3B_PDL=0, which launches every kernel without the
+programmatic-serialization attribute: the outputs must again be identical, so
+the early launch of a grid ahead of its grid-dependency wait changes nothing."""
 import os
 import subprocess
 import sys
@@ -30,7 +37,8 @@ def run_cases():
     """Every case's outputs as numpy arrays (bf16 as uint16 bit patterns)."""
     import oracle as O
     from video_diffusion_transformer_adaln_b200 import h3b, synth
-    from video_diffusion_transformer_adaln_b200.runtime import DeviceBlock, block_forward, dims_of, workspace
+    from video_diffusion_transformer_adaln_b200.runtime import (DeviceBlock, block_forward, blocks_forward, dims_of,
+                                                                workspace)
 
     out = {}
     r = np.random.default_rng(5)
@@ -42,6 +50,13 @@ def run_cases():
         xd = bf16_dev(x)
         block_forward(dims, blk, to_dev(c), xd, workspace(dims))
         out[name] = bf16_host(xd)
+    # a two-block pass (grids of consecutive blocks launched back to back)
+    wl = synth.WORKLOADS["d256_L512"]
+    dims = dims_of(wl)
+    blocks = [DeviceBlock.from_host(synth.block_weights(wl, block=b)) for b in (0, 1)]
+    xd = bf16_dev(synth.x_input(wl))
+    blocks_forward(dims, blocks, to_dev(synth.cond(wl)), xd, workspace(dims))
+    out["blocks2"] = bf16_host(xd)
     # attention at a ragged length
     B, H, L, dh = 2, 2, 777, 128
     qkv = synth.f32_to_bf16_bits(r.standard_normal((3, B, H, L, dh)).astype(np.float32))
@@ -84,6 +99,25 @@ def run_cases():
     Cg = torch.empty((M, N), dtype=torch.int32, device="cuda")
     h3b.h3b_gemm_i8_s32(to_dev(A), to_dev(W), Cg)
     out["gemm_s32"] = Cg.cpu().numpy()
+    # bf16-output epilogues at ragged sizes: 100 rows (a partial 32-row box) and 272 columns
+    # (a partial 32-column chunk); the gated residual's 34 rows per item straddle warps
+    M, N, K = 100, 272, 160
+    A = to_dev(r.integers(-127, 128, (M, K), dtype=np.int8))
+    W = to_dev(r.integers(-127, 128, (N, K), dtype=np.int8))
+    sa = to_dev(r.uniform(1e-3, 1e-2, M).astype(np.float32))
+    sw = to_dev(r.uniform(1e-3, 1e-2, N).astype(np.float32))
+    bias = to_dev((r.standard_normal(N) * 0.1).astype(np.float32))
+    o = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    h3b.h3b_gemm_i8_dequant(A, sa, W, sw, bias, o)
+    out["gemm_dequant"] = bf16_host(o)
+    g = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    am = torch.zeros(M, dtype=torch.float32, device="cuda")
+    h3b.h3b_gemm_i8_gelu(A, sa, W, sw, bias, g, am)
+    out["gemm_gelu"], out["gemm_gelu_absmax"] = bf16_host(g), am.cpu().numpy()
+    xr = bf16_dev(synth.f32_to_bf16_bits(r.standard_normal((M, N)).astype(np.float32)))
+    gate = to_dev(r.standard_normal((3, N)).astype(np.float32))
+    h3b.h3b_gemm_i8_gated_residual(A, sa, W, sw, bias, gate, 34, N, xr)
+    out["gemm_resid"] = bf16_host(xr)
     # QKV projection with RoPE, head-major
     wl = synth.WORKLOADS["d256_L512"]
     raw = synth.block_weights(wl)
@@ -120,4 +154,20 @@ def test_checked_build_matches_the_normal_build_and_records_nothing(tmp_path):
     for k, v in ref.items():
         if k in ("checked", "error_word"):
             continue
+        assert np.array_equal(got[k], v), k
+
+
+def test_launches_without_dependent_launch_match(tmp_path):
+    require_gpu()
+    ref = run_cases()
+    assert ref["checked"][0] == 0 and ref["error_word"][0] == 0
+    path = str(tmp_path / "no_pdl.npz")
+    env = dict(os.environ, H3B_PDL="0")
+    env.pop("H3B_CHECKED", None)
+    code = f"import sys; sys.path[:0] = [{HERE!r}, {os.path.dirname(HERE)!r}]; import test_gpu_checked as t; t.child({path!r})"
+    r = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-3000:]
+    got = dict(np.load(path))
+    assert got["checked"][0] == 0 and got["error_word"][0] == 0
+    for k, v in ref.items():
         assert np.array_equal(got[k], v), k

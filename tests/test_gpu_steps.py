@@ -203,7 +203,7 @@ def test_gemm_i8_dequant(M, N, K):
     no_device_error()
 
 
-@pytest.mark.parametrize("M,N,K", [(512, 1024, 256), (77, 8192, 2048)])
+@pytest.mark.parametrize("M,N,K", [(512, 1024, 256), (77, 8192, 2048), (77, 1040, 256)])
 def test_gemm_i8_gelu(M, N, K):
     qa, sa, qw, sw, bias = _quant_operands(M, N, K, 12)
     g = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
@@ -219,10 +219,12 @@ def test_gemm_i8_gelu(M, N, K):
 
 
 @pytest.mark.parametrize("M,N,K,items", [(512, 256, 256, 1), (256, 2048, 8192, 2), (100, 512, 1024, 1),
-                                         (100, 512, 1024, 3)])
+                                         (100, 512, 1024, 3), (100, 272, 160, 3)])
 def test_gemm_i8_gated_residual(M, N, K, items):
     """items=3 over 100 rows gives 34 rows per item, so some warps' 32 rows straddle two
-    items and read their gates row by row instead of from the staged per-item copy."""
+    items and read their gates row by row instead of from the staged per-item copy.
+    N=272 ends in a half-filled 32-column chunk: its x loads and its TMA-stored box are
+    cut at N."""
     qa, sa, qw, sw, bias = _quant_operands(M, N, K, 13)
     r = _rng(14)
     x = synth.f32_to_bf16_bits(r.standard_normal((M, N)).astype(np.float32))
