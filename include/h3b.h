@@ -31,6 +31,13 @@
  *     device index: use one CUDA context per device, and do not call
  *     cudaDeviceReset between calls (the cached addresses would be stale).
  *   - Every call is asynchronous on `stream` (NULL = legacy default stream).
+ *     Kernels are launched with programmatic stream serialization: a kernel may
+ *     start its setup while the kernel before it on the stream finishes, but it
+ *     waits for that grid (griddepcontrol.wait) before it reads or writes any
+ *     tensor, so stream order is kept for the caller's data. A caller's kernel
+ *     launched after a call without that attribute waits as usual; one launched
+ *     with it must itself wait before reading the call's outputs. The
+ *     environment variable H3B_PDL=0 turns the attribute off.
  *   - bf16 tensors are passed as `void*` (IEEE bfloat16 bit patterns).
  *   - Matrices are row-major. Weights are [out][in] (each output channel's input
  *     weights contiguous).

@@ -28,7 +28,10 @@
 // warp stages its columns' weight scales, bias and gate in shared memory before
 // the accumulator wait, requests the next 32 accumulator columns before
 // processing the current ones, and (QKV) reads the RoPE table from shared
-// memory. Every wait is bounded.
+// memory. The bf16 row-major outputs (dequant, GELU, gated residual) leave
+// through TMA tile stores from a per-warp 32 x 32 staging box, and the gated
+// residual's x arrives by coalesced loads that the same box turns into rows.
+// Every wait is bounded.
 #include <atomic>
 
 #include "h3b_common.cuh"
