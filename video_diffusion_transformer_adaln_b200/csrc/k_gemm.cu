@@ -302,8 +302,6 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, uint32_t tbase,
             v[4 * g] += b.x; v[4 * g + 1] += b.y; v[4 * g + 2] += b.z; v[4 * g + 3] += b.w;
           }
         }
-        // checked build: the last element this row's chunk writes lies inside the output
-        const bool out_ok = H3B_IDX_OK((long long)row * p.N + col0 + valid - 1, (long long)p.M * p.N, p.err);
         if (kEpi == EPI_DEQ) {
 #pragma unroll
           for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
@@ -364,7 +362,6 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, uint32_t tbase,
           if (H3B_IDX_OK((long long)off + 31, (long long)p.M * p.N, p.err))
             store_bf16x32(static_cast<__nv_bfloat16*>(p.out) + off, v, 32);
         }
-        (void)out_ok;
       }
     }
     if (kTmaStore) {
