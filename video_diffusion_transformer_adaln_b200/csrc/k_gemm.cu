@@ -247,7 +247,8 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, uint32_t tbase,
     item = row / p.rows_per_item;
   }
   float amax = 0.0f;
-  // the gated residual keeps its 128 prefetched x columns in registers instead
+  // the gated residual holds its prefetched x (16 vectors per thread) in the
+  // registers a second accumulator chunk would take, so it loads one chunk at a time
   constexpr bool kDoubleBuffer = kEpi != EPI_RESID;
   uint32_t r[kDoubleBuffer ? 2 : 1][32];
   tmem_ld32(tbase, r[0]);
